@@ -1,0 +1,223 @@
+/*
+ * coli_moe.h - C ABI of libcolimoe: one routed Mixture-of-Experts FFN layer with
+ * int4 expert weights (GLM-5.2 shape: hidden 6144, 256 routed experts + 1 shared,
+ * intermediate 2048, top-8), computed by hand-written sm_100a CUDA kernels.
+ *
+ * The layer, per token x (sources are web pages, cited by title and section):
+ *   1. Router   - z = W_r x (f32), s = sigmoid(z), sel = s + b; the k experts with
+ *                 the largest sel (ties to the lower index); weights
+ *                 w_j = s_j / sum(s) * routed_scale when norm_topk, else s_j * scale.
+ *                 ["解密GLM-5.2-colibri-int4-with-int8-mtp" 模型架构深度解析;
+ *                  "github一周涨11k⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.1, 四.3]
+ *   2. Union    - the batch's (token, slot) pairs grouped by expert, so every
+ *                 distinct expert is read once for all positions that chose it.
+ *                 [same article, 三.4 "Batch-union MoE"; "colibrì 實戰指南" 二]
+ *   3. Dequant  - w = float(q) * s, q a signed int4 nibble, s an f32 scale per row
+ *                 or per 64 columns.  ["jlnsrk/GLM-5.2-colibri-int4 - Hugging Face"
+ *                 container paragraph and conversion note; "colibrì 實戰指南" 三]
+ *   4. SwiGLU   - h = silu(W_g x) * (W_u x), silu(a) = a / (1 + exp(-a)).
+ *   5. Combine  - y = sum_j w_j * (W_d h)_j + sum over shared experts (weight 1).
+ *                 ["解密GLM-5.2-colibri-int4-with-int8-mtp" 模型架构深度解析: 1 shared]
+ *
+ * Conventions
+ *  - Every function returns an int: COLI_OK (0) or a negative coli_status.
+ *    coli_moe_last_error() gives a thread-local message for the last failure.
+ *  - The caller owns every buffer.  Pointers documented as "device" must be CUDA
+ *    device memory of the current device; "host" means ordinary host memory.
+ *    Apart from the small coli_moe_layer handle (host memory), the library
+ *    allocates nothing: calls that need scratch space take a device workspace
+ *    whose size coli_moe_workspace_size() reports.
+ *  - Device calls are asynchronous on the given stream (NULL = legacy default
+ *    stream) and never synchronise the host.  Launch errors are returned;
+ *    errors raised while kernels run surface at the next synchronisation.
+ *  - Calls that share a workspace must not overlap on the GPU.
+ *
+ * Matrix conventions: row-major [out, in]; gate and up are [I, H], down is [H, I].
+ *
+ * Container (host) layout of one quantised matrix [R, K] (coli_moe_quantize):
+ *    codes  U8  [R, K/2]    column c in byte c/2, even c in the low nibble,
+ *                           two's-complement signed nibble in [-8, 7]
+ *                           (the quantiser only emits [-7, 7])
+ *    scales F32 [R, K/G]    G = K (group 0, one scale per row) or 64
+ *
+ * Device layout of one expert ("blob", coli_moe_pack_expert): the container
+ * re-tiled for coalesced 16-byte loads; its dequantised values are identical.
+ *    For each matrix m in (gate, up, down) with R rows and K columns:
+ *      codes_m  [R/128][K/32][128][16 bytes]   unit (t, c, r) = row 128t + r,
+ *               columns 32c .. 32c+31 in container byte order
+ *      scales_m [R/128][K/G][128] f32          scale of row 128t + r, group g
+ *    Order: codes_gate, codes_up, codes_down, scales_gate, scales_up,
+ *    scales_down; each section starts on a 256-byte boundary and the blob size
+ *    is a multiple of 256 bytes.  All experts of a layer sit back to back in one
+ *    device buffer: routed experts 0 .. E-1, then the shared experts.
+ *
+ * Limits: H and I multiples of 128; group 0 or 64; 1 <= k <= 32; k <= E <= 1024;
+ * n_shared <= 4; 1 <= T <= 8192 tokens per call.
+ */
+#ifndef COLI_MOE_H
+#define COLI_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* coli_stream_t; /* same object as cudaStream_t */
+
+typedef enum coli_status {
+    COLI_OK = 0,
+    COLI_E_INVAL = -1,       /* bad argument, shape or pointer               */
+    COLI_E_CUDA = -2,        /* a CUDA runtime call or launch failed          */
+    COLI_E_NOMEM = -3,       /* host allocation failed                        */
+    COLI_E_UNSUPPORTED = -4, /* valid request this build does not implement   */
+    COLI_E_WORKSPACE = -5,   /* workspace missing or smaller than required    */
+    COLI_E_TIMEOUT = -6      /* a device-side bounded wait gave up            */
+} coli_status;
+
+typedef enum coli_dtype { COLI_F32 = 0, COLI_BF16 = 1 } coli_dtype;
+
+typedef enum coli_path {
+    COLI_PATH_AUTO = 0, /* choose by batch size                              */
+    COLI_PATH_GEMV = 1, /* CUDA-core int4 GEMV, f32 arithmetic throughout      */
+    COLI_PATH_GEMM = 2  /* tcgen05 grouped GEMM, bf16 operands, f32 accumulate */
+} coli_path;
+
+/* Thread-local description of the last error returned on this thread. */
+const char* coli_moe_last_error(void);
+
+/* ------------------------------------------------------------------------ */
+/* Container                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Quantise a host row-major f32 matrix [rows, cols] into the container layout
+ * ("jlnsrk/GLM-5.2-colibri-int4 - Hugging Face": U8 packed nibbles + F32 scales;
+ * conversion note: np.rint, i.e. round half to even).  Per row (group 0) or per
+ * 64 columns: s = max|w| / 7 (f32 division); q = rint(w / s) clamped to [-7, 7]
+ * (f32 division, half to even); s == 0 gives q = 0.
+ * Host pointers: w [rows*cols], packed [rows*cols/2], scales [rows*cols/G].
+ * Errors: COLI_E_INVAL for NULL pointers, rows < 0, odd cols, group not 0/64 or
+ * cols not a multiple of 64 when grouped. */
+int coli_moe_quantize(const float* w, int64_t rows, int64_t cols, int32_t group,
+                      uint8_t* packed, float* scales);
+
+/* Bytes of one expert blob in the device layout (see top of file). */
+int coli_moe_expert_bytes(int32_t H, int32_t I, int32_t group, size_t* bytes);
+
+/* Re-tile one expert's three container matrices (host memory, as written by
+ * coli_moe_quantize) into one blob in the device layout (host memory, size
+ * coli_moe_expert_bytes).  The blob keeps the three matrices adjacent, as the
+ * engine stores an expert ("colibrì 實戰指南" 二: one read per expert).
+ * Errors: COLI_E_INVAL for NULL pointers or unsupported shapes. */
+int coli_moe_pack_expert(int32_t H, int32_t I, int32_t group,
+                         const uint8_t* gate_codes, const float* gate_scales,
+                         const uint8_t* up_codes, const float* up_scales,
+                         const uint8_t* down_codes, const float* down_scales,
+                         void* blob);
+
+/* Device-side quantise + pack of one expert from f32 masters (device memory:
+ * gate, up [I, H], down [H, I]) straight into a device blob; bit-identical to
+ * coli_moe_quantize followed by coli_moe_pack_expert.  Asynchronous. */
+int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group,
+                                    const float* gate, const float* up,
+                                    const float* down, void* blob,
+                                    coli_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Layer                                                                     */
+/* ------------------------------------------------------------------------ */
+
+typedef struct coli_moe_desc {
+    int32_t H;             /* hidden size                                    */
+    int32_t I;             /* expert intermediate size (routed and shared)   */
+    int32_t E;             /* routed experts                                 */
+    int32_t k;             /* experts per token                              */
+    int32_t n_shared;      /* shared experts, always applied with weight 1   */
+    int32_t group;         /* 0 = per-row scales, 64 = per-64-column scales  */
+    float routed_scale;    /* multiplies the routed weights (1.0 for GLM-5.2)*/
+    int32_t norm_topk;     /* 1: renormalise the k scores to sum to 1        */
+    const float* router_w; /* device f32 [E, H]                              */
+    const float* router_b; /* device f32 [E], selection bias                 */
+    const void* experts;   /* device, (E + n_shared) blobs back to back      */
+} coli_moe_desc;
+
+typedef struct coli_moe_layer coli_moe_layer;
+
+/* Validate a descriptor and make a handle (host memory only; the device
+ * buffers it points to stay owned by the caller and must outlive it). */
+int coli_moe_layer_create(const coli_moe_desc* desc, coli_moe_layer** out);
+int coli_moe_layer_destroy(coli_moe_layer* layer);
+
+/* Workspace bytes that coli_moe_route / coli_moe_forward need for T tokens. */
+int coli_moe_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes);
+
+/* Step 1 alone.  x device [T, H] (f32 or bf16); idx device i32 [T, k] ordered
+ * by (sel desc, expert asc); w device f32 [T, k]. */
+int coli_moe_route(const coli_moe_layer* layer, const void* x, coli_dtype xt,
+                   int32_t T, int32_t* idx, float* w, void* ws, size_t ws_bytes,
+                   coli_stream_t stream);
+
+/* Step 2 alone, for idx device i32 [T, k] with entries in [0, E): offsets
+ * [E+1] (exclusive prefix of per-expert counts), pair_tok / pair_slot [T*k]
+ * (pairs sorted by expert, then token), uniq [E] (ascending experts with at
+ * least one pair; entries past n_uniq are left untouched), n_uniq [1].  All
+ * device i32.  Needs no workspace.  Out-of-range expert ids give undefined
+ * (but in-bounds) output. */
+int coli_moe_union(const int32_t* idx, int32_t T, int32_t k, int32_t E,
+                   int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot,
+                   int32_t* uniq, int32_t* n_uniq, coli_stream_t stream);
+
+/* Steps 1-5: writes y device f32 [T, H] (overwrites; no accumulation). */
+int coli_moe_forward(const coli_moe_layer* layer, const void* x, coli_dtype xt,
+                     int32_t T, float* y, void* ws, size_t ws_bytes,
+                     coli_stream_t stream);
+
+/* Stage boundaries of coli_moe_forward_ex, for optional event timing. */
+typedef enum coli_stage {
+    COLI_STAGE_ROUTER = 0,  /* router logits + sigmoid/top-k              */
+    COLI_STAGE_UNION = 1,   /* batch union and expert work list           */
+    COLI_STAGE_GATEUP = 2,  /* gate/up expert kernel with SwiGLU          */
+    COLI_STAGE_DOWN = 3,    /* down expert kernel                         */
+    COLI_STAGE_COMBINE = 4, /* weighted combine + shared + residual       */
+    COLI_STAGES = 5
+} coli_stage;
+
+/* coli_moe_forward with options: path selects the expert kernels; residual
+ * (device f32 [T, H] or NULL) is added to the output (it may alias y);
+ * idx_out / w_out (device, may be NULL) receive the routing decision.
+ * events (may be NULL) is an array of COLI_STAGES + 1 cudaEvent_t created by
+ * the caller; events[s] is recorded on `stream` just before stage s and
+ * events[COLI_STAGES] after the last one, so cudaEventElapsedTime(events[s],
+ * events[s+1]) is the device time of stage s. */
+int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x,
+                        coli_dtype xt, int32_t T, float* y,
+                        const float* residual, coli_path path, int32_t* idx_out,
+                        float* w_out, void* const* events, void* ws,
+                        size_t ws_bytes, coli_stream_t stream);
+
+/* RMSNorm with unit gain, per row: out = x / sqrt(mean(x^2) + eps).  Device f32
+ * [T, H]; out may alias x. */
+int coli_moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps, float* out,
+                     coli_stream_t stream);
+
+/* L stacked layers on a residual stream x (device f32 [T, H], updated in
+ * place): x <- x + layer_l(rmsnorm(x)) for l = 0 .. L-1.  All layers must share
+ * H; ws must cover the largest coli_moe_workspace_size(layers[l], T) plus
+ * 4*T*H bytes (reported by coli_moe_stack_workspace_size). */
+int coli_moe_stack_workspace_size(const coli_moe_layer* const* layers, int32_t L,
+                                  int32_t T, size_t* bytes);
+int coli_moe_stack_forward(const coli_moe_layer* const* layers, int32_t L,
+                           float* x, int32_t T, float eps, coli_path path,
+                           void* ws, size_t ws_bytes, coli_stream_t stream);
+
+/* Test helper: dequantise matrix `which` (0 gate, 1 up, 2 down) of expert
+ * `expert` (0 .. E + n_shared - 1) from the device blob into out (device f32,
+ * row-major [R, K] in container order). */
+int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert,
+                           int32_t which, float* out, coli_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COLI_MOE_H */

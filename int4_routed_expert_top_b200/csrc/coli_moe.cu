@@ -1,0 +1,487 @@
+// coli_moe.cu - C ABI of libcolimoe (see include/coli_moe.h).
+//
+// Host code validates arguments, plans the caller's workspace and launches the
+// kernels of route.cuh, gemv.cuh, gemm.cuh and misc.cuh on the caller's
+// stream.  Nothing here synchronises the host or allocates device memory.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "coli_moe.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "gemv.cuh"
+#include "misc.cuh"
+#include "route.cuh"
+
+using namespace coli;
+
+struct coli_moe_layer {
+    coli_moe_desc d;
+    BlobLayout L;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int check_launch(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(COLI_E_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return COLI_OK;
+}
+
+cudaStream_t S(coli_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool shape_ok(int H, int I, int group) {
+    return H > 0 && I > 0 && H % 128 == 0 && I % 128 == 0 && (group == 0 || group == 64);
+}
+
+// ---------------------------------------------------------------------------
+// workspace plan
+// ---------------------------------------------------------------------------
+struct WsPlan {
+    int64_t zpart, idx, w, offsets, pair_tok, pair_slot, uniq, n_uniq, inv;
+    int64_t unit_expert, unit_begin, unit_end, n_units, h, o, xb, total;
+};
+
+constexpr int kMaxKS = 8;
+
+WsPlan plan_ws(const coli_moe_desc& d, int T) {
+    WsPlan p;
+    int64_t off = 0;
+    auto take = [&](int64_t bytes) { const int64_t at = off; off = align256(off + bytes); return at; };
+    const int64_t Tk = (int64_t)T * d.k;
+    const int64_t P = (int64_t)T * (d.k + d.n_shared);
+    p.zpart = take((int64_t)kMaxKS * T * d.E * 4);
+    p.idx = take(Tk * 4);
+    p.w = take(Tk * 4);
+    p.offsets = take((int64_t)(d.E + 1) * 4);
+    p.pair_tok = take(P * 4);
+    p.pair_slot = take(Tk * 4);
+    p.uniq = take((int64_t)d.E * 4);
+    p.n_uniq = take(4);
+    p.inv = take(Tk * 4);
+    p.unit_expert = take((int64_t)(d.E + d.n_shared) * 4);
+    p.unit_begin = take((int64_t)(d.E + d.n_shared) * 4);
+    p.unit_end = take((int64_t)(d.E + d.n_shared) * 4);
+    p.n_units = take(4);
+    p.h = take(P * d.I * 4);
+    p.o = take(P * d.H * 4);
+    p.xb = take((int64_t)T * d.H * 2);  // bf16 copy of x for the tensor-core path
+    p.total = off;
+    return p;
+}
+
+template <typename T> T* at(void* ws, int64_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int tokens_ok(const coli_moe_desc& d, int T) {
+    if (T < 1 || T > 8192) return fail(COLI_E_INVAL, "T=%d outside [1, 8192]", T);
+    const int64_t words = (int64_t)d.E * ((T + 31) / 32);
+    if (words > 24576)
+        return fail(COLI_E_UNSUPPORTED, "E*ceil(T/32)=%lld exceeds 24576 (union bitmap)",
+                    (long long)words);
+    return COLI_OK;
+}
+
+int set_smem(const void* fn, int bytes) {
+    if (bytes <= 48 * 1024) return COLI_OK;
+    const cudaError_t e =
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return fail(COLI_E_CUDA, "smem attribute: %s", cudaGetErrorString(e));
+    return COLI_OK;
+}
+
+// router logits into zpart; returns the number of K slices used (or < 0)
+int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, float* zpart,
+                  cudaStream_t st, int* ks_out) {
+    int KS = 1;
+    if (T <= 32) {
+        for (int c : {8, 4, 2, 1})
+            if (d.H % (c * 128) == 0) { KS = c; break; }
+        const int warps = d.E * KS;
+        const dim3 grid((warps + 7) / 8);
+        if (xt == COLI_F32)
+            router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart);
+        else
+            router_gemv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart);
+    } else {
+        const int tiles = ((T + 63) / 64) * ((d.E + 63) / 64);
+        for (int c : {8, 4, 2, 1})
+            if (d.H % (c * 16) == 0 && (tiles * c <= 2 * 148 || c == 1)) { KS = c; break; }
+        const dim3 grid((T + 63) / 64, (d.E + 63) / 64, KS);
+        if (xt == COLI_F32)
+            router_tiled_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart);
+        else
+            router_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart);
+    }
+    *ks_out = KS;
+    return check_launch("router");
+}
+
+int launch_topk(const coli_moe_desc& d, const float* zpart, int KS, int T, int32_t* idx,
+                float* w, cudaStream_t st) {
+    const int smem = kTopkWarps * 2 * d.E * 4;
+    topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, 32 * kTopkWarps, smem, st>>>(
+        zpart, KS, T, d.E, d.router_b, d.k, d.routed_scale, d.norm_topk, idx, w);
+    return check_launch("topk");
+}
+
+int launch_union(const int32_t* idx, int T, int k, int E, const UnionOut& o, cudaStream_t st) {
+    const int W = (T + 31) / 32;
+    const int smem = (int)((int64_t)E * W * 4 + 3 * (int64_t)E * 4);
+    int rc = set_smem((const void*)union_kernel, smem);
+    if (rc) return rc;
+    union_kernel<<<1, kUnionThreads, smem, st>>>(idx, T, k, E, o);
+    return check_launch("union");
+}
+
+template <typename Mark>
+int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const void* x,
+                coli_dtype xt, cudaStream_t st, Mark&& mark) {
+    const coli_moe_desc& d = l->d;
+    GemvArgs a;
+    a.experts = static_cast<const uint8_t*>(d.experts);
+    a.blob_bytes = l->L.bytes;
+    a.L = l->L;
+    a.n_units = at<int32_t>(ws, p.n_units);
+    a.unit_expert = at<int32_t>(ws, p.unit_expert);
+    a.unit_begin = at<int32_t>(ws, p.unit_begin);
+    a.unit_end = at<int32_t>(ws, p.unit_end);
+    a.pair_tok = at<int32_t>(ws, p.pair_tok);
+    a.x = x;
+    a.h = at<float>(ws, p.h);
+    a.o = at<float>(ws, p.o);
+    a.H = d.H; a.I = d.I; a.group = d.group;
+    const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;
+    const int tc = std::min(kGemvTC, T);
+    int rc;
+    const int smem_gu = tc * d.H * 4, smem_dn = tc * d.I * 4;
+    if (xt == COLI_F32) {
+        if ((rc = set_smem((const void*)expert_gemv_kernel<true, float>, smem_gu))) return rc;
+        expert_gemv_kernel<true, float><<<units_max * (d.I / 32), kGemvWarps * 32, smem_gu, st>>>(a);
+    } else {
+        if ((rc = set_smem((const void*)expert_gemv_kernel<true, __nv_bfloat16>, smem_gu))) return rc;
+        expert_gemv_kernel<true, __nv_bfloat16><<<units_max * (d.I / 32), kGemvWarps * 32, smem_gu, st>>>(a);
+    }
+    if ((rc = check_launch("gate/up gemv"))) return rc;
+    if ((rc = mark(COLI_STAGE_DOWN))) return rc;
+    if ((rc = set_smem((const void*)expert_gemv_kernel<false, float>, smem_dn))) return rc;
+    expert_gemv_kernel<false, float><<<units_max * (d.H / 32), kGemvWarps * 32, smem_dn, st>>>(a);
+    return check_launch("down gemv");
+}
+
+int launch_combine(const coli_moe_desc& d, int T, void* ws, const WsPlan& p,
+                   const float* residual, float* y, cudaStream_t st) {
+    const int64_t n = (int64_t)T * (d.H / 4);
+    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        at<float>(ws, p.o), at<int32_t>(ws, p.inv), at<float>(ws, p.w), T, d.k, d.n_shared,
+        d.H, residual, y);
+    return check_launch("combine");
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* coli_moe_last_error(void) { return g_err.c_str(); }
+
+int coli_moe_quantize(const float* w, int64_t rows, int64_t cols, int32_t group,
+                      uint8_t* packed, float* scales) {
+    if (!w || !packed || !scales) return fail(COLI_E_INVAL, "quantize: NULL pointer");
+    if (rows < 0 || cols <= 0 || cols % 2 || (group != 0 && group != 64) ||
+        (group && cols % group))
+        return fail(COLI_E_INVAL, "quantize: bad shape rows=%lld cols=%lld group=%d",
+                    (long long)rows, (long long)cols, group);
+    const int64_t gs = group ? group : cols, ng = cols / gs;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* row = w + r * cols;
+        uint8_t* prow = packed + r * (cols / 2);
+        for (int64_t g = 0; g < ng; ++g) {
+            float m = 0.0f;
+            for (int64_t c = g * gs; c < (g + 1) * gs; ++c) m = std::fmax(m, std::fabs(row[c]));
+            const float s = m / 7.0f;
+            scales[r * ng + g] = s;
+            for (int64_t c = g * gs; c < (g + 1) * gs; c += 2) {
+                int q[2];
+                for (int i = 0; i < 2; ++i) {
+                    float v = s == 0.0f ? 0.0f : std::rint(row[c + i] / s);
+                    v = std::fmin(std::fmax(v, -7.0f), 7.0f);
+                    q[i] = (int)v;
+                }
+                prow[c / 2] = (uint8_t)((q[0] & 15) | ((q[1] & 15) << 4));
+            }
+        }
+    }
+    return COLI_OK;
+}
+
+int coli_moe_expert_bytes(int32_t H, int32_t I, int32_t group, size_t* bytes) {
+    if (!bytes) return fail(COLI_E_INVAL, "expert_bytes: NULL pointer");
+    if (!shape_ok(H, I, group)) return fail(COLI_E_INVAL, "expert_bytes: bad shape");
+    *bytes = (size_t)make_blob_layout(H, I, group).bytes;
+    return COLI_OK;
+}
+
+int coli_moe_pack_expert(int32_t H, int32_t I, int32_t group, const uint8_t* gate_codes,
+                         const float* gate_scales, const uint8_t* up_codes,
+                         const float* up_scales, const uint8_t* down_codes,
+                         const float* down_scales, void* blob) {
+    if (!gate_codes || !gate_scales || !up_codes || !up_scales || !down_codes ||
+        !down_scales || !blob)
+        return fail(COLI_E_INVAL, "pack_expert: NULL pointer");
+    if (!shape_ok(H, I, group)) return fail(COLI_E_INVAL, "pack_expert: bad shape");
+    const BlobLayout L = make_blob_layout(H, I, group);
+    uint8_t* out = static_cast<uint8_t*>(blob);
+    std::memset(out, 0, (size_t)L.bytes);
+    const uint8_t* codes[3] = {gate_codes, up_codes, down_codes};
+    const float* scales[3] = {gate_scales, up_scales, down_scales};
+    for (int m = 0; m < 3; ++m) {
+        const int R = L.rows[m], K = L.cols[m], ng = L.ngroups[m];
+        for (int r = 0; r < R; ++r) {
+            for (int c = 0; c < K / 32; ++c)
+                std::memcpy(out + L.codes[m] + code_unit_offset(r, c, K),
+                            codes[m] + (int64_t)r * (K / 2) + 16 * c, 16);
+            for (int g = 0; g < ng; ++g)
+                reinterpret_cast<float*>(out + L.scales[m])[scale_offset(r, g, ng)] =
+                    scales[m][(int64_t)r * ng + g];
+        }
+    }
+    return COLI_OK;
+}
+
+int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group, const float* gate,
+                                    const float* up, const float* down, void* blob,
+                                    coli_stream_t stream) {
+    if (!gate || !up || !down || !blob) return fail(COLI_E_INVAL, "quantize_expert_device: NULL pointer");
+    if (!shape_ok(H, I, group)) return fail(COLI_E_INVAL, "quantize_expert_device: bad shape");
+    const BlobLayout L = make_blob_layout(H, I, group);
+    uint8_t* b = static_cast<uint8_t*>(blob);
+    const float* src[3] = {gate, up, down};
+    for (int m = 0; m < 3; ++m) {
+        const int R = L.rows[m], K = L.cols[m];
+        const int smem = 8 * (K / 2);
+        int rc = set_smem((const void*)quantize_rows_kernel, smem);
+        if (rc) return rc;
+        quantize_rows_kernel<<<(R + 7) / 8, 256, smem, S(stream)>>>(
+            src[m], R, K, group, b + L.codes[m], reinterpret_cast<float*>(b + L.scales[m]));
+        if ((rc = check_launch("quantize_rows"))) return rc;
+    }
+    return COLI_OK;
+}
+
+int coli_moe_layer_create(const coli_moe_desc* desc, coli_moe_layer** out) {
+    if (!desc || !out) return fail(COLI_E_INVAL, "layer_create: NULL pointer");
+    const coli_moe_desc& d = *desc;
+    if (!shape_ok(d.H, d.I, d.group)) return fail(COLI_E_INVAL, "layer_create: H, I must be multiples of 128, group 0 or 64");
+    if (d.E < 1 || d.E > 1024 || d.k < 1 || d.k > 32 || d.k > d.E || d.n_shared < 0 || d.n_shared > 4)
+        return fail(COLI_E_INVAL, "layer_create: need 1<=k<=min(E,32), E<=1024, 0<=n_shared<=4");
+    if (!d.router_w || !d.router_b || !d.experts) return fail(COLI_E_INVAL, "layer_create: NULL device pointer");
+    if (!(std::isfinite(d.routed_scale))) return fail(COLI_E_INVAL, "layer_create: routed_scale not finite");
+    coli_moe_layer* l = new (std::nothrow) coli_moe_layer;
+    if (!l) return fail(COLI_E_NOMEM, "layer_create: out of host memory");
+    l->d = d;
+    l->L = make_blob_layout(d.H, d.I, d.group);
+    *out = l;
+    return COLI_OK;
+}
+
+int coli_moe_layer_destroy(coli_moe_layer* layer) {
+    delete layer;
+    return COLI_OK;
+}
+
+int coli_moe_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes) {
+    if (!layer || !bytes) return fail(COLI_E_INVAL, "workspace_size: NULL pointer");
+    int rc = tokens_ok(layer->d, T);
+    if (rc) return rc;
+    *bytes = (size_t)plan_ws(layer->d, T).total;
+    return COLI_OK;
+}
+
+int coli_moe_route(const coli_moe_layer* layer, const void* x, coli_dtype xt, int32_t T,
+                   int32_t* idx, float* w, void* ws, size_t ws_bytes, coli_stream_t stream) {
+    if (!layer || !x || !idx || !w) return fail(COLI_E_INVAL, "route: NULL pointer");
+    if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_E_INVAL, "route: bad dtype");
+    int rc = tokens_ok(layer->d, T);
+    if (rc) return rc;
+    const WsPlan p = plan_ws(layer->d, T);
+    if (!ws || ws_bytes < (size_t)p.total)
+        return fail(COLI_E_WORKSPACE, "route: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
+    int KS;
+    if ((rc = launch_router(layer->d, x, xt, T, at<float>(ws, p.zpart), S(stream), &KS))) return rc;
+    return launch_topk(layer->d, at<float>(ws, p.zpart), KS, T, idx, w, S(stream));
+}
+
+int coli_moe_union(const int32_t* idx, int32_t T, int32_t k, int32_t E, int32_t* offsets,
+                   int32_t* pair_tok, int32_t* pair_slot, int32_t* uniq, int32_t* n_uniq,
+                   coli_stream_t stream) {
+    if (!idx || !offsets || !pair_tok || !pair_slot || !uniq || !n_uniq)
+        return fail(COLI_E_INVAL, "union: NULL pointer");
+    if (E < 1 || E > 1024 || k < 1 || k > 32 || T < 1 || T > 8192)
+        return fail(COLI_E_INVAL, "union: bad sizes T=%d k=%d E=%d", T, k, E);
+    if ((int64_t)E * ((T + 31) / 32) > 24576) return fail(COLI_E_UNSUPPORTED, "union: E*ceil(T/32) > 24576");
+    UnionOut o{};
+    o.offsets = offsets; o.pair_tok = pair_tok; o.pair_slot = pair_slot;
+    o.uniq = uniq; o.n_uniq = n_uniq;
+    return launch_union(idx, T, k, E, o, S(stream));
+}
+
+int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype xt, int32_t T,
+                        float* y, const float* residual, coli_path path, int32_t* idx_out,
+                        float* w_out, void* const* events, void* ws, size_t ws_bytes,
+                        coli_stream_t stream) {
+    if (!layer || !x || !y) return fail(COLI_E_INVAL, "forward: NULL pointer");
+    if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_E_INVAL, "forward: bad dtype");
+    if (path != COLI_PATH_AUTO && path != COLI_PATH_GEMV && path != COLI_PATH_GEMM)
+        return fail(COLI_E_INVAL, "forward: bad path");
+    const coli_moe_desc& d = layer->d;
+    int rc = tokens_ok(d, T);
+    if (rc) return rc;
+    const WsPlan p = plan_ws(d, T);
+    if (!ws || ws_bytes < (size_t)p.total)
+        return fail(COLI_E_WORKSPACE, "forward: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
+    if (path == COLI_PATH_AUTO) path = gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV;
+    cudaStream_t st = S(stream);
+    int32_t* idx = at<int32_t>(ws, p.idx);
+    float* w = at<float>(ws, p.w);
+    auto mark = [&](int s) -> int {
+        if (!events || !events[s]) return COLI_OK;
+        if (cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[s]), st) != cudaSuccess)
+            return fail(COLI_E_CUDA, "forward: event record failed");
+        return COLI_OK;
+    };
+    int KS;
+    if ((rc = mark(COLI_STAGE_ROUTER))) return rc;
+    if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), st, &KS))) return rc;
+    if ((rc = launch_topk(d, at<float>(ws, p.zpart), KS, T, idx, w, st))) return rc;
+    UnionOut o{};
+    o.offsets = at<int32_t>(ws, p.offsets);
+    o.pair_tok = at<int32_t>(ws, p.pair_tok);
+    o.pair_slot = at<int32_t>(ws, p.pair_slot);
+    o.uniq = at<int32_t>(ws, p.uniq);
+    o.n_uniq = at<int32_t>(ws, p.n_uniq);
+    o.inv = at<int32_t>(ws, p.inv);
+    o.unit_expert = at<int32_t>(ws, p.unit_expert);
+    o.unit_begin = at<int32_t>(ws, p.unit_begin);
+    o.unit_end = at<int32_t>(ws, p.unit_end);
+    o.n_units = at<int32_t>(ws, p.n_units);
+    o.n_shared = d.n_shared;
+    if ((rc = mark(COLI_STAGE_UNION))) return rc;
+    if ((rc = launch_union(idx, T, d.k, d.E, o, st))) return rc;
+    if ((rc = mark(COLI_STAGE_GATEUP))) return rc;
+    if (path == COLI_PATH_GEMM) {
+        GemmCtx g;
+        g.experts = static_cast<const uint8_t*>(d.experts);
+        g.blob_bytes = layer->L.bytes;
+        g.L = layer->L;
+        g.H = d.H; g.I = d.I; g.group = d.group; g.E = d.E; g.n_shared = d.n_shared;
+        g.T = T; g.k = d.k;
+        g.n_units = o.n_units; g.unit_expert = o.unit_expert;
+        g.unit_begin = o.unit_begin; g.unit_end = o.unit_end; g.pair_tok = o.pair_tok;
+        g.x = x; g.x_bf16 = xt == COLI_BF16;
+        g.xb = at<__nv_bfloat16>(ws, p.xb);
+        g.h = at<__nv_bfloat16>(ws, p.h);
+        g.o = at<float>(ws, p.o);
+        if ((rc = launch_gemm(g, st, mark))) return rc;
+    } else {
+        if ((rc = launch_gemv(layer, T, ws, p, x, xt, st, mark))) return rc;
+    }
+    if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
+    if ((rc = launch_combine(d, T, ws, p, residual, y, st))) return rc;
+    if ((rc = mark(COLI_STAGES))) return rc;
+    if (idx_out) {
+        if (cudaMemcpyAsync(idx_out, idx, sizeof(int32_t) * T * d.k, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return fail(COLI_E_CUDA, "forward: copy idx");
+    }
+    if (w_out) {
+        if (cudaMemcpyAsync(w_out, w, sizeof(float) * T * d.k, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return fail(COLI_E_CUDA, "forward: copy w");
+    }
+    return COLI_OK;
+}
+
+int coli_moe_forward(const coli_moe_layer* layer, const void* x, coli_dtype xt, int32_t T,
+                     float* y, void* ws, size_t ws_bytes, coli_stream_t stream) {
+    return coli_moe_forward_ex(layer, x, xt, T, y, nullptr, COLI_PATH_AUTO, nullptr, nullptr,
+                               nullptr, ws, ws_bytes, stream);
+}
+
+int coli_moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps, float* out,
+                     coli_stream_t stream) {
+    if (!x || !out) return fail(COLI_E_INVAL, "rmsnorm: NULL pointer");
+    if (T < 1 || H < 4 || H % 4) return fail(COLI_E_INVAL, "rmsnorm: bad shape");
+    rmsnorm_kernel<<<T, 256, 0, S(stream)>>>(x, H, eps, out);
+    return check_launch("rmsnorm");
+}
+
+int coli_moe_stack_workspace_size(const coli_moe_layer* const* layers, int32_t L, int32_t T,
+                                  size_t* bytes) {
+    if (!layers || !bytes || L < 1) return fail(COLI_E_INVAL, "stack_workspace_size: bad arguments");
+    size_t mx = 0;
+    for (int l = 0; l < L; ++l) {
+        if (!layers[l]) return fail(COLI_E_INVAL, "stack: NULL layer");
+        size_t b;
+        int rc = coli_moe_workspace_size(layers[l], T, &b);
+        if (rc) return rc;
+        mx = std::max(mx, b);
+        if (layers[l]->d.H != layers[0]->d.H) return fail(COLI_E_INVAL, "stack: layers differ in H");
+    }
+    *bytes = (size_t)align256((int64_t)mx) + (size_t)T * layers[0]->d.H * 4;
+    return COLI_OK;
+}
+
+int coli_moe_stack_forward(const coli_moe_layer* const* layers, int32_t L, float* x, int32_t T,
+                           float eps, coli_path path, void* ws, size_t ws_bytes,
+                           coli_stream_t stream) {
+    size_t need;
+    int rc = coli_moe_stack_workspace_size(layers, L, T, &need);
+    if (rc) return rc;
+    if (!x) return fail(COLI_E_INVAL, "stack_forward: NULL x");
+    if (!ws || ws_bytes < need) return fail(COLI_E_WORKSPACE, "stack_forward: workspace %zu < %zu", ws_bytes, need);
+    const int H = layers[0]->d.H;
+    const size_t layer_ws = need - (size_t)T * H * 4;
+    float* xn = reinterpret_cast<float*>(static_cast<char*>(ws) + layer_ws);
+    for (int l = 0; l < L; ++l) {
+        if ((rc = coli_moe_rmsnorm(x, T, H, eps, xn, stream))) return rc;
+        if ((rc = coli_moe_forward_ex(layers[l], xn, COLI_F32, T, x, x, path, nullptr, nullptr,
+                                      nullptr, ws, layer_ws, stream)))
+            return rc;
+    }
+    return COLI_OK;
+}
+
+int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t which,
+                           float* out, coli_stream_t stream) {
+    if (!layer || !out) return fail(COLI_E_INVAL, "dequant_debug: NULL pointer");
+    const coli_moe_desc& d = layer->d;
+    if (expert < 0 || expert >= d.E + d.n_shared || which < 0 || which > 2)
+        return fail(COLI_E_INVAL, "dequant_debug: expert %d / matrix %d out of range", expert, which);
+    const BlobLayout& L = layer->L;
+    const uint8_t* blob = static_cast<const uint8_t*>(d.experts) + (int64_t)expert * L.bytes;
+    const int R = L.rows[which], K = L.cols[which];
+    const int64_t n = (int64_t)R * (K / 32);
+    dequant_kernel<<<(unsigned)((n + 255) / 256), 256, 0, S(stream)>>>(
+        blob + L.codes[which], reinterpret_cast<const float*>(blob + L.scales[which]), R, K,
+        d.group, out);
+    return check_launch("dequant");
+}
+
+}  // extern "C"

@@ -1,0 +1,99 @@
+// misc.cuh - device quantiser/packer, dequantiser (test helper) and RMSNorm.
+//
+// Quantiser ("jlnsrk/GLM-5.2-colibri-int4 - Hugging Face": container paragraph
+// and conversion note): per row or per 64 columns s = max|w| / 7, q =
+// rint(w / s) in [-7, 7] (IEEE f32 division, round half to even), written
+// straight into the tiled device layout.
+#pragma once
+
+#include "common.cuh"
+
+namespace coli {
+
+__device__ __forceinline__ int quant_one(float v, float s) {
+    if (s == 0.0f) return 0;
+    float q = rintf(__fdiv_rn(v, s));
+    q = fminf(fmaxf(q, -7.0f), 7.0f);
+    return (int)q;
+}
+
+// one warp per row; the row's packed bytes are assembled in shared memory and
+// written out as 16-byte units of the device layout
+__global__ void __launch_bounds__(256)
+quantize_rows_kernel(const float* __restrict__ w, int R, int K, int group,
+                     uint8_t* __restrict__ codes, float* __restrict__ scales) {
+    extern __shared__ uint4 qz_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 8 + warp;
+    if (r >= R) return;
+    uint8_t* buf = reinterpret_cast<uint8_t*>(qz_smem) + (int64_t)warp * (K / 2);
+    const float* row = w + (int64_t)r * K;
+    const int gs = group ? group : K;
+    const int ng = K / gs;
+    for (int g = 0; g < ng; ++g) {
+        float m = 0.0f;
+        for (int c = g * gs + lane; c < (g + 1) * gs; c += 32) m = fmaxf(m, fabsf(row[c]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float s = __fdiv_rn(m, 7.0f);
+        if (lane == 0) scales[scale_offset(r, g, ng)] = s;
+        for (int cp = g * gs / 2 + lane; cp < (g + 1) * gs / 2; cp += 32) {
+            const int q0 = quant_one(row[2 * cp], s), q1 = quant_one(row[2 * cp + 1], s);
+            buf[cp] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
+        }
+    }
+    __syncwarp();
+    for (int c = lane; c < K / 32; c += 32)
+        *reinterpret_cast<uint4*>(codes + code_unit_offset(r, c, K)) =
+            *reinterpret_cast<const uint4*>(buf + 16 * c);
+}
+
+// one thread per (row, 16-byte unit): out[r, c] = (float)q * s
+__global__ void __launch_bounds__(256)
+dequant_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ scales,
+               int R, int K, int group, float* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    const int KC = K / 32;
+    if (i >= (int64_t)R * KC) return;
+    const int r = (int)(i / KC), c = (int)(i % KC);
+    const int ng = group ? K / group : 1;
+    const uint4 v = *reinterpret_cast<const uint4*>(codes + code_unit_offset(r, c, K));
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    for (int j = 0; j < 32; ++j) {
+        const int col = 32 * c + j;
+        int n = (wd[j / 8] >> (4 * (j % 8))) & 15;
+        n = n >= 8 ? n - 16 : n;
+        const float s = scales[scale_offset(r, group ? col / group : 0, ng)];
+        out[(int64_t)r * K + col] = __fmul_rn((float)n, s);
+    }
+}
+
+// RMSNorm with unit gain: one CTA per row, f32 sum of squares
+__global__ void __launch_bounds__(256)
+rmsnorm_kernel(const float* x, int H, float eps, float* out) {
+    __shared__ float part[8];
+    const int64_t t = blockIdx.x;
+    const float* xr = x + t * H;
+    float ss = 0.0f;
+    for (int c = threadIdx.x * 4; c < H; c += 1024) {
+        const float4 v = *reinterpret_cast<const float4*>(xr + c);
+        ss = fmaf(v.x, v.x, ss); ss = fmaf(v.y, v.y, ss);
+        ss = fmaf(v.z, v.z, ss); ss = fmaf(v.w, v.w, ss);
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tot += part[i];
+    const float inv = 1.0f / sqrtf(tot / (float)H + eps);
+    __syncthreads();  // every thread has read part before out (may alias x) changes
+    float* orow = out + t * H;
+    for (int c = threadIdx.x * 4; c < H; c += 1024) {
+        float4 v = *reinterpret_cast<const float4*>(xr + c);
+        v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+        *reinterpret_cast<float4*>(orow + c) = v;
+    }
+}
+
+}  // namespace coli

@@ -27,3 +27,11 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    # compile the oracle and the CUDA library in-tree when they are missing or stale
+    import oracle
+    from int4_routed_expert_top_b200 import build as b
+    oracle.build()
+    b.build()
