@@ -39,7 +39,8 @@ def gap_resampled_tokens(wl, T, wr, b, layer=0, step=0, max_rounds=64):
     wr_np, b_np = wr.cpu().numpy(), b.cpu().numpy()
     for _ in range(max_rounds):
         x = synth.tokens(wl, T, layer, step, redraw)
-        idx, w, gap = oracle.route(x.numpy(), wr_np, b_np, wl.k)
+        idx, w, gap = oracle.route(x.numpy(), wr_np, b_np, wl.k, wl.routed_scale,
+                                   wl.norm_topk)
         bad = np.nonzero(gap < 1e-3)[0]
         if bad.size == 0:
             return x, idx, w, redraw
