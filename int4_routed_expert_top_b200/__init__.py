@@ -202,6 +202,9 @@ def coli_moe_forward_ex(layer, x, T, y, ws, residual=None, path=COLI_PATH_AUTO, 
     ev = None
     if events is not None:
         assert len(events) == COLI_STAGES + 1
+        for e in events:          # torch creates the CUDA event on its first record
+            if not e.cuda_event:
+                e.record()
         ev = (_P * len(events))(*[e.cuda_event for e in events])
     _ok(lib.coli_moe_forward_ex(layer, _ptr(x), _xtype(x), T, _ptr(y), _ptr(residual), path,
                                 _ptr(idx_out), _ptr(w_out), ev, _ptr(ws),
