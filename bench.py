@@ -123,44 +123,59 @@ def build_layers(wl, device):
 # ---------------------------------------------------------------------------
 # CPU baseline: the oracle, as it stands, on a bounded sample
 # ---------------------------------------------------------------------------
-def oracle_sample(wl, T, budget_s=12.0, max_tokens=None):
-    """Time the oracle on whole tokens of the workload until ~budget_s of CPU
-    work: routing on the full router, dequantisation of every expert matrix the
-    token uses, the SwiGLU experts and the combine.  Returns (tokens/s, n, secs)."""
-    import oracle
-    import synth
-    import torch
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    wr, b = synth.router(wl, 0)
-    wr_np, b_np = wr.numpy(), b.numpy()
-    x = synth.tokens(wl, max(T, 1), layer=0, step=0).numpy()
-    cont = {}
+class OracleSampler:
+    """The oracle, as it stands, on whole tokens of the workload: routing on the
+    full router, dequantisation of every expert matrix the token uses, the SwiGLU
+    experts and the combine.  Building the container (quantisation) is offline
+    work and is not timed."""
 
-    def container(e):   # untimed: the container is built offline
-        if e not in cont:
-            cont[e] = []
+    def __init__(self, wl):
+        import synth
+        import torch
+        self.wl = wl
+        self.dev = "cuda" if torch.cuda.is_available() else "cpu"
+        wr, b = synth.router(wl, 0)
+        self.wr, self.b = wr.numpy(), b.numpy()
+        self.x = synth.tokens(wl, max(wl.T, 64), layer=0, step=0).numpy()
+        self.cont = {}
+        self.done = 0
+
+    def _container(self, e):
+        import oracle
+        import synth
+        if e not in self.cont:
+            self.cont[e] = []
             for t in (synth.T_GATE, synth.T_UP, synth.T_DOWN):
-                m = synth.expert_master(wl, 0, t, e, device=dev).cpu().numpy()
-                cont[e].append((oracle.quantize(m, wl.group), m.shape[1]))
-        return cont[e]
+                m = synth.expert_master(self.wl, 0, t, e, device=self.dev).cpu().numpy()
+                self.cont[e].append((oracle.quantize(m, self.wl.group), m.shape[1]))
+        return self.cont[e]
 
-    done, spent = 0, 0.0
-    limit = max_tokens or x.shape[0]
-    while done < limit and (spent < budget_s or done == 0):
-        t = done % x.shape[0]
-        idx, w, _ = oracle.route(x[t:t + 1], wr_np, b_np, wl.k)
-        experts_ids = [int(e) for e in idx[0]] + [wl.E + s for s in range(wl.n_shared)]
-        for e in experts_ids:
-            container(e)
+    def step(self) -> float:
+        """One token through the oracle; returns its CPU seconds."""
+        import oracle
+        wl, t = self.wl, self.done % self.x.shape[0]
+        idx, w, _ = oracle.route(self.x[t:t + 1], self.wr, self.b, wl.k, wl.routed_scale,
+                                 wl.norm_topk)
+        ids = [int(e) for e in idx[0]] + [wl.E + s for s in range(wl.n_shared)]
+        for e in ids:
+            self._container(e)
         t0 = time.perf_counter()
-        idx, w, _ = oracle.route(x[t:t + 1], wr_np, b_np, wl.k)
-        ex = []
-        for e in experts_ids:
-            ex.append(tuple(oracle.dequantize(p, s, K, wl.group) for (p, s), K in container(e)))
-        oracle.token_forward(x[t], w[0], ex, wl.n_shared)
-        spent += time.perf_counter() - t0
-        done += 1
-    return done / spent, done, spent
+        idx, w, _ = oracle.route(self.x[t:t + 1], self.wr, self.b, wl.k, wl.routed_scale,
+                                 wl.norm_topk)
+        ex = [tuple(oracle.dequantize(p, s, K, wl.group) for (p, s), K in self._container(e))
+              for e in ids]
+        oracle.token_forward(self.x[t], w[0], ex, wl.n_shared)
+        self.done += 1
+        return time.perf_counter() - t0
+
+
+def oracle_sample(wl, budget_s=12.0):
+    smp = OracleSampler(wl)
+    spent, n = 0.0, 0
+    while n == 0 or spent < budget_s:
+        spent += smp.step()
+        n += 1
+    return n / spent, n, spent
 
 
 def run_reference(args):
@@ -170,12 +185,12 @@ def run_reference(args):
     wl = workload(args.workload)
     T = args.tokens or wl.T
     per_step = []
-    n_steps = args.warmup + args.steps
+    smp = OracleSampler(wl)
     t_all = time.perf_counter()
-    for i in range(n_steps):
-        if time.perf_counter() - t_all > 150 and i >= args.warmup + 1:
+    for i in range(args.warmup + args.steps):
+        if time.perf_counter() - t_all > 150 and len(per_step) >= 1:
             break                       # keep the reference arm within a few minutes
-        _, n, secs = oracle_sample(wl, T, budget_s=0.0, max_tokens=1)
+        secs = smp.step()
         if i >= args.warmup:
             per_step.append(secs)
     tok_s = len(per_step) / sum(per_step)
@@ -208,6 +223,8 @@ def main():
     ap.add_argument("--path", default="auto", choices=("auto", "gemv", "gemm"))
     ap.add_argument("--impl", default="own", choices=("own", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override routed experts (small-footprint profiling layers)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -232,6 +249,9 @@ def main():
             dist.barrier()
 
     wl = workload(args.workload)
+    if args.experts:
+        import dataclasses
+        wl = dataclasses.replace(wl, E=args.experts)
     T = args.tokens or wl.T
     path = {"auto": cm.COLI_PATH_AUTO, "gemv": cm.COLI_PATH_GEMV, "gemm": cm.COLI_PATH_GEMM}[args.path]
     layers = build_layers(wl, dev)
@@ -258,21 +278,45 @@ def main():
 
     for i in range(args.warmup):
         flush.zero_()
-        step(i)
+        step(i, record_idx=i < args.steps)
+    torch.cuda.synchronize()
+    # routing of every pool slot (deterministic), for the weight-byte count
+    for j in range(n_pool):
+        step(j, record_idx=True)
+    torch.cuda.synchronize()
+    slot_idx = idx_all[:n_pool].cpu().numpy() if wl.layers == 1 else None
+
+    # one CUDA graph per token slot: the forward as a deployment would replay it
+    graphs = []
+    for j in range(n_pool):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(j)
+        graphs.append(g)
+    n_prof = min(n_pool, 16)
+    prof_graphs, prof_ev = [], []
+    if wl.layers == 1:
+        for j in range(n_prof):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(cm.COLI_STAGES + 1)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(j, ev)
+            prof_graphs.append(g)
+            prof_ev.append(ev)
+    for j in range(n_pool):
+        graphs[j].replay()
     torch.cuda.synchronize()
 
     K = args.steps
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    stage_ev = ([[torch.cuda.Event(enable_timing=True) for _ in range(cm.COLI_STAGES + 1)]
-                 for _ in range(K)] if wl.layers == 1 else None)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         for i in range(K):
             flush.zero_()
             starts[i].record(stream)
-            step(i, stage_ev[i] if stage_ev else None, record_idx=wl.layers == 1)
+            graphs[i % n_pool].replay()
             ends[i].record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -284,6 +328,17 @@ def main():
     job_ms = float(tot.item())
     tokens_all = T * K * world
     value = tokens_all / (job_ms / 1e3)
+
+    # per-stage device times: graphs with event nodes at the stage boundaries
+    st_ms = []
+    for i in range(max(n_prof, min(K, 4 * n_prof)) if prof_graphs else 0):
+        j = i % n_prof
+        flush.zero_()
+        prof_graphs[j].replay()
+        torch.cuda.synchronize()
+        st_ms.append([prof_ev[j][s].elapsed_time(prof_ev[j][s + 1])
+                      for s in range(cm.COLI_STAGES)] + [j])
+    st_ms = np.array(st_ms)
 
     # end to end through the public API: pinned host x -> device, forward, y -> host
     xh = torch.empty((n_pool, T, wl.H), dtype=xpool.dtype, pin_memory=True)
@@ -324,28 +379,30 @@ def main():
            "top_k": wl.k, "intermediate": wl.I, "shared": wl.n_shared,
            "scale_group": wl.group or "per-row", "layers": wl.layers,
            "x_dtype": wl.x_dtype, "path": args.path,
-           "l2": "256 MiB buffer written between timed steps (flush), not timed"}
+           "l2": "256 MiB buffer written between timed steps (flush), not timed",
+           "launch": "one CUDA graph per token slot, replayed"}
     if wl.layers == 1:
-        idx_np = idx_all.cpu().numpy()
-        uniq = np.array([len(np.unique(idx_np[i])) for i in range(K)])
+        uniq_slot = np.array([len(np.unique(slot_idx[j])) for j in range(n_pool)])
+        uniq = uniq_slot[np.arange(K) % n_pool]
         nbytes = (uniq + wl.n_shared) * blob
         weight_gbs = nbytes.sum() / (total_ms / 1e3) / 1e9
-        st_ms = np.array([[stage_ev[i][s].elapsed_time(stage_ev[i][s + 1])
-                           for s in range(cm.COLI_STAGES)] for i in range(K)])
-        stage_mean = st_ms.mean(0)
-        L = L0.desc
-        gu_bytes_unit = 2 * (wl.I * wl.H // 2 + wl.I * (1 if wl.group == 0 else wl.H // wl.group) * 4)
-        dn_bytes_unit = wl.H * wl.I // 2 + wl.H * (1 if wl.group == 0 else wl.I // wl.group) * 4
-        units = uniq + wl.n_shared
-        gu_ach = (units * gu_bytes_unit / (st_ms[:, 2] / 1e3)).mean() / 1e9
-        dn_ach = (units * dn_bytes_unit / (st_ms[:, 3] / 1e3)).mean() / 1e9
+        ng_h = 1 if wl.group == 0 else wl.H // wl.group
+        ng_i = 1 if wl.group == 0 else wl.I // wl.group
+        gu_bytes_unit = 2 * (wl.I * wl.H // 2 + wl.I * ng_h * 4)
+        dn_bytes_unit = wl.H * wl.I // 2 + wl.H * ng_i * 4
+        units = uniq_slot[st_ms[:, -1].astype(int)] + wl.n_shared
+        stage_mean = st_ms[:, :-1].mean(0)
+        gu_ach = (units * gu_bytes_unit).sum() / (st_ms[:, 2].sum() / 1e3) / 1e9
+        dn_ach = (units * dn_bytes_unit).sum() / (st_ms[:, 3].sum() / 1e3) / 1e9
         dominant = "gateup" if stage_mean[2] >= stage_mean[3] else "down"
         ach = gu_ach if dominant == "gateup" else dn_ach
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
                             "frac": ach / hbm_gbs, "traffic": None,
                             "kernel": f"expert_gemv_kernel ({dominant})",
-                            "peak_source": peak_src}
+                            "peak_source": peak_src,
+                            "bytes_per_launch": float((units * (gu_bytes_unit if dominant == "gateup" else dn_bytes_unit)).mean())}
         line["stages_us"] = {n: 1e3 * v for n, v in zip(cm.STAGE_NAMES, stage_mean)}
+        line["down_gbs"] = dn_ach
         line["int4_weight_gbs"] = weight_gbs
         line["int4_weight_frac_of_hbm"] = weight_gbs / hbm_gbs
         line["unique_experts_per_step"] = float(uniq.mean())
@@ -358,7 +415,7 @@ def main():
                    "h2d_bytes_per_step": int(xpool[0].numel() * xpool.element_size()),
                    "d2h_bytes_per_step": int(T * wl.H * 4)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, n, secs = oracle_sample(wl, T)
+        tok_s, n, secs = oracle_sample(wl)
         line["cpu_baseline"] = {
             "value": tok_s, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} tokens of {wl.name} through the oracle ({secs:.1f} s): router over "
