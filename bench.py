@@ -298,6 +298,8 @@ def main():
     if wl.layers == 1:
         for j in range(n_prof):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(cm.COLI_STAGES + 1)]
+            for e in ev:
+                e.record(stream)          # create the CUDA events outside the capture
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 step(j, ev)

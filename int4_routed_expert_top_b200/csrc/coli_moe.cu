@@ -364,7 +364,9 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     float* w = at<float>(ws, p.w);
     auto mark = [&](int s) -> int {
         if (!events || !events[s]) return COLI_OK;
-        if (cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[s]), st) != cudaSuccess)
+        // External: inside stream capture the record becomes an event node of the graph
+        if (cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(events[s]), st,
+                                     cudaEventRecordExternal) != cudaSuccess)
             return fail(COLI_E_CUDA, "forward: event record failed");
         return COLI_OK;
     };
