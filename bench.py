@@ -264,7 +264,7 @@ def main():
                           if wl.layers > 1 else 0, L0.workspace_bytes(T)),),
                      dtype=torch.uint8, device=dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
-    idx_all = torch.empty((args.steps, T, wl.k), dtype=torch.int32, device=dev)
+    idx_all = torch.empty((max(args.steps, n_pool), T, wl.k), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(i, events=None, record_idx=False):
