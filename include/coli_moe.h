@@ -41,10 +41,15 @@
  *    scales F32 [R, K/G]    G = K (group 0, one scale per row) or 64
  *
  * Device layout of one expert ("blob", coli_moe_pack_expert): the container
- * re-tiled for coalesced 16-byte loads; its dequantised values are identical.
+ * re-tiled so that one 16-byte load of a lane is one lane's share of a 16x16
+ * tensor-core operand tile; its dequantised values are identical.
  *    For each matrix m in (gate, up, down) with R rows and K columns:
- *      codes_m  [R/128][K/32][128][16 bytes]   unit (t, c, r) = row 128t + r,
- *               columns 32c .. 32c+31 in container byte order
+ *      codes_m  [R/128][K/64][8][32][16 bytes]: unit (t, s, b, l) belongs to
+ *               rows r0 = 128t + 16b + l/4 and r1 = r0 + 8, and holds four
+ *               32-bit words j = 0..3 for columns c0 = 64s + 16j + 4(l%4) ..
+ *               c0+3; in word j, bits 4p..4p+3 hold the signed nibble of
+ *                 p: 0 (r0,c0)  1 (r0,c0+2)  2 (r1,c0)  3 (r1,c0+2)
+ *                    4 (r0,c0+1) 5 (r0,c0+3) 6 (r1,c0+1) 7 (r1,c0+3)
  *      scales_m [R/128][K/G][128] f32          scale of row 128t + r, group g
  *    Order: codes_gate, codes_up, codes_down, scales_gate, scales_up,
  *    scales_down; each section starts on a 256-byte boundary and the blob size
@@ -52,7 +57,7 @@
  *    device buffer: routed experts 0 .. E-1, then the shared experts.
  *
  * Limits: H and I multiples of 128; group 0 or 64; 1 <= k <= 32; k <= E <= 1024;
- * n_shared <= 4; 1 <= T <= 8192 tokens per call.
+ * n_shared <= 4; 1 <= T <= 8192 tokens per call and E * ceil(T/32) <= 24576.
  */
 #ifndef COLI_MOE_H
 #define COLI_MOE_H
@@ -175,11 +180,11 @@ int coli_moe_forward(const coli_moe_layer* layer, const void* x, coli_dtype xt,
 
 /* Stage boundaries of coli_moe_forward_ex, for optional event timing. */
 typedef enum coli_stage {
-    COLI_STAGE_ROUTER = 0,  /* router logits + sigmoid/top-k              */
-    COLI_STAGE_UNION = 1,   /* batch union and expert work list           */
+    COLI_STAGE_ROUTER = 0,  /* router logits (+ the activation operand)   */
+    COLI_STAGE_UNION = 1,   /* sigmoid/top-k, weights and batch union     */
     COLI_STAGE_GATEUP = 2,  /* gate/up expert kernel with SwiGLU          */
-    COLI_STAGE_DOWN = 3,    /* down expert kernel                         */
-    COLI_STAGE_COMBINE = 4, /* weighted combine + shared + residual       */
+    COLI_STAGE_DOWN = 3,    /* down expert kernel (and the fused combine) */
+    COLI_STAGE_COMBINE = 4, /* a separate combine, where the path has one */
     COLI_STAGES = 5
 } coli_stage;
 

@@ -54,10 +54,9 @@ bool shape_ok(int H, int I, int group) {
 // ---------------------------------------------------------------------------
 struct WsPlan {
     int64_t zpart, idx, w, offsets, pair_tok, pair_slot, uniq, n_uniq, inv;
-    int64_t unit_expert, unit_begin, unit_end, n_units, h, o, xb, total;
+    int64_t unit_expert, unit_begin, unit_end, n_units, counters;
+    int64_t xq, xinv, hq, hinv, o, total;
 };
-
-constexpr int kMaxKS = 8;
 
 WsPlan plan_ws(const coli_moe_desc& d, int T) {
     WsPlan p;
@@ -78,9 +77,12 @@ WsPlan plan_ws(const coli_moe_desc& d, int T) {
     p.unit_begin = take((int64_t)(d.E + d.n_shared) * 4);
     p.unit_end = take((int64_t)(d.E + d.n_shared) * 4);
     p.n_units = take(4);
-    p.h = take(P * d.I * 4);
+    p.counters = take((int64_t)(d.H / 64) * 4);
+    p.xq = take((int64_t)T * d.H * 4);          // fp16 hi + lo
+    p.xinv = take((int64_t)T * (d.H / 64) * 4);
+    p.hq = take(P * d.I * 4);                   // fp16 hi + lo
+    p.hinv = take(P * (d.I / 64) * 4);
     p.o = take(P * d.H * 4);
-    p.xb = take((int64_t)T * d.H * 2);  // bf16 copy of x for the tensor-core path
     p.total = off;
     return p;
 }
@@ -106,21 +108,27 @@ int set_smem(const void* fn, int bytes) {
     return COLI_OK;
 }
 
-// router logits into zpart; returns the number of K slices used (or < 0)
+// Router logits into zpart (K slices in *ks_out).  When xq is non-null the
+// fp16 activation operand is produced as well (by extra CTAs of the small-batch
+// router, or by its own launch after the tiled router).
 int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, float* zpart,
-                  cudaStream_t st, int* ks_out) {
-    int KS = 1;
-    if (T <= 32) {
+                  __half* xq, float* xinv, cudaStream_t st, int* ks_out) {
+    int KS = 0;
+    if (T <= 32)
         for (int c : {8, 4, 2, 1})
-            if (d.H % (c * 128) == 0) { KS = c; break; }
-        const int warps = d.E * KS;
-        const dim3 grid((warps + 7) / 8);
+            if (d.H % (c * 128) == 0 && d.H / c <= kRouterMaxSlice) { KS = c; break; }
+    const int qwarps = T * (d.H / 64);
+    if (KS > 0) {
+        const int rblocks = (d.E * KS + 7) / 8;
+        const int qblocks = xq ? (qwarps + 7) / 8 : 0;
+        const dim3 grid(rblocks + qblocks);
         if (xt == COLI_F32)
-            router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart);
+            router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, xq, xinv);
         else
-            router_gemv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart);
+            router_gemv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, xq, xinv);
     } else {
         const int tiles = ((T + 63) / 64) * ((d.E + 63) / 64);
+        KS = 1;
         for (int c : {8, 4, 2, 1})
             if (d.H % (c * 16) == 0 && (tiles * c <= 2 * 148 || c == 1)) { KS = c; break; }
         const dim3 grid((T + 63) / 64, (d.E + 63) / 64, KS);
@@ -128,6 +136,14 @@ int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, f
             router_tiled_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart);
         else
             router_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart);
+        if (xq) {
+            int rc = check_launch("router");
+            if (rc) return rc;
+            if (xt == COLI_F32)
+                act_quant_kernel<float><<<(qwarps + 7) / 8, 256, 0, st>>>((const float*)x, T, d.H, xq, xinv);
+            else
+                act_quant_kernel<__nv_bfloat16><<<(qwarps + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, xq, xinv);
+        }
     }
     *ks_out = KS;
     return check_launch("router");
@@ -141,18 +157,49 @@ int launch_topk(const coli_moe_desc& d, const float* zpart, int KS, int T, int32
     return check_launch("topk");
 }
 
+int union_smem_bytes(int T, int E) {
+    return (int)((int64_t)E * ((T + 31) / 32) * 4 + 3 * (int64_t)E * 4);
+}
+
 int launch_union(const int32_t* idx, int T, int k, int E, const UnionOut& o, cudaStream_t st) {
-    const int W = (T + 31) / 32;
-    const int smem = (int)((int64_t)E * W * 4 + 3 * (int64_t)E * 4);
+    const int smem = union_smem_bytes(T, E);
     int rc = set_smem((const void*)union_kernel, smem);
     if (rc) return rc;
     union_kernel<<<1, kUnionThreads, smem, st>>>(idx, T, k, E, o);
     return check_launch("union");
 }
 
+// top-k + union; one fused single-CTA launch for small batches
+int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int32_t* idx,
+                  float* w, const UnionOut& o, cudaStream_t st) {
+    if (T <= 64) {
+        const int topk_warps = std::max(1, std::min(32, (160 * 1024) / (8 * d.E)));
+        const int smem = std::max(topk_warps * 2 * d.E * 4, union_smem_bytes(T, d.E));
+        int rc = set_smem((const void*)topk_union_kernel, smem);
+        if (rc) return rc;
+        topk_union_kernel<<<1, kUnionThreads, smem, st>>>(zpart, KS, T, d.E, d.router_b, d.k,
+                                                          d.routed_scale, d.norm_topk, idx, w,
+                                                          topk_warps, o);
+        return check_launch("topk+union");
+    }
+    int rc = launch_topk(d, zpart, KS, T, idx, w, st);
+    if (rc) return rc;
+    return launch_union(idx, T, d.k, d.E, o, st);
+}
+
+template <bool GATEUP>
+int launch_gemv_nt(int nt, int grid, const GemvArgs& a, cudaStream_t st) {
+    switch (nt) {
+        case 1: expert_gemv_kernel<GATEUP, 1><<<grid, kGemvWarps * 32, 0, st>>>(a); break;
+        case 2: expert_gemv_kernel<GATEUP, 2><<<grid, kGemvWarps * 32, 0, st>>>(a); break;
+        default: expert_gemv_kernel<GATEUP, 4><<<grid, kGemvWarps * 32, 0, st>>>(a); break;
+    }
+    return check_launch(GATEUP ? "gate/up gemv" : "down gemv");
+}
+
 template <typename Mark>
-int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const void* x,
-                coli_dtype xt, cudaStream_t st, Mark&& mark) {
+int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const float* residual,
+                float* y, cudaStream_t st, Mark&& mark) {
     const coli_moe_desc& d = l->d;
     GemvArgs a;
     a.experts = static_cast<const uint8_t*>(d.experts);
@@ -163,35 +210,24 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
     a.unit_begin = at<int32_t>(ws, p.unit_begin);
     a.unit_end = at<int32_t>(ws, p.unit_end);
     a.pair_tok = at<int32_t>(ws, p.pair_tok);
-    a.x = x;
-    a.h = at<float>(ws, p.h);
+    a.xq = at<__half>(ws, p.xq);
+    a.xinv = at<float>(ws, p.xinv);
+    a.hq = at<__half>(ws, p.hq);
+    a.hinv = at<float>(ws, p.hinv);
     a.o = at<float>(ws, p.o);
+    a.counters = at<int32_t>(ws, p.counters);
+    a.inv = at<int32_t>(ws, p.inv);
+    a.w = at<float>(ws, p.w);
+    a.residual = residual;
+    a.y = y;
+    a.T = T; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;
-    const int tc = std::min(kGemvTC, T);
-    int rc;
-    const int smem_gu = tc * d.H * 4, smem_dn = tc * d.I * 4;
-    if (xt == COLI_F32) {
-        if ((rc = set_smem((const void*)expert_gemv_kernel<true, float>, smem_gu))) return rc;
-        expert_gemv_kernel<true, float><<<units_max * (d.I / 32), kGemvWarps * 32, smem_gu, st>>>(a);
-    } else {
-        if ((rc = set_smem((const void*)expert_gemv_kernel<true, __nv_bfloat16>, smem_gu))) return rc;
-        expert_gemv_kernel<true, __nv_bfloat16><<<units_max * (d.I / 32), kGemvWarps * 32, smem_gu, st>>>(a);
-    }
-    if ((rc = check_launch("gate/up gemv"))) return rc;
+    const int nt = T <= 4 ? 1 : T <= 8 ? 2 : 4;
+    int rc = launch_gemv_nt<true>(nt, units_max * (d.I / 64), a, st);
+    if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;
-    if ((rc = set_smem((const void*)expert_gemv_kernel<false, float>, smem_dn))) return rc;
-    expert_gemv_kernel<false, float><<<units_max * (d.H / 32), kGemvWarps * 32, smem_dn, st>>>(a);
-    return check_launch("down gemv");
-}
-
-int launch_combine(const coli_moe_desc& d, int T, void* ws, const WsPlan& p,
-                   const float* residual, float* y, cudaStream_t st) {
-    const int64_t n = (int64_t)T * (d.H / 4);
-    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-        at<float>(ws, p.o), at<int32_t>(ws, p.inv), at<float>(ws, p.w), T, d.k, d.n_shared,
-        d.H, residual, y);
-    return check_launch("combine");
+    return launch_gemv_nt<false>(nt, units_max * (d.H / 64), a, st);
 }
 
 }  // namespace
@@ -256,9 +292,12 @@ int coli_moe_pack_expert(int32_t H, int32_t I, int32_t group, const uint8_t* gat
     for (int m = 0; m < 3; ++m) {
         const int R = L.rows[m], K = L.cols[m], ng = L.ngroups[m];
         for (int r = 0; r < R; ++r) {
-            for (int c = 0; c < K / 32; ++c)
-                std::memcpy(out + L.codes[m] + code_unit_offset(r, c, K),
-                            codes[m] + (int64_t)r * (K / 2) + 16 * c, 16);
+            for (int c = 0; c < K; ++c) {
+                const uint8_t byte = codes[m][(int64_t)r * (K / 2) + c / 2];
+                const uint32_t nib = (c & 1) ? (byte >> 4) : (byte & 15);
+                uint32_t* word = reinterpret_cast<uint32_t*>(out + L.codes[m] + frag_word_offset(r, c, K));
+                *word |= nib << frag_nibble_shift(r, c);
+            }
             for (int g = 0; g < ng; ++g)
                 reinterpret_cast<float*>(out + L.scales[m])[scale_offset(r, g, ng)] =
                     scales[m][(int64_t)r * ng + g];
@@ -277,10 +316,10 @@ int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group, const f
     const float* src[3] = {gate, up, down};
     for (int m = 0; m < 3; ++m) {
         const int R = L.rows[m], K = L.cols[m];
-        const int smem = 8 * (K / 2);
+        const int smem = 16 * (K / 2);
         int rc = set_smem((const void*)quantize_rows_kernel, smem);
         if (rc) return rc;
-        quantize_rows_kernel<<<(R + 7) / 8, 256, smem, S(stream)>>>(
+        quantize_rows_kernel<<<R / 16, 256, smem, S(stream)>>>(
             src[m], R, K, group, b + L.codes[m], reinterpret_cast<float*>(b + L.scales[m]));
         if ((rc = check_launch("quantize_rows"))) return rc;
     }
@@ -326,7 +365,9 @@ int coli_moe_route(const coli_moe_layer* layer, const void* x, coli_dtype xt, in
     if (!ws || ws_bytes < (size_t)p.total)
         return fail(COLI_E_WORKSPACE, "route: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
     int KS;
-    if ((rc = launch_router(layer->d, x, xt, T, at<float>(ws, p.zpart), S(stream), &KS))) return rc;
+    if ((rc = launch_router(layer->d, x, xt, T, at<float>(ws, p.zpart), nullptr, nullptr,
+                            S(stream), &KS)))
+        return rc;
     return launch_topk(layer->d, at<float>(ws, p.zpart), KS, T, idx, w, S(stream));
 }
 
@@ -370,10 +411,12 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
             return fail(COLI_E_CUDA, "forward: event record failed");
         return COLI_OK;
     };
+    const bool gemm = path == COLI_PATH_GEMM;
     int KS;
     if ((rc = mark(COLI_STAGE_ROUTER))) return rc;
-    if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), st, &KS))) return rc;
-    if ((rc = launch_topk(d, at<float>(ws, p.zpart), KS, T, idx, w, st))) return rc;
+    if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart),
+                            gemm ? nullptr : at<__half>(ws, p.xq), at<float>(ws, p.xinv), st, &KS)))
+        return rc;
     UnionOut o{};
     o.offsets = at<int32_t>(ws, p.offsets);
     o.pair_tok = at<int32_t>(ws, p.pair_tok);
@@ -385,11 +428,13 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     o.unit_begin = at<int32_t>(ws, p.unit_begin);
     o.unit_end = at<int32_t>(ws, p.unit_end);
     o.n_units = at<int32_t>(ws, p.n_units);
+    o.counters = at<int32_t>(ws, p.counters);
+    o.n_counters = d.H / 64;
     o.n_shared = d.n_shared;
     if ((rc = mark(COLI_STAGE_UNION))) return rc;
-    if ((rc = launch_union(idx, T, d.k, d.E, o, st))) return rc;
+    if ((rc = launch_select(d, at<float>(ws, p.zpart), KS, T, idx, w, o, st))) return rc;
     if ((rc = mark(COLI_STAGE_GATEUP))) return rc;
-    if (path == COLI_PATH_GEMM) {
+    if (gemm) {
         GemmCtx g;
         g.experts = static_cast<const uint8_t*>(d.experts);
         g.blob_bytes = layer->L.bytes;
@@ -399,15 +444,13 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         g.n_units = o.n_units; g.unit_expert = o.unit_expert;
         g.unit_begin = o.unit_begin; g.unit_end = o.unit_end; g.pair_tok = o.pair_tok;
         g.x = x; g.x_bf16 = xt == COLI_BF16;
-        g.xb = at<__nv_bfloat16>(ws, p.xb);
-        g.h = at<__nv_bfloat16>(ws, p.h);
         g.o = at<float>(ws, p.o);
-        if ((rc = launch_gemm(g, st, mark))) return rc;
+        if ((rc = launch_gemm(g, st, mark))) return fail(rc, "forward: tensor-core path not available");
+        if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
     } else {
-        if ((rc = launch_gemv(layer, T, ws, p, x, xt, st, mark))) return rc;
+        if ((rc = launch_gemv(layer, T, ws, p, residual, y, st, mark))) return rc;
+        if ((rc = mark(COLI_STAGE_COMBINE))) return rc;   // combine is fused into the down pass
     }
-    if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
-    if ((rc = launch_combine(d, T, ws, p, residual, y, st))) return rc;
     if ((rc = mark(COLI_STAGES))) return rc;
     if (idx_out) {
         if (cudaMemcpyAsync(idx_out, idx, sizeof(int32_t) * T * d.k, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -479,7 +522,7 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t 
     const BlobLayout& L = layer->L;
     const uint8_t* blob = static_cast<const uint8_t*>(d.experts) + (int64_t)expert * L.bytes;
     const int R = L.rows[which], K = L.cols[which];
-    const int64_t n = (int64_t)R * (K / 32);
+    const int64_t n = (int64_t)R * K;
     dequant_kernel<<<(unsigned)((n + 255) / 256), 256, 0, S(stream)>>>(
         blob + L.codes[which], reinterpret_cast<const float*>(blob + L.scales[which]), R, K,
         d.group, out);

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -44,10 +45,33 @@ __host__ __device__ inline BlobLayout make_blob_layout(int H, int I, int group) 
     return L;
 }
 
-// byte offset of code unit (row r, unit c) inside a matrix with K columns
-__host__ __device__ inline int64_t code_unit_offset(int r, int c, int K) {
-    const int t = r / kTileRows, m = r % kTileRows;
-    return (((int64_t)t * (K / kUnitCols) + c) * kTileRows + m) * 16;
+// Fragment tiles.  A matrix [R, K] is cut into 16-row x 64-column blocks; the
+// block is 32 units of 16 bytes, one per lane l = 4*g + t of a warp, so one warp
+// load of 512 bytes fetches a whole block.  Unit l holds rows r0 = 16*b + g and
+// r1 = r0 + 8 of the block, and for each 16-column sub-block j the 4 columns
+// c0 = 16*j + 4*t .. c0 + 3 of both rows: 8 nibbles in word j.  These are the
+// elements that lane owns in a 16x16 tensor-core operand tile (mma.sync A
+// fragment up to a column permutation, and the tcgen05 16x256b TMEM access).
+// Blocks are ordered [R/128][K/64][8][32 lanes], so the eight blocks of a
+// 128-row tile and one 64-column step are 4 KB of contiguous bytes.
+//
+// nibble position of (row r, column c) inside its 32-bit word
+__host__ __device__ inline int frag_nibble_shift(int r, int c) {
+    const int upper = (r % 16) / 8, cc = c % 4;
+    return 4 * (upper * 2 + (cc >> 1)) + 16 * (cc & 1);
+}
+
+// byte offset of the 16-byte unit of lane l, 16-row block b8 (0..7) of tile rt,
+// 64-column step kb, in a matrix with K columns
+__host__ __device__ inline int64_t frag_unit_offset(int rt, int kb, int b8, int lane, int K) {
+    return ((((int64_t)rt * (K / 64) + kb) * 8 + b8) * 32 + lane) * 16;
+}
+
+// byte offset of the word holding (row r, column c)
+__host__ __device__ inline int64_t frag_word_offset(int r, int c, int K) {
+    const int rt = r / kTileRows, b8 = (r % kTileRows) / 16, g = r % 8;
+    const int kb = c / 64, j = (c % 64) / 16, t = (c % 16) / 4;
+    return frag_unit_offset(rt, kb, b8, 4 * g + t, K) + 4 * j;
 }
 
 // element offset of the scale of (row r, group g) with ng groups per row
@@ -83,39 +107,59 @@ __device__ __forceinline__ f2_t f2fma(f2_t a, f2_t b, f2_t c) {
 }
 
 // ---------------------------------------------------------------------------
-// Exact int4 -> f32 decode without integer-to-float conversions.
-//
-// A nibble n sitting at bit position 4p (p <= 4) of a word is masked in place
-// and its sign bit flipped, and the f32 exponent of 2^23 is OR-ed in:
-//   bits = (w & (0xF << 4p)) ^ (0x4B000000 | 0x8 << 4p)
-//   value = 2^23 + 16^p * (n ^ 8) = 2^23 + 16^p * (q + 8)   (q = signed code)
-// Subtracting the constant 2^23 + 8 * 16^p leaves 16^p * q exactly.  The
-// factor 16^p is undone by pre-scaling the activation of that column by
-// 16^-p (exact powers of two), so (16^p q) * (16^-p x) rounds like q * x.
-// Nibbles 5..7 are first moved down by 12 bits to positions 2..4.
-// Column j of a word (j = 0..7) therefore uses position
-//   pos(j) = {0, 1, 2, 3, 4, 2, 3, 4}[j]
+// Exact int4 -> fp16 decode of one word of a fragment tile (see above) into the
+// four f16x2 registers (row r0: c0,c0+1 | row r0: c0+2,c0+3 | row r1: c0,c0+1 |
+// row r1: c0+2,c0+3).  The nibble is masked in place, its sign bit flipped and
+// the fp16 exponent of 1024 OR-ed in: a nibble at bits 0-3 of a half reads as
+// 1024 + (q + 8), one at bits 4-7 as 1024 + 16 (q + 8); one packed subtract or
+// fused multiply-add per two values then leaves q exactly.
 // ---------------------------------------------------------------------------
-__host__ __device__ constexpr float kPosScale(int j) {
-    return j == 0 ? 1.0f : j == 1 ? 0.0625f : (j == 2 || j == 5) ? 0.00390625f
-         : (j == 3 || j == 6) ? 0.000244140625f : 0.0000152587890625f;
+__device__ __forceinline__ uint32_t h2sub_1032(uint32_t v) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0x64086408u));
+    return r;
+}
+__device__ __forceinline__ uint32_t h2fma_16th_m72(uint32_t v) {
+    uint32_t r;  // v * 1/16 - 72
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(0x2C002C00u), "r"(0xD480D480u));
+    return r;
+}
+__device__ __forceinline__ void decode_frag_word(uint32_t w, uint32_t& r0, uint32_t& r1,
+                                                 uint32_t& r2, uint32_t& r3) {
+    const uint32_t w8 = w >> 8;
+    r0 = h2sub_1032((w & 0x000F000Fu) ^ 0x64086408u);
+    r1 = h2fma_16th_m72((w & 0x00F000F0u) ^ 0x64806480u);
+    r2 = h2sub_1032((w8 & 0x000F000Fu) ^ 0x64086408u);
+    r3 = h2fma_16th_m72((w8 & 0x00F000F0u) ^ 0x64806480u);
 }
 
-// decode the 8 nibbles of w into 4 f32 pairs: (c0,c1), (c2,c3), (c4,c5), (c6,c7)
-__device__ __forceinline__ void decode8(uint32_t w, f2_t out[4]) {
-    const uint32_t u = w >> 12;
-    const float a0 = __uint_as_float((w & 0x0000000Fu) ^ 0x4B000008u);
-    const float a1 = __uint_as_float((w & 0x000000F0u) ^ 0x4B000080u);
-    const float a2 = __uint_as_float((w & 0x00000F00u) ^ 0x4B000800u);
-    const float a3 = __uint_as_float((w & 0x0000F000u) ^ 0x4B008000u);
-    const float a4 = __uint_as_float((w & 0x000F0000u) ^ 0x4B080000u);
-    const float a5 = __uint_as_float((u & 0x00000F00u) ^ 0x4B000800u);
-    const float a6 = __uint_as_float((u & 0x0000F000u) ^ 0x4B008000u);
-    const float a7 = __uint_as_float((u & 0x000F0000u) ^ 0x4B080000u);
-    out[0] = f2add(f2pack(a0, a1), f2pack(-8388616.0f, -8388736.0f));
-    out[1] = f2add(f2pack(a2, a3), f2pack(-8390656.0f, -8421376.0f));
-    out[2] = f2add(f2pack(a4, a5), f2pack(-8912896.0f, -8390656.0f));
-    out[3] = f2add(f2pack(a6, a7), f2pack(-8421376.0f, -8912896.0f));
+// D[16x8] (f32) += A[16x16] (f16) * B[16x8] (f16), warp-wide
+__device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Activation operand: power-of-two scale 2^(14 - e) for a group whose largest
+// magnitude is m = 2^e * f (f in [1, 2)), so the scaled values stay below 2^15
+// in fp16; returns the inverse scale.  All-zero groups use 1.
+__device__ __forceinline__ float act_group_scale(float m, float* inv) {
+    if (!(m > 0.0f) || !isfinite(m)) { *inv = 1.0f; return 1.0f; }
+    int e;
+    frexpf(m, &e);                 // m = f * 2^e, f in [0.5, 1)
+    int sh = 15 - e;               // m * 2^sh in [2^14, 2^15)
+    sh = max(-100, min(100, sh));
+    *inv = ldexpf(1.0f, -sh);
+    return ldexpf(1.0f, sh);
+}
+
+// split v (already scaled) into fp16 hi + lo with v ~= hi + lo to ~22 bits
+__device__ __forceinline__ void split_f16(float v, __half& hi, __half& lo) {
+    hi = __float2half_rn(v);
+    lo = __float2half_rn(v - __half2float(hi));
 }
 
 // Read-only 16-byte global load that bypasses L1 allocation (weights are

@@ -18,8 +18,6 @@ struct GemmCtx {
     const int32_t* pair_tok;
     const void* x;
     int x_bf16;
-    __nv_bfloat16* xb;  // bf16 copy of x when x is f32
-    __nv_bfloat16* h;   // [P, I]
     float* o;           // [P, H]
 };
 

@@ -1,20 +1,23 @@
-// gemv.cuh - CUDA-core int4 expert kernels for small batches (decode, MTP
-// verify) and the weighted combine.
+// gemv.cuh - int4 expert kernels for small batches (decode, MTP verify).
 //
-// One CTA owns 32 output rows of one unit (a routed expert picked by the batch,
-// or a shared expert) and every token routed to that unit: the weights are read
-// from HBM once per launch no matter how many of the unit's tokens use them
-// (batch union, "github一周涨11k⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.4).  Lane l of
-// every warp owns row 32*rb + l; the 8 warps split the reduction dimension in
-// 64-column steps.  A lane's 16-byte loads of consecutive rows are adjacent in
-// the device layout, so each warp load is one coalesced 512-byte transaction.
-// Nibbles are decoded in registers exactly (see decode8) and multiplied in f32
-// with packed f32x2 FMAs; partial sums of the 8 warps meet in shared memory.
+// A CTA owns one unit (a routed expert picked by the batch, or a shared expert)
+// and 64 output rows, and every token routed to that unit, so each weight byte
+// is read from HBM once per launch however many of the unit's tokens use it
+// (batch union, "github一周涨11k⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.4).  Warp w
+// takes 16-row block w % 4 and half w / 4 of the reduction.  Every step a lane
+// loads one 16-byte unit of a fragment tile (a whole warp: one coalesced 512-byte
+// block), decodes its 32 nibbles to exact fp16 in registers and feeds them to
+// the tensor cores as mma.sync A fragments.  The activations are the B operand,
+// split into fp16 hi + lo parts scaled by a power of two per 64-column group,
+// so the products carry ~22 significant bits into the f32 accumulators.  After
+// each 64-column group the partial product is multiplied by the weight scale
+// (per row, or per group for gs64) and by the activation group's inverse power
+// of two, in f32.
 //
-// gate/up pass:  h[p, i] = silu(sum_c Wg'[i, c] x[c]) * (sum_c Wu'[i, c] x[c])
-// down pass:     o[p, r] = sum_i Wd'[r, i] h[p, i]
-// combine:       y[t]    = residual[t] + sum_j w[t, j] o[pair(t, j)] + sum_s o_shared
-// with W' = q * s, the scale applied per 64-column step (gs64) or per row.
+//   gate/up: h[p, i] = silu(sum_c Wg'[i, c] x[c]) * (sum_c Wu'[i, c] x[c])
+//            written as fp16 hi/lo per 64-row group with its power-of-two scale
+//   down:    o[p, r] = sum_i Wd'[r, i] h[p, i]  (f32), and the last CTA to finish
+//            a 64-row block forms y = residual + sum_j w_j o_j + sum_s o_shared
 #pragma once
 
 #include "common.cuh"
@@ -22,7 +25,7 @@
 namespace coli {
 
 constexpr int kGemvWarps = 8;
-constexpr int kGemvTC = 4;  // tokens per pass over a unit's weights
+constexpr int kGemvMaxNT = 4;     // up to 4 column groups of 8: 16 tokens per pass
 
 struct GemvArgs {
     const uint8_t* experts;
@@ -33,175 +36,243 @@ struct GemvArgs {
     const int32_t* unit_begin;
     const int32_t* unit_end;
     const int32_t* pair_tok;
-    const void* x;   // [T, H] f32 or bf16 (gate/up input)
-    float* h;        // [P, I] f32: gate/up output, down input
-    float* o;        // [P, H] f32: down output
+    const __half* xq;     // [T][H/64][128]  hi (64) then lo (64), scaled
+    const float* xinv;    // [T][H/64]       inverse power-of-two scales
+    __half* hq;           // [P][I/64][128]
+    float* hinv;          // [P][I/64]
+    float* o;             // [P][H]
+    // combine (down pass)
+    int32_t* counters;    // [H/64], zero on entry
+    const int32_t* inv;   // [T*k] pair of (t, j)
+    const float* w;       // [T*k]
+    const float* residual;
+    float* y;
+    int T, k, n_shared;
     int H, I, group;
 };
 
-template <bool GATEUP, int TC>
-__device__ __forceinline__ void gemv_pass(const GemvArgs& a, const float4* __restrict__ xs4,
-                                          float (*red)[kGemvTC][2][32], int K, int rb,
-                                          const uint8_t* __restrict__ baseA,
-                                          const uint8_t* __restrict__ baseB,
+// One warp: 16 rows (block b16 of this CTA's 64), reduction groups
+// [kb0, kb1), NT column groups of 8.  Column n of group c carries token
+// 4c + (n & 3), hi part for n < 4 and lo part for n >= 4.
+template <bool GATEUP, int NT>
+__device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __restrict__ codesA,
+                                          const uint8_t* __restrict__ codesB,
                                           const float* __restrict__ sA,
-                                          const float* __restrict__ sB, int pc) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int NG64 = K / kGroupCols;
-    const int K4 = K / 4;
-    const bool grouped = a.group != 0;
-    float accA[TC], accB[TC];
+                                          const float* __restrict__ sB, int K, int row0,
+                                          int kb0, int kb1, int pc, int p1,
+                                          float accA[NT][4], float accB[NT][4]) {
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int KB = K / 64;
+    const int rt = row0 / kTileRows, b8 = (row0 % kTileRows) / 16;
+    const int ng = a.group ? KB : 1;
+    // this lane's B column: token pc + 4c + (g & 3), part g >> 2
+    const __half* bsrc[NT];
+    const float* bsig[NT];
+    bool bvalid[NT];
+    // this lane's D columns 2t, 2t+1: tokens pc + 4c + (2t & 3) + {0, 1}
+    const float* dsig[NT][2];
 #pragma unroll
-    for (int t = 0; t < TC; ++t) { accA[t] = 0.0f; accB[t] = 0.0f; }
+    for (int c = 0; c < NT; ++c) {
+        const int pb = pc + 4 * c + (g & 3);
+        bvalid[c] = pb < p1;
+        const int sb = bvalid[c] ? (GATEUP ? a.pair_tok[pb] : pb) : 0;
+        bsrc[c] = (GATEUP ? a.xq : a.hq) + (int64_t)sb * KB * 128 + (g >> 2) * 64 + 4 * t;
+        bsig[c] = (GATEUP ? a.xinv : a.hinv) + (int64_t)sb * KB;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int pd = pc + 4 * c + ((2 * t) & 3) + i;
+            const int sd = pd < p1 ? (GATEUP ? a.pair_tok[pd] : pd) : 0;
+            dsig[c][i] = (GATEUP ? a.xinv : a.hinv) + (int64_t)sd * KB;
+        }
+    }
+    const float* rowsA0 = sA + scale_offset(row0 + g, 0, ng);
+    const float* rowsB0 = sB + scale_offset(row0 + g, 0, ng);
+#pragma unroll
+    for (int c = 0; c < NT; ++c)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { accA[c][i] = 0.0f; accB[c][i] = 0.0f; }
 
 #pragma unroll 2
-    for (int g = warp; g < NG64; g += kGemvWarps) {
-        // two 16-byte units (64 columns) per matrix; a unit step is 128*16 bytes
-        const uint4 a0 = ldg_stream(baseA + (int64_t)(2 * g) * (kTileRows * 16));
-        const uint4 a1 = ldg_stream(baseA + (int64_t)(2 * g + 1) * (kTileRows * 16));
-        uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
-        if (GATEUP) {
-            b0 = ldg_stream(baseB + (int64_t)(2 * g) * (kTileRows * 16));
-            b1 = ldg_stream(baseB + (int64_t)(2 * g + 1) * (kTileRows * 16));
-        }
-        const float scA = grouped ? __ldg(sA + (int64_t)g * kTileRows) : 1.0f;
-        const float scB = (GATEUP && grouped) ? __ldg(sB + (int64_t)g * kTileRows) : 1.0f;
-        const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        f2_t pa[TC], pb[TC];
+    for (int kb = kb0; kb < kb1; ++kb) {
+        const int64_t uoff = frag_unit_offset(rt, kb, b8, lane, K);
+        const uint4 ua = ldg_stream(codesA + uoff);
+        uint4 ub = make_uint4(0, 0, 0, 0);
+        if (GATEUP) ub = ldg_stream(codesB + uoff);
+        // B fragments: 4 fp16 of this lane's column for each 16-column sub-block
+        uint2 bf[NT][4];
 #pragma unroll
-        for (int t = 0; t < TC; ++t) { pa[t] = 0ull; pb[t] = 0ull; }
+        for (int c = 0; c < NT; ++c)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            f2_t da[4], db[4];
-            decode8(wa[i], da);
-            if (GATEUP) decode8(wb[i], db);
+            for (int j = 0; j < 4; ++j)
+                bf[c][j] = bvalid[c] ? *reinterpret_cast<const uint2*>(bsrc[c] + (int64_t)kb * 128 + 16 * j)
+                                     : make_uint2(0u, 0u);
+        float dA[NT][4], dB[NT][4];
 #pragma unroll
-            for (int t = 0; t < TC; ++t) {
-                const float4* xp = xs4 + t * K4 + (g * kGroupCols + 8 * i) / 4;
-                const float4 x0 = xp[0], x1 = xp[1];
-                const f2_t x01 = f2pack(x0.x, x0.y), x23 = f2pack(x0.z, x0.w);
-                const f2_t x45 = f2pack(x1.x, x1.y), x67 = f2pack(x1.z, x1.w);
-                pa[t] = f2fma(da[0], x01, pa[t]);
-                pa[t] = f2fma(da[1], x23, pa[t]);
-                pa[t] = f2fma(da[2], x45, pa[t]);
-                pa[t] = f2fma(da[3], x67, pa[t]);
-                if (GATEUP) {
-                    pb[t] = f2fma(db[0], x01, pb[t]);
-                    pb[t] = f2fma(db[1], x23, pb[t]);
-                    pb[t] = f2fma(db[2], x45, pb[t]);
-                    pb[t] = f2fma(db[3], x67, pb[t]);
-                }
-            }
-        }
+        for (int c = 0; c < NT; ++c)
 #pragma unroll
-        for (int t = 0; t < TC; ++t) {
-            const float2 va = f2unpack(pa[t]);
-            accA[t] = fmaf(scA, va.x + va.y, accA[t]);
+            for (int i = 0; i < 4; ++i) { dA[c][i] = 0.0f; dB[c][i] = 0.0f; }
+        const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
+        const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t r0, r1, r2, r3;
+            decode_frag_word(wa[j], r0, r1, r2, r3);
+            // A fragment: a0 = row g (k 2t,2t+1) <- r0, a1 = row g+8 <- r2,
+            // a2 = row g (k 2t+8, 2t+9) <- r1, a3 = row g+8 <- r3; the column
+            // permutation is matched by the B layout (4 consecutive columns)
+#pragma unroll
+            for (int c = 0; c < NT; ++c) mma_f16_16816(dA[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
             if (GATEUP) {
-                const float2 vb = f2unpack(pb[t]);
-                accB[t] = fmaf(scB, vb.x + vb.y, accB[t]);
+                decode_frag_word(wb[j], r0, r1, r2, r3);
+#pragma unroll
+                for (int c = 0; c < NT; ++c) mma_f16_16816(dB[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
             }
         }
-    }
-#pragma unroll
-    for (int t = 0; t < TC; ++t) {
-        red[warp][t][0][lane] = accA[t];
-        red[warp][t][1][lane] = accB[t];
-    }
-    __syncthreads();
-    if (threadIdx.x < TC * 32) {
-        const int t = threadIdx.x >> 5, r = threadIdx.x & 31;
-        float A = 0.0f, B = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kGemvWarps; ++w) { A += red[w][t][0][r]; B += red[w][t][1][r]; }
-        if (!grouped) {  // per-row scale, applied once after the full sum
-            A *= __ldg(sA);
-            if (GATEUP) B *= __ldg(sB);
+        // group epilogue: weight scale of rows g, g+8 times the activation
+        // group's inverse scale of columns 2t, 2t+1
+        const int sg = a.group ? kb : 0;
+        const float sa0 = __ldg(rowsA0 + (int64_t)sg * kTileRows);
+        const float sa1 = __ldg(rowsA0 + (int64_t)sg * kTileRows + 8);
+        float sb0 = 0.f, sb1 = 0.f;
+        if (GATEUP) {
+            sb0 = __ldg(rowsB0 + (int64_t)sg * kTileRows);
+            sb1 = __ldg(rowsB0 + (int64_t)sg * kTileRows + 8);
         }
-        const int row = rb * 32 + r;
-        if (GATEUP) a.h[(int64_t)(pc + t) * a.I + row] = silu_f(A) * B;
-        else        a.o[(int64_t)(pc + t) * a.H + row] = A;
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+            const float i0 = __ldg(dsig[c][0] + kb), i1 = __ldg(dsig[c][1] + kb);
+            accA[c][0] = fmaf(sa0 * i0, dA[c][0], accA[c][0]);
+            accA[c][1] = fmaf(sa0 * i1, dA[c][1], accA[c][1]);
+            accA[c][2] = fmaf(sa1 * i0, dA[c][2], accA[c][2]);
+            accA[c][3] = fmaf(sa1 * i1, dA[c][3], accA[c][3]);
+            if (GATEUP) {
+                accB[c][0] = fmaf(sb0 * i0, dB[c][0], accB[c][0]);
+                accB[c][1] = fmaf(sb0 * i1, dB[c][1], accB[c][1]);
+                accB[c][2] = fmaf(sb1 * i0, dB[c][2], accB[c][2]);
+                accB[c][3] = fmaf(sb1 * i1, dB[c][3], accB[c][3]);
+            }
+        }
     }
 }
 
-template <bool GATEUP, typename XT>
+template <bool GATEUP, int NT>
+__device__ __forceinline__ void gemv_pass(const GemvArgs& a, float* red, const uint8_t* codesA,
+                                          const uint8_t* codesB, const float* sA,
+                                          const float* sB, int K, int rb64, int pc, int p1) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int b16 = warp & 3, half = warp >> 2;
+    const int KB = K / 64;
+    const int row0 = rb64 * 64 + b16 * 16;
+    float accA[NT][4], accB[NT][4];
+    gemv_warp<GATEUP, NT>(a, codesA, codesB, sA, sB, K, row0, half * (KB / 2),
+                          (half + 1) * (KB / 2), pc, p1, accA, accB);
+    // red layout: [mat 2][half 2][64 rows][8*NT cols]
+    const int C = 8 * NT;
+#pragma unroll
+    for (int c = 0; c < NT; ++c)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = b16 * 16 + g + (i >> 1) * 8, n = 8 * c + 2 * t + (i & 1);
+            red[((0 * 2 + half) * 64 + r) * C + n] = accA[c][i];
+            if (GATEUP) red[((1 * 2 + half) * 64 + r) * C + n] = accB[c][i];
+        }
+    __syncthreads();
+}
+
+template <bool GATEUP, int NT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
 expert_gemv_kernel(GemvArgs a) {
-    extern __shared__ float4 gemv_xs4[];  // [TC][K/4] pre-scaled input rows
-    __shared__ float red[kGemvWarps][kGemvTC][2][32];
+    __shared__ float red[2 * 2 * 64 * 8 * kGemvMaxNT];
+    __shared__ float gmax[16][2];
+    __shared__ int last_flag;
     const int K = GATEUP ? a.H : a.I;
     const int R = GATEUP ? a.I : a.H;
-    const int nb = R / 32;
-    const int u = blockIdx.x / nb, rb = blockIdx.x % nb;
+    const int nrb = R / 64;
+    const int u = blockIdx.x / nrb, rb64 = blockIdx.x % nrb;
     if (u >= *a.n_units) return;
     const int e = a.unit_expert[u], p0 = a.unit_begin[u], p1 = a.unit_end[u];
     const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
-    const int lane = threadIdx.x & 31;
-    const int row = rb * 32 + lane;
     const int mA = GATEUP ? 0 : 2;
-    const int ng = a.L.ngroups[mA];
-    const uint8_t* baseA = blob + a.L.codes[mA] + code_unit_offset(row, 0, K);
-    const uint8_t* baseB = blob + a.L.codes[1] + code_unit_offset(row, 0, K);
-    const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[mA]) + scale_offset(row, 0, ng);
-    const float* sB = reinterpret_cast<const float*>(blob + a.L.scales[1]) + scale_offset(row, 0, ng);
-    const int K4 = K / 4;
+    const uint8_t* codesA = blob + a.L.codes[mA];
+    const uint8_t* codesB = blob + a.L.codes[1];
+    const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[mA]);
+    const float* sB = reinterpret_cast<const float*>(blob + a.L.scales[1]);
+    const int C = 8 * NT;
+    const int tid = threadIdx.x;
 
-    for (int pc = p0; pc < p1; pc += kGemvTC) {
-        const int tc = min(kGemvTC, p1 - pc);
-        __syncthreads();  // previous pass done with xs and red
-        for (int i = threadIdx.x; i < tc * K4; i += kGemvWarps * 32) {
-            const int t = i / K4, c4 = i - t * K4;
-            float4 v;
-            if (GATEUP) {
-                const XT* src = reinterpret_cast<const XT*>(a.x) +
-                                (int64_t)a.pair_tok[pc + t] * a.H + 4 * c4;
-                v = make_float4(to_f32(src[0]), to_f32(src[1]), to_f32(src[2]), to_f32(src[3]));
-            } else {
-                v = *reinterpret_cast<const float4*>(a.h + (int64_t)(pc + t) * a.I + 4 * c4);
+    for (int pc = p0; pc < p1; pc += 4 * NT) {
+        const int tc = min(4 * NT, p1 - pc);
+        __syncthreads();  // previous pass finished with red
+        gemv_pass<GATEUP, NT>(a, red, codesA, codesB, sA, sB, K, rb64, pc, p1);
+        // combine halves and hi/lo: thread -> (token tt, row r)
+        if (GATEUP) {
+            // h for 64 rows x tc tokens, then one power-of-two scale per token
+            for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
+                const int tt = q / 64, r = q % 64;
+                const int c = tt / 4, n = 8 * c + (tt & 3);
+                const float ga = red[((0 * 2 + 0) * 64 + r) * C + n] + red[((0 * 2 + 1) * 64 + r) * C + n] +
+                                 red[((0 * 2 + 0) * 64 + r) * C + n + 4] + red[((0 * 2 + 1) * 64 + r) * C + n + 4];
+                const float ua = red[((1 * 2 + 0) * 64 + r) * C + n] + red[((1 * 2 + 1) * 64 + r) * C + n] +
+                                 red[((1 * 2 + 0) * 64 + r) * C + n + 4] + red[((1 * 2 + 1) * 64 + r) * C + n + 4];
+                const float hv = silu_f(ga) * ua;
+                red[((0 * 2 + 0) * 64 + r) * C + n] = hv;  // reuse: h in slot (0, 0, r, n)
+                float m = fabsf(hv);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if ((q & 31) == 0) gmax[tt][(q >> 5) & 1] = m;
             }
-            const int j = (4 * c4) & 7;  // column position inside its 8-nibble word
-            v.x *= kPosScale(j); v.y *= kPosScale(j + 1);
-            v.z *= kPosScale(j + 2); v.w *= kPosScale(j + 3);
-            gemv_xs4[t * K4 + c4] = v;
-        }
-        __syncthreads();
-        switch (tc) {
-            case 4: gemv_pass<GATEUP, 4>(a, gemv_xs4, red, K, rb, baseA, baseB, sA, sB, pc); break;
-            case 3: gemv_pass<GATEUP, 3>(a, gemv_xs4, red, K, rb, baseA, baseB, sA, sB, pc); break;
-            case 2: gemv_pass<GATEUP, 2>(a, gemv_xs4, red, K, rb, baseA, baseB, sA, sB, pc); break;
-            default: gemv_pass<GATEUP, 1>(a, gemv_xs4, red, K, rb, baseA, baseB, sA, sB, pc); break;
+            __syncthreads();
+            for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
+                const int tt = q / 64, r = q % 64;
+                const int c = tt / 4, n = 8 * c + (tt & 3);
+                const float hv = red[((0 * 2 + 0) * 64 + r) * C + n];
+                float inv;
+                const float sc = act_group_scale(fmaxf(gmax[tt][0], gmax[tt][1]), &inv);
+                __half hi, lo;
+                split_f16(hv * sc, hi, lo);
+                const int64_t p = pc + tt;
+                __half* dst = a.hq + (p * (a.I / 64) + rb64) * 128;
+                dst[r] = hi;
+                dst[64 + r] = lo;
+                if (r == 0) a.hinv[p * (a.I / 64) + rb64] = inv;
+            }
+        } else {
+            for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
+                const int tt = q / 64, r = q % 64;
+                const int c = tt / 4, n = 8 * c + (tt & 3);
+                const float v = red[((0 * 2 + 0) * 64 + r) * C + n] + red[((0 * 2 + 1) * 64 + r) * C + n] +
+                                red[((0 * 2 + 0) * 64 + r) * C + n + 4] + red[((0 * 2 + 1) * 64 + r) * C + n + 4];
+                a.o[(int64_t)(pc + tt) * a.H + rb64 * 64 + r] = v;
+            }
         }
     }
-}
+    if (GATEUP) return;
 
-// y[t] = residual[t] + sum_j w[t, j] * o[inv[t, j]] + sum_s o[T*k + s*T + t]
-__global__ void __launch_bounds__(256)
-combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv,
-               const float* __restrict__ w, int T, int k, int n_shared, int H,
-               const float* residual, float* y) {
-    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    const int H4 = H / 4;
-    if (i >= (int64_t)T * H4) return;
-    const int t = (int)(i / H4), c = (int)(i % H4) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-        const int p = inv[(int64_t)t * k + j];
-        const float wj = w[(int64_t)t * k + j];
-        const float4 v = *reinterpret_cast<const float4*>(o + (int64_t)p * H + c);
-        acc.x = fmaf(wj, v.x, acc.x); acc.y = fmaf(wj, v.y, acc.y);
-        acc.z = fmaf(wj, v.z, acc.z); acc.w = fmaf(wj, v.w, acc.w);
+    // ---- combine: the last unit to finish this 64-row block writes y ----
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const int done = atomicAdd(&a.counters[rb64], 1) + 1;
+        last_flag = done == *a.n_units;
     }
-    for (int s = 0; s < n_shared; ++s) {
-        const int64_t p = (int64_t)T * k + (int64_t)s * T + t;
-        const float4 v = *reinterpret_cast<const float4*>(o + p * H + c);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    __syncthreads();
+    if (!last_flag) return;
+    __threadfence();
+    for (int q = tid; q < a.T * 64; q += kGemvWarps * 32) {
+        const int tt = q / 64, r = rb64 * 64 + q % 64;
+        float acc = 0.0f;
+        for (int j = 0; j < a.k; ++j) {
+            const int p = __ldcg(a.inv + (int64_t)tt * a.k + j);
+            acc = fmaf(__ldcg(a.w + (int64_t)tt * a.k + j), __ldcg(a.o + (int64_t)p * a.H + r), acc);
+        }
+        for (int s = 0; s < a.n_shared; ++s)
+            acc += __ldcg(a.o + ((int64_t)a.T * a.k + (int64_t)s * a.T + tt) * a.H + r);
+        if (a.residual) acc = a.residual[(int64_t)tt * a.H + r] + acc;
+        a.y[(int64_t)tt * a.H + r] = acc;
     }
-    if (residual) {
-        const float4 r = *reinterpret_cast<const float4*>(residual + (int64_t)t * H + c);
-        acc.x = r.x + acc.x; acc.y = r.y + acc.y; acc.z = r.z + acc.z; acc.w = r.w + acc.w;
-    }
-    *reinterpret_cast<float4*>(y + (int64_t)t * H + c) = acc;
+    if (tid == 0) a.counters[rb64] = 0;  // ready for the next call on this workspace
 }
 
 }  // namespace coli

@@ -17,55 +17,69 @@ __device__ __forceinline__ int quant_one(float v, float s) {
     return (int)q;
 }
 
-// one warp per row; the row's packed bytes are assembled in shared memory and
-// written out as 16-byte units of the device layout
+// One CTA per 16-row block of a 128-row tile.  Each warp quantises two rows
+// into shared memory in container byte order, then every thread assembles
+// 16-byte fragment-tile units (see common.cuh) and stores them.
 __global__ void __launch_bounds__(256)
 quantize_rows_kernel(const float* __restrict__ w, int R, int K, int group,
                      uint8_t* __restrict__ codes, float* __restrict__ scales) {
     extern __shared__ uint4 qz_smem[];
+    uint8_t* rows = reinterpret_cast<uint8_t*>(qz_smem);  // [16][K/2]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = blockIdx.x * 8 + warp;
-    if (r >= R) return;
-    uint8_t* buf = reinterpret_cast<uint8_t*>(qz_smem) + (int64_t)warp * (K / 2);
-    const float* row = w + (int64_t)r * K;
+    const int blk = blockIdx.x;                            // 16-row block index
+    const int rt = blk / 8, b8 = blk % 8;
     const int gs = group ? group : K;
     const int ng = K / gs;
-    for (int g = 0; g < ng; ++g) {
-        float m = 0.0f;
-        for (int c = g * gs + lane; c < (g + 1) * gs; c += 32) m = fmaxf(m, fabsf(row[c]));
+    for (int lr = warp; lr < 16; lr += 8) {
+        const int r = blk * 16 + lr;
+        const float* row = w + (int64_t)r * K;
+        uint8_t* buf = rows + (int64_t)lr * (K / 2);
+        for (int g = 0; g < ng; ++g) {
+            float m = 0.0f;
+            for (int c = g * gs + lane; c < (g + 1) * gs; c += 32) m = fmaxf(m, fabsf(row[c]));
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        const float s = __fdiv_rn(m, 7.0f);
-        if (lane == 0) scales[scale_offset(r, g, ng)] = s;
-        for (int cp = g * gs / 2 + lane; cp < (g + 1) * gs / 2; cp += 32) {
-            const int q0 = quant_one(row[2 * cp], s), q1 = quant_one(row[2 * cp + 1], s);
-            buf[cp] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const float s = __fdiv_rn(m, 7.0f);
+            if (lane == 0) scales[scale_offset(r, g, ng)] = s;
+            for (int cp = g * gs / 2 + lane; cp < (g + 1) * gs / 2; cp += 32) {
+                const int q0 = quant_one(row[2 * cp], s), q1 = quant_one(row[2 * cp + 1], s);
+                buf[cp] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
+            }
         }
     }
-    __syncwarp();
-    for (int c = lane; c < K / 32; c += 32)
-        *reinterpret_cast<uint4*>(codes + code_unit_offset(r, c, K)) =
-            *reinterpret_cast<const uint4*>(buf + 16 * c);
+    __syncthreads();
+    for (int i = threadIdx.x; i < (K / 64) * 32; i += 256) {
+        const int kb = i / 32, l = i % 32, g = l >> 2, t = l & 3;
+        uint32_t wd[4];
+        for (int j = 0; j < 4; ++j) {
+            uint32_t word = 0;
+            for (int upper = 0; upper < 2; ++upper)
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int lr = g + 8 * upper, c = kb * 64 + 16 * j + 4 * t + cc;
+                    const uint8_t byte = rows[(int64_t)lr * (K / 2) + c / 2];
+                    const uint32_t nib = (c & 1) ? (byte >> 4) : (byte & 15);
+                    word |= nib << frag_nibble_shift(lr, c);
+                }
+            wd[j] = word;
+        }
+        *reinterpret_cast<uint4*>(codes + frag_unit_offset(rt, kb, b8, l, K)) =
+            make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    }
 }
 
-// one thread per (row, 16-byte unit): out[r, c] = (float)q * s
+// one thread per element: out[r, c] = (float)q * s
 __global__ void __launch_bounds__(256)
 dequant_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ scales,
                int R, int K, int group, float* __restrict__ out) {
     const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    const int KC = K / 32;
-    if (i >= (int64_t)R * KC) return;
-    const int r = (int)(i / KC), c = (int)(i % KC);
+    if (i >= (int64_t)R * K) return;
+    const int r = (int)(i / K), c = (int)(i % K);
     const int ng = group ? K / group : 1;
-    const uint4 v = *reinterpret_cast<const uint4*>(codes + code_unit_offset(r, c, K));
-    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-    for (int j = 0; j < 32; ++j) {
-        const int col = 32 * c + j;
-        int n = (wd[j / 8] >> (4 * (j % 8))) & 15;
-        n = n >= 8 ? n - 16 : n;
-        const float s = scales[scale_offset(r, group ? col / group : 0, ng)];
-        out[(int64_t)r * K + col] = __fmul_rn((float)n, s);
-    }
+    const uint32_t word = *reinterpret_cast<const uint32_t*>(codes + frag_word_offset(r, c, K));
+    int n = (word >> frag_nibble_shift(r, c)) & 15;
+    n = n >= 8 ? n - 16 : n;
+    const float s = scales[scale_offset(r, group ? c / group : 0, ng)];
+    out[i] = __fmul_rn((float)n, s);
 }
 
 // RMSNorm with unit gain: one CTA per row, f32 sum of squares

@@ -1,4 +1,5 @@
-// route.cuh - router logits, sigmoid + bias-corrected top-k, and the batch union.
+// route.cuh - router logits, sigmoid + bias-corrected top-k, the batch union,
+// and the fp16 activation operand of the expert kernels.
 //
 // Router ("解密GLM-5.2-colibri-int4-with-int8-mtp" 模型架构深度解析; "github一周涨11k
 // ⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.1 and 四.3): z = W_r x in f32 (plain FMA on
@@ -12,46 +13,86 @@
 
 namespace coli {
 
+constexpr int kMaxKS = 8;
+
+// ---------------------------------------------------------------------------
+// fp16 hi/lo activation operand: one warp per (token, 64-column group).
+// xq[t][g][0..64) = hi, [64..128) = lo of x * 2^sh, xinv[t][g] = 2^-sh.
+// ---------------------------------------------------------------------------
+template <typename XT>
+__device__ __forceinline__ void act_quant_group(const XT* __restrict__ x, int H, int t, int kb,
+                                                __half* __restrict__ xq, float* __restrict__ xinv) {
+    const int lane = threadIdx.x & 31;
+    const XT* src = x + (int64_t)t * H + kb * 64 + 2 * lane;
+    const float v0 = to_f32(src[0]), v1 = to_f32(src[1]);
+    float m = fmaxf(fabsf(v0), fabsf(v1));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float inv;
+    const float sc = act_group_scale(m, &inv);
+    __half h0, l0, h1, l1;
+    split_f16(v0 * sc, h0, l0);
+    split_f16(v1 * sc, h1, l1);
+    __half* dst = xq + ((int64_t)t * (H / 64) + kb) * 128;
+    *reinterpret_cast<__half2*>(dst + 2 * lane) = __halves2half2(h0, h1);
+    *reinterpret_cast<__half2*>(dst + 64 + 2 * lane) = __halves2half2(l0, l1);
+    if (lane == 0) xinv[(int64_t)t * (H / 64) + kb] = inv;
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+act_quant_kernel(const XT* __restrict__ x, int T, int H, __half* __restrict__ xq,
+                 float* __restrict__ xinv) {
+    const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int KB = H / 64;
+    if (gw >= T * KB) return;
+    act_quant_group(x, H, gw / KB, gw % KB, xq, xinv);
+}
+
 // ---------------------------------------------------------------------------
 // Router logits, small batches: one warp per (expert row, K slice).  The warp
-// streams its slice of W_r once with 16-byte loads and dots it with every
-// token.  Partial sums go to zpart[ks][t][e]; top-k adds the slices in order.
+// issues all of its 16-byte loads of W_r before the first FMA.  Partial sums go
+// to zpart[ks][t][e]; top-k adds the slices in order.  Blocks past the router's
+// share build the fp16 activation operand (xq) when xq != nullptr.
 // ---------------------------------------------------------------------------
+constexpr int kRouterMaxSlice = 1024;  // columns per warp slice (<= 8 loads per lane)
+
 template <typename XT>
 __global__ void __launch_bounds__(256)
 router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restrict__ wr,
-                   int E, int KS, float* __restrict__ zpart) {
+                   int E, int KS, float* __restrict__ zpart, int router_blocks,
+                   __half* __restrict__ xq, float* __restrict__ xinv) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if ((int)blockIdx.x >= router_blocks) {
+        const int gw = (blockIdx.x - router_blocks) * 8 + warp;
+        const int KB = H / 64;
+        if (xq && gw < T * KB) act_quant_group(x, H, gw / KB, gw % KB, xq, xinv);
+        return;
+    }
     const int gw = blockIdx.x * 8 + warp;
     const int e = gw / KS, ks = gw % KS;
     if (e >= E) return;
-    const int SL = H / KS;  // multiple of 128
+    const int SL = H / KS;  // multiple of 128, at most kRouterMaxSlice
     const float* wrow = wr + (int64_t)e * H + (int64_t)ks * SL;
-    for (int t0 = 0; t0 < T; t0 += 8) {
-        const int tn = min(8, T - t0);
-        float acc[8];
+    float4 wv[kRouterMaxSlice / 128];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        for (int c = lane * 4; c < SL; c += 128) {
-            const float4 wv = *reinterpret_cast<const float4*>(wrow + c);
+    for (int i = 0; i < kRouterMaxSlice / 128; ++i)
+        if (i * 128 < SL) wv[i] = __ldg(reinterpret_cast<const float4*>(wrow + i * 128 + lane * 4));
+    for (int t = 0; t < T; ++t) {
+        const XT* xr = x + (int64_t)t * H + (int64_t)ks * SL + lane * 4;
+        float acc = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (i < tn) {
-                    const XT* xp = x + (int64_t)(t0 + i) * H + (int64_t)ks * SL + c;
-                    acc[i] = fmaf(wv.x, to_f32(xp[0]), acc[i]);
-                    acc[i] = fmaf(wv.y, to_f32(xp[1]), acc[i]);
-                    acc[i] = fmaf(wv.z, to_f32(xp[2]), acc[i]);
-                    acc[i] = fmaf(wv.w, to_f32(xp[3]), acc[i]);
-                }
+        for (int i = 0; i < kRouterMaxSlice / 128; ++i) {
+            if (i * 128 < SL) {
+                const XT* xp = xr + i * 128;
+                acc = fmaf(wv[i].x, to_f32(xp[0]), acc);
+                acc = fmaf(wv[i].y, to_f32(xp[1]), acc);
+                acc = fmaf(wv[i].z, to_f32(xp[2]), acc);
+                acc = fmaf(wv[i].w, to_f32(xp[3]), acc);
             }
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (i < tn) {
-                const float v = warp_sum(acc[i]);
-                if (lane == 0) zpart[((int64_t)ks * T + t0 + i) * E + e] = v;
-            }
-        }
+        acc = warp_sum(acc);
+        if (lane == 0) zpart[((int64_t)ks * T + t) * E + e] = acc;
     }
 }
 
@@ -74,7 +115,6 @@ router_tiled_kernel(const XT* __restrict__ x, int T, int H, const float* __restr
     const int tr = (tid / 16) * 4, er = (tid % 16) * 4;
     float acc[4][4] = {};
     for (int k0 = kbeg; k0 < kend; k0 += BK) {
-        // 64 rows x 16 columns of x and of W_r: 1024 values each, 4 per thread
         for (int i = tid; i < BT * BK; i += 256) {
             const int r = i / BK, c = i % BK;
             const int t = t0 + r, e = e0 + r;
@@ -84,13 +124,13 @@ router_tiled_kernel(const XT* __restrict__ x, int T, int H, const float* __restr
         __syncthreads();
 #pragma unroll
         for (int c = 0; c < BK; ++c) {
-            float a[4], b[4];
+            float av[4], bv[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) { a[i] = xs[c][tr + i]; b[i] = ws[c][er + i]; }
+            for (int i = 0; i < 4; ++i) { av[i] = xs[c][tr + i]; bv[i] = ws[c][er + i]; }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
     }
@@ -104,28 +144,27 @@ router_tiled_kernel(const XT* __restrict__ x, int T, int H, const float* __restr
 }
 
 // ---------------------------------------------------------------------------
-// Sigmoid, bias-corrected top-k and weights: one warp per token.  The warp
-// keeps the token's E scores in shared memory and runs k rounds of a warp
-// arg-max over (sel desc, index asc).
+// Sigmoid, bias-corrected top-k and weights for one token, by one warp, with
+// sel / s in shared memory (2E floats).  Writes idx[t, :], w[t, :].
 // ---------------------------------------------------------------------------
-constexpr int kTopkWarps = 4;
-
-__global__ void __launch_bounds__(32 * kTopkWarps)
-topk_kernel(const float* __restrict__ zpart, int KS, int T, int E,
-            const float* __restrict__ bias, int k, float routed_scale, int norm_topk,
-            int32_t* __restrict__ idx, float* __restrict__ w) {
-    extern __shared__ float tk_smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kTopkWarps + warp;
-    if (t >= T) return;
-    float* sel = tk_smem + (int64_t)warp * 2 * E;
-    float* sc = sel + E;
+__device__ __forceinline__ void topk_token(const float* __restrict__ zpart, int KS, int T, int E,
+                                           const float* __restrict__ bias, int k,
+                                           float routed_scale, int norm_topk, int t, float* sel,
+                                           float* sc, int32_t* __restrict__ idx,
+                                           float* __restrict__ w) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll 4
     for (int e = lane; e < E; e += 32) {
+        float zp[kMaxKS];
+#pragma unroll
+        for (int ks = 0; ks < kMaxKS; ++ks)
+            zp[ks] = ks < KS ? __ldcg(zpart + ((int64_t)ks * T + t) * E + e) : 0.0f;
         float z = 0.0f;
-        for (int ks = 0; ks < KS; ++ks) z += zpart[((int64_t)ks * T + t) * E + e];
+#pragma unroll
+        for (int ks = 0; ks < kMaxKS; ++ks) z += zp[ks];
         const float s = 1.0f / (1.0f + expf(-z));
         sc[e] = s;
-        sel[e] = s + bias[e];
+        sel[e] = s + __ldg(bias + e);
     }
     __syncwarp();
     float mine = 0.0f;  // lane j keeps the score of the j-th pick
@@ -148,8 +187,7 @@ topk_kernel(const float* __restrict__ zpart, int KS, int T, int E,
         if (lane == 0) sel[be] = -INFINITY;
         __syncwarp();
     }
-    // renormalise over the k picks in pick order
-    float denom = 0.0f;
+    float denom = 0.0f;  // renormalise over the k picks in pick order
     for (int j = 0; j < k; ++j) denom += __shfl_sync(0xffffffffu, mine, j);
     if (lane < k) {
         idx[(int64_t)t * k + lane] = mine_e;
@@ -157,16 +195,31 @@ topk_kernel(const float* __restrict__ zpart, int KS, int T, int E,
     }
 }
 
+constexpr int kTopkWarps = 4;
+
+__global__ void __launch_bounds__(32 * kTopkWarps)
+topk_kernel(const float* __restrict__ zpart, int KS, int T, int E,
+            const float* __restrict__ bias, int k, float routed_scale, int norm_topk,
+            int32_t* __restrict__ idx, float* __restrict__ w) {
+    extern __shared__ float tk_smem[];
+    const int warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * kTopkWarps + warp;
+    if (t >= T) return;
+    float* sel = tk_smem + (int64_t)warp * 2 * E;
+    topk_token(zpart, KS, T, E, bias, k, routed_scale, norm_topk, t, sel, sel + E, idx, w);
+}
+
 // ---------------------------------------------------------------------------
-// Batch union in one CTA: per-expert counts, an exclusive scan, and a stable
-// scatter.  A pair's rank inside its expert is the number of earlier tokens
-// that chose the same expert, read from a per-expert token bitmap (a token
-// picks an expert at most once), so the order never depends on timing.
-// Optionally also emits the work list the expert kernels consume.
+// Batch union in one CTA of 1024 threads: per-expert counts, an exclusive scan
+// and a stable scatter.  A pair's rank inside its expert is the number of
+// earlier tokens that chose the same expert, read from a per-expert token
+// bitmap (a token picks an expert at most once), so the order never depends on
+// timing.  Optionally also emits the expert kernels' work list and clears the
+// combine counters.
 // ---------------------------------------------------------------------------
 struct UnionOut {
     int32_t* offsets;      // [E+1]
-    int32_t* pair_tok;     // [T*k] (+ T*n_shared shared pairs when units != 0)
+    int32_t* pair_tok;     // [T*k] (+ T*n_shared shared pairs when unit_expert)
     int32_t* pair_slot;    // [T*k]
     int32_t* uniq;         // [E]
     int32_t* n_uniq;       // [1]
@@ -175,23 +228,26 @@ struct UnionOut {
     int32_t* unit_begin;
     int32_t* unit_end;
     int32_t* n_units;      // [1]
+    int32_t* counters;     // combine counters to clear, or nullptr
+    int32_t n_counters;
     int32_t n_shared;
 };
 
 constexpr int kUnionThreads = 1024;
 
-__global__ void __launch_bounds__(kUnionThreads)
-union_kernel(const int32_t* __restrict__ idx, int T, int k, int E, UnionOut o) {
-    extern __shared__ uint32_t un_smem[];
+__device__ __forceinline__ void union_body(const int32_t* idx, int T, int k, int E,
+                                           const UnionOut& o, uint32_t* un_smem) {
     const int W = (T + 31) / 32;
-    uint32_t* bits = un_smem;                       // [E][W]
-    int32_t* cnt = reinterpret_cast<int32_t*>(bits + (int64_t)E * W);  // [E]
-    int32_t* excl = cnt + E;                        // [E]
-    int32_t* uexcl = excl + E;                      // [E]
+    uint32_t* bits = un_smem;                                           // [E][W]
+    int32_t* cnt = reinterpret_cast<int32_t*>(bits + (int64_t)E * W);   // [E]
+    int32_t* excl = cnt + E;                                            // [E]
+    int32_t* uexcl = excl + E;                                          // [E]
     __shared__ int32_t warp_tot[2][32];
     const int tid = threadIdx.x;
     for (int i = tid; i < E * W; i += kUnionThreads) bits[i] = 0u;
     for (int i = tid; i < E; i += kUnionThreads) cnt[i] = 0;
+    if (o.counters)
+        for (int i = tid; i < o.n_counters; i += kUnionThreads) o.counters[i] = 0;
     __syncthreads();
     const int P = T * k;
     for (int i = tid; i < P; i += kUnionThreads) {
@@ -216,7 +272,7 @@ union_kernel(const int32_t* __restrict__ idx, int T, int k, int E, UnionOut o) {
     if (lane == 31) { warp_tot[0][warp] = sc; warp_tot[1][warp] = sf; }
     __syncthreads();
     if (warp == 0) {
-        int a = warp_tot[0][lane], b = warp_tot[1][lane];
+        const int a = warp_tot[0][lane], b = warp_tot[1][lane];
         int pa = a, pb = b;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -263,7 +319,6 @@ union_kernel(const int32_t* __restrict__ idx, int T, int k, int E, UnionOut o) {
                 o.unit_end[u] = excl[e] + cnt[e];
             }
         }
-        __syncthreads();
         const int n_uniq = uexcl[E - 1] + (cnt[E - 1] > 0 ? 1 : 0);
         for (int s = tid; s < o.n_shared; s += kUnionThreads) {
             o.unit_expert[n_uniq + s] = E + s;
@@ -272,6 +327,30 @@ union_kernel(const int32_t* __restrict__ idx, int T, int k, int E, UnionOut o) {
         }
         for (int i = tid; i < o.n_shared * T; i += kUnionThreads) o.pair_tok[P + i] = i % T;
     }
+}
+
+__global__ void __launch_bounds__(kUnionThreads)
+union_kernel(const int32_t* __restrict__ idx, int T, int k, int E, UnionOut o) {
+    extern __shared__ uint32_t un_smem[];
+    union_body(idx, T, k, E, o, un_smem);
+}
+
+// Small batches: top-k of every token (warps take tokens in turn) and the union
+// in one CTA, saving a launch and a round trip through global memory.
+__global__ void __launch_bounds__(kUnionThreads)
+topk_union_kernel(const float* __restrict__ zpart, int KS, int T, int E,
+                  const float* __restrict__ bias, int k, float routed_scale, int norm_topk,
+                  int32_t* idx, float* w, int topk_warps, UnionOut o) {
+    extern __shared__ uint32_t un_smem[];
+    const int warp = threadIdx.x >> 5;
+    if (warp < topk_warps) {
+        float* sel = reinterpret_cast<float*>(un_smem) + (int64_t)warp * 2 * E;
+        for (int t = warp; t < T; t += topk_warps)
+            topk_token(zpart, KS, T, E, bias, k, routed_scale, norm_topk, t, sel, sel + E, idx, w);
+    }
+    __threadfence_block();
+    __syncthreads();
+    union_body(idx, T, k, E, o, un_smem);
 }
 
 }  // namespace coli

@@ -58,11 +58,24 @@ def _unpack_blob(blob, H, I, group):
         scale_off.append(off)
         off = sec_align(off + R * ng * 4)
     assert off == blob.size
+    # word j of unit (t, s, b, l): nibble p at bits 4p.. holds
+    #   p: 0 (r0,c0) 1 (r0,c0+2) 2 (r1,c0) 3 (r1,c0+2) 4 (r0,c0+1) 5 (r0,c0+3)
+    #      6 (r1,c0+1) 7 (r1,c0+3); r0 = 128t + 16b + l//4, r1 = r0 + 8,
+    #   c0 = 64s + 16j + 4(l%4)
+    dr = np.array([0, 0, 8, 8, 0, 0, 8, 8])
+    dc = np.array([0, 2, 0, 2, 1, 3, 1, 3])
     out = []
     for m, (R, K) in enumerate(mats):
         ng = 1 if group == 0 else K // group
-        units = blob[code_off[m]:code_off[m] + R * K // 2].reshape(R // 128, K // 32, 128, 16)
-        codes = units.transpose(0, 2, 1, 3).reshape(R, K // 2)
+        words = blob[code_off[m]:code_off[m] + R * K // 2].view(np.uint32)
+        words = words.reshape(R // 128, K // 64, 8, 32, 4)
+        t, s_, b, l, j = np.meshgrid(*[np.arange(n) for n in words.shape], indexing="ij")
+        r0 = 128 * t + 16 * b + l // 4
+        c0 = 64 * s_ + 16 * j + 4 * (l % 4)
+        q = np.zeros((R, K), np.uint8)
+        for p in range(8):
+            q[r0 + dr[p], c0 + dc[p]] = (words >> (4 * p)) & 15
+        codes = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
         sc = blob[scale_off[m]:scale_off[m] + R * ng * 4].view(np.float32)
         sc = sc.reshape(R // 128, ng, 128).transpose(0, 2, 1).reshape(R, ng)
         out += [codes, sc]
