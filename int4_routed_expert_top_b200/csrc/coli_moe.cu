@@ -173,7 +173,7 @@ int launch_union(const int32_t* idx, int T, int k, int E, const UnionOut& o, cud
 int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int32_t* idx,
                   float* w, const UnionOut& o, cudaStream_t st) {
     if (T <= 64) {
-        const int topk_warps = std::max(1, std::min(32, (160 * 1024) / (8 * d.E)));
+        const int topk_warps = std::max(1, std::min(std::min(32, T), (160 * 1024) / (8 * d.E)));
         const int smem = std::max(topk_warps * 2 * d.E * 4, union_smem_bytes(T, d.E));
         int rc = set_smem((const void*)topk_union_kernel, smem);
         if (rc) return rc;

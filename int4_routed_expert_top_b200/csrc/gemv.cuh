@@ -93,64 +93,86 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
 #pragma unroll
         for (int i = 0; i < 4; ++i) { accA[c][i] = 0.0f; accB[c][i] = 0.0f; }
 
-#pragma unroll 2
-    for (int kb = kb0; kb < kb1; ++kb) {
-        const int64_t uoff = frag_unit_offset(rt, kb, b8, lane, K);
-        const uint4 ua = ldg_stream(codesA + uoff);
-        uint4 ub = make_uint4(0, 0, 0, 0);
-        if (GATEUP) ub = ldg_stream(codesB + uoff);
-        // B fragments: 4 fp16 of this lane's column for each 16-column sub-block
-        uint2 bf[NT][4];
+    // weight-scale rows (hoisted for per-row scales)
+    float sa0 = __ldg(rowsA0), sa1 = __ldg(rowsA0 + 8), sb0 = 0.f, sb1 = 0.f;
+    if (GATEUP) { sb0 = __ldg(rowsB0); sb1 = __ldg(rowsB0 + 8); }
+
+    // register ring: the unit loads of the next D steps are always in flight
+    constexpr int D = NT == 1 ? 8 : NT == 2 ? 4 : 2;
+    uint4 ringA[D], ringB[D];
 #pragma unroll
-        for (int c = 0; c < NT; ++c)
+    for (int i = 0; i < D; ++i) {
+        if (kb0 + i < kb1) {
+            const int64_t uoff = frag_unit_offset(rt, kb0 + i, b8, lane, K);
+            ringA[i] = ldg_stream(codesA + uoff);
+            if (GATEUP) ringB[i] = ldg_stream(codesB + uoff);
+        }
+    }
+    for (int kb_base = kb0; kb_base < kb1; kb_base += D) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                bf[c][j] = bvalid[c] ? *reinterpret_cast<const uint2*>(bsrc[c] + (int64_t)kb * 128 + 16 * j)
-                                     : make_uint2(0u, 0u);
-        float dA[NT][4], dB[NT][4];
-#pragma unroll
-        for (int c = 0; c < NT; ++c)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) { dA[c][i] = 0.0f; dB[c][i] = 0.0f; }
-        const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
-        const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t r0, r1, r2, r3;
-            decode_frag_word(wa[j], r0, r1, r2, r3);
-            // A fragment: a0 = row g (k 2t,2t+1) <- r0, a1 = row g+8 <- r2,
-            // a2 = row g (k 2t+8, 2t+9) <- r1, a3 = row g+8 <- r3; the column
-            // permutation is matched by the B layout (4 consecutive columns)
-#pragma unroll
-            for (int c = 0; c < NT; ++c) mma_f16_16816(dA[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
-            if (GATEUP) {
-                decode_frag_word(wb[j], r0, r1, r2, r3);
-#pragma unroll
-                for (int c = 0; c < NT; ++c) mma_f16_16816(dB[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
+        for (int i = 0; i < D; ++i) {
+            const int kb = kb_base + i;
+            if (kb >= kb1) break;
+            const uint4 ua = ringA[i];
+            const uint4 ub = GATEUP ? ringB[i] : make_uint4(0, 0, 0, 0);
+            if (kb + D < kb1) {
+                const int64_t uoff = frag_unit_offset(rt, kb + D, b8, lane, K);
+                ringA[i] = ldg_stream(codesA + uoff);
+                if (GATEUP) ringB[i] = ldg_stream(codesB + uoff);
             }
-        }
-        // group epilogue: weight scale of rows g, g+8 times the activation
-        // group's inverse scale of columns 2t, 2t+1
-        const int sg = a.group ? kb : 0;
-        const float sa0 = __ldg(rowsA0 + (int64_t)sg * kTileRows);
-        const float sa1 = __ldg(rowsA0 + (int64_t)sg * kTileRows + 8);
-        float sb0 = 0.f, sb1 = 0.f;
-        if (GATEUP) {
-            sb0 = __ldg(rowsB0 + (int64_t)sg * kTileRows);
-            sb1 = __ldg(rowsB0 + (int64_t)sg * kTileRows + 8);
-        }
+            // B fragments: 4 fp16 of this lane's column for each 16-column sub-block
+            uint2 bf[NT][4];
 #pragma unroll
-        for (int c = 0; c < NT; ++c) {
-            const float i0 = __ldg(dsig[c][0] + kb), i1 = __ldg(dsig[c][1] + kb);
-            accA[c][0] = fmaf(sa0 * i0, dA[c][0], accA[c][0]);
-            accA[c][1] = fmaf(sa0 * i1, dA[c][1], accA[c][1]);
-            accA[c][2] = fmaf(sa1 * i0, dA[c][2], accA[c][2]);
-            accA[c][3] = fmaf(sa1 * i1, dA[c][3], accA[c][3]);
-            if (GATEUP) {
-                accB[c][0] = fmaf(sb0 * i0, dB[c][0], accB[c][0]);
-                accB[c][1] = fmaf(sb0 * i1, dB[c][1], accB[c][1]);
-                accB[c][2] = fmaf(sb1 * i0, dB[c][2], accB[c][2]);
-                accB[c][3] = fmaf(sb1 * i1, dB[c][3], accB[c][3]);
+            for (int c = 0; c < NT; ++c)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    bf[c][j] = bvalid[c] ? *reinterpret_cast<const uint2*>(bsrc[c] + (int64_t)kb * 128 + 16 * j)
+                                         : make_uint2(0u, 0u);
+            float dA[NT][4], dB[NT][4];
+#pragma unroll
+            for (int c = 0; c < NT; ++c)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) { dA[c][q] = 0.0f; dB[c][q] = 0.0f; }
+            const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
+            const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t r0, r1, r2, r3;
+                decode_frag_word(wa[j], r0, r1, r2, r3);
+                // A fragment: a0 = row g (k 2t,2t+1) <- r0, a1 = row g+8 <- r2,
+                // a2 = row g (k 2t+8, 2t+9) <- r1, a3 = row g+8 <- r3; the column
+                // permutation is matched by the B layout (4 consecutive columns)
+#pragma unroll
+                for (int c = 0; c < NT; ++c) mma_f16_16816(dA[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
+                if (GATEUP) {
+                    decode_frag_word(wb[j], r0, r1, r2, r3);
+#pragma unroll
+                    for (int c = 0; c < NT; ++c) mma_f16_16816(dB[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
+                }
+            }
+            // group epilogue: weight scale of rows g, g+8 times the activation
+            // group's inverse scale of columns 2t, 2t+1
+            if (a.group) {
+                sa0 = __ldg(rowsA0 + (int64_t)kb * kTileRows);
+                sa1 = __ldg(rowsA0 + (int64_t)kb * kTileRows + 8);
+                if (GATEUP) {
+                    sb0 = __ldg(rowsB0 + (int64_t)kb * kTileRows);
+                    sb1 = __ldg(rowsB0 + (int64_t)kb * kTileRows + 8);
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < NT; ++c) {
+                const float i0 = __ldg(dsig[c][0] + kb), i1 = __ldg(dsig[c][1] + kb);
+                accA[c][0] = fmaf(sa0 * i0, dA[c][0], accA[c][0]);
+                accA[c][1] = fmaf(sa0 * i1, dA[c][1], accA[c][1]);
+                accA[c][2] = fmaf(sa1 * i0, dA[c][2], accA[c][2]);
+                accA[c][3] = fmaf(sa1 * i1, dA[c][3], accA[c][3]);
+                if (GATEUP) {
+                    accB[c][0] = fmaf(sb0 * i0, dB[c][0], accB[c][0]);
+                    accB[c][1] = fmaf(sb0 * i1, dB[c][1], accB[c][1]);
+                    accB[c][2] = fmaf(sb1 * i0, dB[c][2], accB[c][2]);
+                    accB[c][3] = fmaf(sb1 * i1, dB[c][3], accB[c][3]);
+                }
             }
         }
     }
