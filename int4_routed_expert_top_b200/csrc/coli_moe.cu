@@ -117,10 +117,9 @@ int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, f
     if (T <= 32)
         for (int c : {8, 4, 2, 1})
             if (d.H % (c * 128) == 0 && d.H / c <= kRouterMaxSlice) { KS = c; break; }
-    const int qwarps = T * (d.H / 64);
     if (KS > 0) {
         const int rblocks = (d.E * KS + 7) / 8;
-        const int qblocks = xq ? (qwarps + 7) / 8 : 0;
+        const int qblocks = xq ? T : 0;
         const dim3 grid(rblocks + qblocks);
         if (xt == COLI_F32)
             router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, xq, xinv);
@@ -140,9 +139,9 @@ int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, f
             int rc = check_launch("router");
             if (rc) return rc;
             if (xt == COLI_F32)
-                act_quant_kernel<float><<<(qwarps + 7) / 8, 256, 0, st>>>((const float*)x, T, d.H, xq, xinv);
+                act_quant_kernel<float><<<T, 256, 0, st>>>((const float*)x, T, d.H, xq, xinv);
             else
-                act_quant_kernel<__nv_bfloat16><<<(qwarps + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, xq, xinv);
+                act_quant_kernel<__nv_bfloat16><<<T, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, xq, xinv);
         }
     }
     *ks_out = KS;
@@ -187,13 +186,10 @@ int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int
     return launch_union(idx, T, d.k, d.E, o, st);
 }
 
-template <bool GATEUP>
+template <bool GATEUP, bool CHAIN>
 int launch_gemv_nt(int nt, int grid, const GemvArgs& a, cudaStream_t st) {
-    switch (nt) {
-        case 1: expert_gemv_kernel<GATEUP, 1><<<grid, kGemvWarps * 32, 0, st>>>(a); break;
-        case 2: expert_gemv_kernel<GATEUP, 2><<<grid, kGemvWarps * 32, 0, st>>>(a); break;
-        default: expert_gemv_kernel<GATEUP, 4><<<grid, kGemvWarps * 32, 0, st>>>(a); break;
-    }
+    if (nt == 1) expert_gemv_kernel<GATEUP, 1, CHAIN><<<grid, kGemvWarps * 32, 0, st>>>(a);
+    else         expert_gemv_kernel<GATEUP, 2, CHAIN><<<grid, kGemvWarps * 32, 0, st>>>(a);
     return check_launch(GATEUP ? "gate/up gemv" : "down gemv");
 }
 
@@ -223,11 +219,14 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
     a.T = T; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;
-    const int nt = T <= 4 ? 1 : T <= 8 ? 2 : 4;
-    int rc = launch_gemv_nt<true>(nt, units_max * (d.I / 64), a, st);
+    const int nt = T <= 4 ? 1 : 2;
+    // gate/up: per-row weight scales with one activation scale per token let the
+    // MMAs run through K without a per-step epilogue
+    int rc = d.group == 0 ? launch_gemv_nt<true, true>(nt, units_max * (d.I / 64), a, st)
+                          : launch_gemv_nt<true, false>(nt, units_max * (d.I / 64), a, st);
     if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;
-    return launch_gemv_nt<false>(nt, units_max * (d.H / 64), a, st);
+    return launch_gemv_nt<false, false>(nt, units_max * (d.H / 64), a, st);
 }
 
 }  // namespace

@@ -124,23 +124,35 @@ __device__ __forceinline__ uint32_t h2fma_16th_m72(uint32_t v) {
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(0x2C002C00u), "r"(0xD480D480u));
     return r;
 }
-__device__ __forceinline__ void decode_frag_word(uint32_t w, uint32_t& r0, uint32_t& r1,
-                                                 uint32_t& r2, uint32_t& r3) {
+// decode one fragment-tile word straight into an mma.sync A fragment:
+// a[0] = row g (c0, c0+1), a[1] = row g+8 (c0, c0+1), a[2] = row g (c0+2, c0+3),
+// a[3] = row g+8 (c0+2, c0+3).  With logical columns 2t,2t+1 <- c0,c0+1 and
+// 2t+8,2t+9 <- c0+2,c0+3 this is the m16n8k16 row-major A fragment of lane 4g+t.
+__device__ __forceinline__ void decode_frag_word(uint32_t w, uint32_t a[4]) {
     const uint32_t w8 = w >> 8;
-    r0 = h2sub_1032((w & 0x000F000Fu) ^ 0x64086408u);
-    r1 = h2fma_16th_m72((w & 0x00F000F0u) ^ 0x64806480u);
-    r2 = h2sub_1032((w8 & 0x000F000Fu) ^ 0x64086408u);
-    r3 = h2fma_16th_m72((w8 & 0x00F000F0u) ^ 0x64806480u);
+    a[0] = h2sub_1032((w & 0x000F000Fu) ^ 0x64086408u);
+    a[1] = h2sub_1032((w8 & 0x000F000Fu) ^ 0x64086408u);
+    a[2] = h2fma_16th_m72((w & 0x00F000F0u) ^ 0x64806480u);
+    a[3] = h2fma_16th_m72((w8 & 0x00F000F0u) ^ 0x64806480u);
 }
 
-// D[16x8] (f32) += A[16x16] (f16) * B[16x8] (f16), warp-wide
-__device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+// D[16x8] (f32) (+)= A[16x16] (f16) * B[16x8] (f16), warp-wide
+__device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], uint32_t b0,
+                                              uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16_16816_zc(float d[4], const uint32_t a[4], uint32_t b0,
+                                                 uint32_t b1) {
+    const float z = 0.0f;  // C = 0: starts a fresh partial product
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(z));
 }
 
 // Activation operand: power-of-two scale 2^(14 - e) for a group whose largest

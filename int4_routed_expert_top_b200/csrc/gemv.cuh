@@ -25,7 +25,7 @@
 namespace coli {
 
 constexpr int kGemvWarps = 8;
-constexpr int kGemvMaxNT = 4;     // up to 4 column groups of 8: 16 tokens per pass
+constexpr int kGemvMaxNT = 2;     // up to 2 column groups of 8: 8 tokens per pass
 
 struct GemvArgs {
     const uint8_t* experts;
@@ -51,10 +51,16 @@ struct GemvArgs {
     int H, I, group;
 };
 
-// One warp: 16 rows (block b16 of this CTA's 64), reduction groups
-// [kb0, kb1), NT column groups of 8.  Column n of group c carries token
+// One warp: 16 rows (block b16 of this CTA's 64), reduction steps [kb0, kb1)
+// of 64 columns, NT column groups of 8.  Column n of group c carries token
 // 4c + (n & 3), hi part for n < 4 and lo part for n >= 4.
-template <bool GATEUP, int NT>
+//
+// CHAIN (per-row weight scales and one activation scale per token): the MMAs
+// accumulate straight through K and the caller applies both scales at the end.
+// Otherwise every 64-column step ends with acc += (s_row * inv_act) * D_step.
+// A register ring keeps the loads of the next D steps in flight: weight units,
+// activation fragments and (per-step mode) the scales they need.
+template <bool GATEUP, int NT, bool CHAIN>
 __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __restrict__ codesA,
                                           const uint8_t* __restrict__ codesB,
                                           const float* __restrict__ sA,
@@ -66,119 +72,153 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
     const int KB = K / 64;
     const int rt = row0 / kTileRows, b8 = (row0 % kTileRows) / 16;
     const int ng = a.group ? KB : 1;
-    // this lane's B column: token pc + 4c + (g & 3), part g >> 2
-    const __half* bsrc[NT];
-    const float* bsig[NT];
-    bool bvalid[NT];
-    // this lane's D columns 2t, 2t+1: tokens pc + 4c + (2t & 3) + {0, 1}
-    const float* dsig[NT][2];
+    const int n = kb1 - kb0;
+    constexpr int UNIT_STEP = 8 * 32;  // uint4 units between consecutive 64-column steps
+    const uint4* pA = reinterpret_cast<const uint4*>(codesA + frag_unit_offset(rt, kb0, b8, lane, K));
+    const uint4* pB = reinterpret_cast<const uint4*>(codesB + frag_unit_offset(rt, kb0, b8, lane, K));
+    // activation fragments of this lane's B column: 4 fp16 per 16-column sub-block
+    const uint2* pX[NT];
+    bool bval[NT];
+    // inverse activation scales of this lane's D columns 2t, 2t+1
+    const float* pI[NT][2];
 #pragma unroll
     for (int c = 0; c < NT; ++c) {
         const int pb = pc + 4 * c + (g & 3);
-        bvalid[c] = pb < p1;
-        const int sb = bvalid[c] ? (GATEUP ? a.pair_tok[pb] : pb) : 0;
-        bsrc[c] = (GATEUP ? a.xq : a.hq) + (int64_t)sb * KB * 128 + (g >> 2) * 64 + 4 * t;
-        bsig[c] = (GATEUP ? a.xinv : a.hinv) + (int64_t)sb * KB;
+        bval[c] = pb < p1;
+        const int sb = bval[c] ? (GATEUP ? a.pair_tok[pb] : pb) : 0;
+        const __half* base = (GATEUP ? a.xq : a.hq) + ((int64_t)sb * KB + kb0) * 128 + (g >> 2) * 64;
+        pX[c] = reinterpret_cast<const uint2*>(base) + t;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int pd = pc + 4 * c + ((2 * t) & 3) + i;
             const int sd = pd < p1 ? (GATEUP ? a.pair_tok[pd] : pd) : 0;
-            dsig[c][i] = (GATEUP ? a.xinv : a.hinv) + (int64_t)sd * KB;
+            pI[c][i] = (GATEUP ? a.xinv : a.hinv) + (int64_t)sd * KB + kb0;
         }
     }
-    const float* rowsA0 = sA + scale_offset(row0 + g, 0, ng);
-    const float* rowsB0 = sB + scale_offset(row0 + g, 0, ng);
+    const float* pS[2] = {sA + scale_offset(row0 + g, 0, ng), sB + scale_offset(row0 + g, 0, ng)};
 #pragma unroll
     for (int c = 0; c < NT; ++c)
 #pragma unroll
         for (int i = 0; i < 4; ++i) { accA[c][i] = 0.0f; accB[c][i] = 0.0f; }
-
-    // weight-scale rows (hoisted for per-row scales)
-    float sa0 = __ldg(rowsA0), sa1 = __ldg(rowsA0 + 8), sb0 = 0.f, sb1 = 0.f;
-    if (GATEUP) { sb0 = __ldg(rowsB0); sb1 = __ldg(rowsB0 + 8); }
-
-    // register ring: the unit loads of the next D steps are always in flight
-    constexpr int D = NT == 1 ? 8 : NT == 2 ? 4 : 2;
-    uint4 ringA[D], ringB[D];
-#pragma unroll
-    for (int i = 0; i < D; ++i) {
-        if (kb0 + i < kb1) {
-            const int64_t uoff = frag_unit_offset(rt, kb0 + i, b8, lane, K);
-            ringA[i] = ldg_stream(codesA + uoff);
-            if (GATEUP) ringB[i] = ldg_stream(codesB + uoff);
-        }
+    float rowA0 = 0.f, rowA1 = 0.f, rowB0 = 0.f, rowB1 = 0.f;  // per-row scales
+    if (!CHAIN && !a.group) {
+        rowA0 = __ldg(pS[0]); rowA1 = __ldg(pS[0] + 8);
+        if (GATEUP) { rowB0 = __ldg(pS[1]); rowB1 = __ldg(pS[1] + 8); }
     }
-    for (int kb_base = kb0; kb_base < kb1; kb_base += D) {
+
+    constexpr int D = NT == 1 ? 4 : 2;
+    uint4 rA[D], rB[D];
+    uint2 rX[D][NT][4];
+    float rI[D][NT][2], rS[D][4];
+    auto fetch = [&](int slot, int rel) {
+        rA[slot] = ldg_stream(pA + rel * UNIT_STEP);
+        if (GATEUP) rB[slot] = ldg_stream(pB + rel * UNIT_STEP);
 #pragma unroll
-        for (int i = 0; i < D; ++i) {
-            const int kb = kb_base + i;
-            if (kb >= kb1) break;
-            const uint4 ua = ringA[i];
-            const uint4 ub = GATEUP ? ringB[i] : make_uint4(0, 0, 0, 0);
-            if (kb + D < kb1) {
-                const int64_t uoff = frag_unit_offset(rt, kb + D, b8, lane, K);
-                ringA[i] = ldg_stream(codesA + uoff);
-                if (GATEUP) ringB[i] = ldg_stream(codesB + uoff);
-            }
-            // B fragments: 4 fp16 of this lane's column for each 16-column sub-block
-            uint2 bf[NT][4];
+        for (int c = 0; c < NT; ++c)
 #pragma unroll
-            for (int c = 0; c < NT; ++c)
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    bf[c][j] = bvalid[c] ? *reinterpret_cast<const uint2*>(bsrc[c] + (int64_t)kb * 128 + 16 * j)
-                                         : make_uint2(0u, 0u);
-            float dA[NT][4], dB[NT][4];
-#pragma unroll
-            for (int c = 0; c < NT; ++c)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) { dA[c][q] = 0.0f; dB[c][q] = 0.0f; }
-            const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
-            const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t r0, r1, r2, r3;
-                decode_frag_word(wa[j], r0, r1, r2, r3);
-                // A fragment: a0 = row g (k 2t,2t+1) <- r0, a1 = row g+8 <- r2,
-                // a2 = row g (k 2t+8, 2t+9) <- r1, a3 = row g+8 <- r3; the column
-                // permutation is matched by the B layout (4 consecutive columns)
-#pragma unroll
-                for (int c = 0; c < NT; ++c) mma_f16_16816(dA[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
-                if (GATEUP) {
-                    decode_frag_word(wb[j], r0, r1, r2, r3);
-#pragma unroll
-                    for (int c = 0; c < NT; ++c) mma_f16_16816(dB[c], r0, r2, r1, r3, bf[c][j].x, bf[c][j].y);
-                }
-            }
-            // group epilogue: weight scale of rows g, g+8 times the activation
-            // group's inverse scale of columns 2t, 2t+1
-            if (a.group) {
-                sa0 = __ldg(rowsA0 + (int64_t)kb * kTileRows);
-                sa1 = __ldg(rowsA0 + (int64_t)kb * kTileRows + 8);
-                if (GATEUP) {
-                    sb0 = __ldg(rowsB0 + (int64_t)kb * kTileRows);
-                    sb1 = __ldg(rowsB0 + (int64_t)kb * kTileRows + 8);
-                }
-            }
+            for (int j = 0; j < 4; ++j)
+                rX[slot][c][j] = bval[c] ? __ldg(pX[c] + rel * 32 + 4 * j) : make_uint2(0u, 0u);
+        if (!CHAIN) {
 #pragma unroll
             for (int c = 0; c < NT; ++c) {
-                const float i0 = __ldg(dsig[c][0] + kb), i1 = __ldg(dsig[c][1] + kb);
-                accA[c][0] = fmaf(sa0 * i0, dA[c][0], accA[c][0]);
-                accA[c][1] = fmaf(sa0 * i1, dA[c][1], accA[c][1]);
-                accA[c][2] = fmaf(sa1 * i0, dA[c][2], accA[c][2]);
-                accA[c][3] = fmaf(sa1 * i1, dA[c][3], accA[c][3]);
+                rI[slot][c][0] = __ldg(pI[c][0] + rel);
+                rI[slot][c][1] = __ldg(pI[c][1] + rel);
+            }
+            if (a.group) {
+                rS[slot][0] = __ldg(pS[0] + (int64_t)(kb0 + rel) * kTileRows);
+                rS[slot][1] = __ldg(pS[0] + (int64_t)(kb0 + rel) * kTileRows + 8);
                 if (GATEUP) {
-                    accB[c][0] = fmaf(sb0 * i0, dB[c][0], accB[c][0]);
-                    accB[c][1] = fmaf(sb0 * i1, dB[c][1], accB[c][1]);
-                    accB[c][2] = fmaf(sb1 * i0, dB[c][2], accB[c][2]);
-                    accB[c][3] = fmaf(sb1 * i1, dB[c][3], accB[c][3]);
+                    rS[slot][2] = __ldg(pS[1] + (int64_t)(kb0 + rel) * kTileRows);
+                    rS[slot][3] = __ldg(pS[1] + (int64_t)(kb0 + rel) * kTileRows + 8);
+                }
+            }
+        }
+    };
+#pragma unroll
+    for (int sl = 0; sl < D; ++sl)
+        if (sl < n) fetch(sl, sl);
+
+    for (int base = 0; base < n; base += D) {
+#pragma unroll
+        for (int sl = 0; sl < D; ++sl) {
+            const int rel = base + sl;
+            if (rel < n) {
+                const uint4 ua = rA[sl];
+                const uint4 ub = GATEUP ? rB[sl] : ua;
+                uint2 bx[NT][4];
+                float iv[NT][2], sc[4];
+#pragma unroll
+                for (int c = 0; c < NT; ++c) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) bx[c][j] = rX[sl][c][j];
+                    if (!CHAIN) { iv[c][0] = rI[sl][c][0]; iv[c][1] = rI[sl][c][1]; }
+                }
+                if (!CHAIN) {
+                    if (a.group) {
+                        sc[0] = rS[sl][0]; sc[1] = rS[sl][1];
+                        sc[2] = GATEUP ? rS[sl][2] : 0.f; sc[3] = GATEUP ? rS[sl][3] : 0.f;
+                    } else {
+                        sc[0] = rowA0; sc[1] = rowA1; sc[2] = rowB0; sc[3] = rowB1;
+                    }
+                }
+                if (rel + D < n) fetch(sl, rel + D);
+                const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
+                const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
+                if (CHAIN) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t fa[4];
+                        decode_frag_word(wa[j], fa);
+#pragma unroll
+                        for (int c = 0; c < NT; ++c) mma_f16_16816(accA[c], fa, bx[c][j].x, bx[c][j].y);
+                        if (GATEUP) {
+                            uint32_t fb[4];
+                            decode_frag_word(wb[j], fb);
+#pragma unroll
+                            for (int c = 0; c < NT; ++c) mma_f16_16816(accB[c], fb, bx[c][j].x, bx[c][j].y);
+                        }
+                    }
+                } else {
+                    float dA[NT][4], dB[NT][4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t fa[4];
+                        decode_frag_word(wa[j], fa);
+#pragma unroll
+                        for (int c = 0; c < NT; ++c) {
+                            if (j == 0) mma_f16_16816_zc(dA[c], fa, bx[c][j].x, bx[c][j].y);
+                            else        mma_f16_16816(dA[c], fa, bx[c][j].x, bx[c][j].y);
+                        }
+                        if (GATEUP) {
+                            uint32_t fb[4];
+                            decode_frag_word(wb[j], fb);
+#pragma unroll
+                            for (int c = 0; c < NT; ++c) {
+                                if (j == 0) mma_f16_16816_zc(dB[c], fb, bx[c][j].x, bx[c][j].y);
+                                else        mma_f16_16816(dB[c], fb, bx[c][j].x, bx[c][j].y);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < NT; ++c) {
+                        accA[c][0] = fmaf(sc[0] * iv[c][0], dA[c][0], accA[c][0]);
+                        accA[c][1] = fmaf(sc[0] * iv[c][1], dA[c][1], accA[c][1]);
+                        accA[c][2] = fmaf(sc[1] * iv[c][0], dA[c][2], accA[c][2]);
+                        accA[c][3] = fmaf(sc[1] * iv[c][1], dA[c][3], accA[c][3]);
+                        if (GATEUP) {
+                            accB[c][0] = fmaf(sc[2] * iv[c][0], dB[c][0], accB[c][0]);
+                            accB[c][1] = fmaf(sc[2] * iv[c][1], dB[c][1], accB[c][1]);
+                            accB[c][2] = fmaf(sc[3] * iv[c][0], dB[c][2], accB[c][2]);
+                            accB[c][3] = fmaf(sc[3] * iv[c][1], dB[c][3], accB[c][3]);
+                        }
+                    }
                 }
             }
         }
     }
 }
 
-template <bool GATEUP, int NT>
+template <bool GATEUP, int NT, bool CHAIN>
 __device__ __forceinline__ void gemv_pass(const GemvArgs& a, float* red, const uint8_t* codesA,
                                           const uint8_t* codesB, const float* sA,
                                           const float* sB, int K, int rb64, int pc, int p1) {
@@ -188,26 +228,26 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& a, float* red, const u
     const int KB = K / 64;
     const int row0 = rb64 * 64 + b16 * 16;
     float accA[NT][4], accB[NT][4];
-    gemv_warp<GATEUP, NT>(a, codesA, codesB, sA, sB, K, row0, half * (KB / 2),
-                          (half + 1) * (KB / 2), pc, p1, accA, accB);
+    gemv_warp<GATEUP, NT, CHAIN>(a, codesA, codesB, sA, sB, K, row0, half * (KB / 2),
+                                 (half + 1) * (KB / 2), pc, p1, accA, accB);
     // red layout: [mat 2][half 2][64 rows][8*NT cols]
     const int C = 8 * NT;
 #pragma unroll
     for (int c = 0; c < NT; ++c)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int r = b16 * 16 + g + (i >> 1) * 8, n = 8 * c + 2 * t + (i & 1);
-            red[((0 * 2 + half) * 64 + r) * C + n] = accA[c][i];
-            if (GATEUP) red[((1 * 2 + half) * 64 + r) * C + n] = accB[c][i];
+            const int r = b16 * 16 + g + (i >> 1) * 8, nn = 8 * c + 2 * t + (i & 1);
+            red[((0 * 2 + half) * 64 + r) * C + nn] = accA[c][i];
+            if (GATEUP) red[((1 * 2 + half) * 64 + r) * C + nn] = accB[c][i];
         }
     __syncthreads();
 }
 
-template <bool GATEUP, int NT>
+template <bool GATEUP, int NT, bool CHAIN>
 __global__ void __launch_bounds__(kGemvWarps * 32)
 expert_gemv_kernel(GemvArgs a) {
     __shared__ float red[2 * 2 * 64 * 8 * kGemvMaxNT];
-    __shared__ float gmax[16][2];
+    __shared__ float gmax[8 * kGemvMaxNT][2];
     __shared__ int last_flag;
     const int K = GATEUP ? a.H : a.I;
     const int R = GATEUP ? a.I : a.H;
@@ -223,23 +263,30 @@ expert_gemv_kernel(GemvArgs a) {
     const float* sB = reinterpret_cast<const float*>(blob + a.L.scales[1]);
     const int C = 8 * NT;
     const int tid = threadIdx.x;
+    const int KB = K / 64;
 
     for (int pc = p0; pc < p1; pc += 4 * NT) {
         const int tc = min(4 * NT, p1 - pc);
         __syncthreads();  // previous pass finished with red
-        gemv_pass<GATEUP, NT>(a, red, codesA, codesB, sA, sB, K, rb64, pc, p1);
+        gemv_pass<GATEUP, NT, CHAIN>(a, red, codesA, codesB, sA, sB, K, rb64, pc, p1);
         // combine halves and hi/lo: thread -> (token tt, row r)
         if (GATEUP) {
             // h for 64 rows x tc tokens, then one power-of-two scale per token
             for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
                 const int tt = q / 64, r = q % 64;
-                const int c = tt / 4, n = 8 * c + (tt & 3);
-                const float ga = red[((0 * 2 + 0) * 64 + r) * C + n] + red[((0 * 2 + 1) * 64 + r) * C + n] +
-                                 red[((0 * 2 + 0) * 64 + r) * C + n + 4] + red[((0 * 2 + 1) * 64 + r) * C + n + 4];
-                const float ua = red[((1 * 2 + 0) * 64 + r) * C + n] + red[((1 * 2 + 1) * 64 + r) * C + n] +
-                                 red[((1 * 2 + 0) * 64 + r) * C + n + 4] + red[((1 * 2 + 1) * 64 + r) * C + n + 4];
+                const int c = tt / 4, nn = 8 * c + (tt & 3);
+                float ga = red[((0 * 2 + 0) * 64 + r) * C + nn] + red[((0 * 2 + 1) * 64 + r) * C + nn] +
+                           red[((0 * 2 + 0) * 64 + r) * C + nn + 4] + red[((0 * 2 + 1) * 64 + r) * C + nn + 4];
+                float ua = red[((1 * 2 + 0) * 64 + r) * C + nn] + red[((1 * 2 + 1) * 64 + r) * C + nn] +
+                           red[((1 * 2 + 0) * 64 + r) * C + nn + 4] + red[((1 * 2 + 1) * 64 + r) * C + nn + 4];
+                if (CHAIN) {  // per-row weight scale and the token's activation scale
+                    const float inv = __ldg(a.xinv + (int64_t)a.pair_tok[pc + tt] * KB);
+                    const int row = rb64 * 64 + r;
+                    ga *= __ldg(sA + scale_offset(row, 0, 1)) * inv;
+                    ua *= __ldg(sB + scale_offset(row, 0, 1)) * inv;
+                }
                 const float hv = silu_f(ga) * ua;
-                red[((0 * 2 + 0) * 64 + r) * C + n] = hv;  // reuse: h in slot (0, 0, r, n)
+                red[((0 * 2 + 0) * 64 + r) * C + nn] = hv;  // reuse: h in slot (0, 0, r, nn)
                 float m = fabsf(hv);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -248,8 +295,8 @@ expert_gemv_kernel(GemvArgs a) {
             __syncthreads();
             for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
                 const int tt = q / 64, r = q % 64;
-                const int c = tt / 4, n = 8 * c + (tt & 3);
-                const float hv = red[((0 * 2 + 0) * 64 + r) * C + n];
+                const int c = tt / 4, nn = 8 * c + (tt & 3);
+                const float hv = red[((0 * 2 + 0) * 64 + r) * C + nn];
                 float inv;
                 const float sc = act_group_scale(fmaxf(gmax[tt][0], gmax[tt][1]), &inv);
                 __half hi, lo;
@@ -263,9 +310,9 @@ expert_gemv_kernel(GemvArgs a) {
         } else {
             for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
                 const int tt = q / 64, r = q % 64;
-                const int c = tt / 4, n = 8 * c + (tt & 3);
-                const float v = red[((0 * 2 + 0) * 64 + r) * C + n] + red[((0 * 2 + 1) * 64 + r) * C + n] +
-                                red[((0 * 2 + 0) * 64 + r) * C + n + 4] + red[((0 * 2 + 1) * 64 + r) * C + n + 4];
+                const int c = tt / 4, nn = 8 * c + (tt & 3);
+                float v = red[((0 * 2 + 0) * 64 + r) * C + nn] + red[((0 * 2 + 1) * 64 + r) * C + nn] +
+                          red[((0 * 2 + 0) * 64 + r) * C + nn + 4] + red[((0 * 2 + 1) * 64 + r) * C + nn + 4];
                 a.o[(int64_t)(pc + tt) * a.H + rb64 * 64 + r] = v;
             }
         }

@@ -16,37 +16,43 @@ namespace coli {
 constexpr int kMaxKS = 8;
 
 // ---------------------------------------------------------------------------
-// fp16 hi/lo activation operand: one warp per (token, 64-column group).
-// xq[t][g][0..64) = hi, [64..128) = lo of x * 2^sh, xinv[t][g] = 2^-sh.
+// fp16 hi/lo activation operand, one CTA (256 threads) per token: one power of
+// two per token from the row's largest magnitude, xq[t][g][0..64) = hi and
+// [64..128) = lo of x * 2^sh for 64-column group g, xinv[t][g] = 2^-sh.
 // ---------------------------------------------------------------------------
 template <typename XT>
-__device__ __forceinline__ void act_quant_group(const XT* __restrict__ x, int H, int t, int kb,
+__device__ __forceinline__ void act_quant_token(const XT* __restrict__ x, int H, int t,
                                                 __half* __restrict__ xq, float* __restrict__ xinv) {
-    const int lane = threadIdx.x & 31;
-    const XT* src = x + (int64_t)t * H + kb * 64 + 2 * lane;
-    const float v0 = to_f32(src[0]), v1 = to_f32(src[1]);
-    float m = fmaxf(fabsf(v0), fabsf(v1));
+    __shared__ float part[8];
+    const XT* row = x + (int64_t)t * H;
+    float m = 0.0f;
+    for (int c = threadIdx.x; c < H; c += 256) m = fmaxf(m, fabsf(to_f32(row[c])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = part[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) m = fmaxf(m, part[i]);
     float inv;
     const float sc = act_group_scale(m, &inv);
-    __half h0, l0, h1, l1;
-    split_f16(v0 * sc, h0, l0);
-    split_f16(v1 * sc, h1, l1);
-    __half* dst = xq + ((int64_t)t * (H / 64) + kb) * 128;
-    *reinterpret_cast<__half2*>(dst + 2 * lane) = __halves2half2(h0, h1);
-    *reinterpret_cast<__half2*>(dst + 64 + 2 * lane) = __halves2half2(l0, l1);
-    if (lane == 0) xinv[(int64_t)t * (H / 64) + kb] = inv;
+    const int KB = H / 64;
+    for (int c = 2 * threadIdx.x; c < H; c += 512) {
+        __half h0, l0, h1, l1;
+        split_f16(to_f32(row[c]) * sc, h0, l0);
+        split_f16(to_f32(row[c + 1]) * sc, h1, l1);
+        __half* dst = xq + ((int64_t)t * KB + c / 64) * 128 + (c % 64);
+        *reinterpret_cast<__half2*>(dst) = __halves2half2(h0, h1);
+        *reinterpret_cast<__half2*>(dst + 64) = __halves2half2(l0, l1);
+    }
+    for (int kb = threadIdx.x; kb < KB; kb += 256) xinv[(int64_t)t * KB + kb] = inv;
 }
 
 template <typename XT>
 __global__ void __launch_bounds__(256)
 act_quant_kernel(const XT* __restrict__ x, int T, int H, __half* __restrict__ xq,
                  float* __restrict__ xinv) {
-    const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int KB = H / 64;
-    if (gw >= T * KB) return;
-    act_quant_group(x, H, gw / KB, gw % KB, xq, xinv);
+    act_quant_token(x, H, blockIdx.x, xq, xinv);
 }
 
 // ---------------------------------------------------------------------------
@@ -63,10 +69,8 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
                    int E, int KS, float* __restrict__ zpart, int router_blocks,
                    __half* __restrict__ xq, float* __restrict__ xinv) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if ((int)blockIdx.x >= router_blocks) {
-        const int gw = (blockIdx.x - router_blocks) * 8 + warp;
-        const int KB = H / 64;
-        if (xq && gw < T * KB) act_quant_group(x, H, gw / KB, gw % KB, xq, xinv);
+    if ((int)blockIdx.x >= router_blocks) {  // one CTA per token: activation operand
+        if (xq) act_quant_token(x, H, blockIdx.x - router_blocks, xq, xinv);
         return;
     }
     const int gw = blockIdx.x * 8 + warp;
