@@ -222,6 +222,31 @@ int coli_moe_stack_forward(const coli_moe_layer* const* layers, int32_t L,
 int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert,
                            int32_t which, float* out, coli_stream_t stream);
 
+/* coli_moe_forward for callers that cannot allocate device memory.  (The
+ * method on the source pages has no counterpart to this call; it exists for
+ * integration only.)  Some hosts cannot hand this library a workspace: a plugin
+ * running inside a framework that owns every device allocation and exposes no
+ * allocator, or a real-time serving loop that forbids allocator calls once it
+ * has started.  This call allocates nothing: instead of a caller workspace it
+ * uses a scratch array of COLI_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the
+ * library, which every GPU that loads the library keeps until the process
+ * exits.  x, y and the layer's buffers are still the caller's.
+ *  - T is limited to what fits: a call whose coli_moe_workspace_size(layer, T)
+ *    exceeds COLI_NOALLOC_SCRATCH_BYTES returns COLI_E_UNSUPPORTED (for the
+ *    GLM-5.2 shapes that is T <= 24 tokens).
+ *  - The first call on each device looks up that device's copy of the array
+ *    (cudaGetSymbolAddress with the device current); make that first call before
+ *    any stream capture.  Later calls only launch kernels.
+ *  - All calls share the one array, and it keeps whatever the previous call left
+ *    in it (every value a call needs cleared is cleared by its own kernels).
+ *    Calls whose kernels overlap on the GPU (different streams, or different
+ *    host threads on one device) race on the array: serialise them.
+ * Results equal coli_moe_forward with COLI_PATH_AUTO on the same inputs. */
+#define COLI_NOALLOC_SCRATCH_BYTES (8u << 20)
+int coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x,
+                             coli_dtype xt, int32_t T, float* y,
+                             coli_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,7 +21,7 @@ __all__ = [
     "coli_moe_layer_destroy", "coli_moe_workspace_size", "coli_moe_route",
     "coli_moe_union", "coli_moe_forward", "coli_moe_forward_ex", "coli_moe_rmsnorm",
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
-    "Desc",
+    "coli_moe_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "Desc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +37,7 @@ EXPORTS = (
     "coli_moe_layer_destroy", "coli_moe_workspace_size", "coli_moe_route",
     "coli_moe_union", "coli_moe_forward", "coli_moe_forward_ex", "coli_moe_rmsnorm",
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
+    "coli_moe_forward_noalloc",
 )
 
 
@@ -84,6 +85,7 @@ _SIGS = {
     "coli_moe_stack_forward": ([_P, _I32, _P, _I32, ctypes.c_float, ctypes.c_int, _P, _SZ,
                                 _P], ctypes.c_int),
     "coli_moe_dequant_debug": ([_P, _I32, _I32, _P, _P], ctypes.c_int),
+    "coli_moe_forward_noalloc": ([_P, _P, ctypes.c_int, _I32, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -234,3 +236,13 @@ def coli_moe_stack_forward(layers, x, T, eps, ws, path=COLI_PATH_AUTO, stream=No
 
 def coli_moe_dequant_debug(layer, expert: int, which: int, out, stream=None):
     _ok(lib.coli_moe_dequant_debug(layer, expert, which, _ptr(out), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # COLI_NOALLOC_SCRATCH_BYTES in include/coli_moe.h
+
+
+def coli_moe_forward_noalloc(layer, x, T, y, stream=None):
+    """Forward without a caller workspace, for hosts that cannot allocate device
+    memory: the library's built-in scratch array is used instead (see the header
+    for its limit and for the rule that overlapping calls must be serialised)."""
+    _ok(lib.coli_moe_forward_noalloc(layer, _ptr(x), _xtype(x), T, _ptr(y), _stream(stream)))

@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "coli_moe.h"
@@ -526,6 +527,53 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t 
         blob + L.codes[which], reinterpret_cast<const float*>(blob + L.scales[which]), R, K,
         d.group, out);
     return check_launch("dequant");
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward: the workspace is a scratch array compiled into the
+// library (one copy per device), not memory from the caller.
+// ---------------------------------------------------------------------------
+namespace {
+__device__ __align__(256) unsigned char g_noalloc_scratch[COLI_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of this device's copy of the scratch array.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, and cached.
+int noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return fail(COLI_E_CUDA, "forward_noalloc: no usable current device");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(COLI_E_CUDA, "forward_noalloc: scratch lookup failed: %s",
+                        cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return COLI_OK;
+}
+}  // namespace
+
+int coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x, coli_dtype xt,
+                             int32_t T, float* y, coli_stream_t stream) {
+    if (!layer || !x || !y) return fail(COLI_E_INVAL, "forward_noalloc: NULL pointer");
+    size_t need = 0;
+    int rc = coli_moe_workspace_size(layer, T, &need);
+    if (rc) return rc;
+    if (need > (size_t)COLI_NOALLOC_SCRATCH_BYTES)
+        return fail(COLI_E_UNSUPPORTED,
+                    "forward_noalloc: T=%d needs %zu bytes of scratch, the built-in array holds %u",
+                    T, need, (unsigned)COLI_NOALLOC_SCRATCH_BYTES);
+    void* ws = nullptr;
+    if ((rc = noalloc_scratch(&ws))) return rc;
+    return coli_moe_forward(layer, x, xt, T, y, ws, (size_t)COLI_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

@@ -1,0 +1,46 @@
+"""The allocation-free forward (coli_moe_forward_noalloc), for callers that
+cannot allocate device memory, against the ordinary forward with a caller
+workspace.  Kept in its own file, collected last, so that a run stopping at the
+first failure has already run every other test."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import int4_routed_expert_top_b200 as cm
+from tests.workloads import build_layer, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("group", [0, 64])
+def test_noalloc_forward_matches_workspace_forward(group):
+    import dataclasses
+    wl = dataclasses.replace(synth.TINY, group=group, T=5)
+    L = build_layer(wl)
+    y_ref = torch.empty((wl.T, wl.H), dtype=torch.float32, device="cuda")
+    y = torch.empty_like(y_ref)
+    for call in range(2):           # two calls in a row share the built-in scratch
+        x = synth.tokens(wl, wl.T, step=call).cuda()
+        cm.coli_moe_forward(L.handle, x, wl.T, y_ref, L.workspace(wl.T))
+        y.fill_(float("nan"))
+        cm.coli_moe_forward_noalloc(L.handle, x, wl.T, y)
+        torch.cuda.synchronize()
+        err = rel_err(y.cpu().numpy(), y_ref.cpu().numpy())
+        assert err <= 2e-3, (call, err)
+        assert np.isfinite(y.cpu().numpy()).all()
+    L.close()
+
+
+def test_noalloc_rejects_too_many_tokens():
+    wl = synth.TINY
+    L = build_layer(wl)
+    T = 1
+    while cm.coli_moe_workspace_size(L.handle, T) <= cm.NOALLOC_SCRATCH_BYTES:
+        T *= 2
+    x = torch.zeros((T, wl.H), dtype=torch.float32, device="cuda")
+    y = torch.empty_like(x)
+    with pytest.raises(cm.ColiError) as e:
+        cm.coli_moe_forward_noalloc(L.handle, x, T, y)
+    assert e.value.code == -4 and "scratch" in str(e.value)
+    L.close()
