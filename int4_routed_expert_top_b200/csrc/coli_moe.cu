@@ -172,14 +172,12 @@ int launch_union(const int32_t* idx, int T, int k, int E, const UnionOut& o, cud
 // top-k + union; one fused single-CTA launch for small batches
 int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int32_t* idx,
                   float* w, const UnionOut& o, cudaStream_t st) {
-    if (T <= 64) {
-        const int topk_warps = std::max(1, std::min(std::min(32, T), (160 * 1024) / (8 * d.E)));
-        const int smem = std::max(topk_warps * 2 * d.E * 4, union_smem_bytes(T, d.E));
+    if (T * d.E <= kSmallSelect && T <= kSmallSelect / 32) {
+        const int smem = std::max(2 * T * d.E * 4, union_smem_bytes(T, d.E));
         int rc = set_smem((const void*)topk_union_kernel, smem);
         if (rc) return rc;
         topk_union_kernel<<<1, kUnionThreads, smem, st>>>(zpart, KS, T, d.E, d.router_b, d.k,
-                                                          d.routed_scale, d.norm_topk, idx, w,
-                                                          topk_warps, o);
+                                                          d.routed_scale, d.norm_topk, idx, w, o);
         return check_launch("topk+union");
     }
     int rc = launch_topk(d, zpart, KS, T, idx, w, st);
@@ -187,11 +185,20 @@ int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int
     return launch_union(idx, T, d.k, d.E, o, st);
 }
 
-template <bool GATEUP, bool CHAIN>
-int launch_gemv_nt(int nt, int grid, const GemvArgs& a, cudaStream_t st) {
-    if (nt == 1) expert_gemv_kernel<GATEUP, 1, CHAIN><<<grid, kGemvWarps * 32, 0, st>>>(a);
-    else         expert_gemv_kernel<GATEUP, 2, CHAIN><<<grid, kGemvWarps * 32, 0, st>>>(a);
-    return check_launch(GATEUP ? "gate/up gemv" : "down gemv");
+template <int NT>
+int launch_gemv_nt(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st,
+                   int stage_mark_rc) {
+    (void)stage_mark_rc;
+    const int grid = units_max * (d.I / 64);
+    if (d.group == 0) gateup_gemv_kernel<NT, true><<<grid, kGemvWarps * 32, 0, st>>>(a);
+    else              gateup_gemv_kernel<NT, false><<<grid, kGemvWarps * 32, 0, st>>>(a);
+    return check_launch("gate/up gemv");
+}
+
+template <int NT>
+int launch_down_nt(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
+    down_gemv_kernel<NT><<<units_max * (d.H / 64) * kDownSplit, kGemvWarps * 32, 0, st>>>(a);
+    return check_launch("down gemv");
 }
 
 template <typename Mark>
@@ -220,14 +227,12 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
     a.T = T; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;
-    const int nt = T <= 4 ? 1 : 2;
-    // gate/up: per-row weight scales with one activation scale per token let the
-    // MMAs run through K without a per-step epilogue
-    int rc = d.group == 0 ? launch_gemv_nt<true, true>(nt, units_max * (d.I / 64), a, st)
-                          : launch_gemv_nt<true, false>(nt, units_max * (d.I / 64), a, st);
+    // per-row weight scales with one activation scale per token let the gate/up
+    // MMAs run through K without a per-step epilogue (CHAIN)
+    int rc = T <= 4 ? launch_gemv_nt<1>(d, units_max, a, st, 0) : launch_gemv_nt<2>(d, units_max, a, st, 0);
     if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;
-    return launch_gemv_nt<false, false>(nt, units_max * (d.H / 64), a, st);
+    return T <= 4 ? launch_down_nt<1>(d, units_max, a, st) : launch_down_nt<2>(d, units_max, a, st);
 }
 
 }  // namespace

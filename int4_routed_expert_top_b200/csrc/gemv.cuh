@@ -1,36 +1,62 @@
 // gemv.cuh - int4 expert kernels for small batches (decode, MTP verify).
 //
-// A CTA owns one unit (a routed expert picked by the batch, or a shared expert)
-// and 64 output rows, and every token routed to that unit, so each weight byte
-// is read from HBM once per launch however many of the unit's tokens use it
-// (batch union, "github一周涨11k⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.4).  Warp w
-// takes 16-row block w % 4 and half w / 4 of the reduction.  Every step a lane
-// loads one 16-byte unit of a fragment tile (a whole warp: one coalesced 512-byte
-// block), decodes its 32 nibbles to exact fp16 in registers and feeds them to
-// the tensor cores as mma.sync A fragments.  The activations are the B operand,
-// split into fp16 hi + lo parts scaled by a power of two per 64-column group,
-// so the products carry ~22 significant bits into the f32 accumulators.  After
-// each 64-column group the partial product is multiplied by the weight scale
-// (per row, or per group for gs64) and by the activation group's inverse power
-// of two, in f32.
+// A CTA of 4 warps owns one unit (a routed expert picked by the batch, or a
+// shared expert), 64 output rows, and every token routed to that unit, so each
+// weight byte is read from HBM once per launch however many of the unit's
+// tokens use it (batch union, "github一周涨11k⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.4).
+// Warp w streams 16 rows over the whole reduction (gate/up) or half of it (down).
+// Every step a lane loads one 16-byte unit of a fragment tile (a whole warp: one
+// coalesced 512-byte block), decodes its 32 nibbles to exact fp16 in registers
+// and feeds them to the tensor cores as mma.sync A fragments.  The activations
+// are the B operand, split into fp16 hi + lo parts under a power-of-two scale,
+// so the products carry ~22 significant bits into the f32 accumulators.  The
+// weight scale (per row, or per 64-column group for gs64) and the activation's
+// inverse scale are applied in f32: once at the end when both are constant along
+// the reduction (CHAIN), else after every 64-column step.
 //
-//   gate/up: h[p, i] = silu(sum_c Wg'[i, c] x[c]) * (sum_c Wu'[i, c] x[c])
-//            written as fp16 hi/lo per 64-row group with its power-of-two scale
-//   down:    o[p, r] = sum_i Wd'[r, i] h[p, i]  (f32), and the last CTA to finish
-//            a 64-row block forms y = residual + sum_j w_j o_j + sum_s o_shared
+//   gate/up: h[p, i] = silu(sum_c Wg'[i, c] x[c]) * (sum_c Wu'[i, c] x[c]),
+//            stored as fp16 hi/lo with one power of two per 64 rows
+//   down:    o[p, r] = sum_i Wd'[r, i] h[p, i] (f32; the two halves of the sum are
+//            added into o, which the gate/up pass zeroed), and the last CTA to
+//            finish a 64-row block forms y = residual + sum_j w_j o_j + sum_s o_s
 #pragma once
 
 #include "common.cuh"
 
 namespace coli {
 
-constexpr int kGemvWarps = 8;
-constexpr int kGemvMaxNT = 2;     // up to 2 column groups of 8: 8 tokens per pass
+constexpr int kGemvWarps = 4;      // 64 rows per CTA
+constexpr int kGemvMaxNT = 2;      // up to 2 column groups of 8: 8 tokens per pass
+constexpr int kDownSplit = 2;      // the down reduction is split in halves
+
+// fp16 magic constants of the nibble decode, passed as kernel parameters so
+// they are read from the parameter bank instead of being rebuilt per use
+struct DecodeK {
+    uint32_t xlo = 0x64086408u;   // sign flip of a nibble at bits 0-3 + fp16 exponent of 1024
+    uint32_t xhi = 0x64806480u;   // same for a nibble at bits 4-7
+    uint32_t sub = 0x64086408u;   // 1032 = 1024 + 8
+    uint32_t mul = 0x2C002C00u;   // 1/16
+    uint32_t add = 0xD480D480u;   // -72 = -(1024 + 8*16)/16
+};
+
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t a[4], const DecodeK& k) {
+    const uint32_t w8 = w >> 8;
+    uint32_t t0, t1, t2, t3;
+    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t0) : "r"(w), "r"(k.xlo));
+    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t1) : "r"(w8), "r"(k.xlo));
+    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t2) : "r"(w), "r"(k.xhi));
+    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t3) : "r"(w8), "r"(k.xhi));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(a[0]) : "r"(t0), "r"(k.sub));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(a[1]) : "r"(t1), "r"(k.sub));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(a[2]) : "r"(t2), "r"(k.mul), "r"(k.add));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(a[3]) : "r"(t3), "r"(k.mul), "r"(k.add));
+}
 
 struct GemvArgs {
     const uint8_t* experts;
     int64_t blob_bytes;
     BlobLayout L;
+    DecodeK dk;
     const int32_t* n_units;
     const int32_t* unit_expert;
     const int32_t* unit_begin;
@@ -51,15 +77,11 @@ struct GemvArgs {
     int H, I, group;
 };
 
-// One warp: 16 rows (block b16 of this CTA's 64), reduction steps [kb0, kb1)
-// of 64 columns, NT column groups of 8.  Column n of group c carries token
-// 4c + (n & 3), hi part for n < 4 and lo part for n >= 4.
-//
-// CHAIN (per-row weight scales and one activation scale per token): the MMAs
-// accumulate straight through K and the caller applies both scales at the end.
-// Otherwise every 64-column step ends with acc += (s_row * inv_act) * D_step.
-// A register ring keeps the loads of the next D steps in flight: weight units,
-// activation fragments and (per-step mode) the scales they need.
+// One warp: 16 rows starting at row0, reduction steps [kb0, kb1) of 64 columns,
+// NT column groups of 8.  Column n of group c carries token 4c + (n & 3), hi
+// part for n < 4 and lo part for n >= 4.  A register ring keeps the loads of
+// the next D steps in flight: weight units, activation fragments and (per-step
+// mode) the scales they need.
 template <bool GATEUP, int NT, bool CHAIN>
 __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __restrict__ codesA,
                                           const uint8_t* __restrict__ codesB,
@@ -73,13 +95,12 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
     const int rt = row0 / kTileRows, b8 = (row0 % kTileRows) / 16;
     const int ng = a.group ? KB : 1;
     const int n = kb1 - kb0;
+    const DecodeK dk = a.dk;
     constexpr int UNIT_STEP = 8 * 32;  // uint4 units between consecutive 64-column steps
     const uint4* pA = reinterpret_cast<const uint4*>(codesA + frag_unit_offset(rt, kb0, b8, lane, K));
     const uint4* pB = reinterpret_cast<const uint4*>(codesB + frag_unit_offset(rt, kb0, b8, lane, K));
-    // activation fragments of this lane's B column: 4 fp16 per 16-column sub-block
     const uint2* pX[NT];
     bool bval[NT];
-    // inverse activation scales of this lane's D columns 2t, 2t+1
     const float* pI[NT][2];
 #pragma unroll
     for (int c = 0; c < NT; ++c) {
@@ -106,31 +127,21 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
         if (GATEUP) { rowB0 = __ldg(pS[1]); rowB1 = __ldg(pS[1] + 8); }
     }
 
-    constexpr int D = NT == 1 ? 4 : 2;
+    // the ring holds what streams from HBM: weight units and (gs64) their scales;
+    // activation fragments and their inverse scales are L1 hits shared by the
+    // CTA's warps and are loaded when used
+    constexpr int D = 8;
     uint4 rA[D], rB[D];
-    uint2 rX[D][NT][4];
-    float rI[D][NT][2], rS[D][4];
+    float rS[D][4];
     auto fetch = [&](int slot, int rel) {
         rA[slot] = ldg_stream(pA + rel * UNIT_STEP);
         if (GATEUP) rB[slot] = ldg_stream(pB + rel * UNIT_STEP);
-#pragma unroll
-        for (int c = 0; c < NT; ++c)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                rX[slot][c][j] = bval[c] ? __ldg(pX[c] + rel * 32 + 4 * j) : make_uint2(0u, 0u);
-        if (!CHAIN) {
-#pragma unroll
-            for (int c = 0; c < NT; ++c) {
-                rI[slot][c][0] = __ldg(pI[c][0] + rel);
-                rI[slot][c][1] = __ldg(pI[c][1] + rel);
-            }
-            if (a.group) {
-                rS[slot][0] = __ldg(pS[0] + (int64_t)(kb0 + rel) * kTileRows);
-                rS[slot][1] = __ldg(pS[0] + (int64_t)(kb0 + rel) * kTileRows + 8);
-                if (GATEUP) {
-                    rS[slot][2] = __ldg(pS[1] + (int64_t)(kb0 + rel) * kTileRows);
-                    rS[slot][3] = __ldg(pS[1] + (int64_t)(kb0 + rel) * kTileRows + 8);
-                }
+        if (!CHAIN && a.group) {
+            rS[slot][0] = __ldg(pS[0] + (int64_t)(kb0 + rel) * kTileRows);
+            rS[slot][1] = __ldg(pS[0] + (int64_t)(kb0 + rel) * kTileRows + 8);
+            if (GATEUP) {
+                rS[slot][2] = __ldg(pS[1] + (int64_t)(kb0 + rel) * kTileRows);
+                rS[slot][3] = __ldg(pS[1] + (int64_t)(kb0 + rel) * kTileRows + 8);
             }
         }
     };
@@ -150,8 +161,9 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
 #pragma unroll
                 for (int c = 0; c < NT; ++c) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) bx[c][j] = rX[sl][c][j];
-                    if (!CHAIN) { iv[c][0] = rI[sl][c][0]; iv[c][1] = rI[sl][c][1]; }
+                    for (int j = 0; j < 4; ++j)
+                        bx[c][j] = bval[c] ? __ldg(pX[c] + rel * 32 + 4 * j) : make_uint2(0u, 0u);
+                    if (!CHAIN) { iv[c][0] = __ldg(pI[c][0] + rel); iv[c][1] = __ldg(pI[c][1] + rel); }
                 }
                 if (!CHAIN) {
                     if (a.group) {
@@ -168,12 +180,12 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t fa[4];
-                        decode_frag_word(wa[j], fa);
+                        decode_word(wa[j], fa, dk);
 #pragma unroll
                         for (int c = 0; c < NT; ++c) mma_f16_16816(accA[c], fa, bx[c][j].x, bx[c][j].y);
                         if (GATEUP) {
                             uint32_t fb[4];
-                            decode_frag_word(wb[j], fb);
+                            decode_word(wb[j], fb, dk);
 #pragma unroll
                             for (int c = 0; c < NT; ++c) mma_f16_16816(accB[c], fb, bx[c][j].x, bx[c][j].y);
                         }
@@ -183,7 +195,7 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t fa[4];
-                        decode_frag_word(wa[j], fa);
+                        decode_word(wa[j], fa, dk);
 #pragma unroll
                         for (int c = 0; c < NT; ++c) {
                             if (j == 0) mma_f16_16816_zc(dA[c], fa, bx[c][j].x, bx[c][j].y);
@@ -191,7 +203,7 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
                         }
                         if (GATEUP) {
                             uint32_t fb[4];
-                            decode_frag_word(wb[j], fb);
+                            decode_word(wb[j], fb, dk);
 #pragma unroll
                             for (int c = 0; c < NT; ++c) {
                                 if (j == 0) mma_f16_16816_zc(dB[c], fb, bx[c][j].x, bx[c][j].y);
@@ -216,120 +228,162 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
             }
         }
     }
-}
-
-template <bool GATEUP, int NT, bool CHAIN>
-__device__ __forceinline__ void gemv_pass(const GemvArgs& a, float* red, const uint8_t* codesA,
-                                          const uint8_t* codesB, const float* sA,
-                                          const float* sB, int K, int rb64, int pc, int p1) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int b16 = warp & 3, half = warp >> 2;
-    const int KB = K / 64;
-    const int row0 = rb64 * 64 + b16 * 16;
-    float accA[NT][4], accB[NT][4];
-    gemv_warp<GATEUP, NT, CHAIN>(a, codesA, codesB, sA, sB, K, row0, half * (KB / 2),
-                                 (half + 1) * (KB / 2), pc, p1, accA, accB);
-    // red layout: [mat 2][half 2][64 rows][8*NT cols]
-    const int C = 8 * NT;
+    // hi + lo: lanes t and t ^ 2 hold the two parts of the same tokens
 #pragma unroll
     for (int c = 0; c < NT; ++c)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int r = b16 * 16 + g + (i >> 1) * 8, nn = 8 * c + 2 * t + (i & 1);
-            red[((0 * 2 + half) * 64 + r) * C + nn] = accA[c][i];
-            if (GATEUP) red[((1 * 2 + half) * 64 + r) * C + nn] = accB[c][i];
+            accA[c][i] += __shfl_xor_sync(0xffffffffu, accA[c][i], 2);
+            if (GATEUP) accB[c][i] += __shfl_xor_sync(0xffffffffu, accB[c][i], 2);
         }
-    __syncthreads();
 }
 
-template <bool GATEUP, int NT, bool CHAIN>
+// ---------------------------------------------------------------------------
+// gate/up + SwiGLU.  After the shuffle, lane (g, t < 2) holds rows g, g + 8 of
+// the warp's 16 and tokens 4c + 2t + {0, 1}.
+// ---------------------------------------------------------------------------
+template <int NT, bool CHAIN>
 __global__ void __launch_bounds__(kGemvWarps * 32)
-expert_gemv_kernel(GemvArgs a) {
-    __shared__ float red[2 * 2 * 64 * 8 * kGemvMaxNT];
-    __shared__ float gmax[8 * kGemvMaxNT][2];
-    __shared__ int last_flag;
-    const int K = GATEUP ? a.H : a.I;
-    const int R = GATEUP ? a.I : a.H;
-    const int nrb = R / 64;
+gateup_gemv_kernel(GemvArgs a) {
+    __shared__ float wmax[kGemvWarps][8 * kGemvMaxNT];
+    const int nrb = a.I / 64;
     const int u = blockIdx.x / nrb, rb64 = blockIdx.x % nrb;
     if (u >= *a.n_units) return;
     const int e = a.unit_expert[u], p0 = a.unit_begin[u], p1 = a.unit_end[u];
     const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
-    const int mA = GATEUP ? 0 : 2;
-    const uint8_t* codesA = blob + a.L.codes[mA];
+    const uint8_t* codesA = blob + a.L.codes[0];
     const uint8_t* codesB = blob + a.L.codes[1];
-    const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[mA]);
+    const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[0]);
     const float* sB = reinterpret_cast<const float*>(blob + a.L.scales[1]);
-    const int C = 8 * NT;
-    const int tid = threadIdx.x;
-    const int KB = K / 64;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int KB = a.H / 64;
+    const int row0 = rb64 * 64 + warp * 16;
+
+    // zero this CTA's share of the unit's down-projection outputs o[p0:p1, :]
+    {
+        float4* o4 = reinterpret_cast<float4*>(a.o + (int64_t)p0 * a.H);
+        const int64_t n4 = (int64_t)(p1 - p0) * a.H / 4;
+        const int64_t beg = n4 * rb64 / nrb, end = n4 * (rb64 + 1) / nrb;
+        for (int64_t i = beg + threadIdx.x; i < end; i += kGemvWarps * 32)
+            o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 
     for (int pc = p0; pc < p1; pc += 4 * NT) {
-        const int tc = min(4 * NT, p1 - pc);
-        __syncthreads();  // previous pass finished with red
-        gemv_pass<GATEUP, NT, CHAIN>(a, red, codesA, codesB, sA, sB, K, rb64, pc, p1);
-        // combine halves and hi/lo: thread -> (token tt, row r)
-        if (GATEUP) {
-            // h for 64 rows x tc tokens, then one power-of-two scale per token
-            for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
-                const int tt = q / 64, r = q % 64;
-                const int c = tt / 4, nn = 8 * c + (tt & 3);
-                float ga = red[((0 * 2 + 0) * 64 + r) * C + nn] + red[((0 * 2 + 1) * 64 + r) * C + nn] +
-                           red[((0 * 2 + 0) * 64 + r) * C + nn + 4] + red[((0 * 2 + 1) * 64 + r) * C + nn + 4];
-                float ua = red[((1 * 2 + 0) * 64 + r) * C + nn] + red[((1 * 2 + 1) * 64 + r) * C + nn] +
-                           red[((1 * 2 + 0) * 64 + r) * C + nn + 4] + red[((1 * 2 + 1) * 64 + r) * C + nn + 4];
-                if (CHAIN) {  // per-row weight scale and the token's activation scale
+        float accA[NT][4], accB[NT][4];
+        gemv_warp<true, NT, CHAIN>(a, codesA, codesB, sA, sB, a.H, row0, 0, KB, pc, p1, accA, accB);
+        // SwiGLU on rows g, g+8 for tokens 4c + 2t + {0, 1} (lanes t < 2)
+        float hv[NT][4];
+        float mx[NT][2];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+            mx[c][0] = 0.0f; mx[c][1] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int tt = 4 * c + 2 * (t & 1) + (i & 1);
+                const int row = row0 + g + 8 * (i >> 1);
+                float ga = accA[c][i], ua = accB[c][i];
+                if (CHAIN && pc + tt < p1) {
                     const float inv = __ldg(a.xinv + (int64_t)a.pair_tok[pc + tt] * KB);
-                    const int row = rb64 * 64 + r;
                     ga *= __ldg(sA + scale_offset(row, 0, 1)) * inv;
                     ua *= __ldg(sB + scale_offset(row, 0, 1)) * inv;
                 }
-                const float hv = silu_f(ga) * ua;
-                red[((0 * 2 + 0) * 64 + r) * C + nn] = hv;  // reuse: h in slot (0, 0, r, nn)
-                float m = fabsf(hv);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if ((q & 31) == 0) gmax[tt][(q >> 5) & 1] = m;
-            }
-            __syncthreads();
-            for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
-                const int tt = q / 64, r = q % 64;
-                const int c = tt / 4, nn = 8 * c + (tt & 3);
-                const float hv = red[((0 * 2 + 0) * 64 + r) * C + nn];
-                float inv;
-                const float sc = act_group_scale(fmaxf(gmax[tt][0], gmax[tt][1]), &inv);
-                __half hi, lo;
-                split_f16(hv * sc, hi, lo);
-                const int64_t p = pc + tt;
-                __half* dst = a.hq + (p * (a.I / 64) + rb64) * 128;
-                dst[r] = hi;
-                dst[64 + r] = lo;
-                if (r == 0) a.hinv[p * (a.I / 64) + rb64] = inv;
-            }
-        } else {
-            for (int q = tid; q < tc * 64; q += kGemvWarps * 32) {
-                const int tt = q / 64, r = q % 64;
-                const int c = tt / 4, nn = 8 * c + (tt & 3);
-                float v = red[((0 * 2 + 0) * 64 + r) * C + nn] + red[((0 * 2 + 1) * 64 + r) * C + nn] +
-                          red[((0 * 2 + 0) * 64 + r) * C + nn + 4] + red[((0 * 2 + 1) * 64 + r) * C + nn + 4];
-                a.o[(int64_t)(pc + tt) * a.H + rb64 * 64 + r] = v;
+                hv[c][i] = (t < 2 && pc + tt < p1) ? silu_f(ga) * ua : 0.0f;
+                mx[c][i & 1] = fmaxf(mx[c][i & 1], fabsf(hv[c][i]));
             }
         }
+        // max over the warp's 16 rows per token, then over the CTA's 64 rows
+#pragma unroll
+        for (int c = 0; c < NT; ++c)
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float m = mx[c][q];
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                if (g == 0 && t < 2) wmax[warp][4 * c + 2 * t + q] = m;
+            }
+        __syncthreads();
+        if (t < 2) {
+#pragma unroll
+            for (int c = 0; c < NT; ++c)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int tt = 4 * c + 2 * t + q;
+                    if (pc + tt >= p1) continue;
+                    float m = wmax[0][tt];
+#pragma unroll
+                    for (int ww = 1; ww < kGemvWarps; ++ww) m = fmaxf(m, wmax[ww][tt]);
+                    float inv;
+                    const float sc = act_group_scale(m, &inv);
+                    const int64_t p = pc + tt;
+                    __half* dst = a.hq + (p * (a.I / 64) + rb64) * 128;
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        __half hi, lo;
+                        split_f16(hv[c][2 * hr + q] * sc, hi, lo);
+                        const int r = warp * 16 + g + 8 * hr;
+                        dst[r] = hi;
+                        dst[64 + r] = lo;
+                    }
+                    if (warp == 0 && g == 0) a.hinv[p * (a.I / 64) + rb64] = inv;
+                }
+        }
+        __syncthreads();  // wmax reused by the next pass
     }
-    if (GATEUP) return;
+}
 
-    // ---- combine: the last unit to finish this 64-row block writes y ----
+// ---------------------------------------------------------------------------
+// down projection + combine.  CTA = (unit, 64-row block, half of the reduction).
+// ---------------------------------------------------------------------------
+template <int NT>
+__global__ void __launch_bounds__(kGemvWarps * 32)
+down_gemv_kernel(GemvArgs a) {
+    __shared__ int last_flag;
+    const int nrb = a.H / 64;
+    const int u = blockIdx.x / (nrb * kDownSplit);
+    const int rem = blockIdx.x % (nrb * kDownSplit);
+    const int rb64 = rem / kDownSplit, half = rem % kDownSplit;
+    const int n_units = *a.n_units;
+    if (u >= n_units) return;
+    const int e = a.unit_expert[u], p0 = a.unit_begin[u], p1 = a.unit_end[u];
+    const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
+    const uint8_t* codesA = blob + a.L.codes[2];
+    const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[2]);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int KB = a.I / 64;
+    const int kb0 = half * KB / kDownSplit, kb1 = (half + 1) * KB / kDownSplit;
+    const int row0 = rb64 * 64 + warp * 16;
+
+    for (int pc = p0; pc < p1; pc += 4 * NT) {
+        float accA[NT][4], accB[NT][4];
+        gemv_warp<false, NT, false>(a, codesA, codesA, sA, sA, a.I, row0, kb0, kb1, pc, p1, accA, accB);
+        if (t < 2) {
+#pragma unroll
+            for (int c = 0; c < NT; ++c)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tt = 4 * c + 2 * t + (i & 1);
+                    // two addends per element (the halves) into a zeroed o: the sum
+                    // does not depend on which half lands first
+                    if (pc + tt < p1)
+                        atomicAdd(a.o + (int64_t)(pc + tt) * a.H + row0 + g + 8 * (i >> 1), accA[c][i]);
+                }
+        }
+    }
+
+    // ---- combine: the last CTA to finish this 64-row block writes y ----
     __threadfence();
     __syncthreads();
-    if (tid == 0) {
+    if (threadIdx.x == 0) {
         const int done = atomicAdd(&a.counters[rb64], 1) + 1;
-        last_flag = done == *a.n_units;
+        last_flag = done == n_units * kDownSplit;
     }
     __syncthreads();
     if (!last_flag) return;
     __threadfence();
-    for (int q = tid; q < a.T * 64; q += kGemvWarps * 32) {
+    for (int q = threadIdx.x; q < a.T * 64; q += kGemvWarps * 32) {
         const int tt = q / 64, r = rb64 * 64 + q % 64;
         float acc = 0.0f;
         for (int j = 0; j < a.k; ++j) {
@@ -341,7 +395,7 @@ expert_gemv_kernel(GemvArgs a) {
         if (a.residual) acc = a.residual[(int64_t)tt * a.H + r] + acc;
         a.y[(int64_t)tt * a.H + r] = acc;
     }
-    if (tid == 0) a.counters[rb64] = 0;  // ready for the next call on this workspace
+    if (threadIdx.x == 0) a.counters[rb64] = 0;  // ready for the next call on this workspace
 }
 
 }  // namespace coli

@@ -339,18 +339,51 @@ union_kernel(const int32_t* __restrict__ idx, int T, int k, int E, UnionOut o) {
     union_body(idx, T, k, E, o, un_smem);
 }
 
-// Small batches: top-k of every token (warps take tokens in turn) and the union
-// in one CTA, saving a launch and a round trip through global memory.
+// Small batches (T * E <= 4096): top-k of every token and the union in one CTA.
+// Every (token, expert) pair gets a thread that sums the router slices and
+// applies the sigmoid and the bias, then counts the experts that rank before
+// it (higher selection score, or equal score and lower index); the k with rank
+// < k are the picks, in rank order.  Short loops over shared memory, no
+// long single-warp path.
+constexpr int kSmallSelect = 4096;
+
 __global__ void __launch_bounds__(kUnionThreads)
 topk_union_kernel(const float* __restrict__ zpart, int KS, int T, int E,
                   const float* __restrict__ bias, int k, float routed_scale, int norm_topk,
-                  int32_t* idx, float* w, int topk_warps, UnionOut o) {
+                  int32_t* idx, float* w, UnionOut o) {
     extern __shared__ uint32_t un_smem[];
-    const int warp = threadIdx.x >> 5;
-    if (warp < topk_warps) {
-        float* sel = reinterpret_cast<float*>(un_smem) + (int64_t)warp * 2 * E;
-        for (int t = warp; t < T; t += topk_warps)
-            topk_token(zpart, KS, T, E, bias, k, routed_scale, norm_topk, t, sel, sel + E, idx, w);
+    float* sc = reinterpret_cast<float*>(un_smem);  // [T][E] sigmoid scores
+    float* sel = sc + T * E;                         // [T][E] selection scores
+    __shared__ float pick_s[kSmallSelect / 32][32];
+    __shared__ int pick_e[kSmallSelect / 32][32];
+    const int n = T * E;
+    for (int i = threadIdx.x; i < n; i += kUnionThreads) {
+        const int t = i / E, e = i - t * E;
+        float z = 0.0f;
+        for (int ks = 0; ks < KS; ++ks) z += __ldcg(zpart + ((int64_t)ks * T + t) * E + e);
+        const float s = 1.0f / (1.0f + expf(-z));
+        sc[i] = s;
+        sel[i] = s + __ldg(bias + e);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kUnionThreads) {
+        const int t = i / E, e = i - t * E;
+        const float v = sel[i];
+        const float* row = sel + t * E;
+        int r = 0;
+        for (int e2 = 0; e2 < E; ++e2) {
+            const float v2 = row[e2];
+            r += (v2 > v) | ((v2 == v) & (e2 < e));
+        }
+        if (r < k) { pick_e[t][r] = e; pick_s[t][r] = sc[i]; }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * k; i += kUnionThreads) {
+        const int t = i / k, j = i - t * k;
+        float denom = 0.0f;  // in pick order
+        for (int q = 0; q < k; ++q) denom += pick_s[t][q];
+        idx[i] = pick_e[t][j];
+        w[i] = (norm_topk ? pick_s[t][j] / denom : pick_s[t][j]) * routed_scale;
     }
     __threadfence_block();
     __syncthreads();
