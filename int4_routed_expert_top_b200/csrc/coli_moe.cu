@@ -185,19 +185,31 @@ int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int
     return launch_union(idx, T, d.k, d.E, o, st);
 }
 
+// dynamic shared memory of a GEMV CTA: 4*NT staged activation rows of K
+// columns (fp16 hi + lo) and their inverse scales
+int gemv_smem(int NT, int K) { return 4 * NT * (K / 64) * (128 * 2 + 4); }
+
 template <int NT>
-int launch_gemv_nt(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st,
-                   int stage_mark_rc) {
-    (void)stage_mark_rc;
+int launch_gemv_nt(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
     const int grid = units_max * (d.I / 64);
-    if (d.group == 0) gateup_gemv_kernel<NT, true><<<grid, kGemvWarps * 32, 0, st>>>(a);
-    else              gateup_gemv_kernel<NT, false><<<grid, kGemvWarps * 32, 0, st>>>(a);
+    const int smem = gemv_smem(NT, d.H);
+    int rc;
+    if (d.group == 0) {
+        if ((rc = set_smem((const void*)gateup_gemv_kernel<NT, true>, smem))) return rc;
+        gateup_gemv_kernel<NT, true><<<grid, kGemvWarps * 32, smem, st>>>(a);
+    } else {
+        if ((rc = set_smem((const void*)gateup_gemv_kernel<NT, false>, smem))) return rc;
+        gateup_gemv_kernel<NT, false><<<grid, kGemvWarps * 32, smem, st>>>(a);
+    }
     return check_launch("gate/up gemv");
 }
 
 template <int NT>
 int launch_down_nt(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
-    down_gemv_kernel<NT><<<units_max * (d.H / 64) * kDownSplit, kGemvWarps * 32, 0, st>>>(a);
+    const int smem = gemv_smem(NT, d.I);
+    int rc = set_smem((const void*)down_gemv_kernel<NT>, smem);
+    if (rc) return rc;
+    down_gemv_kernel<NT><<<units_max * (d.H / 64) * kDownSplit, kGemvWarps * 32, smem, st>>>(a);
     return check_launch("down gemv");
 }
 
@@ -229,7 +241,7 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
     const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;
     // per-row weight scales with one activation scale per token let the gate/up
     // MMAs run through K without a per-step epilogue (CHAIN)
-    int rc = T <= 4 ? launch_gemv_nt<1>(d, units_max, a, st, 0) : launch_gemv_nt<2>(d, units_max, a, st, 0);
+    int rc = T <= 4 ? launch_gemv_nt<1>(d, units_max, a, st) : launch_gemv_nt<2>(d, units_max, a, st);
     if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;
     return T <= 4 ? launch_down_nt<1>(d, units_max, a, st) : launch_down_nt<2>(d, units_max, a, st);

@@ -80,14 +80,17 @@ struct GemvArgs {
 // One warp: 16 rows starting at row0, reduction steps [kb0, kb1) of 64 columns,
 // NT column groups of 8.  Column n of group c carries token 4c + (n & 3), hi
 // part for n < 4 and lo part for n >= 4.  A register ring keeps the loads of
-// the next D steps in flight: weight units, activation fragments and (per-step
-// mode) the scales they need.
-template <bool GATEUP, int NT, bool CHAIN>
+// the next D steps of weight units (and gs64 scales) in flight; the pass's
+// activation rows and inverse scales are staged in shared memory by stage()
+// (called by every thread of the CTA while the ring fills) as
+// xs[token][K/64][128] fp16 and xi[token][K/64] f32.
+template <bool GATEUP, int NT, bool CHAIN, typename Stage>
 __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __restrict__ codesA,
                                           const uint8_t* __restrict__ codesB,
                                           const float* __restrict__ sA,
                                           const float* __restrict__ sB, int K, int row0,
-                                          int kb0, int kb1, int pc, int p1,
+                                          int kb0, int kb1, int tc, const __half* xs,
+                                          const float* xi, Stage&& stage,
                                           float accA[NT][4], float accB[NT][4]) {
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -104,16 +107,14 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
     const float* pI[NT][2];
 #pragma unroll
     for (int c = 0; c < NT; ++c) {
-        const int pb = pc + 4 * c + (g & 3);
-        bval[c] = pb < p1;
-        const int sb = bval[c] ? (GATEUP ? a.pair_tok[pb] : pb) : 0;
-        const __half* base = (GATEUP ? a.xq : a.hq) + ((int64_t)sb * KB + kb0) * 128 + (g >> 2) * 64;
-        pX[c] = reinterpret_cast<const uint2*>(base) + t;
+        const int tb = 4 * c + (g & 3);
+        bval[c] = tb < tc;
+        pX[c] = reinterpret_cast<const uint2*>(xs + ((int64_t)(bval[c] ? tb : 0) * KB + kb0) * 128 +
+                                               (g >> 2) * 64) + t;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-            const int pd = pc + 4 * c + ((2 * t) & 3) + i;
-            const int sd = pd < p1 ? (GATEUP ? a.pair_tok[pd] : pd) : 0;
-            pI[c][i] = (GATEUP ? a.xinv : a.hinv) + (int64_t)sd * KB + kb0;
+            const int td = 4 * c + ((2 * t) & 3) + i;
+            pI[c][i] = xi + (td < tc ? td : 0) * KB + kb0;
         }
     }
     const float* pS[2] = {sA + scale_offset(row0 + g, 0, ng), sB + scale_offset(row0 + g, 0, ng)};
@@ -148,6 +149,8 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
 #pragma unroll
     for (int sl = 0; sl < D; ++sl)
         if (sl < n) fetch(sl, sl);
+    stage();
+    __syncthreads();
 
     for (int base = 0; base < n; base += D) {
 #pragma unroll
@@ -162,8 +165,8 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
                 for (int c = 0; c < NT; ++c) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        bx[c][j] = bval[c] ? __ldg(pX[c] + rel * 32 + 4 * j) : make_uint2(0u, 0u);
-                    if (!CHAIN) { iv[c][0] = __ldg(pI[c][0] + rel); iv[c][1] = __ldg(pI[c][1] + rel); }
+                        bx[c][j] = bval[c] ? pX[c][rel * 32 + 4 * j] : make_uint2(0u, 0u);
+                    if (!CHAIN) { iv[c][0] = pI[c][0][rel]; iv[c][1] = pI[c][1][rel]; }
                 }
                 if (!CHAIN) {
                     if (a.group) {
@@ -242,10 +245,28 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
 // gate/up + SwiGLU.  After the shuffle, lane (g, t < 2) holds rows g, g + 8 of
 // the warp's 16 and tokens 4c + 2t + {0, 1}.
 // ---------------------------------------------------------------------------
+// stage activation rows src[i] (i < tc) of one pass: [tc][KB][128] fp16 plus
+// [tc][KB] inverse scales, 16-byte copies by every thread of the CTA
+__device__ __forceinline__ void stage_rows(const __half* __restrict__ q, const float* __restrict__ inv,
+                                           const int* src, int tc, int KB, __half* xs, float* xi) {
+    const int per = KB * 16;  // uint4 per row
+    for (int i = threadIdx.x; i < tc * per; i += kGemvWarps * 32) {
+        const int r = i / per, c = i - r * per;
+        reinterpret_cast<uint4*>(xs)[i] =
+            __ldg(reinterpret_cast<const uint4*>(q + (int64_t)src[r] * KB * 128) + c);
+    }
+    for (int i = threadIdx.x; i < tc * KB; i += kGemvWarps * 32) {
+        const int r = i / KB, c = i - r * KB;
+        xi[i] = __ldg(inv + (int64_t)src[r] * KB + c);
+    }
+}
+
 template <int NT, bool CHAIN>
 __global__ void __launch_bounds__(kGemvWarps * 32)
 gateup_gemv_kernel(GemvArgs a) {
+    extern __shared__ uint4 gv_smem[];
     __shared__ float wmax[kGemvWarps][8 * kGemvMaxNT];
+    __shared__ int src[8 * kGemvMaxNT];
     const int nrb = a.I / 64;
     const int u = blockIdx.x / nrb, rb64 = blockIdx.x % nrb;
     if (u >= *a.n_units) return;
@@ -259,6 +280,8 @@ gateup_gemv_kernel(GemvArgs a) {
     const int g = lane >> 2, t = lane & 3;
     const int KB = a.H / 64;
     const int row0 = rb64 * 64 + warp * 16;
+    __half* xs = reinterpret_cast<__half*>(gv_smem);
+    float* xi = reinterpret_cast<float*>(xs + (size_t)4 * NT * KB * 128);
 
     // zero this CTA's share of the unit's down-projection outputs o[p0:p1, :]
     {
@@ -270,8 +293,14 @@ gateup_gemv_kernel(GemvArgs a) {
     }
 
     for (int pc = p0; pc < p1; pc += 4 * NT) {
+        const int tc = min(4 * NT, p1 - pc);
+        __syncthreads();  // the previous pass is done with xs, xi, src and wmax
+        if (threadIdx.x < tc) src[threadIdx.x] = a.pair_tok[pc + threadIdx.x];
+        __syncthreads();
         float accA[NT][4], accB[NT][4];
-        gemv_warp<true, NT, CHAIN>(a, codesA, codesB, sA, sB, a.H, row0, 0, KB, pc, p1, accA, accB);
+        gemv_warp<true, NT, CHAIN>(a, codesA, codesB, sA, sB, a.H, row0, 0, KB, tc, xs, xi,
+                                   [&] { stage_rows(a.xq, a.xinv, src, tc, KB, xs, xi); },
+                                   accA, accB);
         // SwiGLU on rows g, g+8 for tokens 4c + 2t + {0, 1} (lanes t < 2)
         float hv[NT][4];
         float mx[NT][2];
@@ -284,7 +313,7 @@ gateup_gemv_kernel(GemvArgs a) {
                 const int row = row0 + g + 8 * (i >> 1);
                 float ga = accA[c][i], ua = accB[c][i];
                 if (CHAIN && pc + tt < p1) {
-                    const float inv = __ldg(a.xinv + (int64_t)a.pair_tok[pc + tt] * KB);
+                    const float inv = xi[tt * KB];
                     ga *= __ldg(sA + scale_offset(row, 0, 1)) * inv;
                     ua *= __ldg(sB + scale_offset(row, 0, 1)) * inv;
                 }
@@ -329,7 +358,6 @@ gateup_gemv_kernel(GemvArgs a) {
                     if (warp == 0 && g == 0) a.hinv[p * (a.I / 64) + rb64] = inv;
                 }
         }
-        __syncthreads();  // wmax reused by the next pass
     }
 }
 
@@ -339,7 +367,9 @@ gateup_gemv_kernel(GemvArgs a) {
 template <int NT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
 down_gemv_kernel(GemvArgs a) {
+    extern __shared__ uint4 gv_smem[];
     __shared__ int last_flag;
+    __shared__ int src[8 * kGemvMaxNT];
     const int nrb = a.H / 64;
     const int u = blockIdx.x / (nrb * kDownSplit);
     const int rem = blockIdx.x % (nrb * kDownSplit);
@@ -355,10 +385,18 @@ down_gemv_kernel(GemvArgs a) {
     const int KB = a.I / 64;
     const int kb0 = half * KB / kDownSplit, kb1 = (half + 1) * KB / kDownSplit;
     const int row0 = rb64 * 64 + warp * 16;
+    __half* xs = reinterpret_cast<__half*>(gv_smem);
+    float* xi = reinterpret_cast<float*>(xs + (size_t)4 * NT * KB * 128);
 
     for (int pc = p0; pc < p1; pc += 4 * NT) {
+        const int tc = min(4 * NT, p1 - pc);
+        __syncthreads();
+        if (threadIdx.x < tc) src[threadIdx.x] = pc + threadIdx.x;
+        __syncthreads();
         float accA[NT][4], accB[NT][4];
-        gemv_warp<false, NT, false>(a, codesA, codesA, sA, sA, a.I, row0, kb0, kb1, pc, p1, accA, accB);
+        gemv_warp<false, NT, false>(a, codesA, codesA, sA, sA, a.I, row0, kb0, kb1, tc, xs, xi,
+                                    [&] { stage_rows(a.hq, a.hinv, src, tc, KB, xs, xi); },
+                                    accA, accB);
         if (t < 2) {
 #pragma unroll
             for (int c = 0; c < NT; ++c)
