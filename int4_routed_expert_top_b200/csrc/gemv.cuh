@@ -118,10 +118,16 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
         }
     }
     const float* pS[2] = {sA + scale_offset(row0 + g, 0, ng), sB + scale_offset(row0 + g, 0, ng)};
+    float cA[CHAIN ? NT : 1][4][4], cB[CHAIN ? NT : 1][4][4];  // CHAIN accumulators per sub-block
 #pragma unroll
     for (int c = 0; c < NT; ++c)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) { accA[c][i] = 0.0f; accB[c][i] = 0.0f; }
+        for (int i = 0; i < 4; ++i) {
+            accA[c][i] = 0.0f; accB[c][i] = 0.0f;
+            if (CHAIN)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) { cA[c][j][i] = 0.0f; cB[c][j][i] = 0.0f; }
+        }
     float rowA0 = 0.f, rowA1 = 0.f, rowB0 = 0.f, rowB1 = 0.f;  // per-row scales
     if (!CHAIN && !a.group) {
         rowA0 = __ldg(pS[0]); rowA1 = __ldg(pS[0] + 8);
@@ -180,56 +186,73 @@ __device__ __forceinline__ void gemv_warp(const GemvArgs& a, const uint8_t* __re
                 const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
                 const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
                 if (CHAIN) {
+                    // one accumulator per 16-column sub-block: four independent MMA chains
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t fa[4];
                         decode_word(wa[j], fa, dk);
 #pragma unroll
-                        for (int c = 0; c < NT; ++c) mma_f16_16816(accA[c], fa, bx[c][j].x, bx[c][j].y);
+                        for (int c = 0; c < NT; ++c) mma_f16_16816(cA[c][j], fa, bx[c][j].x, bx[c][j].y);
                         if (GATEUP) {
                             uint32_t fb[4];
                             decode_word(wb[j], fb, dk);
 #pragma unroll
-                            for (int c = 0; c < NT; ++c) mma_f16_16816(accB[c], fb, bx[c][j].x, bx[c][j].y);
+                            for (int c = 0; c < NT; ++c) mma_f16_16816(cB[c][j], fb, bx[c][j].x, bx[c][j].y);
                         }
                     }
                 } else {
-                    float dA[NT][4], dB[NT][4];
+                    // two fresh chains per step (sub-blocks 0,2 and 1,3), summed in the epilogue
+                    float dA[NT][2][4], dB[NT][2][4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t fa[4];
                         decode_word(wa[j], fa, dk);
 #pragma unroll
                         for (int c = 0; c < NT; ++c) {
-                            if (j == 0) mma_f16_16816_zc(dA[c], fa, bx[c][j].x, bx[c][j].y);
-                            else        mma_f16_16816(dA[c], fa, bx[c][j].x, bx[c][j].y);
+                            if (j < 2) mma_f16_16816_zc(dA[c][j & 1], fa, bx[c][j].x, bx[c][j].y);
+                            else       mma_f16_16816(dA[c][j & 1], fa, bx[c][j].x, bx[c][j].y);
                         }
                         if (GATEUP) {
                             uint32_t fb[4];
                             decode_word(wb[j], fb, dk);
 #pragma unroll
                             for (int c = 0; c < NT; ++c) {
-                                if (j == 0) mma_f16_16816_zc(dB[c], fb, bx[c][j].x, bx[c][j].y);
-                                else        mma_f16_16816(dB[c], fb, bx[c][j].x, bx[c][j].y);
+                                if (j < 2) mma_f16_16816_zc(dB[c][j & 1], fb, bx[c][j].x, bx[c][j].y);
+                                else       mma_f16_16816(dB[c][j & 1], fb, bx[c][j].x, bx[c][j].y);
                             }
                         }
                     }
 #pragma unroll
                     for (int c = 0; c < NT; ++c) {
-                        accA[c][0] = fmaf(sc[0] * iv[c][0], dA[c][0], accA[c][0]);
-                        accA[c][1] = fmaf(sc[0] * iv[c][1], dA[c][1], accA[c][1]);
-                        accA[c][2] = fmaf(sc[1] * iv[c][0], dA[c][2], accA[c][2]);
-                        accA[c][3] = fmaf(sc[1] * iv[c][1], dA[c][3], accA[c][3]);
+                        float qa[4], qb[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            qa[i] = dA[c][0][i] + dA[c][1][i];
+                            qb[i] = GATEUP ? dB[c][0][i] + dB[c][1][i] : 0.0f;
+                        }
+                        accA[c][0] = fmaf(sc[0] * iv[c][0], qa[0], accA[c][0]);
+                        accA[c][1] = fmaf(sc[0] * iv[c][1], qa[1], accA[c][1]);
+                        accA[c][2] = fmaf(sc[1] * iv[c][0], qa[2], accA[c][2]);
+                        accA[c][3] = fmaf(sc[1] * iv[c][1], qa[3], accA[c][3]);
                         if (GATEUP) {
-                            accB[c][0] = fmaf(sc[2] * iv[c][0], dB[c][0], accB[c][0]);
-                            accB[c][1] = fmaf(sc[2] * iv[c][1], dB[c][1], accB[c][1]);
-                            accB[c][2] = fmaf(sc[3] * iv[c][0], dB[c][2], accB[c][2]);
-                            accB[c][3] = fmaf(sc[3] * iv[c][1], dB[c][3], accB[c][3]);
+                            accB[c][0] = fmaf(sc[2] * iv[c][0], qb[0], accB[c][0]);
+                            accB[c][1] = fmaf(sc[2] * iv[c][1], qb[1], accB[c][1]);
+                            accB[c][2] = fmaf(sc[3] * iv[c][0], qb[2], accB[c][2]);
+                            accB[c][3] = fmaf(sc[3] * iv[c][1], qb[3], accB[c][3]);
                         }
                     }
                 }
             }
         }
+    }
+    if (CHAIN) {
+#pragma unroll
+        for (int c = 0; c < NT; ++c)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                accA[c][i] = (cA[c][0][i] + cA[c][1][i]) + (cA[c][2][i] + cA[c][3][i]);
+                if (GATEUP) accB[c][i] = (cB[c][0][i] + cB[c][1][i]) + (cB[c][2][i] + cB[c][3][i]);
+            }
     }
     // hi + lo: lanes t and t ^ 2 hold the two parts of the same tokens
 #pragma unroll
