@@ -216,6 +216,13 @@ int coli_moe_stack_forward(const coli_moe_layer* const* layers, int32_t L,
                            float* x, int32_t T, float eps, coli_path path,
                            void* ws, size_t ws_bytes, coli_stream_t stream);
 
+/* Device-side status of the most recent coli_moe_forward* call that used this
+ * workspace (ws planned for T tokens): copies the error flags to *flags (host)
+ * after synchronising `stream`.  Returns COLI_E_TIMEOUT if a bounded wait inside
+ * a kernel gave up (its outputs are then invalid), else COLI_OK. */
+int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws,
+                    int32_t* flags, coli_stream_t stream);
+
 /* Test helper: dequantise matrix `which` (0 gate, 1 up, 2 down) of expert
  * `expert` (0 .. E + n_shared - 1) from the device blob into out (device f32,
  * row-major [R, K] in container order). */

@@ -21,7 +21,7 @@ __all__ = [
     "coli_moe_layer_destroy", "coli_moe_workspace_size", "coli_moe_route",
     "coli_moe_union", "coli_moe_forward", "coli_moe_forward_ex", "coli_moe_rmsnorm",
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
-    "coli_moe_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "Desc",
+    "coli_moe_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "coli_moe_status", "Desc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +37,7 @@ EXPORTS = (
     "coli_moe_layer_destroy", "coli_moe_workspace_size", "coli_moe_route",
     "coli_moe_union", "coli_moe_forward", "coli_moe_forward_ex", "coli_moe_rmsnorm",
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
-    "coli_moe_forward_noalloc",
+    "coli_moe_forward_noalloc", "coli_moe_status",
 )
 
 
@@ -86,6 +86,7 @@ _SIGS = {
                                 _P], ctypes.c_int),
     "coli_moe_dequant_debug": ([_P, _I32, _I32, _P, _P], ctypes.c_int),
     "coli_moe_forward_noalloc": ([_P, _P, ctypes.c_int, _I32, _P, _P], ctypes.c_int),
+    "coli_moe_status": ([_P, _I32, _P, ctypes.POINTER(_I32), _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -232,6 +233,13 @@ def coli_moe_stack_workspace_size(layers, T: int) -> int:
 def coli_moe_stack_forward(layers, x, T, eps, ws, path=COLI_PATH_AUTO, stream=None):
     _ok(lib.coli_moe_stack_forward(_layer_array(layers), len(layers), _ptr(x), T, eps, path,
                                    _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def coli_moe_status(layer, T: int, ws, stream=None) -> int:
+    """Error flags of the last forward on this workspace (raises on a timeout)."""
+    flags = _I32(0)
+    _ok(lib.coli_moe_status(layer, T, _ptr(ws), ctypes.byref(flags), _stream(stream)))
+    return flags.value
 
 
 def coli_moe_dequant_debug(layer, expert: int, which: int, out, stream=None):

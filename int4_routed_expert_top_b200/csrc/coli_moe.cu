@@ -55,7 +55,7 @@ bool shape_ok(int H, int I, int group) {
 // ---------------------------------------------------------------------------
 struct WsPlan {
     int64_t zpart, idx, w, offsets, pair_tok, pair_slot, uniq, n_uniq, inv;
-    int64_t unit_expert, unit_begin, unit_end, n_units, counters;
+    int64_t unit_expert, unit_begin, unit_end, n_units, counters, err;
     int64_t xq, xinv, hq, hinv, o, total;
 };
 
@@ -79,6 +79,7 @@ WsPlan plan_ws(const coli_moe_desc& d, int T) {
     p.unit_end = take((int64_t)(d.E + d.n_shared) * 4);
     p.n_units = take(4);
     p.counters = take((int64_t)(d.H / 64) * 4);
+    p.err = take(4);
     p.xq = take((int64_t)T * d.H * 4);          // fp16 hi + lo
     p.xinv = take((int64_t)T * (d.H / 64) * 4);
     p.hq = take(P * d.I * 4);                   // fp16 hi + lo
@@ -185,31 +186,21 @@ int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int
     return launch_union(idx, T, d.k, d.E, o, st);
 }
 
-// dynamic shared memory of a GEMV CTA: 4*NT staged activation rows of K
-// columns (fp16 hi + lo) and their inverse scales
-int gemv_smem(int NT, int K) { return 4 * NT * (K / 64) * (128 * 2 + 4); }
-
-template <int NT>
-int launch_gemv_nt(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
-    const int grid = units_max * (d.I / 64);
-    const int smem = gemv_smem(NT, d.H);
-    int rc;
-    if (d.group == 0) {
-        if ((rc = set_smem((const void*)gateup_gemv_kernel<NT, true>, smem))) return rc;
-        gateup_gemv_kernel<NT, true><<<grid, kGemvWarps * 32, smem, st>>>(a);
-    } else {
-        if ((rc = set_smem((const void*)gateup_gemv_kernel<NT, false>, smem))) return rc;
-        gateup_gemv_kernel<NT, false><<<grid, kGemvWarps * 32, smem, st>>>(a);
-    }
+template <int NT, bool GS>
+int launch_gateup_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
+    const int smem = gemv_ring_bytes<true, GS>() + gemv_act_bytes(NT, d.H);
+    int rc = set_smem((const void*)gateup_gemv_kernel<NT, GS>, smem);
+    if (rc) return rc;
+    gateup_gemv_kernel<NT, GS><<<units_max * (d.I / 64), kGemvThreads, smem, st>>>(a);
     return check_launch("gate/up gemv");
 }
 
-template <int NT>
-int launch_down_nt(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
-    const int smem = gemv_smem(NT, d.I);
-    int rc = set_smem((const void*)down_gemv_kernel<NT>, smem);
+template <int NT, bool GS>
+int launch_down_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
+    const int smem = gemv_ring_bytes<false, GS>() + gemv_act_bytes(NT, d.I);
+    int rc = set_smem((const void*)down_gemv_kernel<NT, GS>, smem);
     if (rc) return rc;
-    down_gemv_kernel<NT><<<units_max * (d.H / 64) * kDownSplit, kGemvWarps * 32, smem, st>>>(a);
+    down_gemv_kernel<NT, GS><<<units_max * (d.H / 64) * kDownSplit, kGemvThreads, smem, st>>>(a);
     return check_launch("down gemv");
 }
 
@@ -236,15 +227,17 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
     a.w = at<float>(ws, p.w);
     a.residual = residual;
     a.y = y;
+    a.err = at<int32_t>(ws, p.err);
     a.T = T; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;
-    // per-row weight scales with one activation scale per token let the gate/up
-    // MMAs run through K without a per-step epilogue (CHAIN)
-    int rc = T <= 4 ? launch_gemv_nt<1>(d, units_max, a, st) : launch_gemv_nt<2>(d, units_max, a, st);
+    const bool gs = d.group != 0;
+    int rc = T <= 4 ? (gs ? launch_gateup_t<1, true>(d, units_max, a, st) : launch_gateup_t<1, false>(d, units_max, a, st))
+                    : (gs ? launch_gateup_t<2, true>(d, units_max, a, st) : launch_gateup_t<2, false>(d, units_max, a, st));
     if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;
-    return T <= 4 ? launch_down_nt<1>(d, units_max, a, st) : launch_down_nt<2>(d, units_max, a, st);
+    return T <= 4 ? (gs ? launch_down_t<1, true>(d, units_max, a, st) : launch_down_t<1, false>(d, units_max, a, st))
+                  : (gs ? launch_down_t<2, true>(d, units_max, a, st) : launch_down_t<2, false>(d, units_max, a, st));
 }
 
 }  // namespace
@@ -447,6 +440,7 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     o.n_units = at<int32_t>(ws, p.n_units);
     o.counters = at<int32_t>(ws, p.counters);
     o.n_counters = d.H / 64;
+    o.err = at<int32_t>(ws, p.err);
     o.n_shared = d.n_shared;
     if ((rc = mark(COLI_STAGE_UNION))) return rc;
     if ((rc = launch_select(d, at<float>(ws, p.zpart), KS, T, idx, w, o, st))) return rc;
@@ -544,6 +538,20 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t 
         blob + L.codes[which], reinterpret_cast<const float*>(blob + L.scales[which]), R, K,
         d.group, out);
     return check_launch("dequant");
+}
+
+int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws, int32_t* flags,
+                    coli_stream_t stream) {
+    if (!layer || !ws || !flags) return fail(COLI_E_INVAL, "status: NULL pointer");
+    int rc = tokens_ok(layer->d, T);
+    if (rc) return rc;
+    const WsPlan p = plan_ws(layer->d, T);
+    cudaStream_t st = S(stream);
+    if (cudaMemcpyAsync(flags, static_cast<const char*>(ws) + p.err, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return fail(COLI_E_CUDA, "status: read failed");
+    if (*flags & kErrWaitTimeout) return fail(COLI_E_TIMEOUT, "a device-side wait timed out; the outputs are invalid");
+    return COLI_OK;
 }
 
 // ---------------------------------------------------------------------------

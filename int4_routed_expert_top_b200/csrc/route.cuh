@@ -234,6 +234,7 @@ struct UnionOut {
     int32_t* n_units;      // [1]
     int32_t* counters;     // combine counters to clear, or nullptr
     int32_t n_counters;
+    int32_t* err;          // device error flags to clear, or nullptr
     int32_t n_shared;
 };
 
@@ -252,6 +253,7 @@ __device__ __forceinline__ void union_body(const int32_t* idx, int T, int k, int
     for (int i = tid; i < E; i += kUnionThreads) cnt[i] = 0;
     if (o.counters)
         for (int i = tid; i < o.n_counters; i += kUnionThreads) o.counters[i] = 0;
+    if (o.err && tid == 0) *o.err = 0;
     __syncthreads();
     const int P = T * k;
     for (int i = tid; i < P; i += kUnionThreads) {
