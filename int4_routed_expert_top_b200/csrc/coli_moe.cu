@@ -188,7 +188,7 @@ int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int
 
 template <int NT, bool GS>
 int launch_gateup_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
-    const int smem = gemv_ring_bytes<true, GS>() + gemv_act_bytes(NT, d.H);
+    const int smem = gemv_ring_bytes<true, GS>() + gemv_act_bytes(a.tok_cap, d.H);
     int rc = set_smem((const void*)gateup_gemv_kernel<NT, GS>, smem);
     if (rc) return rc;
     gateup_gemv_kernel<NT, GS><<<units_max * (d.I / 64), kGemvThreads, smem, st>>>(a);
@@ -197,7 +197,7 @@ int launch_gateup_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cu
 
 template <int NT, bool GS>
 int launch_down_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
-    const int smem = gemv_ring_bytes<false, GS>() + gemv_act_bytes(NT, d.I);
+    const int smem = gemv_ring_bytes<false, GS>() + gemv_act_bytes(a.tok_cap, d.I);
     int rc = set_smem((const void*)down_gemv_kernel<NT, GS>, smem);
     if (rc) return rc;
     down_gemv_kernel<NT, GS><<<units_max * (d.H / 64) * kDownSplit, kGemvThreads, smem, st>>>(a);
@@ -228,6 +228,7 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
     a.residual = residual;
     a.y = y;
     a.err = at<int32_t>(ws, p.err);
+    a.tok_cap = std::min(T <= 4 ? 4 : 8, T);
     a.T = T; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;

@@ -84,6 +84,7 @@ struct GemvArgs {
     const float* residual;
     float* y;
     int32_t* err;         // device error flags
+    int tok_cap;          // activation rows staged per pass (shared memory is sized for it)
     int T, k, n_shared;
     int H, I, group;
 };
@@ -291,7 +292,7 @@ __device__ __forceinline__ void stage_rows(const __half* __restrict__ q, const f
 // dynamic shared memory: ring + staged activations of one pass
 template <bool TWO, bool GS>
 __host__ __device__ constexpr int gemv_ring_bytes() { return kStages * Stage<TWO, GS>::kBytes; }
-__host__ __device__ inline int gemv_act_bytes(int NT, int K) { return 4 * NT * (K / 64) * (128 * 2 + 4); }
+__host__ __device__ inline int gemv_act_bytes(int tok_cap, int K) { return tok_cap * (K / 64) * (128 * 2 + 4); }
 
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU.  After the shuffle, lane (g, t < 2) holds rows g, g + 8 of
@@ -315,10 +316,10 @@ gateup_gemv_kernel(GemvArgs a) {
     const float* sB = reinterpret_cast<const float*>(blob + a.L.scales[1]);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = a.H / 64;
-    const int passes = (p1 - p0 + 4 * NT - 1) / (4 * NT);
+    const int passes = (p1 - p0 + a.tok_cap - 1) / a.tok_cap;
     uint8_t* ring = gv_smem;
     __half* xs = reinterpret_cast<__half*>(gv_smem + gemv_ring_bytes<true, GS>());
-    float* xi = reinterpret_cast<float*>(xs + (size_t)4 * NT * KB * 128);
+    float* xi = reinterpret_cast<float*>(xs + (size_t)a.tok_cap * KB * 128);
     const int rt = (rb64 * 64) / kTileRows, b8_0 = ((rb64 * 64) % kTileRows) / 16;
 
     if (threadIdx.x == 0) {
@@ -345,8 +346,8 @@ gateup_gemv_kernel(GemvArgs a) {
     }
 
     int pass = 0;
-    for (int pc = p0; pc < p1; pc += 4 * NT, ++pass) {
-        const int tc = min(4 * NT, p1 - pc);
+    for (int pc = p0; pc < p1; pc += a.tok_cap, ++pass) {
+        const int tc = min(a.tok_cap, p1 - pc);
         named_sync(32 * kConsumers);  // the previous pass is done with xs, xi, src, wmax
         if (threadIdx.x < tc) src[threadIdx.x] = a.pair_tok[pc + threadIdx.x];
         named_sync(32 * kConsumers);
@@ -439,10 +440,10 @@ down_gemv_kernel(GemvArgs a) {
     const int KB = a.I / 64;
     const int kb0 = half * KB / kDownSplit, kb1 = (half + 1) * KB / kDownSplit;
     const int n = kb1 - kb0;
-    const int passes = (p1 - p0 + 4 * NT - 1) / (4 * NT);
+    const int passes = (p1 - p0 + a.tok_cap - 1) / a.tok_cap;
     uint8_t* ring = gv_smem;
     __half* xs = reinterpret_cast<__half*>(gv_smem + gemv_ring_bytes<false, GS>());
-    float* xi = reinterpret_cast<float*>(xs + (size_t)4 * NT * KB * 128);
+    float* xi = reinterpret_cast<float*>(xs + (size_t)a.tok_cap * KB * 128);
     const int rt = (rb64 * 64) / kTileRows, b8_0 = ((rb64 * 64) % kTileRows) / 16;
 
     if (threadIdx.x == 0) {
@@ -460,8 +461,8 @@ down_gemv_kernel(GemvArgs a) {
     const int g = lane >> 2, t = lane & 3;
     const int row0 = rb64 * 64 + warp * 16;
     int pass = 0;
-    for (int pc = p0; pc < p1; pc += 4 * NT, ++pass) {
-        const int tc = min(4 * NT, p1 - pc);
+    for (int pc = p0; pc < p1; pc += a.tok_cap, ++pass) {
+        const int tc = min(a.tok_cap, p1 - pc);
         named_sync(32 * kConsumers);
         if (threadIdx.x < tc) src[threadIdx.x] = pc + threadIdx.x;
         named_sync(32 * kConsumers);
