@@ -240,7 +240,7 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert,
  * exits.  x, y and the layer's buffers are still the caller's.
  *  - T is limited to what fits: a call whose coli_moe_workspace_size(layer, T)
  *    exceeds COLI_NOALLOC_SCRATCH_BYTES returns COLI_E_UNSUPPORTED (for the
- *    GLM-5.2 shapes that is T <= 24 tokens).
+ *    GLM-5.2 shapes that is T <= 22 tokens).
  *  - The first call on each device looks up that device's copy of the array
  *    (cudaGetSymbolAddress with the device current); make that first call before
  *    any stream capture.  Later calls only launch kernels.

@@ -56,7 +56,7 @@ bool shape_ok(int H, int I, int group) {
 struct WsPlan {
     int64_t zpart, idx, w, offsets, pair_tok, pair_slot, uniq, n_uniq, inv;
     int64_t unit_expert, unit_begin, unit_end, n_units, counters, err;
-    int64_t xq, xinv, hq, hinv, o, total;
+    int64_t xq, xinv, hq, hinv, o, xg, hg, hmax, hsc, total;
 };
 
 WsPlan plan_ws(const coli_moe_desc& d, int T) {
@@ -85,6 +85,11 @@ WsPlan plan_ws(const coli_moe_desc& d, int T) {
     p.hq = take(P * d.I * 4);                   // fp16 hi + lo
     p.hinv = take(P * (d.I / 64) * 4);
     p.o = take(P * d.H * 4);
+    p.xg = p.o;                                 // tensor-core path: gathered fp16 tokens (dead
+                                                //   before the down pass writes o)
+    p.hg = take(P * d.I * 2);                   //   fp16 h of every pair
+    p.hmax = take(P * 4);                       //   per-pair max |h|
+    p.hsc = take(P * 4);                        //   per-pair inverse scale of h
     p.total = off;
     return p;
 }
@@ -185,6 +190,107 @@ int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int
     if (rc) return rc;
     return launch_union(idx, T, d.k, d.E, o, st);
 }
+
+// ---------------------------------------------------------------------------
+// tensor-core path
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// [rows][cols] fp16, boxes of 16 rows x 64 columns, 128-byte swizzle
+int encode_b_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(COLI_E_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(COLI_E_CUDA, "tensor map encode failed (%d)", (int)r);
+    return COLI_OK;
+}
+
+int gemm_grid() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    return sms;
+}
+
+template <typename Mark>
+int launch_gemm(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, cudaStream_t st,
+                Mark&& mark) {
+    const coli_moe_desc& d = l->d;
+    const int P = T * (d.k + d.n_shared);
+    int rc;
+    {
+        const int64_t n = (int64_t)P * (d.H / 8);
+        gather_x_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+            at<__half>(ws, p.xq), at<int32_t>(ws, p.pair_tok), P, d.H, at<__half>(ws, p.xg),
+            at<uint32_t>(ws, p.hmax));
+        if ((rc = check_launch("gather x"))) return rc;
+    }
+    if ((rc = set_smem((const void*)moe_gemm_kernel, kGemmSmem))) return rc;
+    GemmArgs g;
+    g.experts = static_cast<const uint8_t*>(d.experts);
+    g.blob_bytes = l->L.bytes;
+    g.L = l->L;
+    g.n_units = at<int32_t>(ws, p.n_units);
+    g.unit_expert = at<int32_t>(ws, p.unit_expert);
+    g.unit_begin = at<int32_t>(ws, p.unit_begin);
+    g.unit_end = at<int32_t>(ws, p.unit_end);
+    g.pair_tok = at<int32_t>(ws, p.pair_tok);
+    g.group = d.group;
+    g.hf = at<float>(ws, p.hq);
+    g.hmax = at<uint32_t>(ws, p.hmax);
+    g.o = at<float>(ws, p.o);
+    g.err = at<int32_t>(ws, p.err);
+    g.I = d.I; g.H = d.H;
+    CUtensorMap xmap, hmap;
+    if ((rc = encode_b_map(&xmap, at<__half>(ws, p.xg), P, d.H))) return rc;
+    g.two = 1; g.K = d.H; g.R = d.I;
+    g.act_inv = at<float>(ws, p.xinv);
+    moe_gemm_kernel<<<gemm_grid(), kGemmThreads, kGemmSmem, st>>>(xmap, g);
+    if ((rc = check_launch("gate/up gemm"))) return rc;
+    if ((rc = mark(COLI_STAGE_DOWN))) return rc;
+    {
+        const int64_t n = (int64_t)P * d.I / 2;
+        convert_h_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+            at<float>(ws, p.hq), at<uint32_t>(ws, p.hmax), P, d.I, at<__half>(ws, p.hg),
+            at<float>(ws, p.hsc));
+        if ((rc = check_launch("convert h"))) return rc;
+    }
+    if ((rc = encode_b_map(&hmap, at<__half>(ws, p.hg), P, d.I))) return rc;
+    g.two = 0; g.K = d.I; g.R = d.H;
+    g.act_inv = at<float>(ws, p.hsc);
+    moe_gemm_kernel<<<gemm_grid(), kGemmThreads, kGemmSmem, st>>>(hmap, g);
+    return check_launch("down gemm");
+}
+
+// tensor cores from this many tokens on (the GEMV path below)
+constexpr int kGemmMinTokens = 48;
+bool gemm_path_preferred(const coli_moe_desc&, int T) { return T >= kGemmMinTokens; }
 
 template <int NT, bool GS>
 int launch_gateup_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
@@ -425,8 +531,8 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     const bool gemm = path == COLI_PATH_GEMM;
     int KS;
     if ((rc = mark(COLI_STAGE_ROUTER))) return rc;
-    if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart),
-                            gemm ? nullptr : at<__half>(ws, p.xq), at<float>(ws, p.xinv), st, &KS)))
+    if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), at<__half>(ws, p.xq),
+                            at<float>(ws, p.xinv), st, &KS)))
         return rc;
     UnionOut o{};
     o.offsets = at<int32_t>(ws, p.offsets);
@@ -447,18 +553,13 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     if ((rc = launch_select(d, at<float>(ws, p.zpart), KS, T, idx, w, o, st))) return rc;
     if ((rc = mark(COLI_STAGE_GATEUP))) return rc;
     if (gemm) {
-        GemmCtx g;
-        g.experts = static_cast<const uint8_t*>(d.experts);
-        g.blob_bytes = layer->L.bytes;
-        g.L = layer->L;
-        g.H = d.H; g.I = d.I; g.group = d.group; g.E = d.E; g.n_shared = d.n_shared;
-        g.T = T; g.k = d.k;
-        g.n_units = o.n_units; g.unit_expert = o.unit_expert;
-        g.unit_begin = o.unit_begin; g.unit_end = o.unit_end; g.pair_tok = o.pair_tok;
-        g.x = x; g.x_bf16 = xt == COLI_BF16;
-        g.o = at<float>(ws, p.o);
-        if ((rc = launch_gemm(g, st, mark))) return fail(rc, "forward: tensor-core path not available");
+        if ((rc = launch_gemm(layer, T, ws, p, st, mark))) return rc;
         if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
+        const int64_t n4 = (int64_t)T * (d.H / 4);
+        combine_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
+            at<float>(ws, p.o), at<int32_t>(ws, p.inv), at<float>(ws, p.w), T, d.k, d.n_shared,
+            d.H, residual, y);
+        if ((rc = check_launch("combine"))) return rc;
     } else {
         if ((rc = launch_gemv(layer, T, ws, p, residual, y, st, mark))) return rc;
         if ((rc = mark(COLI_STAGE_COMBINE))) return rc;   // combine is fused into the down pass

@@ -39,29 +39,6 @@ constexpr int kStages = 8;
 constexpr int kGemvMaxNT = 2;   // up to 2 column groups of 8: 8 tokens per pass
 constexpr int kDownSplit = 2;   // the down reduction is split in halves
 
-// fp16 magic constants of the nibble decode, passed as kernel parameters so
-// they are read from the parameter bank instead of being rebuilt per use
-struct DecodeK {
-    uint32_t xlo = 0x64086408u;   // sign flip of a nibble at bits 0-3 + fp16 exponent of 1024
-    uint32_t xhi = 0x64806480u;   // same for a nibble at bits 4-7
-    uint32_t sub = 0x64086408u;   // 1032 = 1024 + 8
-    uint32_t mul = 0x2C002C00u;   // 1/16
-    uint32_t add = 0xD480D480u;   // -72 = -(1024 + 8*16)/16
-};
-
-__device__ __forceinline__ void decode_word(uint32_t w, uint32_t a[4], const DecodeK& k) {
-    const uint32_t w8 = w >> 8;
-    uint32_t t0, t1, t2, t3;
-    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t0) : "r"(w), "r"(k.xlo));
-    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t1) : "r"(w8), "r"(k.xlo));
-    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t2) : "r"(w), "r"(k.xhi));
-    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t3) : "r"(w8), "r"(k.xhi));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(a[0]) : "r"(t0), "r"(k.sub));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(a[1]) : "r"(t1), "r"(k.sub));
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(a[2]) : "r"(t2), "r"(k.mul), "r"(k.add));
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(a[3]) : "r"(t3), "r"(k.mul), "r"(k.add));
-}
-
 struct GemvArgs {
     const uint8_t* experts;
     int64_t blob_bytes;
