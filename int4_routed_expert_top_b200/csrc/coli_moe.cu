@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 #include <string>
 
 #include "coli_moe.h"
@@ -107,11 +108,24 @@ int tokens_ok(const coli_moe_desc& d, int T) {
     return COLI_OK;
 }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` (static + dynamic
+// above 48 KB needs the opt-in).  The largest value set per (device, kernel) is
+// remembered so that a forward normally makes no attribute call.
 int set_smem(const void* fn, int bytes) {
-    if (bytes <= 48 * 1024) return COLI_OK;
+    struct Entry { int dev; const void* fn; int bytes; };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(COLI_E_CUDA, "smem attribute: no device");
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& en : done)
+        if (en.dev == dev && en.fn == fn && en.bytes >= bytes) return COLI_OK;
     const cudaError_t e =
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return fail(COLI_E_CUDA, "smem attribute: %s", cudaGetErrorString(e));
+    for (Entry& en : done)
+        if (en.dev == dev && en.fn == fn) { en.bytes = bytes; return COLI_OK; }
+    done.push_back({dev, fn, bytes});
     return COLI_OK;
 }
 
@@ -334,7 +348,12 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
     a.residual = residual;
     a.y = y;
     a.err = at<int32_t>(ws, p.err);
+    // tokens staged per pass: as many as the MMA tiles take, but ring + staging
+    // must fit one CTA's shared memory for the longer reduction
     a.tok_cap = std::min(T <= 4 ? 4 : 8, T);
+    while (a.tok_cap > 1 &&
+           gemv_ring_bytes<true, true>() + gemv_act_bytes(a.tok_cap, std::max(d.H, d.I)) > kGemvSmemMax)
+        --a.tok_cap;
     a.T = T; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int units_max = (int)std::min<int64_t>(d.E, (int64_t)T * d.k) + d.n_shared;

@@ -3,25 +3,28 @@
 // work to be a dense contraction.
 //
 // Orientation ("swap AB"): D[r, n] = sum_k W[r, k] * X[n, k] with the weight
-// rows as the MMA M dimension (a 128-row tile) and the unit's tokens as N, so a
-// unit with few tokens does not waste a 128-token tile.  Per CTA (persistent,
-// one per SM, all 512 TMEM columns):
-//   warp 0      producer: 1-D bulk copies of the int4 fragment tiles of a
-//               128-row tile and one 64-column step (4 KB per matrix, plus the
-//               step's scales for gs64) and 2-D TMA loads of the B tile (the
-//               unit's tokens as fp16, 128-byte swizzle) into a 4-stage ring;
-//   warp 1      one lane issues tcgen05.mma (kind::f16, f32 accumulators in
-//               TMEM) with A read from TMEM and B from shared memory;
-//   warps 4-7   decode matrix 0 (gate, or down): each lane turns its 16-byte
-//               unit into exact fp16 (q, or q*s for gs64) and writes it to TMEM
-//               with tcgen05.st.16x256b, whose lane/column layout is that of the
-//               fragment tiles; these warps also run the epilogue;
-//   warps 8-11  decode matrix 1 (up) for the gate/up pass.
-// TMEM columns: D0 [0, 128), D1 [128, 256), A stage s at 256 + 64 s (matrix 0)
-// and 256 + 64 s + 32 (matrix 1).
+// rows as the MMA M dimension (a 128-row tile) and up to 64 of a unit's tokens
+// as N.  At these batch sizes the layer streams every expert once and does
+// little arithmetic per weight byte, so the kernel is built to keep HBM busy and
+// the int4 decode off the critical path.  Per CTA (persistent, one per SM, all
+// 512 TMEM columns, 24 warps):
+//   warp 0       producer: 1-D bulk copies of the int4 fragment tiles (8 KB a
+//                stage: gate and up of one 64-column step, or two steps of down)
+//                with their gs64 scales, and 2-D TMA loads of the tokens (fp16,
+//                128-byte swizzle) into an 8-stage ring;
+//   warp 1       one lane issues tcgen05.mma (kind::f16, f32 accumulators in
+//                TMEM), A from TMEM and B from shared memory;
+//   warps 4-7    epilogue: TMEM accumulators -> registers -> global;
+//   warps 8-23   decode: each warp turns one 16-row x 64-column unit block of a
+//                stage (512 B of nibbles) into exact fp16 (q, or q*s for gs64)
+//                and writes it to TMEM with tcgen05.st.16x256b, whose lane and
+//                column layout is that of the fragment tiles.
+// TMEM columns: accumulators [0, 256) as two buffers of 128 (gate at +0, up at
+// +64; down at +0), so the epilogue of one tile overlaps the next tile's main
+// loop; A stages at 256 + 64 a (a = 0..3), 32 columns per slot.
 //
 // Epilogues: gate/up writes h = silu(a) * u in f32 and the per-pair max |h|;
-// down writes o in f32.  Weight scales (per row) and the activations' powers of
+// down writes o in f32.  Per-row weight scales and the activations' powers of
 // two are applied there in f32.
 #pragma once
 
@@ -33,16 +36,20 @@
 
 namespace coli {
 
-constexpr int kGemmThreads = 384;
-constexpr int kGemmStages = 4;
-constexpr int kGemmMaxN = 128;
-constexpr int kStageB = 16384;                       // B tile: up to 128 rows x 128 B
-constexpr int kStageCodes = 4096;                    // one matrix, 128 rows x 64 columns
-constexpr int kStageBytes = kStageB + 2 * kStageCodes + 2 * 512;   // 25600, 1 KB multiple
-// + alignment slack; the request is kept above half of the SM's shared memory so
-// that exactly one CTA (which takes all 512 TMEM columns) is resident per SM
-constexpr int kGemmSmem = 120 * 1024;
-static_assert(kGemmStages * kStageBytes + 1024 <= kGemmSmem, "gemm ring does not fit");
+constexpr int kGemmThreads = 768;
+constexpr int kGemmStages = 8;                        // shared-memory ring
+constexpr int kGemmAStages = 4;                       // TMEM A ring
+constexpr int kGemmMaxN = 64;                         // tokens per tile
+constexpr int kGemmDecodeWarp0 = 8;
+constexpr int kGemmDecodeWarps = 16;
+constexpr int kGemmEpiWarp0 = 4;
+constexpr int kAtomBytes = kGemmMaxN * 128;           // one 64-column B atom, 64 rows
+constexpr int kStageB = 2 * kAtomBytes;               // two atoms (down: two k-steps)
+constexpr int kStageCodes = 2 * 4096;                 // two 128 x 64 nibble blocks
+constexpr int kStageScales = 2 * 512;
+constexpr int kStageBytes = kStageB + kStageCodes + kStageScales;   // 25600, 1 KB multiple
+constexpr int kGemmSmem = kGemmStages * kStageBytes + 1024;        // + alignment slack
+static_assert(kStageBytes % 1024 == 0, "stages must stay 1 KB aligned for the swizzle");
 constexpr uint32_t kTmemCols = 512;
 
 struct GemmArgs {
@@ -88,6 +95,29 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a, uint64_t bdesc
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}"
         ::"r"(d), "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+// elected-lane forms (see pipeline.cuh): the whole warp executes them
+__device__ __forceinline__ void tc_commit_elect(uint64_t* bar) {
+    asm volatile(
+        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+        " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}"
+        ::"r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts_elect(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}"
+        ::"r"(d), "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void tma_load_2d_elect(void* dst, const CUtensorMap* map, int x, int y,
+                                                  uint64_t* bar) {
+    asm volatile(
+        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+        " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n}"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t r[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
@@ -131,24 +161,40 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
     return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// tile index -> (unit, first token of the n-tile, n, row tile); tiles are
-// ordered unit by unit, n-tile by n-tile, row tile fastest
-__device__ __forceinline__ bool gemm_tile(const GemmArgs& a, int n_units, int idx, int& u, int& p0,
-                                          int& n, int& rt) {
-    const int RT = a.R / kTileRows;
-    for (u = 0; u < n_units; ++u) {
-        const int b = a.unit_begin[u], e = a.unit_end[u];
-        const int nt = (e - b + kGemmMaxN - 1) / kGemmMaxN;
-        if (idx < nt * RT) {
-            const int j = idx / RT;
-            rt = idx % RT;
-            p0 = b + j * kGemmMaxN;
-            n = min(kGemmMaxN, e - p0);
-            return true;
+// Walks the tiles of one CTA in increasing order: unit by unit, N tile by N
+// tile, row tile fastest (so CTAs running at the same time share a unit's
+// tokens in L2).  The cursor only moves forward, so a CTA scans the unit list
+// once.
+struct TileCursor {
+    int u = 0, base = 0;
+    __device__ __forceinline__ bool next(const GemmArgs& a, int n_units, int RT, int tile, int& p0,
+                                         int& n, int& rt) {
+        for (; u < n_units; ++u) {
+            const int b = a.unit_begin[u], e = a.unit_end[u];
+            const int cnt = (e - b + kGemmMaxN - 1) / kGemmMaxN * RT;
+            if (tile < base + cnt) {
+                const int idx = tile - base, j = idx / RT;
+                rt = idx - j * RT;
+                p0 = b + j * kGemmMaxN;
+                n = min(kGemmMaxN, e - p0);
+                return true;
+            }
+            base += cnt;
         }
-        idx -= nt * RT;
+        return false;
     }
-    return false;
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ float lds32f(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -156,26 +202,31 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
     extern __shared__ uint8_t gm_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gm_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages];
-    __shared__ __align__(8) uint64_t afull[kGemmStages], aempty[kGemmStages];
-    __shared__ __align__(8) uint64_t accfull, accempty;
+    __shared__ __align__(8) uint64_t afull[kGemmAStages], aempty[kGemmAStages];
+    __shared__ __align__(8) uint64_t accfull[2], accempty[2];
     __shared__ uint32_t tmem_slot;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_units = *a.n_units;
     const int KB = a.K / 64;
     const int ng = a.group ? KB : 1;
-    const int ndec = a.two ? 8 : 4;  // decode warps
+    const int KS = a.two ? KB : KB / 2;          // ring stages per tile
+    const int RT = a.R / kTileRows;
     const int mA = a.two ? 0 : 2;
 
     if (warp == 0) tmem_alloc(&tmem_slot, kTmemCols);
     if (threadIdx.x == 32) {
         for (int s = 0; s < kGemmStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], ndec + 1);
-            mbar_init(&afull[s], ndec);
+            mbar_init(&empty[s], kGemmDecodeWarps + 1);
+        }
+        for (int s = 0; s < kGemmAStages; ++s) {
+            mbar_init(&afull[s], kGemmDecodeWarps);
             mbar_init(&aempty[s], 1);
         }
-        mbar_init(&accfull, 1);
-        mbar_init(&accempty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accfull[b], 1);
+            mbar_init(&accempty[b], 4);
+        }
         fence_mbar_init();
     }
     tc_fence_before();
@@ -183,160 +234,195 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
     bool ok = true;  // cleared by a timed-out wait: then no further waits, every barrier kept
+    TileCursor cur;
 
     if (warp == 0) {
-      if (lane == 0) {
-        // ---------------- producer ----------------
-        int it = 0;
-        for (int tile = blockIdx.x;; tile += gridDim.x) {
-            int u, p0, n, rt;
-            if (!gemm_tile(a, n_units, tile, u, p0, n, rt)) break;
-            const uint8_t* blob = a.experts + (int64_t)a.unit_expert[u] * a.blob_bytes;
+        // ---------------- producer (whole warp, elected lane issues) ----------------
+        int u = 0;
+        int p0, n, rt;
+        for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x) {
+            const uint8_t* blob = a.experts + (int64_t)a.unit_expert[cur.u] * a.blob_bytes;
             const uint8_t* c0 = blob + a.L.codes[mA];
             const uint8_t* c1 = blob + a.L.codes[1];
             const float* s0 = reinterpret_cast<const float*>(blob + a.L.scales[mA]);
             const float* s1 = reinterpret_cast<const float*>(blob + a.L.scales[1]);
             const int nb = (n + 15) / 16;
-            const uint32_t bytes = (uint32_t)(nb * 2048 + kStageCodes * (a.two ? 2 : 1) +
-                                              (a.group ? 512 * (a.two ? 2 : 1) : 0));
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-                const int s = it % kGemmStages;
-                if (it >= kGemmStages && ok && !mbar_wait(&empty[s], ((it / kGemmStages) - 1) & 1, a.err)) ok = false;
+            const uint32_t bytes = (uint32_t)(kStageCodes + (a.group ? kStageScales : 0) +
+                                              nb * 2048 * (a.two ? 1 : 2));
+            for (int ks = 0; ks < KS; ++ks, ++u) {
+                const int s = u % kGemmStages;
+                if (u >= kGemmStages && ok && !mbar_wait_warp(&empty[s], ((u / kGemmStages) - 1) & 1, a.err)) ok = false;
                 uint8_t* st = smem + s * kStageBytes;
-                mbar_expect_tx(&full[s], bytes);
-                const int64_t uoff = frag_unit_offset(rt, kb, 0, 0, a.K);
-                bulk_g2s(st + kStageB, c0 + uoff, kStageCodes, &full[s]);
-                if (a.two) bulk_g2s(st + kStageB + kStageCodes, c1 + uoff, kStageCodes, &full[s]);
-                if (a.group) {
-                    const int64_t soff = ((int64_t)rt * ng + kb) * kTileRows;
-                    bulk_g2s(st + kStageB + 2 * kStageCodes, s0 + soff, 512, &full[s]);
-                    if (a.two) bulk_g2s(st + kStageB + 2 * kStageCodes + 512, s1 + soff, 512, &full[s]);
+                uint8_t* sc = st + kStageB;
+                mbar_expect_tx_elect(&full[s], bytes);
+                if (a.two) {
+                    const int64_t uoff = frag_unit_offset(rt, ks, 0, 0, a.K);
+                    bulk_g2s_elect(sc, c0 + uoff, 4096, &full[s]);
+                    bulk_g2s_elect(sc + 4096, c1 + uoff, 4096, &full[s]);
+                    if (a.group) {
+                        const int64_t soff = ((int64_t)rt * ng + ks) * kTileRows;
+                        bulk_g2s_elect(sc + kStageCodes, s0 + soff, 512, &full[s]);
+                        bulk_g2s_elect(sc + kStageCodes + 512, s1 + soff, 512, &full[s]);
+                    }
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d_elect(st + i * 2048, &bmap, ks * 64, p0 + 16 * i, &full[s]);
+                } else {
+                    // two consecutive 64-column steps of down: contiguous in the layout
+                    const int kb = 2 * ks;
+                    bulk_g2s_elect(sc, c0 + frag_unit_offset(rt, kb, 0, 0, a.K), kStageCodes, &full[s]);
+                    if (a.group)
+                        bulk_g2s_elect(sc + kStageCodes, s0 + ((int64_t)rt * ng + kb) * kTileRows, kStageScales,
+                                       &full[s]);
+                    for (int h = 0; h < 2; ++h)
+                        for (int i = 0; i < nb; ++i)
+                            tma_load_2d_elect(st + h * kAtomBytes + i * 2048, &bmap, (kb + h) * 64, p0 + 16 * i,
+                                              &full[s]);
                 }
-                for (int i = 0; i < nb; ++i) tma_load_2d(st + i * 2048, &bmap, kb * 64, p0 + 16 * i, &full[s]);
             }
         }
-      }
-      __syncwarp();
     } else if (warp == 1) {
-      if (lane == 0) {
-        // ---------------- MMA issuer ----------------
-        int it = 0, tcount = 0;
-        for (int tile = blockIdx.x;; tile += gridDim.x, ++tcount) {
-            int u, p0, n, rt;
-            if (!gemm_tile(a, n_units, tile, u, p0, n, rt)) break;
+        // ---------------- MMA issuer (whole warp, elected lane issues) ----------------
+        int u = 0, tcount = 0;
+        int p0, n, rt;
+        for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x, ++tcount) {
             const int np = (n + 15) / 16 * 16;  // N: multiple of 16 for M = 128
             const uint32_t idesc = idesc_f16_f32(np);
-            if (tcount > 0 && ok && !mbar_wait(&accempty, (tcount - 1) & 1, a.err)) ok = false;
+            const int buf = tcount & 1;
+            if (tcount >= 2 && ok && !mbar_wait_warp(&accempty[buf], ((tcount >> 1) - 1) & 1, a.err)) ok = false;
             tc_fence_after();
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-                const int s = it % kGemmStages;
-                if (ok && !mbar_wait(&afull[s], (it / kGemmStages) & 1, a.err)) ok = false;
-                if (ok && !mbar_wait(&full[s], (it / kGemmStages) & 1, a.err)) ok = false;
+            const uint32_t dacc = tmem + 128 * buf;
+            for (int ks = 0; ks < KS; ++ks, ++u) {
+                const int s = u % kGemmStages, as = u % kGemmAStages;
+                if (ok && !mbar_wait_warp(&afull[as], (u / kGemmAStages) & 1, a.err)) ok = false;
+                if (ok && !mbar_wait_warp(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
                 tc_fence_after();
                 const uint64_t bdesc = smem_desc_sw128(smem + s * kStageBytes);
-                const uint32_t a0 = tmem + 256 + 64 * s;
+                const uint32_t a0 = tmem + 256 + 64 * as;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
-                    tc_mma_ts(tmem + 0, a0 + 8 * j, bdesc + 2 * j, idesc, acc);
-                    if (a.two) tc_mma_ts(tmem + 128, a0 + 32 + 8 * j, bdesc + 2 * j, idesc, acc);
-                }
-                tc_commit(&aempty[s]);
-                tc_commit(&empty[s]);
-            }
-            tc_commit(&accfull);
-        }
-      }
-      __syncwarp();
-    } else if (warp >= 4 && warp < 4 + ndec) {
-        // ---------------- decode (+ epilogue on warps 4-7) ----------------
-        const int grp = (warp - 4) / 4;           // 0: matrix 0, 1: matrix 1
-        const int q = warp & 3;                   // TMEM lane quarter of this warp
-        const int g = lane >> 2;
-        const DecodeK dk = a.dk;
-        int it = 0, tcount = 0;
-        for (int tile = blockIdx.x;; tile += gridDim.x, ++tcount) {
-            int u, p0, n, rt;
-            if (!gemm_tile(a, n_units, tile, u, p0, n, rt)) break;
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-                const int s = it % kGemmStages;
-                if (ok && !mbar_wait(&full[s], (it / kGemmStages) & 1, a.err)) ok = false;
-                if (it >= kGemmStages && ok && !mbar_wait(&aempty[s], ((it / kGemmStages) - 1) & 1, a.err)) ok = false;
-                tc_fence_after();
-                const uint8_t* st = smem + s * kStageBytes + kStageB + grp * kStageCodes;
-                const float* ss = reinterpret_cast<const float*>(smem + s * kStageBytes + kStageB + 2 * kStageCodes + grp * 512);
-#pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int b8 = 2 * q + hb;
-                    const uint4 un = reinterpret_cast<const uint4*>(st)[b8 * 32 + lane];
-                    const uint32_t wd[4] = {un.x, un.y, un.z, un.w};
-                    uint32_t r[16];
+                for (int slot = 0; slot < 2; ++slot)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        uint32_t f[4];
-                        decode_word(wd[j], f, dk);
-                        // 16x256b register order: (row g, c0..c0+1), (row g, c0+2..),
-                        // (row g+8, c0..), (row g+8, c0+2..)
-                        r[4 * j + 0] = f[0]; r[4 * j + 1] = f[2];
-                        r[4 * j + 2] = f[1]; r[4 * j + 3] = f[3];
-                    }
-                    if (a.group) {  // gs64: A = fp16(q * s)
-                        const __half2 s0 = __float2half2_rn(ss[b8 * 16 + g]);
-                        const __half2 s1 = __float2half2_rn(ss[b8 * 16 + g + 8]);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            __half2* h = reinterpret_cast<__half2*>(r + 4 * j);
-                            h[0] = __hmul2(h[0], s0); h[1] = __hmul2(h[1], s0);
-                            h[2] = __hmul2(h[2], s1); h[3] = __hmul2(h[3], s1);
+                        if (a.two) {
+                            tc_mma_ts_elect(dacc + 64 * slot, a0 + 32 * slot + 8 * j, bdesc + 2 * j, idesc,
+                                            (ks > 0 || j > 0) ? 1u : 0u);
+                        } else {
+                            tc_mma_ts_elect(dacc, a0 + 32 * slot + 8 * j,
+                                            bdesc + (uint64_t)((slot * kAtomBytes) >> 4) + 2 * j, idesc,
+                                            (ks > 0 || slot > 0 || j > 0) ? 1u : 0u);
                         }
                     }
-                    const uint32_t taddr = tmem + ((uint32_t)(32 * q + 16 * hb) << 16) + 256 + 64 * s + 32 * grp;
-                    tmem_st_16x256b_x4(taddr, r);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) { mbar_arrive(&afull[s]); mbar_arrive(&empty[s]); }
+                tc_commit_elect(&aempty[as]);
+                tc_commit_elect(&empty[s]);
             }
-            if (grp != 0) continue;
-            // ---------------- epilogue: rows 32q + lane of the tile ----------------
-            if (ok && !mbar_wait(&accfull, tcount & 1, a.err)) ok = false;
-            tc_fence_after();
+            tc_commit_elect(&accfull[buf]);
+        }
+    } else if (warp >= kGemmEpiWarp0 && warp < kGemmEpiWarp0 + 4) {
+        // ---------------- epilogue: rows 32q + lane of the tile ----------------
+        const int q = warp & 3;
+        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+        int tcount = 0;
+        int p0, n, rt;
+        for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x, ++tcount) {
+            const int buf = tcount & 1;
             const int row = rt * kTileRows + 32 * q + lane;
-            const uint8_t* blob = a.experts + (int64_t)a.unit_expert[u] * a.blob_bytes;
+            const uint8_t* blob = a.experts + (int64_t)a.unit_expert[cur.u] * a.blob_bytes;
             const float srow0 = a.group ? 1.0f
                 : __ldg(reinterpret_cast<const float*>(blob + a.L.scales[mA]) + scale_offset(row, 0, 1));
             const float srow1 = (a.group || !a.two) ? 1.0f
                 : __ldg(reinterpret_cast<const float*>(blob + a.L.scales[1]) + scale_offset(row, 0, 1));
-            const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+            // the activation scale of columns lane and 32 + lane, broadcast below
+            float cinv[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c = 32 * h + lane;
+                cinv[h] = 0.0f;
+                if (c < n) {
+                    const int p = p0 + c;
+                    cinv[h] = a.two ? __ldg(a.act_inv + (int64_t)a.pair_tok[p] * (a.H / 64))
+                                    : __ldg(a.act_inv + p);
+                }
+            }
+            if (ok && !mbar_wait_warp(&accfull[buf], (tcount >> 1) & 1, a.err)) ok = false;
+            tc_fence_after();
+            const uint32_t dacc = tmem + lane_off + 128 * buf;
             for (int c0 = 0; c0 < n; c0 += 16) {
                 uint32_t d0[16], d1[16];
-                tmem_ld_32x32b_x16(tmem + lane_off + c0, d0);
-                if (a.two) tmem_ld_32x32b_x16(tmem + lane_off + 128 + c0, d1);
+                tmem_ld_32x32b_x16(dacc + c0, d0);
+                if (a.two) tmem_ld_32x32b_x16(dacc + 64 + c0, d1);
                 tmem_wait_ld();
+                const float ci = c0 < 32 ? cinv[0] : cinv[1];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int nn = c0 + i;
-                    const bool valid = nn < n;
-                    const int p = p0 + (valid ? nn : 0);
+                    const float inv = __shfl_sync(0xffffffffu, ci, (c0 + i) & 31);
+                    if (nn >= n) continue;               // uniform across the warp
+                    const int64_t p = p0 + nn;
                     if (a.two) {
-                        const float inv = valid ? __ldg(a.act_inv + (int64_t)a.pair_tok[p] * (a.H / 64)) : 0.f;
                         const float ga = __uint_as_float(d0[i]) * srow0 * inv;
                         const float ua = __uint_as_float(d1[i]) * srow1 * inv;
                         const float h = silu_f(ga) * ua;
-                        if (valid) a.hf[(int64_t)p * a.I + row] = h;
-                        float m = valid ? fabsf(h) : 0.0f;
+                        a.hf[p * a.I + row] = h;
+                        float m = fabsf(h);
 #pragma unroll
                         for (int o2 = 16; o2 > 0; o2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o2));
-                        if (lane == 0 && valid) atomicMax(a.hmax + p, __float_as_uint(m));
-                    } else if (valid) {
-                        a.o[(int64_t)p * a.H + row] = __uint_as_float(d0[i]) * srow0 * __ldg(a.act_inv + p);
+                        if (lane == 0) atomicMax(a.hmax + p, __float_as_uint(m));
+                    } else {
+                        a.o[p * a.H + row] = __uint_as_float(d0[i]) * srow0 * inv;
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&accempty);
+            if (lane == 0) mbar_arrive(&accempty[buf]);
+        }
+    } else if (warp >= kGemmDecodeWarp0) {
+        // ---------------- decode: one 16-row unit block per stage ----------------
+        const int dw = warp - kGemmDecodeWarp0;
+        const int q = warp & 3;                   // TMEM lane quarter of this warp
+        const int hb = (dw >> 2) & 1, slot = dw >> 3;
+        const int b8 = 2 * q + hb;
+        const int g = lane >> 2;
+        const DecodeK dk = a.dk;
+        const uint32_t sbase = smem_u32(smem);
+        const uint32_t tlane = tmem + ((uint32_t)(32 * q + 16 * hb) << 16) + 256 + 32 * slot;
+        int u = 0;
+        int p0, n, rt;
+        for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x) {
+            for (int ks = 0; ks < KS; ++ks, ++u) {
+                const int s = u % kGemmStages, as = u % kGemmAStages;
+                if (ok && !mbar_wait_warp(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
+                if (u >= kGemmAStages && ok && !mbar_wait_warp(&aempty[as], ((u / kGemmAStages) - 1) & 1, a.err)) ok = false;
+                tc_fence_after();
+                const uint32_t sc = sbase + s * kStageBytes + kStageB;
+                const uint4 un = lds128(sc + slot * 4096 + (b8 * 32 + lane) * 16);
+                const uint32_t wd[4] = {un.x, un.y, un.z, un.w};
+                uint32_t r[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t f[4];
+                    decode_word(wd[j], f, dk);
+                    // 16x256b register order: (row g, c0..c0+1), (row g, c0+2..),
+                    // (row g+8, c0..), (row g+8, c0+2..)
+                    r[4 * j + 0] = f[0]; r[4 * j + 1] = f[2];
+                    r[4 * j + 2] = f[1]; r[4 * j + 3] = f[3];
+                }
+                if (a.group) {  // gs64: A = fp16(q * s)
+                    const uint32_t sa = sc + kStageCodes + slot * 512 + (b8 * 16 + g) * 4;
+                    const __half2 s0 = __float2half2_rn(lds32f(sa));
+                    const __half2 s1 = __float2half2_rn(lds32f(sa + 32));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        __half2* h = reinterpret_cast<__half2*>(r + 4 * j);
+                        h[0] = __hmul2(h[0], s0); h[1] = __hmul2(h[1], s0);
+                        h[2] = __hmul2(h[2], s1); h[3] = __hmul2(h[3], s1);
+                    }
+                }
+                tmem_st_16x256b_x4(tlane + 64 * as, r);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) { mbar_arrive(&afull[as]); mbar_arrive(&empty[s]); }
+            }
         }
     }
     tc_fence_before();

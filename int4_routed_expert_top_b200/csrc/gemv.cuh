@@ -5,7 +5,7 @@
 // read from HBM once per launch however many of the unit's tokens use it (batch
 // union, "github一周涨11k⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.4).
 //
-// Data movement: one producer lane streams the unit's fragment tiles with bulk
+// Data movement: a producer warp (one elected lane issuing) streams the unit's fragment tiles with bulk
 // copies (the TMA engine, no tensor map) into an 8-stage shared-memory ring.
 // One stage is one 64-column step of the CTA's 64 rows: 2 KB of codes per matrix
 // (four contiguous 512-byte blocks), plus the step's 64 scales for gs64.  Stages
@@ -75,7 +75,7 @@ struct Stage {
     static constexpr int kBytes = (TWO ? 4096 : 2048) + (GS ? (TWO ? 512 : 256) : 0);
 };
 
-// Producer (one lane): `passes` sweeps over steps kb0 .. kb0+n-1 of the 64 rows
+// Producer (whole warp, elected lane issues): `passes` sweeps over steps kb0 .. kb0+n-1 of the 64 rows
 // starting at 16-row block b8_0 of tile rt.
 template <bool TWO, bool GS>
 __device__ __forceinline__ void gemv_produce(const uint8_t* cA, const uint8_t* cB,
@@ -89,22 +89,22 @@ __device__ __forceinline__ void gemv_produce(const uint8_t* cA, const uint8_t* c
     int it = 0;
     for (; it < total; ++it) {
         const int s = it % kStages;
-        if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, err)) break;
+        if (it >= kStages && !mbar_wait_warp(&empty[s], ((it / kStages) - 1) & 1, err)) break;
         const int kb = kb0 + it % n;
         uint8_t* st = ring + s * S::kBytes;
-        mbar_expect_tx(&full[s], S::kBytes);
+        mbar_expect_tx_elect(&full[s], S::kBytes);
         const int64_t uoff = frag_unit_offset(rt, kb, b8_0, 0, K);
-        bulk_g2s(st, cA + uoff, 2048, &full[s]);
-        if (TWO) bulk_g2s(st + S::kB, cB + uoff, 2048, &full[s]);
+        bulk_g2s_elect(st, cA + uoff, 2048, &full[s]);
+        if (TWO) bulk_g2s_elect(st + S::kB, cB + uoff, 2048, &full[s]);
         if (GS) {
             const int64_t soff = ((int64_t)rt * ng + kb) * kTileRows + b8_0 * 16;
-            bulk_g2s(st + S::kSA, sA + soff, 256, &full[s]);
-            if (TWO) bulk_g2s(st + S::kSB, sB + soff, 256, &full[s]);
+            bulk_g2s_elect(st + S::kSA, sA + soff, 256, &full[s]);
+            if (TWO) bulk_g2s_elect(st + S::kSB, sB + soff, 256, &full[s]);
         }
     }
     if (it < total) {  // abandoned: let the copies already issued land before leaving
         for (int j = it > kStages ? it - kStages : 0; j < it; ++j)
-            mbar_wait(&full[j % kStages], (j / kStages) & 1, nullptr);
+            mbar_wait_warp(&full[j % kStages], (j / kStages) & 1, nullptr);
     }
 }
 
@@ -161,7 +161,7 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& a, int K, int row0,
     for (int rel = 0; rel < n; ++rel) {
         const int it = it0 + rel;
         const int s = it % kStages;
-        if (ok && !mbar_wait(&full[s], (it / kStages) & 1, a.err)) ok = false;
+        if (ok && !mbar_wait_warp(&full[s], (it / kStages) & 1, a.err)) ok = false;
         const uint8_t* st = ring + s * S::kBytes;
         const uint4 ua = reinterpret_cast<const uint4*>(st)[warp * 32 + lane];
         const uint4 ub = GATEUP ? reinterpret_cast<const uint4*>(st + S::kB)[warp * 32 + lane] : ua;
@@ -270,6 +270,8 @@ __device__ __forceinline__ void stage_rows(const __half* __restrict__ q, const f
 template <bool TWO, bool GS>
 __host__ __device__ constexpr int gemv_ring_bytes() { return kStages * Stage<TWO, GS>::kBytes; }
 __host__ __device__ inline int gemv_act_bytes(int tok_cap, int K) { return tok_cap * (K / 64) * (128 * 2 + 4); }
+// dynamic shared memory a GEMV CTA may ask for (the opt-in limit less the static part)
+constexpr int kGemvSmemMax = 227 * 1024 - 2048;
 
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU.  After the shuffle, lane (g, t < 2) holds rows g, g + 8 of
@@ -305,8 +307,7 @@ gateup_gemv_kernel(GemvArgs a) {
     }
     __syncthreads();
     if (warp == kConsumers) {  // producer warp
-        if (lane == 0)
-            gemv_produce<true, GS>(codesA, codesB, sA, sB, a.H, rt, b8_0, 0, KB, passes, ring,
+        gemv_produce<true, GS>(codesA, codesB, sA, sB, a.H, rt, b8_0, 0, KB, passes, ring,
                                    full, empty, a.err);
         return;
     }
@@ -429,8 +430,7 @@ down_gemv_kernel(GemvArgs a) {
     }
     __syncthreads();
     if (warp == kConsumers) {
-        if (lane == 0)
-            gemv_produce<false, GS>(codesA, codesA, sA, sA, a.I, rt, b8_0, kb0, n, passes, ring,
+        gemv_produce<false, GS>(codesA, codesA, sA, sA, a.I, rt, b8_0, kb0, n, passes, ring,
                                     full, empty, a.err);
         return;
     }

@@ -57,12 +57,44 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     return false;
 }
 
+// Warp-wide wait: lane 0 polls the barrier while the other lanes sleep at the
+// warp barrier, which then orders their reads after lane 0's acquire.  Keeps the
+// mbarrier unit free for the arrivals and transaction counts that make progress
+// (every lane polling floods it).  Every lane gets lane 0's result.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int32_t* err) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // global -> shared bulk copy, completion counted in bytes on `bar`.  Both
 // addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// The *_elect variants are executed by every lane of a converged warp with
+// warp-uniform operands; one lane elected by elect.sync issues the operation.
+// Issued that way the operands stay in uniform registers, which makes the
+// async-copy and tensor-core instructions several times cheaper to issue than
+// from a lone lane in a divergent branch.
+__device__ __forceinline__ void mbar_expect_tx_elect(uint64_t* bar, uint32_t bytes) {
+    asm volatile(
+        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+        " @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n}"
+        ::"r"(smem_u32(bar)), "r"(bytes)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s_elect(void* dst, const void* src, uint32_t bytes,
+                                               uint64_t* bar) {
+    asm volatile(
+        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+        " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}"
         ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }

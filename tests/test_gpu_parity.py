@@ -212,6 +212,25 @@ def test_glm_decode_full_layer(glm_decode_layer):
         assert err <= TOL_F32, err
 
 
+def test_glm_gemv_batch_over_staging_cap(glm_decode_layer):
+    """A batch of 16 tokens at full size on the GEMV path: more tokens than one
+    pass stages in shared memory, so units of several pairs run several passes.
+    Selection of all tokens exact; two tokens' outputs against the oracle."""
+    wl = synth.GLM_DECODE
+    L = glm_decode_layer
+    wr, b = L.router_w.cpu(), L.router_b.cpu()
+    x, idx_ref, w_ref, _ = gap_resampled_tokens(wl, 16, wr, b, step=7)
+    y, idx, w = forward(L, x.cuda(), 16)
+    same_selection(idx, idx_ref)
+    check_weights(idx, w, idx_ref, w_ref)
+    experts = OracleExperts(wl)
+    for t in (0, 15):
+        y_ref = oracle_tokens(wl, experts, x.numpy()[t:t + 1], idx_ref[t:t + 1], w_ref[t:t + 1])
+        err = rel_err(y[t:t + 1], y_ref)
+        assert err <= TOL_F32, (t, err)
+        experts.cache.clear()
+
+
 @pytest.fixture(scope="module")
 def glm_mtp_layer():
     L = build_layer(synth.GLM_MTP)
