@@ -2,7 +2,7 @@
 """Benchmark of the routed int4 MoE layer (libcolimoe) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--tokens T] [--path auto|gemv|gemm] [--impl own|reference]
+                    [--tokens T] [--path auto|gemv|gemm|fused] [--impl own|reference]
 
 A step is one forward of the layer (router, union, int4 experts, SwiGLU, combine)
 over one batch of synthetic tokens already resident in HBM.  Between timed steps
@@ -220,7 +220,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="glm_decode")
     ap.add_argument("--tokens", type=int, default=0, help="override tokens per step")
-    ap.add_argument("--path", default="auto", choices=("auto", "gemv", "gemm"))
+    ap.add_argument("--path", default="auto", choices=("auto", "gemv", "gemm", "fused"))
     ap.add_argument("--impl", default="own", choices=("own", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
@@ -253,7 +253,11 @@ def main():
         import dataclasses
         wl = dataclasses.replace(wl, E=args.experts)
     T = args.tokens or wl.T
-    path = {"auto": cm.COLI_PATH_AUTO, "gemv": cm.COLI_PATH_GEMV, "gemm": cm.COLI_PATH_GEMM}[args.path]
+    path = {"auto": cm.COLI_PATH_AUTO, "gemv": cm.COLI_PATH_GEMV, "gemm": cm.COLI_PATH_GEMM,
+            "fused": cm.COLI_PATH_FUSED}[args.path]
+    # the path AUTO resolves to (include/coli_moe.h): the fused kernel for small batches
+    fused = args.path == "fused" or (args.path == "auto" and T <= 16 and wl.E <= 256
+                                     and wl.k <= 32 and wl.n_shared <= 4)
     layers = build_layers(wl, dev)
     L0 = layers[0]
     n_pool = 64 if T <= 16 else 2
@@ -394,21 +398,30 @@ def main():
         dn_bytes_unit = wl.H * wl.I // 2 + wl.H * ng_i * 4
         units = uniq_slot[st_ms[:, -1].astype(int)] + wl.n_shared
         stage_mean = st_ms[:, :-1].mean(0)
-        gu_ach = (units * gu_bytes_unit).sum() / (st_ms[:, 2].sum() / 1e3) / 1e9
-        dn_ach = (units * dn_bytes_unit).sum() / (st_ms[:, 3].sum() / 1e3) / 1e9
-        dominant = "gateup" if stage_mean[2] >= stage_mean[3] else "down"
-        ach = gu_ach if dominant == "gateup" else dn_ach
+        if fused:
+            # one kernel: top-k, union, gate/up, down and combine; its time is the
+            # "gateup" stage (the union/down/combine marks bracket nothing)
+            kern_bytes = units * (gu_bytes_unit + dn_bytes_unit)
+            ach = kern_bytes.sum() / (st_ms[:, 2].sum() / 1e3) / 1e9
+            kname = "moe_fused_kernel (top-k, union, gate/up, down, combine)"
+            line["stages_us"] = {"router": 1e3 * stage_mean[0], "fused": 1e3 * stage_mean[2]}
+        else:
+            gu_ach = (units * gu_bytes_unit).sum() / (st_ms[:, 2].sum() / 1e3) / 1e9
+            dn_ach = (units * dn_bytes_unit).sum() / (st_ms[:, 3].sum() / 1e3) / 1e9
+            dominant = "gateup" if stage_mean[2] >= stage_mean[3] else "down"
+            ach = gu_ach if dominant == "gateup" else dn_ach
+            kern_bytes = units * (gu_bytes_unit if dominant == "gateup" else dn_bytes_unit)
+            kname = f"{dominant}_gemv_kernel"
+            line["stages_us"] = {n: 1e3 * v for n, v in zip(cm.STAGE_NAMES, stage_mean)}
+            line["down_gbs"] = dn_ach
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
-                            "frac": ach / hbm_gbs, "traffic": None,
-                            "kernel": f"expert_gemv_kernel ({dominant})",
+                            "frac": ach / hbm_gbs, "traffic": None, "kernel": kname,
                             "peak_source": peak_src,
-                            "bytes_per_launch": float((units * (gu_bytes_unit if dominant == "gateup" else dn_bytes_unit)).mean())}
-        line["stages_us"] = {n: 1e3 * v for n, v in zip(cm.STAGE_NAMES, stage_mean)}
-        line["down_gbs"] = dn_ach
+                            "bytes_per_launch": float(kern_bytes.mean())}
         line["int4_weight_gbs"] = weight_gbs
         line["int4_weight_frac_of_hbm"] = weight_gbs / hbm_gbs
         line["unique_experts_per_step"] = float(uniq.mean())
-        line["gpu_launches"] = 6 * K
+        line["gpu_launches"] = (2 if fused else 6) * K
     else:
         line["gpu_launches"] = 7 * wl.layers * K
     line["config"] = cfg

@@ -84,9 +84,14 @@ typedef enum coli_status {
 typedef enum coli_dtype { COLI_F32 = 0, COLI_BF16 = 1 } coli_dtype;
 
 typedef enum coli_path {
-    COLI_PATH_AUTO = 0, /* choose by batch size                              */
-    COLI_PATH_GEMV = 1, /* CUDA-core int4 GEMV, f32 arithmetic throughout      */
-    COLI_PATH_GEMM = 2  /* tcgen05 grouped GEMM, bf16 operands, f32 accumulate */
+    COLI_PATH_AUTO = 0,  /* FUSED when it applies, else GEMV below 48 tokens,
+                            else GEMM                                          */
+    COLI_PATH_GEMV = 1,  /* per-unit int4 GEMV kernels (mma.sync, fp16 hi/lo
+                            activation digits, f32 accumulation)               */
+    COLI_PATH_GEMM = 2,  /* tcgen05 grouped GEMM, fp16 operands, f32 accumulate */
+    COLI_PATH_FUSED = 3  /* one persistent kernel for top-k, union, experts and
+                            combine (mma.sync s8, exact int32 step sums);
+                            T <= 16, E <= 256, k <= 32, n_shared <= 4         */
 } coli_path;
 
 /* Thread-local description of the last error returned on this thread. */

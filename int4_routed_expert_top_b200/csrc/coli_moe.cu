@@ -13,6 +13,7 @@
 
 #include "coli_moe.h"
 #include "common.cuh"
+#include "fused.cuh"
 #include "gemm.cuh"
 #include "gemv.cuh"
 #include "misc.cuh"
@@ -57,8 +58,14 @@ bool shape_ok(int H, int I, int group) {
 struct WsPlan {
     int64_t zpart, idx, w, offsets, pair_tok, pair_slot, uniq, n_uniq, inv;
     int64_t unit_expert, unit_begin, unit_end, n_units, counters, err;
-    int64_t xq, xinv, hq, hinv, o, xg, hg, hmax, hsc, total;
+    int64_t xq, xinv, hq, hinv, o, xg, hg, hmax, hsc;
+    int64_t xq8, xinv8, hq8, fsync;  // fused small-batch kernel (T <= kFzMaxT only)
+    int64_t total;
 };
+
+bool fused_fits(const coli_moe_desc& d, int T) {
+    return T <= kFzMaxT && d.E <= kFzMaxE && d.k <= kFzMaxK && d.n_shared <= 4;
+}
 
 WsPlan plan_ws(const coli_moe_desc& d, int T) {
     WsPlan p;
@@ -91,6 +98,15 @@ WsPlan plan_ws(const coli_moe_desc& d, int T) {
     p.hg = take(P * d.I * 2);                   //   fp16 h of every pair
     p.hmax = take(P * 4);                       //   per-pair max |h|
     p.hsc = take(P * 4);                        //   per-pair inverse scale of h
+    if (fused_fits(d, T)) {
+        const int ns_dn = fz_ns_down(d.I);
+        p.xq8 = take((int64_t)T * d.H * 2);
+        p.xinv8 = take((int64_t)T * 4);
+        p.hq8 = take((int64_t)(d.I / 64 / ns_dn) * P * fz_rec_bytes(ns_dn));
+        p.fsync = take((int64_t)fz_sync_ints(d.H) * 4);
+    } else {
+        p.xq8 = p.xinv8 = p.hq8 = p.fsync = 0;
+    }
     p.total = off;
     return p;
 }
@@ -133,19 +149,25 @@ int set_smem(const void* fn, int bytes) {
 // fp16 activation operand is produced as well (by extra CTAs of the small-batch
 // router, or by its own launch after the tiled router).
 int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, float* zpart,
-                  __half* xq, float* xinv, cudaStream_t st, int* ks_out) {
+                  __half* xq, float* xinv, cudaStream_t st, int* ks_out,
+                  const RouterExtras* fused = nullptr) {
     int KS = 0;
     if (T <= 32)
         for (int c : {8, 4, 2, 1})
             if (d.H % (c * 128) == 0 && d.H / c <= kRouterMaxSlice) { KS = c; break; }
     if (KS > 0) {
         const int rblocks = (d.E * KS + 7) / 8;
-        const int qblocks = xq ? T : 0;
-        const dim3 grid(rblocks + qblocks);
+        RouterExtras ex;
+        if (fused) ex = *fused;
+        ex.xq = xq;
+        ex.xinv = xinv;
+        const int qblocks = (ex.xq || ex.xq8) ? T : 0;
+        const int zblocks = ex.zero_n > 0 ? 1 : 0;
+        const dim3 grid(rblocks + qblocks + zblocks);
         if (xt == COLI_F32)
-            router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, xq, xinv);
+            router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
         else
-            router_gemv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, xq, xinv);
+            router_gemv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
     } else {
         const int tiles = ((T + 63) / 64) * ((d.E + 63) / 64);
         KS = 1;
@@ -366,6 +388,58 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
                   : (gs ? launch_down_t<2, true>(d, units_max, a, st) : launch_down_t<2, false>(d, units_max, a, st));
 }
 
+// ---------------------------------------------------------------------------
+// fused small-batch path
+// ---------------------------------------------------------------------------
+int sm_count() { return gemm_grid(); }
+
+template <int NT, bool GS>
+int launch_fused_t(const FusedArgs& a, cudaStream_t st) {
+    const int smem = a.slots * a.slot_bytes;
+    int rc = set_smem((const void*)moe_fused_kernel<NT, GS>, smem);
+    if (rc) return rc;
+    moe_fused_kernel<NT, GS><<<sm_count(), kFzThreads, smem, st>>>(a);
+    return check_launch("fused moe");
+}
+
+int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int KS,
+                 const float* residual, float* y, cudaStream_t st) {
+    const coli_moe_desc& d = l->d;
+    FusedArgs a;
+    a.experts = static_cast<const uint8_t*>(d.experts);
+    a.blob_bytes = l->L.bytes;
+    a.L = l->L;
+    a.zpart = at<float>(ws, p.zpart);
+    a.KS = KS;
+    a.bias = d.router_b;
+    a.routed_scale = d.routed_scale;
+    a.norm_topk = d.norm_topk;
+    a.xq8 = at<int8_t>(ws, p.xq8);
+    a.xinv8 = at<float>(ws, p.xinv8);
+    a.hq8 = at<int8_t>(ws, p.hq8);
+    a.o = at<float>(ws, p.o);
+    a.sync = at<int32_t>(ws, p.fsync);
+    a.idx = at<int32_t>(ws, p.idx);
+    a.w = at<float>(ws, p.w);
+    a.residual = residual;
+    a.y = y;
+    a.err = at<int32_t>(ws, p.err);
+    a.T = T; a.E = d.E; a.k = d.k; a.n_shared = d.n_shared;
+    a.H = d.H; a.I = d.I; a.group = d.group;
+    const int NT = T <= 4 ? 1 : (T <= 8 ? 2 : 4);
+    const int rec = std::max(fz_rec_bytes(fz_ns_gateup(d.H)), fz_rec_bytes(fz_ns_down(d.I)));
+    a.slot_bytes = (int)align256(kFzActOff + 4 * NT * rec);
+    const int budget = 227 * 1024 - (int)sizeof(FusedShared) - 1024;
+    a.slots = std::min(kFzMaxSlots, budget / a.slot_bytes);
+    if (a.slots < 2) return fail(COLI_E_UNSUPPORTED, "fused: ring does not fit");
+    const bool gs = d.group != 0;
+    switch (NT) {
+        case 1: return gs ? launch_fused_t<1, true>(a, st) : launch_fused_t<1, false>(a, st);
+        case 2: return gs ? launch_fused_t<2, true>(a, st) : launch_fused_t<2, false>(a, st);
+        default: return gs ? launch_fused_t<4, true>(a, st) : launch_fused_t<4, false>(a, st);
+    }
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -527,7 +601,8 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
                         coli_stream_t stream) {
     if (!layer || !x || !y) return fail(COLI_E_INVAL, "forward: NULL pointer");
     if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_E_INVAL, "forward: bad dtype");
-    if (path != COLI_PATH_AUTO && path != COLI_PATH_GEMV && path != COLI_PATH_GEMM)
+    if (path != COLI_PATH_AUTO && path != COLI_PATH_GEMV && path != COLI_PATH_GEMM &&
+        path != COLI_PATH_FUSED)
         return fail(COLI_E_INVAL, "forward: bad path");
     const coli_moe_desc& d = layer->d;
     int rc = tokens_ok(d, T);
@@ -535,7 +610,12 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     const WsPlan p = plan_ws(d, T);
     if (!ws || ws_bytes < (size_t)p.total)
         return fail(COLI_E_WORKSPACE, "forward: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
-    if (path == COLI_PATH_AUTO) path = gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV;
+    if (path == COLI_PATH_FUSED && !fused_fits(d, T))
+        return fail(COLI_E_UNSUPPORTED, "forward: fused path needs T<=%d, E<=%d, k<=%d, n_shared<=4",
+                    kFzMaxT, kFzMaxE, kFzMaxK);
+    if (path == COLI_PATH_AUTO)
+        path = fused_fits(d, T) ? COLI_PATH_FUSED
+                                : (gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV);
     cudaStream_t st = S(stream);
     int32_t* idx = at<int32_t>(ws, p.idx);
     float* w = at<float>(ws, p.w);
@@ -549,6 +629,31 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     };
     const bool gemm = path == COLI_PATH_GEMM;
     int KS;
+    if (path == COLI_PATH_FUSED) {
+        if ((rc = mark(COLI_STAGE_ROUTER))) return rc;
+        RouterExtras ex;
+        ex.xq8 = at<int8_t>(ws, p.xq8);
+        ex.xinv8 = at<float>(ws, p.xinv8);
+        ex.zero = at<int32_t>(ws, p.fsync);
+        ex.zero_n = fz_sync_ints(d.H);
+        ex.err = at<int32_t>(ws, p.err);
+        if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), nullptr, nullptr, st, &KS, &ex)))
+            return rc;
+        // the fused kernel is the union, gate/up, down and combine stages at once
+        if ((rc = mark(COLI_STAGE_UNION))) return rc;
+        if ((rc = mark(COLI_STAGE_GATEUP))) return rc;
+        if ((rc = launch_fused(layer, T, ws, p, KS, residual, y, st))) return rc;
+        if ((rc = mark(COLI_STAGE_DOWN))) return rc;
+        if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
+        if ((rc = mark(COLI_STAGES))) return rc;
+        if (idx_out && cudaMemcpyAsync(idx_out, idx, sizeof(int32_t) * T * d.k,
+                                       cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return fail(COLI_E_CUDA, "forward: copy idx");
+        if (w_out && cudaMemcpyAsync(w_out, w, sizeof(float) * T * d.k,
+                                     cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return fail(COLI_E_CUDA, "forward: copy w");
+        return COLI_OK;
+    }
     if ((rc = mark(COLI_STAGE_ROUTER))) return rc;
     if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), at<__half>(ws, p.xq),
                             at<float>(ws, p.xinv), st, &KS)))

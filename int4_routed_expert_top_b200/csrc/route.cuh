@@ -63,14 +63,101 @@ act_quant_kernel(const XT* __restrict__ x, int T, int H, __half* __restrict__ xq
 // ---------------------------------------------------------------------------
 constexpr int kRouterMaxSlice = 1024;  // columns per warp slice (<= 8 loads per lane)
 
+// ---------------------------------------------------------------------------
+// s8 activation operand of the fused small-batch kernel (fused.cuh): each value
+// becomes two signed 8-bit digits of a 15-bit fixed-point number under one
+// power-of-two scale per token.
+// ---------------------------------------------------------------------------
+// Byte position of column c (0..63) of a 64-column step in the activation
+// operand: lane t's 16 bytes hold columns 4t..4t+3, 16+4t.., 32+4t.., 48+4t..,
+// i.e. its B registers of the two k32 halves of the step.
+__host__ __device__ inline int fz_act_pos(int c) {
+    return 16 * ((c % 16) / 4) + 4 * (c / 16) + (c % 4);
+}
+
+// Power-of-two scale for a block whose largest magnitude is m: returns sh with
+// m * 2^sh in [2^13, 2^14) and *inv = 2^-sh (1 for an all-zero block).
+__device__ __forceinline__ float fz_scale(float m, float* inv) {
+    if (!(m > 0.0f) || !isfinite(m)) { *inv = 1.0f; return 1.0f; }
+    int e;
+    frexpf(m, &e);
+    const int sh = max(-100, min(100, 14 - e));
+    *inv = ldexpf(1.0f, -sh);
+    return ldexpf(1.0f, sh);
+}
+
+// x16 = rint(v * sc) split into hi (high digit) and lo (low digit)
+__device__ __forceinline__ void fz_split(float v, float sc, int& hi, int& lo) {
+    const int x = __float2int_rn(v * sc);
+    hi = (x + 128) >> 8;
+    lo = x - 256 * hi;
+}
+
+// s8 activation operand of one token, one CTA of 256 threads: xq8[t][step]
+// (64 hi bytes then 64 lo bytes, columns in fz_act_pos order), xinv8[t].
+template <typename XT>
+__device__ __forceinline__ void act_quant8_token(const XT* __restrict__ x, int H, int t,
+                                                 int8_t* __restrict__ xq8,
+                                                 float* __restrict__ xinv8) {
+    __shared__ float part8[8];
+    const XT* row = x + (int64_t)t * H;
+    float m = 0.0f;
+    for (int c = threadIdx.x; c < H; c += 256) m = fmaxf(m, fabsf(to_f32(row[c])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) part8[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = part8[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) m = fmaxf(m, part8[i]);
+    float inv;
+    const float sc = fz_scale(m, &inv);
+    // four consecutive columns per thread -> one 32-bit word of hi, one of lo
+    for (int c = 4 * threadIdx.x; c < H; c += 1024) {
+        uint32_t wh = 0, wl = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int hi, lo;
+            fz_split(to_f32(row[c + i]), sc, hi, lo);
+            wh |= (uint32_t)(hi & 0xFF) << (8 * i);
+            wl |= (uint32_t)(lo & 0xFF) << (8 * i);
+        }
+        int8_t* step = xq8 + ((int64_t)t * (H / 64) + c / 64) * 128;
+        const int pos = fz_act_pos(c % 64);
+        *reinterpret_cast<uint32_t*>(step + pos) = wh;
+        *reinterpret_cast<uint32_t*>(step + 64 + pos) = wl;
+    }
+    if (threadIdx.x == 0) xinv8[t] = inv;
+}
+
+// Extra blocks after the router's: one per token for the activation operand
+// (fp16 hi/lo into xq, or s8 digits into xq8 for the fused kernel), then one
+// that clears `zero_n` ints at `zero` (the fused kernel's counters).
+struct RouterExtras {
+    __half* xq = nullptr;
+    float* xinv = nullptr;
+    int8_t* xq8 = nullptr;
+    float* xinv8 = nullptr;
+    int32_t* zero = nullptr;
+    int zero_n = 0;
+    int32_t* err = nullptr;  // device error flags, cleared by the same block
+};
+
 template <typename XT>
 __global__ void __launch_bounds__(256)
 router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restrict__ wr,
                    int E, int KS, float* __restrict__ zpart, int router_blocks,
-                   __half* __restrict__ xq, float* __restrict__ xinv) {
+                   RouterExtras ex) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if ((int)blockIdx.x >= router_blocks) {  // one CTA per token: activation operand
-        if (xq) act_quant_token(x, H, blockIdx.x - router_blocks, xq, xinv);
+    if ((int)blockIdx.x >= router_blocks) {
+        const int b = blockIdx.x - router_blocks;
+        if (b < T) {  // one CTA per token: activation operand
+            if (ex.xq) act_quant_token(x, H, b, ex.xq, ex.xinv);
+            if (ex.xq8) act_quant8_token(x, H, b, ex.xq8, ex.xinv8);
+        } else {
+            for (int i = threadIdx.x; i < ex.zero_n; i += 256) ex.zero[i] = 0;
+            if (threadIdx.x == 0 && ex.err) *ex.err = 0;
+        }
         return;
     }
     const int gw = blockIdx.x * 8 + warp;

@@ -1,7 +1,8 @@
 """GPU parity: libcolimoe (through the C ABI) against the CPU oracle on the same
 seeded inputs.  Bit-exact for container bytes, scales, dequantised weights,
 selected expert sets and union lists; layer outputs within a norm-wise relative
-error of 2e-3 on the f32 path (GEMV)."""
+error of 2e-3 on the small-batch paths (GEMV: fp16 digits, f32 accumulation;
+FUSED: s8 digits, exact int32 step sums, f32 across steps)."""
 import dataclasses
 
 import numpy as np
@@ -140,28 +141,39 @@ VARIANTS = {
 }
 
 
+SMALL_PATHS = {"gemv": cm.COLI_PATH_GEMV, "fused": cm.COLI_PATH_FUSED}
+
+
+def fused_applies(wl, T):
+    return T <= 16 and wl.E <= 256 and wl.k <= 32 and wl.n_shared <= 4
+
+
+@pytest.mark.parametrize("path", list(SMALL_PATHS))
 @pytest.mark.parametrize("name", list(VARIANTS))
-def test_layer_parity_small(name):
+def test_layer_parity_small(name, path):
     wl = dataclasses.replace(synth.TINY, **VARIANTS[name])
+    if path == "fused" and not fused_applies(wl, wl.T):
+        pytest.skip("outside the fused kernel's limits (covered by the rejection test)")
     wr, b = synth.router(wl)
     x, idx_ref, w_ref, _ = gap_resampled_tokens(wl, wl.T, wr, b)
     y_ref = oracle_tokens(wl, OracleExperts(wl), x.numpy(), idx_ref, w_ref)
     L = build_layer(wl, router=(wr, b))
-    y, idx, w = forward(L, device_x(x, wl), wl.T)
+    y, idx, w = forward(L, device_x(x, wl), wl.T, path=SMALL_PATHS[path])
     same_selection(idx, idx_ref, ordered_ok(x.numpy(), wr.numpy(), b.numpy(), idx_ref, wl.k))
     check_weights(idx, w, idx_ref, w_ref)
     err = rel_err(y, y_ref)
     assert err <= TOL_F32, err
     # deterministic: a second run gives the same bytes
-    y2, _, _ = forward(L, device_x(x, wl), wl.T)
+    y2, _, _ = forward(L, device_x(x, wl), wl.T, path=SMALL_PATHS[path])
     np.testing.assert_array_equal(y2.view(np.uint32), y.view(np.uint32))
 
 
-def test_residual_and_zero_input():
+@pytest.mark.parametrize("path", list(SMALL_PATHS))
+def test_residual_and_zero_input(path):
     wl = dataclasses.replace(synth.TINY, group=64)
     L = build_layer(wl)
     x = torch.zeros((3, wl.H), dtype=torch.float32, device="cuda")
-    y, _, _ = forward(L, x, 3)
+    y, _, _ = forward(L, x, 3, path=SMALL_PATHS[path])
     np.testing.assert_array_equal(y, 0.0)          # x = 0 -> y = 0 exactly
     wr, b = synth.router(wl)
     xr, idx_ref, w_ref, _ = gap_resampled_tokens(wl, 4, wr, b)
@@ -169,9 +181,30 @@ def test_residual_and_zero_input():
     res = torch.randn((4, wl.H), device="cuda")
     out = res.clone()
     cm.coli_moe_forward_ex(L.handle, xr.cuda(), 4, out, L.workspace(4), residual=out,
-                           path=cm.COLI_PATH_GEMV)
+                           path=SMALL_PATHS[path])
     torch.cuda.synchronize()
     assert rel_err(out.cpu().numpy() - res.cpu().numpy(), y_ref) <= TOL_F32
+
+
+def test_fused_rejects_sizes_outside_its_limits():
+    wl = dataclasses.replace(synth.TINY, T=17)
+    L = build_layer(wl)
+    x = torch.randn((17, wl.H), device="cuda")
+    y = torch.empty((17, wl.H), device="cuda")
+    with pytest.raises(cm.ColiError) as ei:
+        cm.coli_moe_forward_ex(L.handle, x, 17, y, L.workspace(17), path=cm.COLI_PATH_FUSED)
+    assert ei.value.code == -4   # COLI_E_UNSUPPORTED
+
+
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_auto_small_batches_equal_fused(T):
+    """AUTO picks the fused kernel for small batches: same bytes as asking for it."""
+    wl = dataclasses.replace(synth.TINY, T=T, group=64)
+    L = build_layer(wl)
+    x = torch.randn((T, wl.H), device="cuda")
+    ya, _, _ = forward(L, x, T, path=cm.COLI_PATH_AUTO)
+    yf, _, _ = forward(L, x, T, path=cm.COLI_PATH_FUSED)
+    np.testing.assert_array_equal(ya.view(np.uint32), yf.view(np.uint32))
 
 
 def test_rmsnorm_matches_oracle():
@@ -196,7 +229,8 @@ def glm_decode_layer():
     torch.cuda.empty_cache()
 
 
-def test_glm_decode_full_layer(glm_decode_layer):
+@pytest.mark.parametrize("path", list(SMALL_PATHS))
+def test_glm_decode_full_layer(glm_decode_layer, path):
     """Decode, T = 1, per-row scales, 257 resident experts: all 6144 outputs."""
     wl = synth.GLM_DECODE
     L = glm_decode_layer
@@ -204,7 +238,7 @@ def test_glm_decode_full_layer(glm_decode_layer):
     experts = OracleExperts(wl)
     for step in range(2):
         x, idx_ref, w_ref, _ = gap_resampled_tokens(wl, 1, wr, b, step=step)
-        y, idx, w = forward(L, x.cuda(), 1)
+        y, idx, w = forward(L, x.cuda(), 1, path=SMALL_PATHS[path])
         same_selection(idx, idx_ref)
         check_weights(idx, w, idx_ref, w_ref)
         y_ref = oracle_tokens(wl, experts, x.numpy(), idx_ref, w_ref)
@@ -212,15 +246,17 @@ def test_glm_decode_full_layer(glm_decode_layer):
         assert err <= TOL_F32, err
 
 
-def test_glm_gemv_batch_over_staging_cap(glm_decode_layer):
-    """A batch of 16 tokens at full size on the GEMV path: more tokens than one
-    pass stages in shared memory, so units of several pairs run several passes.
+@pytest.mark.parametrize("path", list(SMALL_PATHS))
+def test_glm_gemv_batch_over_staging_cap(glm_decode_layer, path):
+    """A batch of 16 tokens at full size: on the GEMV path more tokens than one
+    pass stages in shared memory, so units of several pairs run several passes;
+    on the fused path the largest column-group count (16 pairs per unit).
     Selection of all tokens exact; two tokens' outputs against the oracle."""
     wl = synth.GLM_DECODE
     L = glm_decode_layer
     wr, b = L.router_w.cpu(), L.router_b.cpu()
     x, idx_ref, w_ref, _ = gap_resampled_tokens(wl, 16, wr, b, step=7)
-    y, idx, w = forward(L, x.cuda(), 16)
+    y, idx, w = forward(L, x.cuda(), 16, path=SMALL_PATHS[path])
     same_selection(idx, idx_ref)
     check_weights(idx, w, idx_ref, w_ref)
     experts = OracleExperts(wl)
@@ -240,7 +276,8 @@ def glm_mtp_layer():
     torch.cuda.empty_cache()
 
 
-def test_glm_mtp_verify_steps(glm_mtp_layer):
+@pytest.mark.parametrize("path", list(SMALL_PATHS))
+def test_glm_mtp_verify_steps(glm_mtp_layer, path):
     """MTP verify: 64 steps of 3 positions, gs64.  Every step's selection and union
     is checked exactly; outputs of two steps are checked element by element."""
     wl = synth.GLM_MTP
@@ -249,7 +286,7 @@ def test_glm_mtp_verify_steps(glm_mtp_layer):
     experts = OracleExperts(wl)
     for step in range(wl.steps):
         x, idx_ref, w_ref, _ = gap_resampled_tokens(wl, wl.T, wr, b, step=step)
-        y, idx, w = forward(L, x.cuda(), wl.T)
+        y, idx, w = forward(L, x.cuda(), wl.T, path=SMALL_PATHS[path])
         same_selection(idx, idx_ref)
         ref = oracle.union(idx_ref, wl.E)
         d = {n: torch.empty((s,), dtype=torch.int32, device="cuda") for n, s in
