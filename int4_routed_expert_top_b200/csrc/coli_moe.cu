@@ -145,14 +145,15 @@ int set_smem(const void* fn, int bytes) {
     return COLI_OK;
 }
 
-// Router logits into zpart (K slices in *ks_out).  When xq is non-null the
+// Router logits into zpart ([*ks_out][T][E] K slices; the small-batch router
+// sums its slices itself and reports one).  When xq is non-null the
 // fp16 activation operand is produced as well (by extra CTAs of the small-batch
 // router, or by its own launch after the tiled router).
 int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, float* zpart,
                   __half* xq, float* xinv, cudaStream_t st, int* ks_out,
                   const RouterExtras* fused = nullptr) {
     int KS = 0;
-    if (T <= 32)
+    if (T <= kRouterMaxT)
         for (int c : {8, 4, 2, 1})
             if (d.H % (c * 128) == 0 && d.H / c <= kRouterMaxSlice) { KS = c; break; }
     if (KS > 0) {
@@ -168,6 +169,8 @@ int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, f
             router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
         else
             router_gemv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
+        *ks_out = 1;
+        return check_launch("router");
     } else {
         const int tiles = ((T + 63) / 64) * ((d.E + 63) / 64);
         KS = 1;

@@ -44,7 +44,10 @@
 namespace coli {
 
 constexpr int kFzWarps = 16;                     // consumer warps
-constexpr int kFzThreads = 32 * (kFzWarps + 1);  // + one producer warp
+constexpr int kFzProducer = kFzWarps;            // warp that streams the ring
+constexpr int kFzService = kFzWarps + 1;         // warp that publishes finished items
+constexpr int kFzThreads = 32 * (kFzWarps + 2);
+constexpr int kFzHand = 4;                       // finished-item records in flight
 constexpr int kFzMaxT = 16;                      // tokens per call on this path
 constexpr int kFzMaxE = 256;                     // routed experts on this path
 constexpr int kFzMaxUnits = kFzMaxE + 4;
@@ -127,37 +130,50 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 namespace coli {
 
+
 // ---------------------------------------------------------------------------
 // Shared memory of a fused CTA besides the ring (static).
 // ---------------------------------------------------------------------------
 struct FusedShared {
     uint64_t full[kFzMaxSlots], empty[kFzMaxSlots];
+    uint64_t hand_full[kFzHand], hand_empty[kFzHand];
+    uint64_t cbar;
     int meta_item[kFzMaxSlots], meta_st[kFzMaxSlots];
+    int hand_item[kFzHand];
     int u_exp[kFzMaxUnits], u_p0[kFzMaxUnits], u_p1[kFzMaxUnits];
     int pair_tok[kFzMaxT * (kFzMaxK + 4)];
     int inv[kFzMaxT * kFzMaxK];
     int pick_e[kFzMaxT * kFzMaxK];
     float pick_w[kFzMaxT * kFzMaxK];
+    float xinv[kFzMaxT];
     float xch[8][16][kFzMaxT];   // epilogue exchange between warp pairs
     float wmax[8][kFzMaxT];
-    int n_uniq, last;
+    int n_uniq;
 };
 
 // Top-k of token t by one warp (E <= 256: up to 8 candidates per lane).
 // Order: selection score descending, expert index ascending.
 __device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, FusedShared& sh) {
     const int lane = threadIdx.x & 31;
-    float sc[8], sel[8];
+    float z[8], sc[8], sel[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        z[i] = e < a.E ? __ldcg(a.zpart + (int64_t)t * a.E + e) : 0.0f;
+    }
+    for (int ks = 1; ks < a.KS; ++ks)  // further K slices, in slice order
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            if (e < a.E) z[i] += __ldcg(a.zpart + ((int64_t)ks * a.T + t) * a.E + e);
+        }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
         sc[i] = 0.0f;
         sel[i] = -INFINITY;
         if (e < a.E) {
-            float z = 0.0f;
-            for (int ks = 0; ks < a.KS; ++ks)
-                z += __ldcg(a.zpart + ((int64_t)ks * a.T + t) * a.E + e);
-            const float s = 1.0f / (1.0f + expf(-z));
+            const float s = 1.0f / (1.0f + expf(-z[i]));
             sc[i] = s;
             sel[i] = s + __ldg(a.bias + e);
         }
@@ -196,12 +212,14 @@ __device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, FusedSh
 // scratch: 3 * E ints (any shared memory not yet in use).  Returns the units.
 __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& sh,
                                               int* scratch) {
+    constexpr int kAllWarps = kFzThreads / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int* cnt = scratch;
     uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + a.E);
     int* excl = scratch + 2 * a.E;
     for (int e = threadIdx.x; e < a.E; e += kFzThreads) { cnt[e] = 0; bits[e] = 0u; }
-    for (int t = warp; t < a.T; t += kFzWarps + 1) fz_topk_token(a, t, sh);
+    for (int t = threadIdx.x; t < a.T; t += kFzThreads) sh.xinv[t] = __ldcg(a.xinv8 + t);
+    for (int t = warp; t < a.T; t += kAllWarps) fz_topk_token(a, t, sh);
     __syncthreads();
     const int Tk = a.T * a.k;
     for (int i = threadIdx.x; i < Tk; i += kFzThreads) {
@@ -261,10 +279,6 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
     return nu + a.n_shared;
 }
 
-}  // namespace coli
-
-namespace coli {
-
 // D = A * B with C = 0 (a fresh 64-column partial sum)
 __device__ __forceinline__ void mma_s8_16832_zc(int d[4], const uint32_t a[4], uint32_t b0,
                                                 uint32_t b1) {
@@ -306,8 +320,29 @@ __device__ __forceinline__ void fz_decode_step(const uint8_t* p, uint32_t A0[4],
     decode_word_s8(u.w, A1[2], A1[3]);
 }
 
+// Work item -> (gate/up?, unit, 128-row tile).  Items: all gate/up tiles of all
+// units first (unit-major), then all down tiles.
+struct FzItem {
+    int gu, u, rt;
+};
+__device__ __forceinline__ FzItem fz_item(int item, int n_units, int TG, int TD) {
+    FzItem r;
+    r.gu = item < n_units * TG;
+    const int rel = r.gu ? item : item - n_units * TG;
+    const int per = r.gu ? TG : TD;
+    r.u = rel / per;
+    r.rt = rel - r.u * per;
+    return r;
+}
+
+}  // namespace coli
+
+namespace coli {
+
 // ---------------------------------------------------------------------------
 // Producer warp: claim items, stream their stages, then the end marker.
+// Ring position: slot s, lap parity lap (flips whenever s wraps to 0).  An
+// item's last stage also carries its tile's per-row weight scales.
 // ---------------------------------------------------------------------------
 template <bool GS>
 __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, uint8_t* ring,
@@ -320,48 +355,50 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
     const int rec_gu = fz_rec_bytes(ns_gu), rec_dn = fz_rec_bytes(ns_dn);
     int32_t* queue = a.sync;
     const int32_t* gu_done = a.sync + 1;
-    int it = 0;
+    int s = 0, issued = 0;
+    uint32_t lap = 0;
     bool ok = true;
     while (ok) {
         int item = 0;
         if (lane == 0) item = atomicAdd(queue, 1);
         item = __shfl_sync(0xffffffffu, item, 0);
         if (item >= n_items) break;
-        const bool gu = item < n_units * TG;
-        const int u = gu ? item / TG : (item - n_units * TG) / TD;
-        const int rt = gu ? item % TG : (item - n_units * TG) % TD;
-        const int e = sh.u_exp[u], p0 = sh.u_p0[u], np = sh.u_p1[u] - p0;
+        const FzItem w = fz_item(item, n_units, TG, TD);
+        const int e = sh.u_exp[w.u], p0 = sh.u_p0[w.u], np = sh.u_p1[w.u] - p0;
         const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
-        const int ns = gu ? ns_gu : ns_dn;
-        const int K = gu ? a.H : a.I;
+        const int ns = w.gu ? ns_gu : ns_dn;
+        const int K = w.gu ? a.H : a.I;
         const int nst = K / 64 / ns, ng = GS ? K / 64 : 1;
-        const uint8_t* cA = blob + a.L.codes[gu ? 0 : 2];
+        const uint8_t* cA = blob + a.L.codes[w.gu ? 0 : 2];
         const uint8_t* cB = blob + a.L.codes[1];
-        const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[gu ? 0 : 2]);
+        const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[w.gu ? 0 : 2]);
         const float* sB = reinterpret_cast<const float*>(blob + a.L.scales[1]);
-        const int mats = gu ? 2 : 1;
-        for (int st = 0; st < nst && ok; ++st, ++it) {
-            const int s = it % a.slots;
-            if (it >= a.slots && !fz_wait(&sh.empty[s], ((it / a.slots) - 1) & 1, a.err)) {
-                ok = false;
-                break;
-            }
+        const int mats = w.gu ? 2 : 1;
+        const uint32_t cbytes = (uint32_t)ns * 4096, sbytes = GS ? (uint32_t)ns * 512 : 0u;
+        const uint32_t abytes = w.gu ? (uint32_t)(np * ns * 128) : (uint32_t)(np * rec_dn);
+        const uint32_t tx = mats * (cbytes + sbytes) + abytes;
+        for (int st = 0; st < nst; ++st) {
+            if (issued >= a.slots && !fz_wait(&sh.empty[s], lap ^ 1u, a.err)) { ok = false; break; }
             if (lane == 0) { sh.meta_item[s] = item; sh.meta_st[s] = st; }
             __syncwarp();
             uint8_t* sl = ring + (int64_t)s * a.slot_bytes;
             const int kb0 = st * ns;
-            const uint32_t cbytes = (uint32_t)ns * 4096, sbytes = GS ? (uint32_t)ns * 512 : 0u;
-            const uint32_t abytes = gu ? (uint32_t)(np * ns * 128) : (uint32_t)(np * rec_dn);
-            mbar_expect_tx_elect(&sh.full[s], mats * (cbytes + sbytes) + abytes);
-            const int64_t coff = frag_unit_offset(rt, kb0, 0, 0, K);
+            const bool rowsc = !GS && st == nst - 1;
+            mbar_expect_tx_elect(&sh.full[s], tx + (rowsc ? mats * 512u : 0u));
+            const int64_t coff = frag_unit_offset(w.rt, kb0, 0, 0, K);
             bulk_g2s_elect(sl, cA + coff, cbytes, &sh.full[s]);
-            if (gu) bulk_g2s_elect(sl + cbytes, cB + coff, cbytes, &sh.full[s]);
+            if (w.gu) bulk_g2s_elect(sl + cbytes, cB + coff, cbytes, &sh.full[s]);
             if (GS) {
-                const int64_t soff = ((int64_t)rt * ng + kb0) * kTileRows;
+                const int64_t soff = ((int64_t)w.rt * ng + kb0) * kTileRows;
                 bulk_g2s_elect(sl + kFzScaleOff, sA + soff, sbytes, &sh.full[s]);
-                if (gu) bulk_g2s_elect(sl + kFzScaleOff + sbytes, sB + soff, sbytes, &sh.full[s]);
+                if (w.gu) bulk_g2s_elect(sl + kFzScaleOff + sbytes, sB + soff, sbytes, &sh.full[s]);
             }
-            if (gu) {
+            if (rowsc) {  // per-row scales of the tile, for the epilogue
+                bulk_g2s_elect(sl + kFzScaleOff, sA + (int64_t)w.rt * kTileRows, 512u, &sh.full[s]);
+                if (w.gu) bulk_g2s_elect(sl + kFzScaleOff + 512, sB + (int64_t)w.rt * kTileRows, 512u,
+                                         &sh.full[s]);
+            }
+            if (w.gu) {
                 for (int pp = 0; pp < np; ++pp) {
                     const int tok = sh.pair_tok[p0 + pp];
                     bulk_g2s_elect(sl + kFzActOff + pp * rec_gu,
@@ -369,147 +406,197 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
                                    (uint32_t)ns * 128, &sh.full[s]);
                 }
             } else {
-                if (st == 0) {  // h of this unit: every gate/up tile must be done
+                if (st == 0) {  // h of this unit: every gate/up tile must be published
                     int done = 1;
                     if (lane == 0) {
                         done = 0;
                         for (uint32_t i = 0; i < kWaitTries; ++i) {
-                            if (ld_acquire_gpu(gu_done + u) >= TG) { done = 1; break; }
-                            __nanosleep(128);
+                            if (ld_acquire_gpu(gu_done + w.u) >= TG) { done = 1; break; }
+                            __nanosleep(64);
                         }
                         if (!done) atomicOr(a.err, kErrWaitTimeout);
                     }
                     __syncwarp();
                     fence_proxy_async_global();
                 }
-                bulk_g2s_elect(sl + kFzActOff,
-                               a.hq8 + ((int64_t)st * P + p0) * rec_dn, abytes, &sh.full[s]);
+                bulk_g2s_elect(sl + kFzActOff, a.hq8 + ((int64_t)st * P + p0) * rec_dn, abytes,
+                               &sh.full[s]);
+            }
+            ++issued;
+            if (++s == a.slots) { s = 0; lap ^= 1u; }
+        }
+    }
+    if (ok && (issued < a.slots || fz_wait(&sh.empty[s], lap ^ 1u, a.err))) {  // end marker
+        if (lane == 0) sh.meta_item[s] = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.full[s]);
+        ++issued;
+    }
+    // leave only once every copy issued into the ring has landed
+    for (int j = issued > a.slots ? issued - a.slots : 0; j < issued; ++j)
+        fz_wait(&sh.full[j % a.slots], (j / a.slots) & 1, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// Per-stage tensor-core work of a consumer warp.  Warp w: gate/up -> matrix
+// w / 8 (gate, up), 16-row block w % 8, every step of the stage; down -> 16-row
+// block w % 8, half w / 8 of the stage's steps.  After an MMA, lane (g, t)
+// holds rows g, g + 8 and columns 2t, 2t + 1 of an 8-column group c: column n
+// carries pair 4c + (n & 3), high digit for n < 4, low digit for n >= 4, so
+// lanes t and t ^ 2 hold the two digits of the same pairs.
+// ---------------------------------------------------------------------------
+template <int NT, bool GS>
+__device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int ns, int m, int rb, int lane,
+                                                int rec_gu, int acc_i[NT][4], float acc_f[NT][4]) {
+    const int g = lane >> 2, t = lane & 3;
+    const float lanefac = t < 2 ? 256.0f : 1.0f;
+    const uint8_t* cp = sl + m * ns * 4096 + rb * 512 + lane * 16;
+    const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + (g & 3) * rec_gu;
+    const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff + m * ns * 512) + 16 * rb + g;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (j < ns) {
+            uint32_t A0[4], A1[4];
+            fz_decode_step(cp + j * 4096, A0, A1);
+            if (GS) {
+                const float s0 = scl[j * 128] * lanefac, s1 = scl[j * 128 + 8] * lanefac;
+#pragma unroll
+                for (int c = 0; c < NT; ++c) {
+                    const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
+                    int d[4];
+                    mma_s8_16832_zc(d, A0, b.x, b.y);
+                    mma_s8_16832(d, A1, b.z, b.w);
+                    acc_f[c][0] = fmaf((float)d[0], s0, acc_f[c][0]);
+                    acc_f[c][1] = fmaf((float)d[1], s0, acc_f[c][1]);
+                    acc_f[c][2] = fmaf((float)d[2], s1, acc_f[c][2]);
+                    acc_f[c][3] = fmaf((float)d[3], s1, acc_f[c][3]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < NT; ++c) {
+                    const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
+                    mma_s8_16832(acc_i[c], A0, b.x, b.y);
+                    mma_s8_16832(acc_i[c], A1, b.z, b.w);
+                }
             }
         }
     }
-    if (ok) {  // end marker
-        const int s = it % a.slots;
-        if (it < a.slots || fz_wait(&sh.empty[s], ((it / a.slots) - 1) & 1, a.err)) {
-            if (lane == 0) sh.meta_item[s] = -1;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.full[s]);
-            ++it;
+}
+
+template <int NT, bool GS>
+__device__ __forceinline__ void fz_stage_down(const uint8_t* sl, int ns, int half, int rb, int lane,
+                                              int rec_dn, float acc_f[NT][4]) {
+    const int g = lane >> 2, t = lane & 3;
+    const float lanefac = t < 2 ? 256.0f : 1.0f;
+    const int nsh = ns / 2, j0 = half * nsh;
+    const uint8_t* cp = sl + (j0 * 8 + rb) * 512 + lane * 16;
+    const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + (g & 3) * rec_dn + j0 * 128;
+    // inverse scales of h for the two pairs of this lane's columns
+    const float* hsc = reinterpret_cast<const float*>(sl + kFzActOff + ns * 128 + 2 * (t & 1) * rec_dn) + j0 / 2;
+    const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff) + j0 * 128 + 16 * rb + g;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        if (jj < nsh) {
+            uint32_t A0[4], A1[4];
+            fz_decode_step(cp + jj * 4096, A0, A1);
+            const float s0 = GS ? scl[jj * 128] * lanefac : lanefac;
+            const float s1 = GS ? scl[jj * 128 + 8] * lanefac : lanefac;
+#pragma unroll
+            for (int c = 0; c < NT; ++c) {
+                const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_dn + jj * 128);
+                int d[4];
+                mma_s8_16832_zc(d, A0, b.x, b.y);
+                mma_s8_16832(d, A1, b.z, b.w);
+                const float* hs = reinterpret_cast<const float*>(
+                    reinterpret_cast<const uint8_t*>(hsc) + 4 * c * rec_dn) + jj / 2;
+                const float h0 = hs[0];
+                const float h1 = *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(hs) + rec_dn);
+                acc_f[c][0] = fmaf((float)d[0], s0 * h0, acc_f[c][0]);
+                acc_f[c][1] = fmaf((float)d[1], s0 * h1, acc_f[c][1]);
+                acc_f[c][2] = fmaf((float)d[2], s1 * h0, acc_f[c][2]);
+                acc_f[c][3] = fmaf((float)d[3], s1 * h1, acc_f[c][3]);
+            }
         }
     }
-    // leave only once every copy issued into the ring has landed
-    for (int j = it > a.slots ? it - a.slots : 0; j < it; ++j)
-        fz_wait(&sh.full[j % a.slots], (j / a.slots) & 1, nullptr);
 }
 
 }  // namespace coli
 
 namespace coli {
 
+// Hand a finished item to the service warp: every consumer warp arrives on
+// the record's barrier after its own global writes (warp 0 writes the record).
+struct FzHand {
+    int slot = 0, pushed = 0;
+    uint32_t lap = 0;
+};
+__device__ __forceinline__ bool fz_hand_push(FusedShared& sh, FzHand& h, int item, int32_t* err) {
+    const int lane = threadIdx.x & 31;
+    if (h.pushed >= kFzHand && !fz_wait(&sh.hand_empty[h.slot], h.lap ^ 1u, err)) return false;
+    if (threadIdx.x == 0) sh.hand_item[h.slot] = item;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.hand_full[h.slot]);
+    ++h.pushed;
+    if (++h.slot == kFzHand) { h.slot = 0; h.lap ^= 1u; }
+    return true;
+}
+
 // ---------------------------------------------------------------------------
-// Consumer warps.  Warp w: gate/up -> matrix w / 8 (gate, up), 16-row block
-// w % 8, every step of the stage; down -> 16-row block w % 8, half w / 8 of the
-// stage's steps.  Accumulators: acc_i (int32, exact) and acc_f (f32).  After an
-// MMA, lane (g, t) holds rows g, g + 8 and columns 2t, 2t + 1 of an 8-column
-// group c: column n carries pair 4c + (n & 3), high digit for n < 4, low digit
-// for n >= 4, so lanes t and t ^ 2 hold the two digits of the same pairs.
+// Consumer warps: stages, then per item an epilogue that exchanges partial
+// results through shared memory, writes h (gate/up) or o (down) to global
+// memory and hands the item to the service warp.
 // ---------------------------------------------------------------------------
 template <int NT, bool GS>
 __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, uint8_t* ring,
-                                           uint64_t* cbar, int n_units) {
+                                           int n_units) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int rb = warp & 7, half = warp >> 3;
-    const int TG = a.I / 128;
+    const int TG = a.I / 128, TD = a.H / 128;
     const int P = a.T * (a.k + a.n_shared);
     const int ns_gu = fz_ns_gateup(a.H), ns_dn = fz_ns_down(a.I);
     const int rec_gu = fz_rec_bytes(ns_gu), rec_dn = fz_rec_bytes(ns_dn);
     const float lanefac = t < 2 ? 256.0f : 1.0f;
-    int32_t* gu_done = a.sync + 1;
-    int32_t* dn_done = a.sync + 1 + kFzMaxUnits;
-    uint32_t cphase = 0;
-
+    const bool wr = t < 2;  // after the digit combine: lanes holding results
+    uint32_t cphase = 0, lap = 0;
+    int s = 0;
+    FzHand hand;
+    FzItem w{0, 0, 0};
+    int p0 = 0, np = 0, nst = 0;
+    float sw0 = 1.0f, sw1 = 1.0f;  // per-row weight scales of rows g, g + 8
     int acc_i[NT][4];
     float acc_f[NT][4];
-    for (int it = 0;; ++it) {
-        const int s = it % a.slots;
-        if (!fz_wait(&sh.full[s], (it / a.slots) & 1, a.err)) return;
+    for (;;) {
+        if (!fz_wait(&sh.full[s], lap, a.err)) return;
         const int item = sh.meta_item[s], st = sh.meta_st[s];
-        if (item < 0) return;
-        const bool gu = item < n_units * TG;
-        const int u = gu ? item / TG : (item - n_units * TG) / (a.H / 128);
-        const int rt = gu ? item % TG : (item - n_units * TG) % (a.H / 128);
-        const int p0 = sh.u_p0[u], np = sh.u_p1[u] - p0;
-        const int ns = gu ? ns_gu : ns_dn;
-        const int nst = (gu ? a.H : a.I) / 64 / ns;
-        if (st == 0) {
+        if (item < 0) {
+            fz_hand_push(sh, hand, -1, a.err);
+            return;
+        }
+        if (st == 0) {  // a new item
+            w = fz_item(item, n_units, TG, TD);
+            p0 = sh.u_p0[w.u];
+            np = sh.u_p1[w.u] - p0;
+            nst = w.gu ? a.H / 64 / ns_gu : a.I / 64 / ns_dn;
 #pragma unroll
             for (int c = 0; c < NT; ++c)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) { acc_i[c][i] = 0; acc_f[c][i] = 0.0f; }
         }
         const uint8_t* sl = ring + (int64_t)s * a.slot_bytes;
-        if (gu) {
-            const int m = half;
-            const uint8_t* codes = sl + m * ns * 4096 + rb * 512 + lane * 16;
-            const uint8_t* act = sl + kFzActOff + (g >> 2) * 64 + t * 16 + (g & 3) * rec_gu;
-            const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff + m * ns * 512) + 16 * rb + g;
-            for (int j = 0; j < ns; ++j) {
-                uint32_t A0[4], A1[4];
-                fz_decode_step(codes + j * 4096, A0, A1);
-                if (GS) {
-                    const float s0 = scl[j * 128] * lanefac, s1 = scl[j * 128 + 8] * lanefac;
-#pragma unroll
-                    for (int c = 0; c < NT; ++c) {
-                        const uint4 b = *reinterpret_cast<const uint4*>(act + 4 * c * rec_gu + j * 128);
-                        int d[4];
-                        mma_s8_16832_zc(d, A0, b.x, b.y);
-                        mma_s8_16832(d, A1, b.z, b.w);
-                        acc_f[c][0] = fmaf((float)d[0], s0, acc_f[c][0]);
-                        acc_f[c][1] = fmaf((float)d[1], s0, acc_f[c][1]);
-                        acc_f[c][2] = fmaf((float)d[2], s1, acc_f[c][2]);
-                        acc_f[c][3] = fmaf((float)d[3], s1, acc_f[c][3]);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < NT; ++c) {
-                        const uint4 b = *reinterpret_cast<const uint4*>(act + 4 * c * rec_gu + j * 128);
-                        mma_s8_16832(acc_i[c], A0, b.x, b.y);
-                        mma_s8_16832(acc_i[c], A1, b.z, b.w);
-                    }
-                }
-            }
-        } else {
-            const uint8_t* codes = sl + rb * 512 + lane * 16;
-            const uint8_t* act = sl + kFzActOff + (g >> 2) * 64 + t * 16 + (g & 3) * rec_dn;
-            const uint8_t* hsc = sl + kFzActOff + ns * 128 + 2 * (t & 1) * rec_dn;
-            const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff) + 16 * rb + g;
-            const int j0 = half * (ns / 2), j1 = j0 + ns / 2;
-            for (int j = j0; j < j1; ++j) {
-                uint32_t A0[4], A1[4];
-                fz_decode_step(codes + j * 4096, A0, A1);
-                const float s0 = GS ? scl[j * 128] * lanefac : lanefac;
-                const float s1 = GS ? scl[j * 128 + 8] * lanefac : lanefac;
-#pragma unroll
-                for (int c = 0; c < NT; ++c) {
-                    const uint4 b = *reinterpret_cast<const uint4*>(act + 4 * c * rec_dn + j * 128);
-                    int d[4];
-                    mma_s8_16832_zc(d, A0, b.x, b.y);
-                    mma_s8_16832(d, A1, b.z, b.w);
-                    // inverse scales of h for the two pairs of this lane's columns
-                    const float* hs = reinterpret_cast<const float*>(hsc + 4 * c * rec_dn) + j / 2;
-                    const float h0 = hs[0];
-                    const float h1 = *reinterpret_cast<const float*>(
-                        reinterpret_cast<const uint8_t*>(hs) + rec_dn);
-                    acc_f[c][0] = fmaf((float)d[0], s0 * h0, acc_f[c][0]);
-                    acc_f[c][1] = fmaf((float)d[1], s0 * h1, acc_f[c][1]);
-                    acc_f[c][2] = fmaf((float)d[2], s1 * h0, acc_f[c][2]);
-                    acc_f[c][3] = fmaf((float)d[3], s1 * h1, acc_f[c][3]);
-                }
-            }
+        if (w.gu) fz_stage_gateup<NT, GS>(sl, ns_gu, half, rb, lane, rec_gu, acc_i, acc_f);
+        else      fz_stage_down<NT, GS>(sl, ns_dn, half, rb, lane, rec_dn, acc_f);
+        const bool last = st == nst - 1;
+        if (!GS && last) {
+            const float* rs = reinterpret_cast<const float*>(sl + kFzScaleOff + (w.gu ? half * 512 : 0)) +
+                              16 * rb + g;
+            sw0 = rs[0];
+            sw1 = rs[8];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[s]);
-        if (st != nst - 1) continue;
+        if (++s == a.slots) { s = 0; lap ^= 1u; }
+        if (!last) continue;
 
         // ---------------- epilogue of the item ----------------
         float v[NT][4];
@@ -517,28 +604,25 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
         for (int c = 0; c < NT; ++c)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float x = (gu && !GS) ? (float)acc_i[c][i] * lanefac : acc_f[c][i];
+                float x = (w.gu && !GS) ? (float)acc_i[c][i] * lanefac : acc_f[c][i];
                 x += __shfl_xor_sync(0xffffffffu, x, 2);  // high digit * 256 + low digit
+                if (!GS) x *= (i >> 1) ? sw1 : sw0;
                 v[c][i] = x;
             }
         // lanes t < 2 now hold rows g + 8 (i >> 1), pairs 4c + 2t + (i & 1)
-        const bool wr = t < 2;
-        if (gu) {
+        if (w.gu) {
             const int m = half;
-            const float* sw = reinterpret_cast<const float*>(a.experts + (int64_t)sh.u_exp[u] * a.blob_bytes +
-                                                             a.L.scales[m]) + (int64_t)rt * 128 + 16 * rb;
 #pragma unroll
             for (int c = 0; c < NT; ++c)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int pp = 4 * c + 2 * t + (i & 1), rr = g + 8 * (i >> 1);
-                    float x = v[c][i];
-                    if (!GS) x *= __ldg(sw + rr);
-                    if (wr && pp < np) x *= __ldg(a.xinv8 + sh.pair_tok[p0 + pp]) * 0.0625f;
-                    v[c][i] = x;
-                    if (m == 1 && wr && pp < np) sh.xch[rb][rr][pp] = x;
+                    if (wr && pp < np) {
+                        v[c][i] *= sh.xinv[sh.pair_tok[p0 + pp]] * 0.0625f;
+                        if (m == 1) sh.xch[rb][rr][pp] = v[c][i];
+                    }
                 }
-            if (!fz_cbar(cbar, cphase, a.err)) return;
+            if (!fz_cbar(&sh.cbar, cphase, a.err)) return;
             if (m == 0) {
 #pragma unroll
                 for (int c = 0; c < NT; ++c) {
@@ -562,9 +646,9 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                     }
                 }
             }
-            if (!fz_cbar(cbar, cphase, a.err)) return;
+            if (!fz_cbar(&sh.cbar, cphase, a.err)) return;
             if (m == 0 && wr) {
-                const int dstep = 2 * rt + rb / 4;          // down step holding these rows of h
+                const int dstep = 2 * w.rt + rb / 4;  // down step holding these rows of h
                 const int sd = dstep / ns_dn, jj = dstep % ns_dn;
 #pragma unroll
                 for (int c = 0; c < NT; ++c)
@@ -587,15 +671,10 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                             rec[jj * 128 + 64 + pos] = (int8_t)lo;
                         }
                         if (rb == 0 && g == 0)
-                            reinterpret_cast<float*>(rec + ns_dn * 128)[(2 * rt % ns_dn) / 2] = inv;
+                            reinterpret_cast<float*>(rec + ns_dn * 128)[(2 * w.rt % ns_dn) / 2] = inv;
                     }
             }
-            __threadfence();
-            if (!fz_cbar(cbar, cphase, a.err)) return;
-            if (threadIdx.x == 0) atomicAdd(gu_done + u, 1);
         } else {
-            const float* sw = reinterpret_cast<const float*>(a.experts + (int64_t)sh.u_exp[u] * a.blob_bytes +
-                                                             a.L.scales[2]) + (int64_t)rt * 128 + 16 * rb;
             if (half == 1 && wr) {
 #pragma unroll
                 for (int c = 0; c < NT; ++c)
@@ -605,7 +684,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                         if (pp < np) sh.xch[rb][rr][pp] = v[c][i];
                     }
             }
-            if (!fz_cbar(cbar, cphase, a.err)) return;
+            if (!fz_cbar(&sh.cbar, cphase, a.err)) return;
             if (half == 0 && wr) {
 #pragma unroll
                 for (int c = 0; c < NT; ++c)
@@ -613,33 +692,68 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                     for (int i = 0; i < 4; ++i) {
                         const int pp = 4 * c + 2 * t + (i & 1), rr = g + 8 * (i >> 1);
                         if (pp >= np) continue;
-                        float x = v[c][i] + sh.xch[rb][rr][pp];
-                        x *= (GS ? 1.0f : __ldg(sw + rr)) * 0.0625f;
-                        a.o[(int64_t)(p0 + pp) * a.H + rt * 128 + 16 * rb + rr] = x;
+                        // the half-1 partial was scaled by its lanes too
+                        const float x = (v[c][i] + sh.xch[rb][rr][pp]) * 0.0625f;
+                        a.o[(int64_t)(p0 + pp) * a.H + w.rt * 128 + 16 * rb + rr] = x;
                     }
             }
-            __threadfence();
-            if (!fz_cbar(cbar, cphase, a.err)) return;
-            if (threadIdx.x == 0) sh.last = atomicAdd(dn_done + rt, 1) == n_units - 1;
-            if (!fz_cbar(cbar, cphase, a.err)) return;
-            if (sh.last) {  // every unit's o of this 128-row block is written: form y
-                __threadfence();
-                const int Tk = a.T * a.k;
-                for (int q = threadIdx.x; q < a.T * 128; q += 32 * kFzWarps) {
-                    const int tt = q >> 7, r = rt * 128 + (q & 127);
-                    float acc = 0.0f;
-                    for (int j = 0; j < a.k; ++j) {
-                        const int p = sh.inv[tt * a.k + j];
-                        acc = fmaf(sh.pick_w[tt * a.k + j], __ldcg(a.o + (int64_t)p * a.H + r), acc);
-                    }
-                    for (int s2 = 0; s2 < a.n_shared; ++s2)
-                        acc += __ldcg(a.o + ((int64_t)Tk + (int64_t)s2 * a.T + tt) * a.H + r);
-                    if (a.residual) acc = a.residual[(int64_t)tt * a.H + r] + acc;
-                    a.y[(int64_t)tt * a.H + r] = acc;
-                }
-            }
-            // sh.last is rewritten only after the next item's barriers
         }
+        if (!fz_hand_push(sh, hand, item, a.err)) return;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Service warp: for every finished item, make its global writes visible and
+// count it (gate/up: per unit; down: per 128-row block of y).  The item that
+// completes a block of y has this warp form y there: for each token, the sum
+// over its picks in pick order of w_j * o_j, then the shared experts, then the
+// residual.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fz_service(const FusedArgs& a, FusedShared& sh, int n_units) {
+    const int lane = threadIdx.x & 31;
+    const int TG = a.I / 128, TD = a.H / 128;
+    int32_t* gu_done = a.sync + 1;
+    int32_t* dn_done = a.sync + 1 + kFzMaxUnits;
+    const int Tk = a.T * a.k;
+    int hs = 0;
+    uint32_t hlap = 0;
+    for (;;) {
+        if (!fz_wait(&sh.hand_full[hs], hlap, a.err)) return;
+        const int item = sh.hand_item[hs];
+        if (item < 0) return;
+        const FzItem w = fz_item(item, n_units, TG, TD);
+        int last = 0;
+        if (lane == 0) {
+            __threadfence();  // the consumers' writes of this item, before the count
+            if (w.gu) atomicAdd(gu_done + w.u, 1);
+            else last = atomicAdd(dn_done + w.rt, 1) == n_units - 1;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {  // every unit's o of this 128-row block is written: form y
+            __threadfence();
+            for (int q = lane; q < a.T * 128; q += 32) {
+                const int tt = q >> 7, r = w.rt * 128 + (q & 127);
+                float acc = 0.0f;
+                for (int j0 = 0; j0 < a.k; j0 += 8) {  // loads of 8 picks in flight
+                    float ov[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        ov[jj] = j0 + jj < a.k
+                                     ? __ldcg(a.o + (int64_t)sh.inv[tt * a.k + j0 + jj] * a.H + r)
+                                     : 0.0f;
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        if (j0 + jj < a.k) acc = fmaf(sh.pick_w[tt * a.k + j0 + jj], ov[jj], acc);
+                }
+                for (int s2 = 0; s2 < a.n_shared; ++s2)
+                    acc += __ldcg(a.o + ((int64_t)Tk + (int64_t)s2 * a.T + tt) * a.H + r);
+                if (a.residual) acc = a.residual[(int64_t)tt * a.H + r] + acc;
+                a.y[(int64_t)tt * a.H + r] = acc;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.hand_empty[hs]);
+        if (++hs == kFzHand) { hs = 0; hlap ^= 1u; }
     }
 }
 
@@ -648,16 +762,18 @@ __global__ void __launch_bounds__(kFzThreads, 1)
 moe_fused_kernel(FusedArgs a) {
     extern __shared__ __align__(128) uint8_t fz_smem[];
     __shared__ FusedShared sh;
-    __shared__ __align__(8) uint64_t cbar;
     const int n_units = fz_route_union(a, sh, reinterpret_cast<int*>(fz_smem));
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.slots; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kFzWarps); }
-        mbar_init(&cbar, kFzWarps);
+        for (int h = 0; h < kFzHand; ++h) { mbar_init(&sh.hand_full[h], kFzWarps); mbar_init(&sh.hand_empty[h], 1); }
+        mbar_init(&sh.cbar, kFzWarps);
         fence_mbar_init();
     }
     __syncthreads();
-    if ((threadIdx.x >> 5) == kFzWarps) fz_produce<GS>(a, sh, fz_smem, n_units);
-    else fz_consume<NT, GS>(a, sh, fz_smem, &cbar, n_units);
+    const int warp = threadIdx.x >> 5;
+    if (warp == kFzProducer) fz_produce<GS>(a, sh, fz_smem, n_units);
+    else if (warp == kFzService) fz_service(a, sh, n_units);
+    else fz_consume<NT, GS>(a, sh, fz_smem, n_units);
 }
 
 }  // namespace coli

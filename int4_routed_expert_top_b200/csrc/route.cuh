@@ -62,6 +62,7 @@ act_quant_kernel(const XT* __restrict__ x, int T, int H, __half* __restrict__ xq
 // share build the fp16 activation operand (xq) when xq != nullptr.
 // ---------------------------------------------------------------------------
 constexpr int kRouterMaxSlice = 1024;  // columns per warp slice (<= 8 loads per lane)
+constexpr int kRouterMaxT = 32;        // tokens per call of the small-batch router
 
 // ---------------------------------------------------------------------------
 // s8 activation operand of the fused small-batch kernel (fused.cuh): each value
@@ -160,30 +161,44 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
         }
         return;
     }
+    // The CTA's 8 warps are the KS slices of 8 / KS experts (KS divides 8): the
+    // slices are summed here, in slice order, and z[t][e] is written.
+    __shared__ float part[8][kRouterMaxT];
     const int gw = blockIdx.x * 8 + warp;
     const int e = gw / KS, ks = gw % KS;
-    if (e >= E) return;
+    const bool valid = e < E;
     const int SL = H / KS;  // multiple of 128, at most kRouterMaxSlice
-    const float* wrow = wr + (int64_t)e * H + (int64_t)ks * SL;
-    float4 wv[kRouterMaxSlice / 128];
+    if (valid) {
+        const float* wrow = wr + (int64_t)e * H + (int64_t)ks * SL;
+        float4 wv[kRouterMaxSlice / 128];
 #pragma unroll
-    for (int i = 0; i < kRouterMaxSlice / 128; ++i)
-        if (i * 128 < SL) wv[i] = __ldg(reinterpret_cast<const float4*>(wrow + i * 128 + lane * 4));
-    for (int t = 0; t < T; ++t) {
-        const XT* xr = x + (int64_t)t * H + (int64_t)ks * SL + lane * 4;
-        float acc = 0.0f;
+        for (int i = 0; i < kRouterMaxSlice / 128; ++i)
+            if (i * 128 < SL) wv[i] = __ldg(reinterpret_cast<const float4*>(wrow + i * 128 + lane * 4));
+        for (int t = 0; t < T; ++t) {
+            const XT* xr = x + (int64_t)t * H + (int64_t)ks * SL + lane * 4;
+            float acc = 0.0f;
 #pragma unroll
-        for (int i = 0; i < kRouterMaxSlice / 128; ++i) {
-            if (i * 128 < SL) {
-                const XT* xp = xr + i * 128;
-                acc = fmaf(wv[i].x, to_f32(xp[0]), acc);
-                acc = fmaf(wv[i].y, to_f32(xp[1]), acc);
-                acc = fmaf(wv[i].z, to_f32(xp[2]), acc);
-                acc = fmaf(wv[i].w, to_f32(xp[3]), acc);
+            for (int i = 0; i < kRouterMaxSlice / 128; ++i) {
+                if (i * 128 < SL) {
+                    const XT* xp = xr + i * 128;
+                    acc = fmaf(wv[i].x, to_f32(xp[0]), acc);
+                    acc = fmaf(wv[i].y, to_f32(xp[1]), acc);
+                    acc = fmaf(wv[i].z, to_f32(xp[2]), acc);
+                    acc = fmaf(wv[i].w, to_f32(xp[3]), acc);
+                }
             }
+            acc = warp_sum(acc);
+            if (lane == 0) part[warp][t] = acc;
         }
-        acc = warp_sum(acc);
-        if (lane == 0) zpart[((int64_t)ks * T + t) * E + e] = acc;
+    }
+    __syncthreads();
+    const int per = 8 / KS;  // experts of this CTA
+    for (int j = threadIdx.x; j < per * T; j += 256) {
+        const int el = j / T, t = j % T, ee = blockIdx.x * per + el;
+        if (ee >= E) continue;
+        float z = 0.0f;
+        for (int k2 = 0; k2 < KS; ++k2) z += part[el * KS + k2][t];
+        zpart[(int64_t)t * E + ee] = z;
     }
 }
 
