@@ -399,12 +399,13 @@ def main():
         units = uniq_slot[st_ms[:, -1].astype(int)] + wl.n_shared
         stage_mean = st_ms[:, :-1].mean(0)
         if fused:
-            # one kernel: top-k, union, gate/up, down and combine; its time is the
-            # "gateup" stage (the union/down/combine marks bracket nothing)
+            # moe_fused_kernel (top-k, union, gate/up, down partials) is the
+            # "gateup" stage, moe_combine_kernel the "combine" stage
             kern_bytes = units * (gu_bytes_unit + dn_bytes_unit)
             ach = kern_bytes.sum() / (st_ms[:, 2].sum() / 1e3) / 1e9
-            kname = "moe_fused_kernel (top-k, union, gate/up, down, combine)"
-            line["stages_us"] = {"router": 1e3 * stage_mean[0], "fused": 1e3 * stage_mean[2]}
+            kname = "moe_fused_kernel (top-k, union, gate/up, down partial products)"
+            line["stages_us"] = {"router": 1e3 * stage_mean[0], "fused": 1e3 * stage_mean[2],
+                                 "combine": 1e3 * stage_mean[4]}
         else:
             gu_ach = (units * gu_bytes_unit).sum() / (st_ms[:, 2].sum() / 1e3) / 1e9
             dn_ach = (units * dn_bytes_unit).sum() / (st_ms[:, 3].sum() / 1e3) / 1e9
@@ -421,7 +422,7 @@ def main():
         line["int4_weight_gbs"] = weight_gbs
         line["int4_weight_frac_of_hbm"] = weight_gbs / hbm_gbs
         line["unique_experts_per_step"] = float(uniq.mean())
-        line["gpu_launches"] = (2 if fused else 6) * K
+        line["gpu_launches"] = (3 if fused else (4 if T < 48 else 9)) * K
     else:
         line["gpu_launches"] = 7 * wl.layers * K
     line["config"] = cfg

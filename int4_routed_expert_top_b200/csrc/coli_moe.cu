@@ -59,7 +59,7 @@ struct WsPlan {
     int64_t zpart, idx, w, offsets, pair_tok, pair_slot, uniq, n_uniq, inv;
     int64_t unit_expert, unit_begin, unit_end, n_units, counters, err;
     int64_t xq, xinv, hq, hinv, o, xg, hg, hmax, hsc;
-    int64_t xq8, xinv8, hq8, fsync;  // fused small-batch kernel (T <= kFzMaxT only)
+    int64_t xq8, xinv8, part, queue, sel;  // fused small-batch kernel (T <= kFzMaxT only)
     int64_t total;
 };
 
@@ -99,13 +99,13 @@ WsPlan plan_ws(const coli_moe_desc& d, int T) {
     p.hmax = take(P * 4);                       //   per-pair max |h|
     p.hsc = take(P * 4);                        //   per-pair inverse scale of h
     if (fused_fits(d, T)) {
-        const int ns_dn = fz_ns_down(d.I);
         p.xq8 = take((int64_t)T * d.H * 2);
         p.xinv8 = take((int64_t)T * 4);
-        p.hq8 = take((int64_t)(d.I / 64 / ns_dn) * P * fz_rec_bytes(ns_dn));
-        p.fsync = take((int64_t)fz_sync_ints(d.H) * 4);
+        p.part = take(P * (d.I / 128) * d.H * 4);
+        p.queue = take(4);
+        p.sel = take((int64_t)T * d.E * 4);
     } else {
-        p.xq8 = p.xinv8 = p.hq8 = p.fsync = 0;
+        p.xq8 = p.xinv8 = p.part = p.queue = p.sel = 0;
     }
     p.total = off;
     return p;
@@ -396,51 +396,81 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
 // ---------------------------------------------------------------------------
 int sm_count() { return gemm_grid(); }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous one (router, then fused) finishes; it waits
+// (griddepcontrol.wait) before reading what that kernel wrote.
+template <typename... Args>
+int launch_pdl(void (*kern)(Args...), dim3 grid, int threads, int smem, cudaStream_t st,
+               const char* what, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) return fail(COLI_E_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return check_launch(what);
+}
+
 template <int NT, bool GS>
 int launch_fused_t(const FusedArgs& a, cudaStream_t st) {
     const int smem = a.slots * a.slot_bytes;
     int rc = set_smem((const void*)moe_fused_kernel<NT, GS>, smem);
     if (rc) return rc;
-    moe_fused_kernel<NT, GS><<<sm_count(), kFzThreads, smem, st>>>(a);
-    return check_launch("fused moe");
+    return launch_pdl(moe_fused_kernel<NT, GS>, dim3(sm_count()), kFzThreads, smem, st, "fused moe", a);
 }
 
+template <typename Mark>
 int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int KS,
-                 const float* residual, float* y, cudaStream_t st) {
+                 const float* residual, float* y, cudaStream_t st, Mark&& mark) {
     const coli_moe_desc& d = l->d;
     FusedArgs a;
     a.experts = static_cast<const uint8_t*>(d.experts);
     a.blob_bytes = l->L.bytes;
     a.L = l->L;
-    a.zpart = at<float>(ws, p.zpart);
-    a.KS = KS;
-    a.bias = d.router_b;
+    (void)KS;  // the small-batch router leaves one slice: the scores themselves
+    a.score = at<float>(ws, p.zpart);
+    a.sel = at<float>(ws, p.sel);
     a.routed_scale = d.routed_scale;
     a.norm_topk = d.norm_topk;
     a.xq8 = at<int8_t>(ws, p.xq8);
     a.xinv8 = at<float>(ws, p.xinv8);
-    a.hq8 = at<int8_t>(ws, p.hq8);
-    a.o = at<float>(ws, p.o);
-    a.sync = at<int32_t>(ws, p.fsync);
+    a.part = at<float>(ws, p.part);
+    a.queue = at<int32_t>(ws, p.queue);
     a.idx = at<int32_t>(ws, p.idx);
     a.w = at<float>(ws, p.w);
-    a.residual = residual;
-    a.y = y;
+    a.inv = at<int32_t>(ws, p.inv);
     a.err = at<int32_t>(ws, p.err);
     a.T = T; a.E = d.E; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int NT = T <= 4 ? 1 : (T <= 8 ? 2 : 4);
-    const int rec = std::max(fz_rec_bytes(fz_ns_gateup(d.H)), fz_rec_bytes(fz_ns_down(d.I)));
-    a.slot_bytes = (int)align256(kFzActOff + 4 * NT * rec);
+    a.slot_bytes = (int)align256(kFzActOff + 4 * NT * fz_rec_bytes(fz_ns_gateup(d.H)));
     const int budget = 227 * 1024 - (int)sizeof(FusedShared) - 1024;
-    a.slots = std::min(kFzMaxSlots, budget / a.slot_bytes);
+    a.slots = std::min(kFzSlots, budget / a.slot_bytes);
     if (a.slots < 2) return fail(COLI_E_UNSUPPORTED, "fused: ring does not fit");
     const bool gs = d.group != 0;
+    int rc;
     switch (NT) {
-        case 1: return gs ? launch_fused_t<1, true>(a, st) : launch_fused_t<1, false>(a, st);
-        case 2: return gs ? launch_fused_t<2, true>(a, st) : launch_fused_t<2, false>(a, st);
-        default: return gs ? launch_fused_t<4, true>(a, st) : launch_fused_t<4, false>(a, st);
+        case 1: rc = gs ? launch_fused_t<1, true>(a, st) : launch_fused_t<1, false>(a, st); break;
+        case 2: rc = gs ? launch_fused_t<2, true>(a, st) : launch_fused_t<2, false>(a, st); break;
+        default: rc = gs ? launch_fused_t<4, true>(a, st) : launch_fused_t<4, false>(a, st); break;
     }
+    if (rc) return rc;
+    if ((rc = mark(COLI_STAGE_DOWN))) return rc;
+    if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
+    CombineArgs c;
+    c.part = a.part;
+    c.inv = a.inv;
+    c.w = a.w;
+    c.residual = residual;
+    c.y = y;
+    c.T = T; c.k = d.k; c.n_shared = d.n_shared; c.H = d.H; c.TG = d.I / 128;
+    return launch_pdl(moe_combine_kernel, dim3(T * (d.H / 32)), 256, 0, st, "fused combine", c);
 }
 
 }  // namespace
@@ -637,17 +667,17 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         RouterExtras ex;
         ex.xq8 = at<int8_t>(ws, p.xq8);
         ex.xinv8 = at<float>(ws, p.xinv8);
-        ex.zero = at<int32_t>(ws, p.fsync);
-        ex.zero_n = fz_sync_ints(d.H);
+        ex.zero = at<int32_t>(ws, p.queue);
+        ex.zero_n = 1;
         ex.err = at<int32_t>(ws, p.err);
+        ex.sel = at<float>(ws, p.sel);
+        ex.bias = d.router_b;
         if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), nullptr, nullptr, st, &KS, &ex)))
             return rc;
-        // the fused kernel is the union, gate/up, down and combine stages at once
+        // the fused kernel is the union, gate/up and down stages at once
         if ((rc = mark(COLI_STAGE_UNION))) return rc;
         if ((rc = mark(COLI_STAGE_GATEUP))) return rc;
-        if ((rc = launch_fused(layer, T, ws, p, KS, residual, y, st))) return rc;
-        if ((rc = mark(COLI_STAGE_DOWN))) return rc;
-        if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
+        if ((rc = launch_fused(layer, T, ws, p, KS, residual, y, st, mark))) return rc;
         if ((rc = mark(COLI_STAGES))) return rc;
         if (idx_out && cudaMemcpyAsync(idx_out, idx, sizeof(int32_t) * T * d.k,
                                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)

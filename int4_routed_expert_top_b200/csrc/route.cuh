@@ -142,6 +142,10 @@ struct RouterExtras {
     int32_t* zero = nullptr;
     int zero_n = 0;
     int32_t* err = nullptr;  // device error flags, cleared by the same block
+    // scores for the fused kernel: when set, zpart receives s = sigmoid(z) and
+    // sel receives s + bias instead of the logits
+    float* sel = nullptr;
+    const float* bias = nullptr;
 };
 
 template <typename XT>
@@ -150,6 +154,9 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
                    int E, int KS, float* __restrict__ zpart, int router_blocks,
                    RouterExtras ex) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the dependent fused kernel may start its prologue (it waits for this
+    // grid's completion before reading anything written here)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if ((int)blockIdx.x >= router_blocks) {
         const int b = blockIdx.x - router_blocks;
         if (b < T) {  // one CTA per token: activation operand
@@ -198,7 +205,13 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
         if (ee >= E) continue;
         float z = 0.0f;
         for (int k2 = 0; k2 < KS; ++k2) z += part[el * KS + k2][t];
-        zpart[(int64_t)t * E + ee] = z;
+        if (ex.sel) {
+            const float sc = 1.0f / (1.0f + expf(-z));
+            zpart[(int64_t)t * E + ee] = sc;
+            ex.sel[(int64_t)t * E + ee] = sc + __ldg(ex.bias + ee);
+        } else {
+            zpart[(int64_t)t * E + ee] = z;
+        }
     }
 }
 
