@@ -47,9 +47,11 @@
  *      codes_m  [R/128][K/64][8][32][16 bytes]: unit (t, s, b, l) belongs to
  *               rows r0 = 128t + 16b + l/4 and r1 = r0 + 8, and holds four
  *               32-bit words j = 0..3 for columns c0 = 64s + 16j + 4(l%4) ..
- *               c0+3; in word j, bits 4p..4p+3 hold the signed nibble of
- *                 p: 0 (r0,c0)  1 (r0,c0+2)  2 (r1,c0)  3 (r1,c0+2)
- *                    4 (r0,c0+1) 5 (r0,c0+3) 6 (r1,c0+1) 7 (r1,c0+3)
+ *               c0+3; in word j, byte i holds column c0 + i: row r0's signed
+ *               nibble in bits 4-7, row r1's in bits 0-3, i.e. bits 4p..4p+3
+ *               hold the nibble of
+ *                 p: 0 (r1,c0)   1 (r0,c0)   2 (r1,c0+1) 3 (r0,c0+1)
+ *                    4 (r1,c0+2) 5 (r0,c0+2) 6 (r1,c0+3) 7 (r0,c0+3)
  *      scales_m [R/128][K/G][128] f32          scale of row 128t + r, group g
  *    Order: codes_gate, codes_up, codes_down, scales_gate, scales_up,
  *    scales_down; each section starts on a 256-byte boundary and the blob size

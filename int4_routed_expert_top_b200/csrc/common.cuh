@@ -49,16 +49,19 @@ __host__ __device__ inline BlobLayout make_blob_layout(int H, int I, int group) 
 // block is 32 units of 16 bytes, one per lane l = 4*g + t of a warp, so one warp
 // load of 512 bytes fetches a whole block.  Unit l holds rows r0 = 16*b + g and
 // r1 = r0 + 8 of the block, and for each 16-column sub-block j the 4 columns
-// c0 = 16*j + 4*t .. c0 + 3 of both rows: 8 nibbles in word j.  These are the
-// elements that lane owns in a 16x16 tensor-core operand tile (mma.sync A
-// fragment up to a column permutation, and the tcgen05 16x256b TMEM access).
-// Blocks are ordered [R/128][K/64][8][32 lanes], so the eight blocks of a
-// 128-row tile and one 64-column step are 4 KB of contiguous bytes.
+// c0 = 16*j + 4*t .. c0 + 3 of both rows: 8 nibbles in word j, byte i of the
+// word holding column c0 + i, row r0 in its high nibble and row r1 in its low
+// nibble.  These are the elements that lane owns in a 16x16 tensor-core operand
+// tile (mma.sync A fragment up to a column permutation, and the tcgen05
+// 16x256b TMEM access).  Blocks are ordered [R/128][K/64][8][32 lanes], so the
+// eight blocks of a 128-row tile and one 64-column step are 4 KB of contiguous
+// bytes.  With row r0 in the high nibbles, w & 0xF0F0F0F0 is row r0's four
+// values times 16 as signed bytes, and (w << 4) & 0xF0F0F0F0 row r1's.
 //
 // nibble position of (row r, column c) inside its 32-bit word
 __host__ __device__ inline int frag_nibble_shift(int r, int c) {
     const int upper = (r % 16) / 8, cc = c % 4;
-    return 4 * (upper * 2 + (cc >> 1)) + 16 * (cc & 1);
+    return 8 * cc + (upper ? 0 : 4);
 }
 
 // byte offset of the 16-byte unit of lane l, 16-row block b8 (0..7) of tile rt,
@@ -124,18 +127,6 @@ __device__ __forceinline__ uint32_t h2fma_16th_m72(uint32_t v) {
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(0x2C002C00u), "r"(0xD480D480u));
     return r;
 }
-// decode one fragment-tile word straight into an mma.sync A fragment:
-// a[0] = row g (c0, c0+1), a[1] = row g+8 (c0, c0+1), a[2] = row g (c0+2, c0+3),
-// a[3] = row g+8 (c0+2, c0+3).  With logical columns 2t,2t+1 <- c0,c0+1 and
-// 2t+8,2t+9 <- c0+2,c0+3 this is the m16n8k16 row-major A fragment of lane 4g+t.
-__device__ __forceinline__ void decode_frag_word(uint32_t w, uint32_t a[4]) {
-    const uint32_t w8 = w >> 8;
-    a[0] = h2sub_1032((w & 0x000F000Fu) ^ 0x64086408u);
-    a[1] = h2sub_1032((w8 & 0x000F000Fu) ^ 0x64086408u);
-    a[2] = h2fma_16th_m72((w & 0x00F000F0u) ^ 0x64806480u);
-    a[3] = h2fma_16th_m72((w8 & 0x00F000F0u) ^ 0x64806480u);
-}
-
 // D[16x8] (f32) (+)= A[16x16] (f16) * B[16x8] (f16), warp-wide
 __device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], uint32_t b0,
                                               uint32_t b1) {
@@ -165,17 +156,23 @@ struct DecodeK {
     uint32_t add = 0xD480D480u;   // -72 = -(1024 + 8*16)/16
 };
 
+// Decode one fragment-tile word straight into an mma.sync m16n8k16 A fragment:
+// a[0] = row r0 (c0, c0+1), a[1] = row r1 (c0, c0+1), a[2] = row r0 (c0+2, c0+3),
+// a[3] = row r1 (c0+2, c0+3).  Swapping the word's middle bytes puts columns
+// c0, c0+1 in the two 16-bit halves (row r0 at bits 4-7, row r1 at bits 0-3);
+// shifted right by 8, columns c0+2, c0+3 sit the same way.
 __device__ __forceinline__ void decode_word(uint32_t w, uint32_t a[4], const DecodeK& k) {
-    const uint32_t w8 = w >> 8;
+    const uint32_t p = __byte_perm(w, 0u, 0x3120);
+    const uint32_t p8 = p >> 8;
     uint32_t t0, t1, t2, t3;
-    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t0) : "r"(w), "r"(k.xlo));
-    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t1) : "r"(w8), "r"(k.xlo));
-    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t2) : "r"(w), "r"(k.xhi));
-    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t3) : "r"(w8), "r"(k.xhi));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(a[0]) : "r"(t0), "r"(k.sub));
+    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t0) : "r"(p), "r"(k.xhi));
+    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t1) : "r"(p), "r"(k.xlo));
+    asm("lop3.b32 %0, %1, 0x00F000F0, %2, 0x6a;" : "=r"(t2) : "r"(p8), "r"(k.xhi));
+    asm("lop3.b32 %0, %1, 0x000F000F, %2, 0x6a;" : "=r"(t3) : "r"(p8), "r"(k.xlo));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(a[0]) : "r"(t0), "r"(k.mul), "r"(k.add));
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(a[1]) : "r"(t1), "r"(k.sub));
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(a[2]) : "r"(t2), "r"(k.mul), "r"(k.add));
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(a[3]) : "r"(t3), "r"(k.mul), "r"(k.add));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(a[3]) : "r"(t3), "r"(k.sub));
 }
 
 // Activation operand: power-of-two scale 2^(14 - e) for a group whose largest

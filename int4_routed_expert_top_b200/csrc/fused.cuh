@@ -102,12 +102,11 @@ __device__ __forceinline__ void mma_s8_16832(int d[4], const uint32_t a[4], uint
 
 // One fragment-tile word (rows r0, r1 = r0 + 8; columns c0..c0+3, nibble order
 // documented in common.cuh) into two s8x4 registers: row r0 then row r1, each
-// holding 16 q for columns c0, c0+1, c0+2, c0+3 in byte order.
+// holding 16 q for columns c0, c0+1, c0+2, c0+3 in byte order (the nibble in
+// the high half of a byte reads as the signed byte 16 q).
 __device__ __forceinline__ void decode_word_s8(uint32_t w, uint32_t& r0, uint32_t& r1) {
-    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;  // (r0,c0) (r1,c0) (r0,c0+1) (r1,c0+1)
-    const uint32_t hi = w & 0xF0F0F0F0u;         // (r0,c0+2) (r1,c0+2) (r0,c0+3) (r1,c0+3)
-    r0 = __byte_perm(lo, hi, 0x6420);
-    r1 = __byte_perm(lo, hi, 0x7531);
+    r0 = w & 0xF0F0F0F0u;
+    r1 = (w << 4) & 0xF0F0F0F0u;
 }
 
 // L2 policy for data read exactly once (weights streamed into the ring)

@@ -148,8 +148,10 @@ struct RouterExtras {
     const float* bias = nullptr;
 };
 
+// (at most 48 registers, so that a CTA fits beside a CTA of the dependent
+// fused kernel, which then starts while the router finishes)
 template <typename XT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 5)
 router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restrict__ wr,
                    int E, int KS, float* __restrict__ zpart, int router_blocks,
                    RouterExtras ex) {

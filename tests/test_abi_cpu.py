@@ -59,11 +59,11 @@ def _unpack_blob(blob, H, I, group):
         off = sec_align(off + R * ng * 4)
     assert off == blob.size
     # word j of unit (t, s, b, l): nibble p at bits 4p.. holds
-    #   p: 0 (r0,c0) 1 (r0,c0+2) 2 (r1,c0) 3 (r1,c0+2) 4 (r0,c0+1) 5 (r0,c0+3)
-    #      6 (r1,c0+1) 7 (r1,c0+3); r0 = 128t + 16b + l//4, r1 = r0 + 8,
+    #   p: 0 (r1,c0) 1 (r0,c0) 2 (r1,c0+1) 3 (r0,c0+1) 4 (r1,c0+2) 5 (r0,c0+2)
+    #      6 (r1,c0+3) 7 (r0,c0+3); r0 = 128t + 16b + l//4, r1 = r0 + 8,
     #   c0 = 64s + 16j + 4(l%4)
-    dr = np.array([0, 0, 8, 8, 0, 0, 8, 8])
-    dc = np.array([0, 2, 0, 2, 1, 3, 1, 3])
+    dr = np.array([8, 0, 8, 0, 8, 0, 8, 0])
+    dc = np.array([0, 0, 1, 1, 2, 2, 3, 3])
     out = []
     for m, (R, K) in enumerate(mats):
         ng = 1 if group == 0 else K // group
