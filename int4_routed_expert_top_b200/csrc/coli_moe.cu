@@ -64,7 +64,8 @@ struct WsPlan {
 };
 
 bool fused_fits(const coli_moe_desc& d, int T) {
-    return T <= kFzMaxT && d.E <= kFzMaxE && d.k <= kFzMaxK && d.n_shared <= 4;
+    return T <= kFzMaxT && d.E <= kFzMaxE && d.k <= kFzMaxK && d.n_shared <= 4 &&
+           d.I / 128 <= kCombineMaxTiles;
 }
 
 WsPlan plan_ws(const coli_moe_desc& d, int T) {
@@ -470,7 +471,8 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     c.residual = residual;
     c.y = y;
     c.T = T; c.k = d.k; c.n_shared = d.n_shared; c.H = d.H; c.TG = d.I / 128;
-    return launch_pdl(moe_combine_kernel, dim3(T * (d.H / 32)), 256, 0, st, "fused combine", c);
+    const int warps = std::min(32, d.k + d.n_shared);
+    return launch_pdl(moe_combine_kernel, dim3(T * (d.H / 32)), 32 * warps, 0, st, "fused combine", c);
 }
 
 }  // namespace

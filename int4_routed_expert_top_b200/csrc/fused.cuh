@@ -49,7 +49,7 @@ constexpr int kFzMaxE = 256;                     // routed experts on this path
 constexpr int kFzMaxUnits = kFzMaxE + 4;
 constexpr int kFzMaxK = 32;
 constexpr int kFzMaxSlots = 6;
-constexpr int kFzSlots = 4;                      // ring stages (deeper rings stream slower)
+constexpr int kFzSlots = 5;                      // ring stages
 constexpr int kFzCodeBytes = 32768;              // int4 codes per stage
 constexpr int kFzScaleOff = kFzCodeBytes;        // gs64 scales, up to 4 KB
 constexpr int kFzActOff = kFzCodeBytes + 4096;   // activation records
@@ -725,11 +725,13 @@ moe_fused_kernel(FusedArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// y from the partial down products.  CTA (token t, 32 rows): warp w sums the
-// I/128 partials of pairs j = w, w + 8, .. (k routed picks, then the shared
-// experts) in tile order; warp 0 then adds them up in pick order, weighted,
-// then the shared experts, then the residual.
+// y from the partial down products.  CTA (token t, 32 rows), one warp per pick
+// j (k routed picks, then the shared experts): the warp sums pair j's I/128
+// partials in tile order (all loads in flight at once); warp 0 then adds the
+// picks up in pick order, weighted, then the shared experts, then the residual.
 // ---------------------------------------------------------------------------
+constexpr int kCombineMaxTiles = 32;  // I <= 4096
+
 struct CombineArgs {
     const float* part;     // [P][TG][H]
     const int32_t* inv;    // [T*k]
@@ -739,26 +741,26 @@ struct CombineArgs {
     int T, k, n_shared, H, TG;
 };
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(1024)
 moe_combine_kernel(CombineArgs c) {
     __shared__ float oj[kFzMaxK + 4][32];
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
     const int nrg = c.H / 32;
     const int t = blockIdx.x / nrg, r = (blockIdx.x - t * nrg) * 32 + lane;
     const int Tk = c.T * c.k, J = c.k + c.n_shared;
-    for (int j = warp; j < J; j += 8) {
+    for (int j = warp; j < J; j += nw) {
         const int p = j < c.k ? __ldg(c.inv + t * c.k + j) : Tk + (j - c.k) * c.T + t;
         const float* src = c.part + (int64_t)p * c.TG * c.H + r;
+        float pv[kCombineMaxTiles];
+#pragma unroll
+        for (int i = 0; i < kCombineMaxTiles; ++i)
+            pv[i] = i < c.TG ? __ldcg(src + (int64_t)i * c.H) : 0.0f;
         float o = 0.0f;
-        for (int t0 = 0; t0 < c.TG; t0 += 8) {  // eight tiles' loads in flight
-            float pv[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) pv[i] = t0 + i < c.TG ? __ldcg(src + (int64_t)(t0 + i) * c.H) : 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (t0 + i < c.TG) o += pv[i];
-        }
+        for (int i = 0; i < kCombineMaxTiles; ++i)
+            if (i < c.TG) o += pv[i];
         oj[j][lane] = o;
     }
     __syncthreads();
