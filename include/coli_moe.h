@@ -94,7 +94,7 @@ typedef enum coli_path {
     COLI_PATH_FUSED = 3  /* one persistent kernel for top-k, union, experts and
                             combine (mma.sync s8, exact int32 step sums);
                             T <= 16, E <= 256, k <= 32, n_shared <= 4,
-                            I <= 4096                                         */
+                            H a multiple of 256, I <= 4096                   */
 } coli_path;
 
 /* Thread-local description of the last error returned on this thread. */

@@ -65,7 +65,7 @@ struct WsPlan {
 
 bool fused_fits(const coli_moe_desc& d, int T) {
     return T <= kFzMaxT && d.E <= kFzMaxE && d.k <= kFzMaxK && d.n_shared <= 4 &&
-           d.I / 128 <= kCombineMaxTiles;
+           d.H % 256 == 0 && d.I / 128 <= kCombineMaxTiles;
 }
 
 WsPlan plan_ws(const coli_moe_desc& d, int T) {
@@ -466,7 +466,6 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
     CombineArgs c;
     c.part = a.part;
-    c.inv = a.inv;
     c.w = a.w;
     c.residual = residual;
     c.y = y;

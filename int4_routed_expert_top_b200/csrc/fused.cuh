@@ -60,8 +60,9 @@ constexpr int kFzRecH = 320;                     // h record of a pair: 2 steps 
 // records are 64 bytes apart modulo 128 (conflict-free 16-byte shared loads).
 __host__ __device__ constexpr int fz_rec_bytes(int ns) { return ns * 128 + 64; }
 
-// Steps (64 columns) per gate/up stage (both matrices).
-__host__ __device__ inline int fz_ns_gateup(int H) { return (H / 64) % 4 == 0 ? 4 : 2; }
+// Steps (64 columns) per gate/up stage (both matrices); the fused path needs
+// H to be a multiple of 256.
+__host__ __device__ inline int fz_ns_gateup(int) { return 4; }
 
 struct FusedArgs {
     const uint8_t* experts;
@@ -73,7 +74,7 @@ struct FusedArgs {
     int norm_topk;
     const int8_t* xq8;      // [T][H/64][128]  hi (64 B) + lo (64 B) per step, permuted
     const float* xinv8;     // [T] inverse activation scale
-    float* part;            // [P][I/128][H] partial down products
+    float* part;            // [T][k + n_shared][I/128][H] partial down products
     int32_t* queue;         // work-item counter, zeroed by the router kernel
     int32_t* idx;           // [T*k] picks (written by CTA 0)
     float* w;               // [T*k] weights
@@ -162,6 +163,7 @@ struct FusedShared {
     int meta_item[kFzMaxSlots], meta_st[kFzMaxSlots];
     int u_exp[kFzMaxUnits], u_p0[kFzMaxUnits], u_p1[kFzMaxUnits];
     int pair_tok[kFzMaxT * (kFzMaxK + 4)];
+    int pair_pick[kFzMaxT * (kFzMaxK + 4)];      // t * (k + n_shared) + j of each pair
     int pick_e[kFzMaxT * kFzMaxK];
     float pick_w[kFzMaxT * kFzMaxK];
     float xinv[kFzMaxT];
@@ -268,6 +270,7 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
         const int t = i / a.k, e = sh.pick_e[i];
         const int p = excl[e] + __popc(bits[e] & ((1u << t) - 1u));
         sh.pair_tok[p] = t;
+        sh.pair_pick[p] = t * (a.k + a.n_shared) + (i - t * a.k);
         if (blockIdx.x == 0) {
             a.idx[i] = e;
             a.w[i] = sh.pick_w[i];
@@ -279,7 +282,11 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
         sh.u_p0[nu + s] = Tk + s * a.T;
         sh.u_p1[nu + s] = Tk + (s + 1) * a.T;
     }
-    for (int i = threadIdx.x; i < a.n_shared * a.T; i += kFzThreads) sh.pair_tok[Tk + i] = i % a.T;
+    for (int i = threadIdx.x; i < a.n_shared * a.T; i += kFzThreads) {
+        const int t = i % a.T;
+        sh.pair_tok[Tk + i] = t;
+        sh.pair_pick[Tk + i] = t * (a.k + a.n_shared) + a.k + i / a.T;
+    }
     __syncthreads();
     return nu + a.n_shared;
 }
@@ -452,16 +459,17 @@ namespace coli {
 // lanes t and t ^ 2 hold the two digits of the same pairs.
 // ---------------------------------------------------------------------------
 template <int NT, bool GS>
-__device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int ns, int m, int rb, int lane,
-                                                int rec_gu, int acc_i[NT][4], float acc_f[NT][4]) {
+__device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb, int lane,
+                                                int rec_gu, int acc_i[2][NT][4], float acc_f[NT][4]) {
+    constexpr int ns = 4;
     const int g = lane >> 2, t = lane & 3;
     const float lanefac = t < 2 ? 256.0f : 1.0f;
     const uint8_t* cp = sl + m * ns * 4096 + rb * 512 + lane * 16;
     const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + (g & 3) * rec_gu;
     const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff + m * ns * 512) + 16 * rb + g;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        if (j < ns) {
+    for (int j = 0; j < ns; ++j) {
+        {
             uint32_t A0[4], A1[4];
             fz_decode_step(cp + j * 4096, A0, A1);
             if (GS) {
@@ -479,10 +487,10 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int ns, int m
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < NT; ++c) {
+                for (int c = 0; c < NT; ++c) {  // two accumulator chains: even and odd steps
                     const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
-                    mma_s8_16832(acc_i[c], A0, b.x, b.y);
-                    mma_s8_16832(acc_i[c], A1, b.z, b.w);
+                    mma_s8_16832(acc_i[j & 1][c], A0, b.x, b.y);
+                    mma_s8_16832(acc_i[j & 1][c], A1, b.z, b.w);
                 }
             }
         }
@@ -535,9 +543,12 @@ __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedSha
                     v[c][1] = fmaf((float)d[1], s0, v[c][1]);
                     v[c][2] = fmaf((float)d[2], s1, v[c][2]);
                     v[c][3] = fmaf((float)d[3], s1, v[c][3]);
-                } else {
-                    mma_s8_16832(acc[c], A0, b.x, b.y);
-                    mma_s8_16832(acc[c], A1, b.z, b.w);
+                } else {  // one chain per step, added below
+                    int d[4];
+                    mma_s8_16832_zc(d, A0, b.x, b.y);
+                    mma_s8_16832(d, A1, b.z, b.w);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[c][i] += d[i];
                 }
             }
         }
@@ -554,7 +565,7 @@ __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedSha
                 x += __shfl_xor_sync(0xffffffffu, x, 2);  // high digit * 256 + low digit
                 const int pp = 4 * c + 2 * t + (i & 1);
                 if (t < 2 && pp < np)
-                    a.part[((int64_t)(p0 + pp) * TG + tc) * a.H + r0 + 8 * (i >> 1)] = x;
+                    a.part[((int64_t)sh.pair_pick[p0 + pp] * TG + tc) * a.H + r0 + 8 * (i >> 1)] = x;
             }
         }
     }
@@ -583,7 +594,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
     int s = 0;
     int u = 0, tc = 0, p0 = 0, np = 0;
     float sw0 = 1.0f, sw1 = 1.0f;  // per-row weight scales of rows g, g + 8
-    int acc_i[NT][4];
+    int acc_i[2][NT][4];
     float acc_f[NT][4];
     for (;;) {
         if (!fz_wait(&sh.full[s], lap, a.err)) return;
@@ -598,11 +609,11 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
 #pragma unroll
             for (int c = 0; c < NT; ++c)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) { acc_i[c][i] = 0; acc_f[c][i] = 0.0f; }
+                for (int i = 0; i < 4; ++i) { acc_i[0][c][i] = 0; acc_i[1][c][i] = 0; acc_f[c][i] = 0.0f; }
         }
         const bool gu = st < z.nst_gu;
         if (gu) {
-            fz_stage_gateup<NT, GS>(sl, z.ns_gu, m, rb, lane, rec_gu, acc_i, acc_f);
+            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, acc_i, acc_f);
             if (!GS && st == z.nst_gu - 1) {
                 const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
                 sw0 = rsc[0];
@@ -622,7 +633,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
         for (int c = 0; c < NT; ++c)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float x = GS ? acc_f[c][i] : (float)acc_i[c][i] * lanefac;
+                float x = GS ? acc_f[c][i] : (float)(acc_i[0][c][i] + acc_i[1][c][i]) * lanefac;
                 x += __shfl_xor_sync(0xffffffffu, x, 2);  // high digit * 256 + low digit
                 if (!GS) x *= (i >> 1) ? sw1 : sw0;
                 v[c][i] = x;
@@ -726,15 +737,14 @@ moe_fused_kernel(FusedArgs a) {
 
 // ---------------------------------------------------------------------------
 // y from the partial down products.  CTA (token t, 32 rows), one warp per pick
-// j (k routed picks, then the shared experts): the warp sums pair j's I/128
+// j (k routed picks, then the shared experts): the warp sums pick j's I/128
 // partials in tile order (all loads in flight at once); warp 0 then adds the
 // picks up in pick order, weighted, then the shared experts, then the residual.
 // ---------------------------------------------------------------------------
 constexpr int kCombineMaxTiles = 32;  // I <= 4096
 
 struct CombineArgs {
-    const float* part;     // [P][TG][H]
-    const int32_t* inv;    // [T*k]
+    const float* part;     // [T][k + n_shared][TG][H]
     const float* w;        // [T*k]
     const float* residual; // [T][H] or nullptr
     float* y;              // [T][H]
@@ -749,10 +759,9 @@ moe_combine_kernel(CombineArgs c) {
     const int nw = blockDim.x >> 5;
     const int nrg = c.H / 32;
     const int t = blockIdx.x / nrg, r = (blockIdx.x - t * nrg) * 32 + lane;
-    const int Tk = c.T * c.k, J = c.k + c.n_shared;
+    const int J = c.k + c.n_shared;
     for (int j = warp; j < J; j += nw) {
-        const int p = j < c.k ? __ldg(c.inv + t * c.k + j) : Tk + (j - c.k) * c.T + t;
-        const float* src = c.part + (int64_t)p * c.TG * c.H + r;
+        const float* src = c.part + ((int64_t)t * J + j) * c.TG * c.H + r;
         float pv[kCombineMaxTiles];
 #pragma unroll
         for (int i = 0; i < kCombineMaxTiles; ++i)
@@ -761,12 +770,12 @@ moe_combine_kernel(CombineArgs c) {
 #pragma unroll
         for (int i = 0; i < kCombineMaxTiles; ++i)
             if (i < c.TG) o += pv[i];
-        oj[j][lane] = o;
+        oj[j][lane] = j < c.k ? o * __ldcg(c.w + t * c.k + j) : o;
     }
     __syncthreads();
     if (warp == 0) {
         float acc = 0.0f;
-        for (int j = 0; j < c.k; ++j) acc = fmaf(__ldg(c.w + t * c.k + j), oj[j][lane], acc);
+        for (int j = 0; j < c.k; ++j) acc += oj[j][lane];
         for (int s = 0; s < c.n_shared; ++s) acc += oj[c.k + s][lane];
         if (c.residual) acc = c.residual[(int64_t)t * c.H + r] + acc;
         c.y[(int64_t)t * c.H + r] = acc;

@@ -145,7 +145,8 @@ SMALL_PATHS = {"gemv": cm.COLI_PATH_GEMV, "fused": cm.COLI_PATH_FUSED}
 
 
 def fused_applies(wl, T):
-    return T <= 16 and wl.E <= 256 and wl.k <= 32 and wl.n_shared <= 4
+    return (T <= 16 and wl.E <= 256 and wl.k <= 32 and wl.n_shared <= 4 and wl.H % 256 == 0
+            and wl.I <= 4096)
 
 
 @pytest.mark.parametrize("path", list(SMALL_PATHS))
