@@ -503,18 +503,34 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
 // columns of I) against h of the item in shared memory.  Writes the partial
 // products of pairs p0 .. p0 + np - 1 for these 32 rows.
 // ---------------------------------------------------------------------------
+template <int NT>
+// hf[c][q]: lanefac * (inverse scale of h) / 16 of pair 4c + 2(t & 1) + q;
+// dst[c][q]: element offset in part of that pair's row 0 (-1: not written by
+// this lane).  Both are constant over the down stages of an item.
+__device__ __forceinline__ void fz_stage_down_prep(const FusedArgs& a, const FusedShared& sh,
+                                                   int tc, int p0, int np, int lane,
+                                                   float (*hf)[2], int (*dst)[2]) {
+    const int t = lane & 3;
+    const float lanefac = t < 2 ? 256.0f : 1.0f;
+    const int TG = a.I / 128;
+    for (int c = 0; c < NT; ++c)
+        for (int q = 0; q < 2; ++q) {
+            const int ph = 4 * c + 2 * (t & 1) + q;  // pair of this lane's digit columns
+            hf[c][q] = lanefac * *reinterpret_cast<const float*>(sh.hbuf + ph * kFzRecH + 256) * 0.0625f;
+            const int pw = 4 * c + 2 * t + q;         // pair this lane writes (t < 2)
+            dst[c][q] = (t < 2 && pw < np) ? (sh.pair_pick[p0 + pw] * TG + tc) * a.H : -1;
+        }
+}
+
 template <int NT, bool GS>
 __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedShared& sh,
-                                              const uint8_t* sl, int rs, int rt0, int tc,
-                                              int p0, int np, int warp, int lane) {
+                                              const uint8_t* sl, int rs, int rt0,
+                                              const float (*hf)[2], const int (*dst)[2],
+                                              int warp, int lane) {
     const int q = warp >> 2;
     if (q >= rs) return;
     const int g = lane >> 2, t = lane & 3;
-    const float lanefac = t < 2 ? 256.0f : 1.0f;
-    const int TG = a.I / 128;
     const int8_t* hb = sh.hbuf + (g >> 2) * 64 + t * 16 + (g & 3) * kFzRecH;
-    // inverse scales of h for the two pairs of this lane's columns (per group c)
-    const int8_t* hs = sh.hbuf + 256 + 2 * (t & 1) * kFzRecH;
 #pragma unroll
     for (int bb = 0; bb < 2; ++bb) {
         const int b8 = 2 * (warp & 3) + bb;
@@ -556,16 +572,13 @@ __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedSha
         const int r0 = (rt0 + q) * 128 + 16 * b8 + g;
 #pragma unroll
         for (int c = 0; c < NT; ++c) {
-            const float h0 = *reinterpret_cast<const float*>(hs + 4 * c * kFzRecH);
-            const float h1 = *reinterpret_cast<const float*>(hs + (4 * c + 1) * kFzRecH);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float x = GS ? v[c][i] : (float)acc[c][i] * ((i >> 1) ? sw1 : sw0);
-                x *= lanefac * ((i & 1) ? h1 : h0) * 0.0625f;
+                x *= hf[c][i & 1];
                 x += __shfl_xor_sync(0xffffffffu, x, 2);  // high digit * 256 + low digit
-                const int pp = 4 * c + 2 * t + (i & 1);
-                if (t < 2 && pp < np)
-                    a.part[((int64_t)sh.pair_pick[p0 + pp] * TG + tc) * a.H + r0 + 8 * (i >> 1)] = x;
+                const int o = dst[c][i & 1];
+                if (o >= 0) a.part[(int64_t)o + r0 + 8 * (i >> 1)] = x;
             }
         }
     }
@@ -594,6 +607,8 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
     int s = 0;
     int u = 0, tc = 0, p0 = 0, np = 0;
     float sw0 = 1.0f, sw1 = 1.0f;  // per-row weight scales of rows g, g + 8
+    float hf[NT][2];               // down part: digit and h scale factors
+    int dst[NT][2];                //            partial-product offsets
     int acc_i[2][NT][4];
     float acc_f[NT][4];
     for (;;) {
@@ -620,7 +635,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 sw1 = rsc[8];
             }
         } else {
-            fz_stage_down<NT, GS>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, tc, p0, np, warp, lane);
+            fz_stage_down<NT, GS>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, hf, dst, warp, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[s]);
@@ -700,6 +715,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 }
         }
         if (!fz_cbar(&sh.cbar, cphase, a.err)) return;  // h complete before the down stages
+        fz_stage_down_prep<NT>(a, sh, tc, p0, np, lane, hf, dst);
     }
 }
 
