@@ -87,6 +87,24 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def profiled_traffic(kernel_src: str, profile: str):
+    """DRAM bytes per launch (read + write) from the ncu summary in profiles/,
+    valid only while the kernel source still has the hash the capture names."""
+    import hashlib
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        digest = hashlib.sha256(open(os.path.join(ROOT, kernel_src), "rb").read()).hexdigest()
+    except OSError:
+        return None
+    want = traffic = None
+    for line in text.splitlines():
+        if "sha256 prefix" in line:
+            want = line.split("sha256 prefix")[1].split()[0]
+        if line.startswith("| traffic_bytes_per_launch |"):
+            traffic = float(line.split("|")[2])
+    return traffic if want and digest.startswith(want) else None
+
+
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
@@ -415,8 +433,12 @@ def main():
             kname = f"{dominant}_gemv_kernel"
             line["stages_us"] = {n: 1e3 * v for n, v in zip(cm.STAGE_NAMES, stage_mean)}
             line["down_gbs"] = dn_ach
+        traffic = None
+        if fused and wl.name == "glm_decode" and T == 1:
+            traffic = profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
+                                       "moe_fused_kernel_glm_decode.md")
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
-                            "frac": ach / hbm_gbs, "traffic": None, "kernel": kname,
+                            "frac": ach / hbm_gbs, "traffic": traffic, "kernel": kname,
                             "peak_source": peak_src,
                             "bytes_per_launch": float(kern_bytes.mean())}
         line["int4_weight_gbs"] = weight_gbs
