@@ -162,7 +162,8 @@ typedef struct coli_moe_layer coli_moe_layer;
 int coli_moe_layer_create(const coli_moe_desc* desc, coli_moe_layer** out);
 int coli_moe_layer_destroy(coli_moe_layer* layer);
 
-/* Workspace bytes that coli_moe_route / coli_moe_forward need for T tokens. */
+/* Workspace bytes that coli_moe_route / coli_moe_forward need for T tokens
+ * (enough for every path; the GEMV and GEMM paths use only a prefix). */
 int coli_moe_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes);
 
 /* Step 1 alone.  x device [T, H] (f32 or bf16); idx device i32 [T, k] ordered
@@ -246,9 +247,11 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert,
  * uses a scratch array of COLI_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the
  * library, which every GPU that loads the library keeps until the process
  * exits.  x, y and the layer's buffers are still the caller's.
- *  - T is limited to what fits: a call whose coli_moe_workspace_size(layer, T)
- *    exceeds COLI_NOALLOC_SCRATCH_BYTES returns COLI_E_UNSUPPORTED (for the
- *    GLM-5.2 shapes that is T <= 22 tokens).
+ *  - T is limited to what fits.  The call takes the path coli_moe_forward
+ *    would take when coli_moe_workspace_size(layer, T) fits the array, else
+ *    the GEMV or GEMM path, which needs only part of that workspace; when
+ *    neither fits it returns COLI_E_UNSUPPORTED (GLM-5.2 shapes: T <= 22; the
+ *    fused path for T <= 2).
  *  - The first call on each device looks up that device's copy of the array
  *    (cudaGetSymbolAddress with the device current); make that first call before
  *    any stream capture.  Later calls only launch kernels.
@@ -256,7 +259,7 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert,
  *    in it (every value a call needs cleared is cleared by its own kernels).
  *    Calls whose kernels overlap on the GPU (different streams, or different
  *    host threads on one device) race on the array: serialise them.
- * Results equal coli_moe_forward with COLI_PATH_AUTO on the same inputs. */
+ * Results equal coli_moe_forward_ex with the path taken (see above). */
 #define COLI_NOALLOC_SCRATCH_BYTES (8u << 20)
 int coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x,
                              coli_dtype xt, int32_t T, float* y,

@@ -68,7 +68,9 @@ bool fused_fits(const coli_moe_desc& d, int T) {
            d.H % 256 == 0 && d.I / 128 <= kCombineMaxTiles;
 }
 
-WsPlan plan_ws(const coli_moe_desc& d, int T) {
+// with_fused: also the fused path's buffers (placed last, so the plan without
+// them is a prefix of the plan with them)
+WsPlan plan_ws(const coli_moe_desc& d, int T, bool with_fused = true) {
     WsPlan p;
     int64_t off = 0;
     auto take = [&](int64_t bytes) { const int64_t at = off; off = align256(off + bytes); return at; };
@@ -99,7 +101,7 @@ WsPlan plan_ws(const coli_moe_desc& d, int T) {
     p.hg = take(P * d.I * 2);                   //   fp16 h of every pair
     p.hmax = take(P * 4);                       //   per-pair max |h|
     p.hsc = take(P * 4);                        //   per-pair inverse scale of h
-    if (fused_fits(d, T)) {
+    if (with_fused && fused_fits(d, T)) {
         p.xq8 = take((int64_t)T * d.H * 2);
         p.xinv8 = take((int64_t)T * 4);
         p.part = take(P * (d.I / 128) * d.H * 4);
@@ -641,15 +643,17 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     const coli_moe_desc& d = layer->d;
     int rc = tokens_ok(d, T);
     if (rc) return rc;
-    const WsPlan p = plan_ws(d, T);
-    if (!ws || ws_bytes < (size_t)p.total)
-        return fail(COLI_E_WORKSPACE, "forward: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
     if (path == COLI_PATH_FUSED && !fused_fits(d, T))
-        return fail(COLI_E_UNSUPPORTED, "forward: fused path needs T<=%d, E<=%d, k<=%d, n_shared<=4",
+        return fail(COLI_E_UNSUPPORTED,
+                    "forward: fused path needs T<=%d, E<=%d, k<=%d, n_shared<=4, H%%256==0, I<=4096",
                     kFzMaxT, kFzMaxE, kFzMaxK);
     if (path == COLI_PATH_AUTO)
         path = fused_fits(d, T) ? COLI_PATH_FUSED
                                 : (gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV);
+    // the GEMV and GEMM paths need only a prefix of the full workspace
+    const WsPlan p = plan_ws(d, T, path == COLI_PATH_FUSED);
+    if (!ws || ws_bytes < (size_t)p.total)
+        return fail(COLI_E_WORKSPACE, "forward: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
     cudaStream_t st = S(stream);
     int32_t* idx = at<int32_t>(ws, p.idx);
     float* w = at<float>(ws, p.w);
@@ -849,16 +853,24 @@ int noalloc_scratch(void** out) {
 int coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x, coli_dtype xt,
                              int32_t T, float* y, coli_stream_t stream) {
     if (!layer || !x || !y) return fail(COLI_E_INVAL, "forward_noalloc: NULL pointer");
-    size_t need = 0;
-    int rc = coli_moe_workspace_size(layer, T, &need);
+    int rc = tokens_ok(layer->d, T);
     if (rc) return rc;
-    if (need > (size_t)COLI_NOALLOC_SCRATCH_BYTES)
+    // the path AUTO would take if its workspace fits the array, else the
+    // GEMV/GEMM path, whose workspace is a prefix of the full one
+    coli_path path = COLI_PATH_AUTO;
+    int64_t need = plan_ws(layer->d, T, true).total;
+    if (need > (int64_t)COLI_NOALLOC_SCRATCH_BYTES) {
+        path = gemm_path_preferred(layer->d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV;
+        need = plan_ws(layer->d, T, false).total;
+    }
+    if (need > (int64_t)COLI_NOALLOC_SCRATCH_BYTES)
         return fail(COLI_E_UNSUPPORTED,
-                    "forward_noalloc: T=%d needs %zu bytes of scratch, the built-in array holds %u",
-                    T, need, (unsigned)COLI_NOALLOC_SCRATCH_BYTES);
+                    "forward_noalloc: T=%d needs %lld bytes of scratch, the built-in array holds %u",
+                    T, (long long)need, (unsigned)COLI_NOALLOC_SCRATCH_BYTES);
     void* ws = nullptr;
     if ((rc = noalloc_scratch(&ws))) return rc;
-    return coli_moe_forward(layer, x, xt, T, y, ws, (size_t)COLI_NOALLOC_SCRATCH_BYTES, stream);
+    return coli_moe_forward_ex(layer, x, xt, T, y, nullptr, path, nullptr, nullptr, nullptr, ws,
+                               (size_t)COLI_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

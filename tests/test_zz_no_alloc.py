@@ -44,3 +44,28 @@ def test_noalloc_rejects_too_many_tokens():
         cm.coli_moe_forward_noalloc(L.handle, x, T, y)
     assert e.value.code == -4 and "scratch" in str(e.value)
     L.close()
+
+
+def test_noalloc_uses_the_gemv_path_when_the_fused_scratch_does_not_fit():
+    """H 4096, I 1024, 16 tokens: the fused path's partial products need more than
+    the built-in array, the GEMV path's workspace fits, so the call runs the GEMV
+    path and gives exactly its bytes (and the oracle-checked path's values)."""
+    import dataclasses
+    wl = dataclasses.replace(synth.TINY, H=4096, I=1024, T=16)
+    L = build_layer(wl)
+    assert cm.coli_moe_workspace_size(L.handle, wl.T) > cm.NOALLOC_SCRATCH_BYTES
+    x = synth.tokens(wl, wl.T).cuda()
+    y_gemv = torch.empty((wl.T, wl.H), dtype=torch.float32, device="cuda")
+    y_auto = torch.empty_like(y_gemv)
+    y = torch.empty_like(y_gemv)
+    ws = L.workspace(wl.T)
+    cm.coli_moe_forward_ex(L.handle, x, wl.T, y_gemv, ws, path=cm.COLI_PATH_GEMV)
+    cm.coli_moe_forward_ex(L.handle, x, wl.T, y_auto, ws, path=cm.COLI_PATH_AUTO)
+    for _ in range(2):
+        y.fill_(float("nan"))
+        cm.coli_moe_forward_noalloc(L.handle, x, wl.T, y)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32),
+                                      y_gemv.cpu().numpy().view(np.uint32))
+    assert rel_err(y.cpu().numpy(), y_auto.cpu().numpy()) <= 2e-3
+    L.close()
