@@ -460,7 +460,8 @@ namespace coli {
 // ---------------------------------------------------------------------------
 template <int NT, bool GS>
 __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb, int lane,
-                                                int rec_gu, int acc_i[2][NT][4], float acc_f[NT][4]) {
+                                                int rec_gu, int ntc, int acc_i[2][NT][4],
+                                                float acc_f[NT][4]) {
     constexpr int ns = 4;
     const int g = lane >> 2, t = lane & 3;
     const float lanefac = t < 2 ? 256.0f : 1.0f;
@@ -476,6 +477,7 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
                 const float s0 = scl[j * 128] * lanefac, s1 = scl[j * 128 + 8] * lanefac;
 #pragma unroll
                 for (int c = 0; c < NT; ++c) {
+                    if (NT > 1 && c >= ntc) break;  // column groups with no pair of this item
                     const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
                     int d[4];
                     mma_s8_16832_zc(d, A0, b.x, b.y);
@@ -488,6 +490,7 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
             } else {
 #pragma unroll
                 for (int c = 0; c < NT; ++c) {  // two accumulator chains: even and odd steps
+                    if (NT > 1 && c >= ntc) break;
                     const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
                     mma_s8_16832(acc_i[j & 1][c], A0, b.x, b.y);
                     mma_s8_16832(acc_i[j & 1][c], A1, b.z, b.w);
@@ -524,7 +527,7 @@ __device__ __forceinline__ void fz_stage_down_prep(const FusedArgs& a, const Fus
 
 template <int NT, bool GS>
 __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedShared& sh,
-                                              const uint8_t* sl, int rs, int rt0,
+                                              const uint8_t* sl, int rs, int rt0, int ntc,
                                               const float (*hf)[2], const int (*dst)[2],
                                               int warp, int lane) {
     const int q = warp >> 2;
@@ -549,6 +552,7 @@ __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedSha
             fz_decode_step(cp + j * 4096, A0, A1);
 #pragma unroll
             for (int c = 0; c < NT; ++c) {
+                if (NT > 1 && c >= ntc) break;
                 const uint4 b = *reinterpret_cast<const uint4*>(hb + 4 * c * kFzRecH + j * 128);
                 if (GS) {
                     int d[4];
@@ -572,6 +576,7 @@ __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedSha
         const int r0 = (rt0 + q) * 128 + 16 * b8 + g;
 #pragma unroll
         for (int c = 0; c < NT; ++c) {
+            if (NT > 1 && c >= ntc) break;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float x = GS ? v[c][i] : (float)acc[c][i] * ((i >> 1) ? sw1 : sw0);
@@ -628,14 +633,15 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
         }
         const bool gu = st < z.nst_gu;
         if (gu) {
-            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, acc_i, acc_f);
+            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, (np + 3) >> 2, acc_i, acc_f);
             if (!GS && st == z.nst_gu - 1) {
                 const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
                 sw0 = rsc[0];
                 sw1 = rsc[8];
             }
         } else {
-            fz_stage_down<NT, GS>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, hf, dst, warp, lane);
+            fz_stage_down<NT, GS>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, (np + 3) >> 2, hf, dst, warp,
+                                  lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[s]);
