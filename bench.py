@@ -274,8 +274,9 @@ def main():
     path = {"auto": cm.COLI_PATH_AUTO, "gemv": cm.COLI_PATH_GEMV, "gemm": cm.COLI_PATH_GEMM,
             "fused": cm.COLI_PATH_FUSED}[args.path]
     # the path AUTO resolves to (include/coli_moe.h): the fused kernel for small batches
-    fused = args.path == "fused" or (args.path == "auto" and T <= 16 and wl.E <= 256
-                                     and wl.k <= 32 and wl.n_shared <= 4)
+    fused = args.path == "fused" or (
+        args.path == "auto" and T <= 64 and T * (wl.k + wl.n_shared) <= 640 and wl.E <= 256
+        and wl.k <= 32 and wl.n_shared <= 4 and wl.H % 256 == 0 and wl.I <= 4096)
     layers = build_layers(wl, dev)
     L0 = layers[0]
     n_pool = 64 if T <= 16 else 2

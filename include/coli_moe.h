@@ -91,10 +91,11 @@ typedef enum coli_path {
     COLI_PATH_GEMV = 1,  /* per-unit int4 GEMV kernels (mma.sync, fp16 hi/lo
                             activation digits, f32 accumulation)               */
     COLI_PATH_GEMM = 2,  /* tcgen05 grouped GEMM, fp16 operands, f32 accumulate */
-    COLI_PATH_FUSED = 3  /* one persistent kernel for top-k, union, experts and
-                            combine (mma.sync s8, exact int32 step sums);
-                            T <= 16, E <= 256, k <= 32, n_shared <= 4,
-                            H a multiple of 256, I <= 4096                   */
+    COLI_PATH_FUSED = 3  /* one persistent kernel for top-k, union and experts,
+                            then a combine kernel (mma.sync s8, exact int32
+                            step sums); T <= 64, T * (k + n_shared) <= 640,
+                            E <= 256, k <= 32, n_shared <= 4, H a multiple
+                            of 256, I <= 4096                                 */
 } coli_path;
 
 /* Thread-local description of the last error returned on this thread. */

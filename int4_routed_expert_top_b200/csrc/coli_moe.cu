@@ -64,8 +64,8 @@ struct WsPlan {
 };
 
 bool fused_fits(const coli_moe_desc& d, int T) {
-    return T <= kFzMaxT && d.E <= kFzMaxE && d.k <= kFzMaxK && d.n_shared <= 4 &&
-           d.H % 256 == 0 && d.I / 128 <= kCombineMaxTiles;
+    return T <= kFzMaxT && T * (d.k + d.n_shared) <= kFzMaxPairs && d.E <= kFzMaxE &&
+           d.k <= kFzMaxK && d.n_shared <= 4 && d.H % 256 == 0 && d.I / 128 <= kCombineMaxTiles;
 }
 
 // with_fused: also the fused path's buffers (placed last, so the plan without
@@ -645,8 +645,8 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     if (rc) return rc;
     if (path == COLI_PATH_FUSED && !fused_fits(d, T))
         return fail(COLI_E_UNSUPPORTED,
-                    "forward: fused path needs T<=%d, E<=%d, k<=%d, n_shared<=4, H%%256==0, I<=4096",
-                    kFzMaxT, kFzMaxE, kFzMaxK);
+                    "forward: fused path needs T<=%d, T*(k+n_shared)<=%d, E<=%d, k<=%d, n_shared<=4, "
+                    "H%%256==0, I<=4096", kFzMaxT, kFzMaxPairs, kFzMaxE, kFzMaxK);
     if (path == COLI_PATH_AUTO)
         path = fused_fits(d, T) ? COLI_PATH_FUSED
                                 : (gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV);

@@ -44,7 +44,9 @@ namespace coli {
 constexpr int kFzWarps = 16;                     // consumer warps
 constexpr int kFzProducer = kFzWarps;            // warp that streams the ring
 constexpr int kFzThreads = 32 * (kFzWarps + 1);
-constexpr int kFzMaxT = 16;                      // tokens per call on this path
+constexpr int kFzMaxT = 64;                      // tokens per call on this path
+constexpr int kFzChunk = 16;                     // pairs per work item (a unit's pairs in chunks)
+constexpr int kFzMaxPairs = 640;                 // T * (k + n_shared) on this path
 constexpr int kFzMaxE = 256;                     // routed experts on this path
 constexpr int kFzMaxUnits = kFzMaxE + 4;
 constexpr int kFzMaxK = 32;
@@ -162,20 +164,38 @@ struct FusedShared {
     uint64_t cbar;
     int meta_item[kFzMaxSlots], meta_st[kFzMaxSlots];
     int u_exp[kFzMaxUnits], u_p0[kFzMaxUnits], u_p1[kFzMaxUnits];
-    int pair_tok[kFzMaxT * (kFzMaxK + 4)];
-    int pair_pick[kFzMaxT * (kFzMaxK + 4)];      // t * (k + n_shared) + j of each pair
-    int pick_e[kFzMaxT * kFzMaxK];
-    float pick_w[kFzMaxT * kFzMaxK];
+    int u_item0[kFzMaxUnits + 1];                 // first work item of each unit
+    int pair_tok[kFzMaxPairs];
+    int pair_pick[kFzMaxPairs];                   // t * (k + n_shared) + j of each pair
     float xinv[kFzMaxT];
-    float xch[8][16][kFzMaxT];                    // up values for the gate warps
-    float wmax[8][kFzMaxT];                       // per-warp max |h| of each pair
-    __align__(16) int8_t hbuf[kFzMaxT * kFzRecH]; // h of the current item, s8 digits
-    int n_uniq;
+    float xch[8][16][kFzChunk];                   // up values for the gate warps
+    float wmax[8][kFzChunk];                      // per-warp max |h| of each pair
+    __align__(16) int8_t hbuf[kFzChunk * kFzRecH]; // h of the current item, s8 digits
+    int n_uniq, n_items;
 };
+
+// Top-k and union scratch in the (not yet used) ring: per expert a count, a
+// 64-bit token mask and an exclusive prefix; per pick its expert and weight.
+struct FzScratch {
+    int* cnt;
+    unsigned long long* bits;
+    int* excl;
+    int* pick_e;
+    float* pick_w;
+};
+__device__ __forceinline__ FzScratch fz_scratch(uint8_t* ring, int E) {
+    FzScratch r;
+    r.bits = reinterpret_cast<unsigned long long*>(ring);
+    r.cnt = reinterpret_cast<int*>(ring + 8 * E);
+    r.excl = r.cnt + E;
+    r.pick_e = r.excl + E;
+    r.pick_w = reinterpret_cast<float*>(r.pick_e + kFzMaxT * kFzMaxK);
+    return r;
+}
 
 // Top-k of token t by one warp (E <= 256: up to 8 candidates per lane).
 // Order: selection score descending, expert index ascending.
-__device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, FusedShared& sh) {
+__device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, const FzScratch& sc8) {
     const int lane = threadIdx.x & 31;
     float sc[8], sel[8];
 #pragma unroll
@@ -210,70 +230,95 @@ __device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, FusedSh
     float denom = 0.0f;  // over the picks in pick order
     for (int j = 0; j < a.k; ++j) denom += __shfl_sync(0xffffffffu, mine, j);
     if (lane < a.k) {
-        sh.pick_e[t * a.k + lane] = mine_e;
-        sh.pick_w[t * a.k + lane] = (a.norm_topk ? mine / denom : mine) * a.routed_scale;
+        sc8.pick_e[t * a.k + lane] = mine_e;
+        sc8.pick_w[t * a.k + lane] = (a.norm_topk ? mine / denom : mine) * a.routed_scale;
     }
 }
 
-// Top-k of every token and the batch union, in this CTA's shared memory.
-// scratch: 3 * E ints (any shared memory not yet in use).  CTA 0 also
-// publishes the picks, weights and pair indices.  Returns the units.
-__device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& sh,
-                                              int* scratch) {
+// Top-k of every token and the batch union, in this CTA's shared memory, and
+// the work items: unit u's pairs in chunks of kFzChunk, I/128 items per chunk.
+// CTA 0 also publishes the picks, weights and pair indices.  Returns the units.
+__device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& sh, uint8_t* ring) {
     constexpr int kAllWarps = kFzThreads / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int* cnt = scratch;
-    uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + a.E);
-    int* excl = scratch + 2 * a.E;
-    for (int e = threadIdx.x; e < a.E; e += kFzThreads) { cnt[e] = 0; bits[e] = 0u; }
+    const FzScratch sc8 = fz_scratch(ring, a.E);
+    for (int e = threadIdx.x; e < a.E; e += kFzThreads) { sc8.cnt[e] = 0; sc8.bits[e] = 0ull; }
     for (int t = threadIdx.x; t < a.T; t += kFzThreads) sh.xinv[t] = __ldcg(a.xinv8 + t);
-    for (int t = warp; t < a.T; t += kAllWarps) fz_topk_token(a, t, sh);
+    for (int t = warp; t < a.T; t += kAllWarps) fz_topk_token(a, t, sc8);
     __syncthreads();
+    if (threadIdx.x == 32 * kFzProducer) {
+        // The shared experts are used whatever the routing: while the union is
+        // formed, pull this CTA's slice of their blobs into L2 (issued after
+        // the score loads, which it would otherwise slow down).
+        const int64_t total = (int64_t)a.n_shared * a.blob_bytes;
+        const int64_t chunk = ((total + gridDim.x - 1) / gridDim.x + 255) & ~int64_t(255);
+        const int64_t beg = (int64_t)blockIdx.x * chunk;
+        const int64_t end = beg + chunk < total ? beg + chunk : total;
+        const uint8_t* base = a.experts + (int64_t)a.E * a.blob_bytes;
+        for (int64_t off = beg; off < end; off += 65536) {
+            const uint32_t n = (uint32_t)(end - off < 65536 ? end - off : 65536);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(n) : "memory");
+        }
+    }
     const int Tk = a.T * a.k;
     for (int i = threadIdx.x; i < Tk; i += kFzThreads) {
-        const int e = sh.pick_e[i];
-        atomicAdd(&cnt[e], 1);
-        atomicOr(&bits[e], 1u << (i / a.k));
+        const int e = sc8.pick_e[i];
+        atomicAdd(&sc8.cnt[e], 1);
+        atomicOr(&sc8.bits[e], 1ull << (i / a.k));
     }
     __syncthreads();
-    if (warp == 0) {  // exclusive scans of counts and of (count > 0): 8 experts per lane
-        int c[8], f[8], sc = 0, sf = 0;
+    const int TG = a.I / 128;
+    if (warp == 0) {  // exclusive scans of counts, of (count > 0) and of items: 8 experts per lane
+        int c[8], f[8], sc = 0, sf = 0, si = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int e = 8 * lane + i;
-            c[i] = e < a.E ? cnt[e] : 0;
+            c[i] = e < a.E ? sc8.cnt[e] : 0;
             f[i] = c[i] > 0;
-            sc += c[i]; sf += f[i];
+            sc += c[i]; sf += f[i]; si += (c[i] + kFzChunk - 1) / kFzChunk;
         }
-        int ic = sc, jf = sf;
+        int ic = sc, jf = sf, ki = si;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const int x = __shfl_up_sync(0xffffffffu, ic, d);
             const int y = __shfl_up_sync(0xffffffffu, jf, d);
-            if (lane >= d) { ic += x; jf += y; }
+            const int z = __shfl_up_sync(0xffffffffu, ki, d);
+            if (lane >= d) { ic += x; jf += y; ki += z; }
         }
-        int ec = ic - sc, ef = jf - sf;
+        int ec = ic - sc, ef = jf - sf, ei = ki - si;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int e = 8 * lane + i;
             if (e < a.E) {
-                excl[e] = ec;
-                if (f[i]) { sh.u_exp[ef] = e; sh.u_p0[ef] = ec; sh.u_p1[ef] = ec + c[i]; }
+                sc8.excl[e] = ec;
+                if (f[i]) {
+                    sh.u_exp[ef] = e; sh.u_p0[ef] = ec; sh.u_p1[ef] = ec + c[i];
+                    sh.u_item0[ef] = ei * TG;
+                }
             }
-            ec += c[i]; ef += f[i];
+            ec += c[i]; ef += f[i]; ei += (c[i] + kFzChunk - 1) / kFzChunk;
         }
-        if (lane == 31) sh.n_uniq = ef;
+        if (lane == 31) {
+            sh.n_uniq = ef;
+            int item = ei * TG;  // the shared experts follow, T pairs each
+            for (int s2 = 0; s2 < a.n_shared; ++s2) {
+                sh.u_item0[ef + s2] = item;
+                item += (a.T + kFzChunk - 1) / kFzChunk * TG;
+            }
+            sh.u_item0[ef + a.n_shared] = item;
+            sh.n_items = item;
+        }
     }
     __syncthreads();
     const int nu = sh.n_uniq;
     for (int i = threadIdx.x; i < Tk; i += kFzThreads) {
-        const int t = i / a.k, e = sh.pick_e[i];
-        const int p = excl[e] + __popc(bits[e] & ((1u << t) - 1u));
+        const int t = i / a.k, e = sc8.pick_e[i];
+        const int p = sc8.excl[e] + __popcll(sc8.bits[e] & ((1ull << t) - 1ull));
         sh.pair_tok[p] = t;
         sh.pair_pick[p] = t * (a.k + a.n_shared) + (i - t * a.k);
         if (blockIdx.x == 0) {
             a.idx[i] = e;
-            a.w[i] = sh.pick_w[i];
+            a.w[i] = sc8.pick_w[i];
             a.inv[i] = p;
         }
     }
@@ -289,6 +334,27 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
     }
     __syncthreads();
     return nu + a.n_shared;
+}
+
+// Work item -> (unit, its pairs p0 .. p0 + np - 1, 128-row tile tc of I):
+// the unit by binary search over the units' first items.
+struct FzWork {
+    int u, p0, np, tc;
+};
+__device__ __forceinline__ FzWork fz_work(const FusedShared& sh, int n_units, int TG, int item) {
+    int lo = 0, hi = n_units - 1;  // last unit whose first item is <= item
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sh.u_item0[mid] <= item) lo = mid; else hi = mid - 1;
+    }
+    FzWork w;
+    w.u = lo;
+    const int rel = item - sh.u_item0[lo];
+    const int ch = rel / TG;
+    w.tc = rel - ch * TG;
+    w.p0 = sh.u_p0[lo] + ch * kFzChunk;
+    w.np = min(kFzChunk, sh.u_p1[lo] - w.p0);
+    return w;
 }
 
 // D = A * B with C = 0 (a fresh 64-column partial sum)
@@ -366,7 +432,7 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
                                            int n_units) {
     const int lane = threadIdx.x & 31;
     const FzShape z = fz_shape(a);
-    const int n_items = n_units * z.TG;
+    const int n_items = sh.n_items;
     const int rec_gu = fz_rec_bytes(z.ns_gu);
     const int ngH = GS ? a.H / 64 : 1, ngI = GS ? a.I / 64 : 1;
     const uint64_t pol = l2_evict_first_policy();
@@ -375,8 +441,9 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
     bool ok = true;
     int item = blockIdx.x;  // first item: by CTA index; later ones from the queue
     while (ok && item < n_items) {
-        const int u = item / z.TG, tc = item - u * z.TG;
-        const int e = sh.u_exp[u], p0 = sh.u_p0[u], np = sh.u_p1[u] - p0;
+        const FzWork wk = fz_work(sh, n_units, z.TG, item);
+        const int tc = wk.tc, p0 = wk.p0, np = wk.np;
+        const int e = sh.u_exp[wk.u];
         const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
         const uint8_t* cG = blob + a.L.codes[0];
         const uint8_t* cU = blob + a.L.codes[1];
@@ -622,10 +689,11 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
         if (item < 0) return;
         const uint8_t* sl = ring + (int64_t)s * a.slot_bytes;
         if (st == 0) {  // a new item
-            u = item / z.TG;
-            tc = item - u * z.TG;
-            p0 = sh.u_p0[u];
-            np = sh.u_p1[u] - p0;
+            const FzWork wk = fz_work(sh, n_units, z.TG, item);
+            u = wk.u;
+            tc = wk.tc;
+            p0 = wk.p0;
+            np = wk.np;
 #pragma unroll
             for (int c = 0; c < NT; ++c)
 #pragma unroll
@@ -737,22 +805,9 @@ moe_fused_kernel(FusedArgs a) {
     }
     // the combine kernel may be scheduled now; it waits for this grid to finish
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (threadIdx.x == 32 * kFzProducer) {
-        // The shared experts are used whatever the routing: while the router
-        // finishes, pull this CTA's slice of their blobs into L2.
-        const int64_t total = (int64_t)a.n_shared * a.blob_bytes;
-        const int64_t chunk = ((total + gridDim.x - 1) / gridDim.x + 255) & ~int64_t(255);
-        const int64_t beg = (int64_t)blockIdx.x * chunk;
-        const int64_t end = beg + chunk < total ? beg + chunk : total;
-        const uint8_t* base = a.experts + (int64_t)a.E * a.blob_bytes;
-        for (int64_t off = beg; off < end; off += 65536) {
-            const uint32_t n = (uint32_t)(end - off < 65536 ? end - off : 65536);
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(n) : "memory");
-        }
-    }
     // everything below reads what the router kernel wrote
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int n_units = fz_route_union(a, sh, reinterpret_cast<int*>(fz_smem));
+    const int n_units = fz_route_union(a, sh, fz_smem);
     if ((threadIdx.x >> 5) == kFzProducer) fz_produce<GS>(a, sh, fz_smem, n_units);
     else fz_consume<NT, GS>(a, sh, fz_smem, n_units);
 }

@@ -62,7 +62,7 @@ act_quant_kernel(const XT* __restrict__ x, int T, int H, __half* __restrict__ xq
 // share build the fp16 activation operand (xq) when xq != nullptr.
 // ---------------------------------------------------------------------------
 constexpr int kRouterMaxSlice = 1024;  // columns per warp slice (<= 8 loads per lane)
-constexpr int kRouterMaxT = 32;        // tokens per call of the small-batch router
+constexpr int kRouterMaxT = 64;        // tokens per call of the small-batch router
 
 // ---------------------------------------------------------------------------
 // s8 activation operand of the fused small-batch kernel (fused.cuh): each value

@@ -130,6 +130,7 @@ VARIANTS = {
     "T1": dict(T=1),
     "T7_gs64": dict(T=7, group=64),
     "T40_tiled_router": dict(T=40),
+    "T64_chunked_units": dict(T=64, E=8, k=2, group=64),
     "no_shared": dict(n_shared=0),
     "two_shared": dict(n_shared=2),
     "k1": dict(k=1),
@@ -145,8 +146,8 @@ SMALL_PATHS = {"gemv": cm.COLI_PATH_GEMV, "fused": cm.COLI_PATH_FUSED}
 
 
 def fused_applies(wl, T):
-    return (T <= 16 and wl.E <= 256 and wl.k <= 32 and wl.n_shared <= 4 and wl.H % 256 == 0
-            and wl.I <= 4096)
+    return (T <= 64 and T * (wl.k + wl.n_shared) <= 640 and wl.E <= 256 and wl.k <= 32
+            and wl.n_shared <= 4 and wl.H % 256 == 0 and wl.I <= 4096)
 
 
 @pytest.mark.parametrize("path", list(SMALL_PATHS))
@@ -188,16 +189,16 @@ def test_residual_and_zero_input(path):
 
 
 def test_fused_rejects_sizes_outside_its_limits():
-    wl = dataclasses.replace(synth.TINY, T=17)
+    wl = dataclasses.replace(synth.TINY, T=65)
     L = build_layer(wl)
-    x = torch.randn((17, wl.H), device="cuda")
-    y = torch.empty((17, wl.H), device="cuda")
+    x = torch.randn((65, wl.H), device="cuda")
+    y = torch.empty((65, wl.H), device="cuda")
     with pytest.raises(cm.ColiError) as ei:
-        cm.coli_moe_forward_ex(L.handle, x, 17, y, L.workspace(17), path=cm.COLI_PATH_FUSED)
+        cm.coli_moe_forward_ex(L.handle, x, 65, y, L.workspace(65), path=cm.COLI_PATH_FUSED)
     assert ei.value.code == -4   # COLI_E_UNSUPPORTED
 
 
-@pytest.mark.parametrize("T", [1, 5, 16])
+@pytest.mark.parametrize("T", [1, 5, 16, 33, 64])
 def test_auto_small_batches_equal_fused(T):
     """AUTO picks the fused kernel for small batches: same bytes as asking for it."""
     wl = dataclasses.replace(synth.TINY, T=T, group=64)
