@@ -251,7 +251,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
                                               nb * 2048 * (a.two ? 1 : 2));
             for (int ks = 0; ks < KS; ++ks, ++u) {
                 const int s = u % kGemmStages;
-                if (u >= kGemmStages && ok && !mbar_wait_warp(&empty[s], ((u / kGemmStages) - 1) & 1, a.err)) ok = false;
+                if (u >= kGemmStages && ok && !mbar_wait_warp_sleep(&empty[s], ((u / kGemmStages) - 1) & 1, a.err)) ok = false;
                 uint8_t* st = smem + s * kStageBytes;
                 uint8_t* sc = st + kStageB;
                 mbar_expect_tx_elect(&full[s], bytes);
@@ -288,13 +288,13 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
             const int np = (n + 15) / 16 * 16;  // N: multiple of 16 for M = 128
             const uint32_t idesc = idesc_f16_f32(np);
             const int buf = tcount & 1;
-            if (tcount >= 2 && ok && !mbar_wait_warp(&accempty[buf], ((tcount >> 1) - 1) & 1, a.err)) ok = false;
+            if (tcount >= 2 && ok && !mbar_wait_warp_sleep(&accempty[buf], ((tcount >> 1) - 1) & 1, a.err)) ok = false;
             tc_fence_after();
             const uint32_t dacc = tmem + 128 * buf;
             for (int ks = 0; ks < KS; ++ks, ++u) {
                 const int s = u % kGemmStages, as = u % kGemmAStages;
-                if (ok && !mbar_wait_warp(&afull[as], (u / kGemmAStages) & 1, a.err)) ok = false;
-                if (ok && !mbar_wait_warp(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
+                if (ok && !mbar_wait_warp_sleep(&afull[as], (u / kGemmAStages) & 1, a.err)) ok = false;
+                if (ok && !mbar_wait_warp_sleep(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
                 tc_fence_after();
                 const uint64_t bdesc = smem_desc_sw128(smem + s * kStageBytes);
                 const uint32_t a0 = tmem + 256 + 64 * as;
@@ -342,7 +342,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
                                     : __ldg(a.act_inv + p);
                 }
             }
-            if (ok && !mbar_wait_warp(&accfull[buf], (tcount >> 1) & 1, a.err)) ok = false;
+            if (ok && !mbar_wait_warp_sleep(&accfull[buf], (tcount >> 1) & 1, a.err)) ok = false;
             tc_fence_after();
             const uint32_t dacc = tmem + lane_off + 128 * buf;
             for (int c0 = 0; c0 < n; c0 += 16) {
@@ -390,8 +390,8 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x) {
             for (int ks = 0; ks < KS; ++ks, ++u) {
                 const int s = u % kGemmStages, as = u % kGemmAStages;
-                if (ok && !mbar_wait_warp(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
-                if (u >= kGemmAStages && ok && !mbar_wait_warp(&aempty[as], ((u / kGemmAStages) - 1) & 1, a.err)) ok = false;
+                if (ok && !mbar_wait_warp_sleep(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
+                if (u >= kGemmAStages && ok && !mbar_wait_warp_sleep(&aempty[as], ((u / kGemmAStages) - 1) & 1, a.err)) ok = false;
                 tc_fence_after();
                 const uint32_t sc = sbase + s * kStageBytes + kStageB;
                 const uint4 un = lds128(sc + slot * 4096 + (b8 * 32 + lane) * 16);

@@ -57,6 +57,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     return false;
 }
 
+// Warp-wide wait in which each try may sleep until the phase completes or 20 us
+// pass (a suspend-time hint), so that a waiting warp issues almost nothing: for
+// kernels with many warps waiting at once.  At most kSleepTries tries (about a
+// second), then kErrWaitTimeout as for mbar_wait.
+constexpr uint32_t kSleepTries = 1u << 16;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.b32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_warp_sleep(uint64_t* bar, uint32_t parity, int32_t* err) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) {
+        ok = 0;
+        for (uint32_t i = 0; i < kSleepTries; ++i)
+            if (mbar_try_wait_sleep(bar, parity)) { ok = 1; break; }
+        if (!ok && err) atomicOr(err, kErrWaitTimeout);
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // Warp-wide wait: lane 0 polls the barrier while the other lanes sleep at the
 // warp barrier, which then orders their reads after lane 0's acquire.  Keeps the
 // mbarrier unit free for the arrivals and transaction counts that make progress
