@@ -431,7 +431,9 @@ def main():
             dominant = "gateup" if stage_mean[2] >= stage_mean[3] else "down"
             ach = gu_ach if dominant == "gateup" else dn_ach
             kern_bytes = units * (gu_bytes_unit if dominant == "gateup" else dn_bytes_unit)
-            kname = f"{dominant}_gemv_kernel"
+            gemm = args.path == "gemm" or (args.path == "auto" and T >= 48)
+            kname = (f"moe_gemm_kernel ({'gate/up' if dominant == 'gateup' else 'down'})"
+                     if gemm else f"{dominant}_gemv_kernel")
             line["stages_us"] = {n: 1e3 * v for n, v in zip(cm.STAGE_NAMES, stage_mean)}
             line["down_gbs"] = dn_ach
         traffic = None

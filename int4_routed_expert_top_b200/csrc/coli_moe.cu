@@ -254,13 +254,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows][cols] fp16, boxes of 16 rows x 64 columns, 128-byte swizzle
+// [rows][cols] fp16, boxes of 64 rows x 64 columns, 128-byte swizzle
 int encode_b_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(COLI_E_CUDA, "cuTensorMapEncodeTiled is not available");
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kGemmMaxN};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

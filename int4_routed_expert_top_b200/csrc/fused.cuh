@@ -112,33 +112,6 @@ __device__ __forceinline__ void decode_word_s8(uint32_t w, uint32_t& r0, uint32_
     r1 = (w << 4) & 0xF0F0F0F0u;
 }
 
-// L2 policy for data read exactly once (weights streamed into the ring)
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-// global -> shared bulk copy with an L2 cache policy (warp-uniform operands;
-// one elected lane issues)
-__device__ __forceinline__ void bulk_g2s_hint_elect(void* dst, const void* src, uint32_t bytes,
-                                                    uint64_t* bar, uint64_t pol) {
-    asm volatile(
-        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
-        " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1], %2, [%3], %4;\n}"
-        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
-}
-
-__device__ __forceinline__ void prefetch_l2_elect(const void* src, uint32_t bytes) {
-    asm volatile(
-        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
-        " @e cp.async.bulk.prefetch.L2.global [%0], %1;\n}"
-        ::"l"(src), "r"(bytes)
-        : "memory");
-}
-
 __device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

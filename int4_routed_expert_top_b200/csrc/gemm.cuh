@@ -8,15 +8,16 @@
 // little arithmetic per weight byte, so the kernel is built to keep HBM busy and
 // the int4 decode off the critical path.  Per CTA (persistent, one per SM, all
 // 512 TMEM columns, 24 warps):
-//   warp 0       producer: 1-D bulk copies of the int4 fragment tiles (8 KB a
-//                stage: gate and up of one 64-column step, or two steps of down)
-//                with their gs64 scales, and 2-D TMA loads of the tokens (fp16,
-//                128-byte swizzle) into an 8-stage ring;
+//   warp 0       producer: 1-D bulk copies of the int4 fragment tiles (32 KB
+//                a stage: gate and up of four 64-column steps, or eight steps of
+//                down) with their gs64 scales, and one 2-D TMA load of the
+//                tokens (fp16, 128-byte swizzle, a 64 x 64 box) per step into a
+//                3-stage ring of 68 KB stages;
 //   warp 1       one lane issues tcgen05.mma (kind::f16, f32 accumulators in
 //                TMEM), A from TMEM and B from shared memory;
 //   warps 4-7    epilogue: TMEM accumulators -> registers -> global;
-//   warps 8-23   decode: each warp turns one 16-row x 64-column unit block of a
-//                stage (512 B of nibbles) into exact fp16 (q, or q*s for gs64)
+//   warps 8-23   decode: each warp turns one 16-row x 64-column block of an A
+//                unit (512 B of nibbles) into exact fp16 (q, or q*s for gs64)
 //                and writes it to TMEM with tcgen05.st.16x256b, whose lane and
 //                column layout is that of the fragment tiles.
 // TMEM columns: accumulators [0, 256) as two buffers of 128 (gate at +0, up at
@@ -37,17 +38,21 @@
 namespace coli {
 
 constexpr int kGemmThreads = 768;
-constexpr int kGemmStages = 8;                        // shared-memory ring
+constexpr int kGemmStages = 3;                        // shared-memory ring (68 KB stages)
 constexpr int kGemmAStages = 4;                       // TMEM A ring
 constexpr int kGemmMaxN = 64;                         // tokens per tile
 constexpr int kGemmDecodeWarp0 = 8;
 constexpr int kGemmDecodeWarps = 16;
 constexpr int kGemmEpiWarp0 = 4;
+// A ring stage holds four 64-column steps of the tokens (B atoms) and the int4
+// codes that meet them: for gate/up four A units (one step of gate and of up,
+// 8 KB of codes each), for down two A units (two steps of down each).
 constexpr int kAtomBytes = kGemmMaxN * 128;           // one 64-column B atom, 64 rows
-constexpr int kStageB = 2 * kAtomBytes;               // two atoms (down: two k-steps)
-constexpr int kStageCodes = 2 * 4096;                 // two 128 x 64 nibble blocks
-constexpr int kStageScales = 2 * 512;
-constexpr int kStageBytes = kStageB + kStageCodes + kStageScales;   // 25600, 1 KB multiple
+constexpr int kStageAtoms = 4;
+constexpr int kStageB = kStageAtoms * kAtomBytes;     // 32 KB
+constexpr int kStageCodes = 8 * 4096;                 // 32 KB: eight 128 x 64 nibble blocks
+constexpr int kStageScales = 8 * 512;
+constexpr int kStageBytes = kStageB + kStageCodes + kStageScales;   // 68 KB, 1 KB multiple
 constexpr int kGemmSmem = kGemmStages * kStageBytes + 1024;        // + alignment slack
 static_assert(kStageBytes % 1024 == 0, "stages must stay 1 KB aligned for the swizzle");
 constexpr uint32_t kTmemCols = 512;
@@ -209,7 +214,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
     const int n_units = *a.n_units;
     const int KB = a.K / 64;
     const int ng = a.group ? KB : 1;
-    const int KS = a.two ? KB : KB / 2;          // ring stages per tile
+    const int SPS = KB % 4 == 0 ? 4 : 2;         // 64-column steps per ring stage (KB is even)
+    const int KS = KB / SPS;                     // ring stages per tile
+    const int APS = a.two ? SPS : SPS / 2;       // A units per ring stage
+    const int KA = KS * APS;                     // A units per tile
     const int RT = a.R / kTileRows;
     const int mA = a.two ? 0 : 2;
 
@@ -238,6 +246,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
 
     if (warp == 0) {
         // ---------------- producer (whole warp, elected lane issues) ----------------
+        const uint64_t pol = l2_evict_first_policy();
         int u = 0;
         int p0, n, rt;
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x) {
@@ -246,38 +255,28 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
             const uint8_t* c1 = blob + a.L.codes[1];
             const float* s0 = reinterpret_cast<const float*>(blob + a.L.scales[mA]);
             const float* s1 = reinterpret_cast<const float*>(blob + a.L.scales[1]);
-            const int nb = (n + 15) / 16;
-            const uint32_t bytes = (uint32_t)(kStageCodes + (a.group ? kStageScales : 0) +
-                                              nb * 2048 * (a.two ? 1 : 2));
+            // a stage: APS A units; gate/up: steps kb0 .. kb0 + SPS - 1 of gate and of
+            // up, down: the same steps of down; B: those steps of the tile's tokens
+            const uint32_t cbytes = (uint32_t)SPS * 4096;            // per matrix
+            const uint32_t sbytes = a.group ? (uint32_t)SPS * 512 : 0u;
+            const uint32_t bytes = (cbytes + sbytes) * (a.two ? 2u : 1u) + (uint32_t)SPS * kAtomBytes;
             for (int ks = 0; ks < KS; ++ks, ++u) {
                 const int s = u % kGemmStages;
                 if (u >= kGemmStages && ok && !mbar_wait_warp_sleep(&empty[s], ((u / kGemmStages) - 1) & 1, a.err)) ok = false;
                 uint8_t* st = smem + s * kStageBytes;
                 uint8_t* sc = st + kStageB;
                 mbar_expect_tx_elect(&full[s], bytes);
-                if (a.two) {
-                    const int64_t uoff = frag_unit_offset(rt, ks, 0, 0, a.K);
-                    bulk_g2s_elect(sc, c0 + uoff, 4096, &full[s]);
-                    bulk_g2s_elect(sc + 4096, c1 + uoff, 4096, &full[s]);
-                    if (a.group) {
-                        const int64_t soff = ((int64_t)rt * ng + ks) * kTileRows;
-                        bulk_g2s_elect(sc + kStageCodes, s0 + soff, 512, &full[s]);
-                        bulk_g2s_elect(sc + kStageCodes + 512, s1 + soff, 512, &full[s]);
-                    }
-                    for (int i = 0; i < nb; ++i)
-                        tma_load_2d_elect(st + i * 2048, &bmap, ks * 64, p0 + 16 * i, &full[s]);
-                } else {
-                    // two consecutive 64-column steps of down: contiguous in the layout
-                    const int kb = 2 * ks;
-                    bulk_g2s_elect(sc, c0 + frag_unit_offset(rt, kb, 0, 0, a.K), kStageCodes, &full[s]);
-                    if (a.group)
-                        bulk_g2s_elect(sc + kStageCodes, s0 + ((int64_t)rt * ng + kb) * kTileRows, kStageScales,
-                                       &full[s]);
-                    for (int h = 0; h < 2; ++h)
-                        for (int i = 0; i < nb; ++i)
-                            tma_load_2d_elect(st + h * kAtomBytes + i * 2048, &bmap, (kb + h) * 64, p0 + 16 * i,
-                                              &full[s]);
+                const int kb0 = SPS * ks;
+                const int64_t uoff = frag_unit_offset(rt, kb0, 0, 0, a.K);
+                bulk_g2s_hint_elect(sc, c0 + uoff, cbytes, &full[s], pol);
+                if (a.two) bulk_g2s_hint_elect(sc + cbytes, c1 + uoff, cbytes, &full[s], pol);
+                if (a.group) {
+                    const int64_t soff = ((int64_t)rt * ng + kb0) * kTileRows;
+                    bulk_g2s_elect(sc + kStageCodes, s0 + soff, sbytes, &full[s]);
+                    if (a.two) bulk_g2s_elect(sc + kStageCodes + sbytes, s1 + soff, sbytes, &full[s]);
                 }
+                for (int i = 0; i < SPS; ++i)
+                    tma_load_2d_elect(st + i * kAtomBytes, &bmap, (kb0 + i) * 64, p0, &full[s]);
             }
         }
     } else if (warp == 1) {
@@ -291,28 +290,34 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
             if (tcount >= 2 && ok && !mbar_wait_warp_sleep(&accempty[buf], ((tcount >> 1) - 1) & 1, a.err)) ok = false;
             tc_fence_after();
             const uint32_t dacc = tmem + 128 * buf;
-            for (int ks = 0; ks < KS; ++ks, ++u) {
-                const int s = u % kGemmStages, as = u % kGemmAStages;
+            for (int ka = 0; ka < KA; ++ka, ++u) {
+                const int su = u / APS, w = u - su * APS;  // ring stage, A unit inside it
+                const int s = su % kGemmStages, as = u % kGemmAStages;
                 if (ok && !mbar_wait_warp_sleep(&afull[as], (u / kGemmAStages) & 1, a.err)) ok = false;
-                if (ok && !mbar_wait_warp_sleep(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
+                if (ok && !mbar_wait_warp_sleep(&full[s], (su / kGemmStages) & 1, a.err)) ok = false;
                 tc_fence_after();
-                const uint64_t bdesc = smem_desc_sw128(smem + s * kStageBytes);
+                uint8_t* st = smem + s * kStageBytes;
                 const uint32_t a0 = tmem + 256 + 64 * as;
+                if (a.two) {
+                    const uint64_t bdesc = smem_desc_sw128(st + w * kAtomBytes);
 #pragma unroll
-                for (int slot = 0; slot < 2; ++slot)
+                    for (int slot = 0; slot < 2; ++slot)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (a.two) {
+                        for (int j = 0; j < 4; ++j)
                             tc_mma_ts_elect(dacc + 64 * slot, a0 + 32 * slot + 8 * j, bdesc + 2 * j, idesc,
-                                            (ks > 0 || j > 0) ? 1u : 0u);
-                        } else {
-                            tc_mma_ts_elect(dacc, a0 + 32 * slot + 8 * j,
-                                            bdesc + (uint64_t)((slot * kAtomBytes) >> 4) + 2 * j, idesc,
-                                            (ks > 0 || slot > 0 || j > 0) ? 1u : 0u);
-                        }
+                                            (ka > 0 || j > 0) ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int slot = 0; slot < 2; ++slot) {
+                        const uint64_t bdesc = smem_desc_sw128(st + (2 * w + slot) * kAtomBytes);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tc_mma_ts_elect(dacc, a0 + 32 * slot + 8 * j, bdesc + 2 * j, idesc,
+                                            (ka > 0 || slot > 0 || j > 0) ? 1u : 0u);
                     }
+                }
                 tc_commit_elect(&aempty[as]);
-                tc_commit_elect(&empty[s]);
+                if (w == APS - 1) tc_commit_elect(&empty[s]);
             }
             tc_commit_elect(&accfull[buf]);
         }
@@ -388,13 +393,16 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
         int u = 0;
         int p0, n, rt;
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x) {
-            for (int ks = 0; ks < KS; ++ks, ++u) {
-                const int s = u % kGemmStages, as = u % kGemmAStages;
-                if (ok && !mbar_wait_warp_sleep(&full[s], (u / kGemmStages) & 1, a.err)) ok = false;
+            for (int ka = 0; ka < KA; ++ka, ++u) {
+                const int su = u / APS, w = u - su * APS;  // ring stage, A unit inside it
+                const int s = su % kGemmStages, as = u % kGemmAStages;
+                if (ok && !mbar_wait_warp_sleep(&full[s], (su / kGemmStages) & 1, a.err)) ok = false;
                 if (u >= kGemmAStages && ok && !mbar_wait_warp_sleep(&aempty[as], ((u / kGemmAStages) - 1) & 1, a.err)) ok = false;
                 tc_fence_after();
                 const uint32_t sc = sbase + s * kStageBytes + kStageB;
-                const uint4 un = lds128(sc + slot * 4096 + (b8 * 32 + lane) * 16);
+                // gate/up: matrix `slot`, step w; down: step 2w + slot
+                const int blk = a.two ? slot * SPS + w : 2 * w + slot;
+                const uint4 un = lds128(sc + blk * 4096 + (b8 * 32 + lane) * 16);
                 const uint32_t wd[4] = {un.x, un.y, un.z, un.w};
                 uint32_t r[16];
 #pragma unroll
@@ -407,7 +415,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
                     r[4 * j + 2] = f[1]; r[4 * j + 3] = f[3];
                 }
                 if (a.group) {  // gs64: A = fp16(q * s)
-                    const uint32_t sa = sc + kStageCodes + slot * 512 + (b8 * 16 + g) * 4;
+                    const uint32_t sa = sc + kStageCodes + blk * 512 + (b8 * 16 + g) * 4;
                     const __half2 s0 = __float2half2_rn(lds32f(sa));
                     const __half2 s1 = __float2half2_rn(lds32f(sa + 32));
 #pragma unroll
@@ -421,7 +429,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) { mbar_arrive(&afull[as]); mbar_arrive(&empty[s]); }
+                if (lane == 0) {
+                    mbar_arrive(&afull[as]);
+                    if (w == APS - 1) mbar_arrive(&empty[s]);
+                }
             }
         }
     }
