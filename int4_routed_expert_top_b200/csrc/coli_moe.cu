@@ -155,6 +155,23 @@ int set_smem(const void* fn, int bytes) {
 int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, float* zpart,
                   __half* xq, float* xinv, cudaStream_t st, int* ks_out,
                   const RouterExtras* fused = nullptr) {
+    const bool row_ok = T <= kRouterRowMaxT && d.H <= kRouterRowMaxH && d.H % 4 == 0 &&
+                        (reinterpret_cast<uintptr_t>(d.router_w) & 15) == 0;
+    if (row_ok) {
+        RouterExtras ex;
+        if (fused) ex = *fused;
+        ex.xq = xq;
+        ex.xinv = xinv;
+        const int qblocks = (ex.xq || ex.xq8) ? T : 0;
+        const int zblocks = ex.zero_n > 0 ? 1 : 0;
+        const dim3 grid(d.E + qblocks + zblocks);
+        if (xt == COLI_F32)
+            router_row_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, zpart, ex);
+        else
+            router_row_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, zpart, ex);
+        *ks_out = 1;
+        return check_launch("router");
+    }
     int KS = 0;
     if (T <= kRouterMaxT)
         for (int c : {8, 4, 2, 1})
@@ -677,6 +694,8 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         ex.err = at<int32_t>(ws, p.err);
         ex.sel = at<float>(ws, p.sel);
         ex.bias = d.router_b;
+        ex.l2_prefetch = static_cast<const uint8_t*>(d.experts) + (int64_t)d.E * layer->L.bytes;
+        ex.l2_prefetch_bytes = (int64_t)d.n_shared * layer->L.bytes;
         if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), nullptr, nullptr, st, &KS, &ex)))
             return rc;
         // the fused kernel is the union, gate/up and down stages at once

@@ -166,39 +166,50 @@ __device__ __forceinline__ FzScratch fz_scratch(uint8_t* ring, int E) {
     return r;
 }
 
+// Order-preserving key of a selection score: a larger float gives a larger
+// key; -0 and +0 give the same key (they compare equal as floats).
+__device__ __forceinline__ uint32_t fz_order_key(float f) {
+    const uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Top-k of token t by one warp (E <= 256: up to 8 candidates per lane).
-// Order: selection score descending, expert index ascending.
+// Order: selection score descending, expert index ascending.  Each round takes
+// every lane's best remaining candidate (largest key, then smallest expert),
+// the warp's largest key by redux.sync and, among the lanes holding it, the
+// smallest expert; that lane retires the candidate.
 __device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, const FzScratch& sc8) {
     const int lane = threadIdx.x & 31;
-    float sc[8], sel[8];
+    float sc[8];
+    uint32_t key[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
         const bool ok = e < a.E;
         sc[i] = ok ? __ldcg(a.score + (int64_t)t * a.E + e) : 0.0f;
-        sel[i] = ok ? __ldcg(a.sel + (int64_t)t * a.E + e) : -INFINITY;
+        key[i] = ok ? fz_order_key(__ldcg(a.sel + (int64_t)t * a.E + e)) : 0u;  // 0: none
     }
     float mine = 0.0f;
     int mine_e = 0;
     for (int j = 0; j < a.k; ++j) {
-        float bv = -INFINITY, bs = 0.0f;
-        int be = 0x7fffffff;
+        uint32_t bk = key[0];
+        int bi = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane + 32 * i;
-            if (sel[i] > bv || (sel[i] == bv && e < be)) { bv = sel[i]; be = e; bs = sc[i]; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; bs = os; }
-        }
-        if (lane == j) { mine = bs; mine_e = be; }
+        for (int i = 1; i < 8; ++i)
+            if (key[i] > bk) { bk = key[i]; bi = i; }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t we = __reduce_min_sync(0xffffffffu, bk == wk ? (uint32_t)(lane + 32 * bi) : 0xffffffffu);
+        float bs = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            if (lane + 32 * i == be) sel[i] = -INFINITY;
+            if (i == bi) bs = sc[i];
+        const float ws = __shfl_sync(0xffffffffu, bs, (int)(we & 31u));
+        if (lane == (int)(we & 31u)) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i == bi) key[i] = 0u;
+        }
+        if (lane == j) { mine = ws; mine_e = (int)we; }
     }
     float denom = 0.0f;  // over the picks in pick order
     for (int j = 0; j < a.k; ++j) denom += __shfl_sync(0xffffffffu, mine, j);
@@ -216,23 +227,12 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const FzScratch sc8 = fz_scratch(ring, a.E);
     for (int e = threadIdx.x; e < a.E; e += kFzThreads) { sc8.cnt[e] = 0; sc8.bits[e] = 0ull; }
-    for (int t = threadIdx.x; t < a.T; t += kFzThreads) sh.xinv[t] = __ldcg(a.xinv8 + t);
     for (int t = warp; t < a.T; t += kAllWarps) fz_topk_token(a, t, sc8);
-    __syncthreads();
-    if (threadIdx.x == 32 * kFzProducer) {
-        // The shared experts are used whatever the routing: while the union is
-        // formed, pull this CTA's slice of their blobs into L2 (issued after
-        // the score loads, which it would otherwise slow down).
-        const int64_t total = (int64_t)a.n_shared * a.blob_bytes;
-        const int64_t chunk = ((total + gridDim.x - 1) / gridDim.x + 255) & ~int64_t(255);
-        const int64_t beg = (int64_t)blockIdx.x * chunk;
-        const int64_t end = beg + chunk < total ? beg + chunk : total;
-        const uint8_t* base = a.experts + (int64_t)a.E * a.blob_bytes;
-        for (int64_t off = beg; off < end; off += 65536) {
-            const uint32_t n = (uint32_t)(end - off < 65536 ? end - off : 65536);
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(n) : "memory");
-        }
+    {   // from the last threads, which have no token's top-k before them when T is small
+        const int t = kFzThreads - 1 - (int)threadIdx.x;
+        if (t < a.T) sh.xinv[t] = __ldcg(a.xinv8 + t);
     }
+    __syncthreads();
     const int Tk = a.T * a.k;
     for (int i = threadIdx.x; i < Tk; i += kFzThreads) {
         const int e = sc8.pick_e[i];

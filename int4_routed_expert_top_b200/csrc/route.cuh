@@ -10,10 +10,21 @@
 #pragma once
 
 #include "common.cuh"
+#include "pipeline.cuh"
 
 namespace coli {
 
 constexpr int kMaxKS = 8;
+
+// Four consecutive activations as f32 (16-byte f32 or 8-byte bf16 load).
+__device__ __forceinline__ float4 load4_f32(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ float4 load4_f32(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+}
 
 // ---------------------------------------------------------------------------
 // fp16 hi/lo activation operand, one CTA (256 threads) per token: one power of
@@ -96,14 +107,35 @@ __device__ __forceinline__ void fz_split(float v, float sc, int& hi, int& lo) {
 
 // s8 activation operand of one token, one CTA of 256 threads: xq8[t][step]
 // (64 hi bytes then 64 lo bytes, columns in fz_act_pos order), xinv8[t].
+// Thread tid owns columns 4 tid + 1024 j; for H <= 8192 the row is read once,
+// with every load in flight together, and kept in registers for both passes.
 template <typename XT>
 __device__ __forceinline__ void act_quant8_token(const XT* __restrict__ x, int H, int t,
                                                  int8_t* __restrict__ xq8,
                                                  float* __restrict__ xinv8) {
+    constexpr int kJ = 8;
     __shared__ float part8[8];
     const XT* row = x + (int64_t)t * H;
+    const bool in_regs = H <= 1024 * kJ;
+    const bool vec = (reinterpret_cast<uintptr_t>(row) & (4 * sizeof(XT) - 1)) == 0;
+    float4 v[kJ];
     float m = 0.0f;
-    for (int c = threadIdx.x; c < H; c += 256) m = fmaxf(m, fabsf(to_f32(row[c])));
+    if (in_regs) {
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const int c = 4 * threadIdx.x + 1024 * j;
+            v[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (c < H)
+                v[j] = vec ? load4_f32(row + c)
+                           : make_float4(to_f32(row[c]), to_f32(row[c + 1]), to_f32(row[c + 2]),
+                                         to_f32(row[c + 3]));
+        }
+#pragma unroll
+        for (int j = 0; j < kJ; ++j)
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
+    } else {
+        for (int c = threadIdx.x; c < H; c += 256) m = fmaxf(m, fabsf(to_f32(row[c])));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((threadIdx.x & 31) == 0) part8[threadIdx.x >> 5] = m;
@@ -114,7 +146,25 @@ __device__ __forceinline__ void act_quant8_token(const XT* __restrict__ x, int H
     float inv;
     const float sc = fz_scale(m, &inv);
     // four consecutive columns per thread -> one 32-bit word of hi, one of lo
-    for (int c = 4 * threadIdx.x; c < H; c += 1024) {
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+        const int c = 4 * threadIdx.x + 1024 * j;
+        if (!in_regs || c >= H) break;
+        const float f[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+        uint32_t wh = 0, wl = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int hi, lo;
+            fz_split(f[i], sc, hi, lo);
+            wh |= (uint32_t)(hi & 0xFF) << (8 * i);
+            wl |= (uint32_t)(lo & 0xFF) << (8 * i);
+        }
+        int8_t* step = xq8 + ((int64_t)t * (H / 64) + c / 64) * 128;
+        const int pos = fz_act_pos(c % 64);
+        *reinterpret_cast<uint32_t*>(step + pos) = wh;
+        *reinterpret_cast<uint32_t*>(step + 64 + pos) = wl;
+    }
+    for (int c = 4 * threadIdx.x; !in_regs && c < H; c += 1024) {
         uint32_t wh = 0, wl = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -146,12 +196,16 @@ struct RouterExtras {
     // sel receives s + bias instead of the logits
     float* sel = nullptr;
     const float* bias = nullptr;
+    // bytes the dependent kernel reads whatever the routing (the shared
+    // experts' blobs): pulled into L2 by the router CTAs, each its slice, once
+    // their own weight loads are in flight, while HBM is otherwise idle
+    const uint8_t* l2_prefetch = nullptr;
+    int64_t l2_prefetch_bytes = 0;
 };
 
-// (at most 48 registers, so that a CTA fits beside a CTA of the dependent
-// fused kernel, which then starts while the router finishes)
+
 template <typename XT>
-__global__ void __launch_bounds__(256, 5)
+__global__ void __launch_bounds__(256)
 router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restrict__ wr,
                    int E, int KS, float* __restrict__ zpart, int router_blocks,
                    RouterExtras ex) {
@@ -177,12 +231,32 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
     const int e = gw / KS, ks = gw % KS;
     const bool valid = e < E;
     const int SL = H / KS;  // multiple of 128, at most kRouterMaxSlice
+    const int per = 8 / KS;  // experts of this CTA
+    // this thread's first output's bias, loaded beside the weights
+    float bias0 = 0.0f;
+    if (ex.sel && (int)threadIdx.x < per * T) {
+        const int ee = blockIdx.x * per + (int)threadIdx.x / T;
+        if (ee < E) bias0 = __ldg(ex.bias + ee);
+    }
     if (valid) {
         const float* wrow = wr + (int64_t)e * H + (int64_t)ks * SL;
         float4 wv[kRouterMaxSlice / 128];
 #pragma unroll
         for (int i = 0; i < kRouterMaxSlice / 128; ++i)
             if (i * 128 < SL) wv[i] = __ldg(reinterpret_cast<const float4*>(wrow + i * 128 + lane * 4));
+        if (threadIdx.x == 0 && ex.l2_prefetch) {
+            const int64_t total = ex.l2_prefetch_bytes;
+            const int64_t chunk = ((total + router_blocks - 1) / router_blocks + 255) & ~int64_t(255);
+            const int64_t beg = (int64_t)blockIdx.x * chunk;
+            const int64_t end = beg + chunk < total ? beg + chunk : total;
+            for (int64_t off = beg; off < end; off += 65536) {
+                const uint32_t n = (uint32_t)(end - off < 65536 ? end - off : 65536) & ~15u;
+                if (n) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                                    ::"l"(ex.l2_prefetch + off), "r"(n) : "memory");
+            }
+        }
+        // vector loads when the rows are aligned for them (H is a multiple of 128)
+        const bool vec = (reinterpret_cast<uintptr_t>(x) & (4 * sizeof(XT) - 1)) == 0;
         for (int t = 0; t < T; ++t) {
             const XT* xr = x + (int64_t)t * H + (int64_t)ks * SL + lane * 4;
             float acc = 0.0f;
@@ -190,10 +264,13 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
             for (int i = 0; i < kRouterMaxSlice / 128; ++i) {
                 if (i * 128 < SL) {
                     const XT* xp = xr + i * 128;
-                    acc = fmaf(wv[i].x, to_f32(xp[0]), acc);
-                    acc = fmaf(wv[i].y, to_f32(xp[1]), acc);
-                    acc = fmaf(wv[i].z, to_f32(xp[2]), acc);
-                    acc = fmaf(wv[i].w, to_f32(xp[3]), acc);
+                    const float4 xv = vec ? load4_f32(xp)
+                                          : make_float4(to_f32(xp[0]), to_f32(xp[1]),
+                                                        to_f32(xp[2]), to_f32(xp[3]));
+                    acc = fmaf(wv[i].x, xv.x, acc);
+                    acc = fmaf(wv[i].y, xv.y, acc);
+                    acc = fmaf(wv[i].z, xv.z, acc);
+                    acc = fmaf(wv[i].w, xv.w, acc);
                 }
             }
             acc = warp_sum(acc);
@@ -201,7 +278,6 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
         }
     }
     __syncthreads();
-    const int per = 8 / KS;  // experts of this CTA
     for (int j = threadIdx.x; j < per * T; j += 256) {
         const int el = j / T, t = j % T, ee = blockIdx.x * per + el;
         if (ee >= E) continue;
@@ -210,10 +286,115 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
         if (ex.sel) {
             const float sc = 1.0f / (1.0f + expf(-z));
             zpart[(int64_t)t * E + ee] = sc;
-            ex.sel[(int64_t)t * E + ee] = sc + __ldg(ex.bias + ee);
+            ex.sel[(int64_t)t * E + ee] = sc + (j == (int)threadIdx.x ? bias0 : __ldg(ex.bias + ee));
         } else {
             zpart[(int64_t)t * E + ee] = z;
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Router for a few tokens (T <= kRouterRowMaxT, H <= kRouterRowMaxH), one CTA
+// per expert e: the expert's router row (H f32, contiguous) arrives in shared
+// memory by one bulk copy while every thread loads its activation columns
+// c = 4 tid + 1024 j of the first token, so that the CTA waits for about one
+// trip to memory.  Each thread sums its columns in j order, the warp by
+// warp_sum, then the 8 warps in warp order.  The CTAs after the E routers
+// build the activation operands and clear the work queue and error flag, as
+// in router_gemv_kernel; the flag is cleared within microseconds of the launch
+// and a bounded wait here gives up only after about a second, so a timeout it
+// reports is not lost to the clearing.
+// ---------------------------------------------------------------------------
+constexpr int kRouterRowMaxT = 4;
+constexpr int kRouterRowMaxH = 8192;
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+router_row_kernel(const XT* __restrict__ x, int T, int H, const float* __restrict__ wr, int E,
+                  float* __restrict__ zout, RouterExtras ex) {
+    constexpr int kJ = kRouterRowMaxH / 1024;
+    __shared__ __align__(128) float wrow[kRouterRowMaxH];
+    __shared__ float part[8][kRouterRowMaxT];
+    __shared__ __align__(8) uint64_t bar;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int e = blockIdx.x;
+    if (e >= E) {
+        const int b = e - E;
+        if (b < T) {
+            if (ex.xq) act_quant_token(x, H, b, ex.xq, ex.xinv);
+            if (ex.xq8) act_quant8_token(x, H, b, ex.xq8, ex.xinv8);
+        } else {
+            for (int i = threadIdx.x; i < ex.zero_n; i += 256) ex.zero[i] = 0;
+            if (threadIdx.x == 0 && ex.err) *ex.err = 0;
+        }
+        return;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_expect_tx(&bar, (uint32_t)H * 4u);
+        bulk_g2s(wrow, wr + (int64_t)e * H, (uint32_t)H * 4u, &bar);
+        if (ex.l2_prefetch) {
+            const int64_t total = ex.l2_prefetch_bytes;
+            const int64_t chunk = ((total + E - 1) / E + 255) & ~int64_t(255);
+            const int64_t beg = (int64_t)e * chunk;
+            const int64_t end = beg + chunk < total ? beg + chunk : total;
+            for (int64_t off = beg; off < end; off += 65536) {
+                const uint32_t n = (uint32_t)(end - off < 65536 ? end - off : 65536) & ~15u;
+                if (n) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                                    ::"l"(ex.l2_prefetch + off), "r"(n) : "memory");
+            }
+        }
+    }
+    const float bias = (ex.sel && (int)threadIdx.x < T) ? __ldg(ex.bias + e) : 0.0f;
+    const bool vec = (reinterpret_cast<uintptr_t>(x) & (4 * sizeof(XT) - 1)) == 0;
+    auto load_token = [&](int t, float4 (&xv)[kJ]) {
+        const XT* xr = x + (int64_t)t * H;
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const int c = 4 * threadIdx.x + 1024 * j;
+            if (c < H)
+                xv[j] = vec ? load4_f32(xr + c)
+                            : make_float4(to_f32(xr[c]), to_f32(xr[c + 1]), to_f32(xr[c + 2]),
+                                          to_f32(xr[c + 3]));
+        }
+    };
+    float4 cur[kJ], nxt[kJ];
+    load_token(0, cur);
+    __syncthreads();  // the barrier's initialisation, before anyone waits on it
+    const bool ok = mbar_wait_warp(&bar, 0, ex.err);
+    for (int t = 0; t < T; ++t) {
+        if (t + 1 < T) load_token(t + 1, nxt);
+        float acc = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const int c = 4 * threadIdx.x + 1024 * j;
+            if (c < H) {
+                const float4 w = *reinterpret_cast<const float4*>(wrow + c);
+                acc = fmaf(w.x, cur[j].x, acc);
+                acc = fmaf(w.y, cur[j].y, acc);
+                acc = fmaf(w.z, cur[j].z, acc);
+                acc = fmaf(w.w, cur[j].w, acc);
+            }
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) part[warp][t] = acc;
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) cur[j] = nxt[j];
+    }
+    __syncthreads();
+    if (!ok || (int)threadIdx.x >= T) return;
+    const int t = threadIdx.x;
+    float z = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) z += part[w][t];
+    if (ex.sel) {
+        const float sc = 1.0f / (1.0f + expf(-z));
+        zout[(int64_t)t * E + e] = sc;
+        ex.sel[(int64_t)t * E + e] = sc + bias;
+    } else {
+        zout[(int64_t)t * E + e] = z;
     }
 }
 
