@@ -144,6 +144,8 @@ struct FusedShared {
     float xch[8][16][kFzChunk];                   // up values for the gate warps
     float wmax[8][kFzChunk];                      // per-warp max |h| of each pair
     __align__(16) int8_t hbuf[kFzChunk * kFzRecH]; // h of the current item, s8 digits
+    int pick1_e[kFzMaxK];                         // one token: its picks (outside the ring,
+    float pick1_w[kFzMaxK];                       // which fills while they are read)
     int n_uniq, n_items;
 };
 
@@ -219,6 +221,74 @@ __device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, const F
     }
 }
 
+// The batch union by one warp when there are at most 32 picks, in the order
+// the picks first name their experts: units in order of first appearance in
+// (token, slot) order, pairs inside a unit in token order.  The work order is
+// a scheduling choice only: partial products are indexed by pick, so y does
+// not depend on it.  Lane i holds pick i; __match_any_sync finds the picks of
+// the same expert, a ballot the first ones, and one shuffle scan of packed
+// (pairs, items) gives every unit's first pair and first item.
+__device__ __forceinline__ void fz_union_warp(const FusedArgs& a, FusedShared& sh,
+                                              const FzScratch& sc8) {
+    const int lane = threadIdx.x & 31;
+    const int Tk = a.T * a.k, TG = a.I / 128;
+    const bool valid = lane < Tk;
+    const int e = valid ? sc8.pick_e[lane] : 0;
+    const int t = valid ? lane / a.k : 0;
+    const unsigned lt = (1u << lane) - 1u;
+    const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);  // idle lanes: one group
+    const bool first = valid && (same & lt) == 0u;
+    const unsigned firsts = __ballot_sync(0xffffffffu, first);
+    const int nu = __popc(firsts);
+    const int cnt = __popc(same);
+    const int items = first ? (cnt + kFzChunk - 1) / kFzChunk * TG : 0;
+    // inclusive scan of (pairs | items << 16) over the first lanes, lane order
+    int incl = first ? (cnt | (items << 16)) : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+    }
+    const int excl_p = (incl & 0xffff) - (first ? cnt : 0);
+    const int excl_i = (incl >> 16) - items;
+    const int routed_items = __shfl_sync(0xffffffffu, incl, 31) >> 16;
+    // every pick's pair: its unit's first pair plus the earlier picks of the unit
+    const int p = __shfl_sync(0xffffffffu, excl_p, __ffs(same) - 1) + __popc(same & lt);
+    if (first) {
+        const int u = __popc(firsts & lt);
+        sh.u_exp[u] = e;
+        sh.u_p0[u] = excl_p;
+        sh.u_p1[u] = excl_p + cnt;
+        sh.u_item0[u] = excl_i;
+    }
+    if (valid) {
+        sh.pair_tok[p] = t;
+        sh.pair_pick[p] = t * (a.k + a.n_shared) + (lane - t * a.k);
+        if (blockIdx.x == 0) {
+            a.idx[lane] = e;
+            a.w[lane] = sc8.pick_w[lane];
+            a.inv[lane] = p;
+        }
+    }
+    const int per_shared = (a.T + kFzChunk - 1) / kFzChunk * TG;
+    if (lane < a.n_shared) {
+        sh.u_exp[nu + lane] = a.E + lane;
+        sh.u_p0[nu + lane] = Tk + lane * a.T;
+        sh.u_p1[nu + lane] = Tk + (lane + 1) * a.T;
+        sh.u_item0[nu + lane] = routed_items + lane * per_shared;
+    }
+    for (int i = lane; i < a.n_shared * a.T; i += 32) {
+        const int tt = i % a.T;
+        sh.pair_tok[Tk + i] = tt;
+        sh.pair_pick[Tk + i] = tt * (a.k + a.n_shared) + a.k + i / a.T;
+    }
+    if (lane == 0) {
+        sh.n_uniq = nu;
+        sh.u_item0[nu + a.n_shared] = routed_items + a.n_shared * per_shared;
+        sh.n_items = routed_items + a.n_shared * per_shared;
+    }
+}
+
 // Top-k of every token and the batch union, in this CTA's shared memory, and
 // the work items: unit u's pairs in chunks of kFzChunk, I/128 items per chunk.
 // CTA 0 also publishes the picks, weights and pair indices.  Returns the units.
@@ -226,14 +296,21 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
     constexpr int kAllWarps = kFzThreads / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const FzScratch sc8 = fz_scratch(ring, a.E);
-    for (int e = threadIdx.x; e < a.E; e += kFzThreads) { sc8.cnt[e] = 0; sc8.bits[e] = 0ull; }
+    const int Tk = a.T * a.k;
+    const bool small = Tk <= 32;
+    if (!small)
+        for (int e = threadIdx.x; e < a.E; e += kFzThreads) { sc8.cnt[e] = 0; sc8.bits[e] = 0ull; }
     for (int t = warp; t < a.T; t += kAllWarps) fz_topk_token(a, t, sc8);
     {   // from the last threads, which have no token's top-k before them when T is small
         const int t = kFzThreads - 1 - (int)threadIdx.x;
         if (t < a.T) sh.xinv[t] = __ldcg(a.xinv8 + t);
     }
     __syncthreads();
-    const int Tk = a.T * a.k;
+    if (small) {
+        if (warp == 0) fz_union_warp(a, sh, sc8);
+        __syncthreads();
+        return sh.n_uniq + a.n_shared;
+    }
     for (int i = threadIdx.x; i < Tk; i += kFzThreads) {
         const int e = sc8.pick_e[i];
         atomicAdd(&sc8.cnt[e], 1);
@@ -402,10 +479,12 @@ __device__ __forceinline__ FzShape fz_shape(const FusedArgs& a) {
 // ---------------------------------------------------------------------------
 template <bool GS>
 __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, uint8_t* ring,
-                                           int n_units) {
+                                           int n_units, bool one) {
     const int lane = threadIdx.x & 31;
     const FzShape z = fz_shape(a);
-    const int n_items = sh.n_items;
+    // one token: unit u = item / TG is pick u (slot order), then the shared
+    // experts, one pair each (pair u, token 0); no tables needed
+    const int n_items = one ? n_units * z.TG : sh.n_items;
     const int rec_gu = fz_rec_bytes(z.ns_gu);
     const int ngH = GS ? a.H / 64 : 1, ngI = GS ? a.I / 64 : 1;
     const uint64_t pol = l2_evict_first_policy();
@@ -414,9 +493,19 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
     bool ok = true;
     int item = blockIdx.x;  // first item: by CTA index; later ones from the queue
     while (ok && item < n_items) {
-        const FzWork wk = fz_work(sh, n_units, z.TG, item);
+        FzWork wk;
+        int e;
+        if (one) {
+            wk.u = item / z.TG;
+            wk.tc = item - wk.u * z.TG;
+            wk.p0 = wk.u;
+            wk.np = 1;
+            e = wk.u < a.k ? sh.pick1_e[wk.u] : a.E + (wk.u - a.k);
+        } else {
+            wk = fz_work(sh, n_units, z.TG, item);
+            e = sh.u_exp[wk.u];
+        }
         const int tc = wk.tc, p0 = wk.p0, np = wk.np;
-        const int e = sh.u_exp[wk.u];
         const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
         const uint8_t* cG = blob + a.L.codes[0];
         const uint8_t* cU = blob + a.L.codes[1];
@@ -449,7 +538,7 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
                     bulk_g2s_elect(sl + kFzScaleOff + 512, sU + (int64_t)tc * kTileRows, 512u, &sh.full[s]);
                 }
                 for (int pp = 0; pp < np; ++pp) {
-                    const int tok = sh.pair_tok[p0 + pp];
+                    const int tok = one ? 0 : sh.pair_tok[p0 + pp];
                     bulk_g2s_elect(sl + kFzActOff + pp * rec_gu,
                                    a.xq8 + ((int64_t)tok * (a.H / 64) + kb0) * 128,
                                    (uint32_t)z.ns_gu * 128, &sh.full[s]);
@@ -780,8 +869,36 @@ moe_fused_kernel(FusedArgs a) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // everything below reads what the router kernel wrote
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int warp = threadIdx.x >> 5;
+    if (a.T == 1) {
+        // One token: the producer needs only the picks (named barrier 2: warp
+        // 0 and the producer), so it starts streaming while warp 0 writes the
+        // unit and pair tables for the consumer warps (named barrier 1).
+        __syncthreads();  // barrier initialisation, before any wait on them
+        const int n_units = a.k + a.n_shared;  // the k picks are distinct experts
+        if (warp == kFzProducer) {
+            asm volatile("bar.sync 2, %0;" ::"n"(64) : "memory");
+            fz_produce<GS>(a, sh, fz_smem, n_units, true);
+            return;
+        }
+        if (warp == 0) {
+            FzScratch one;
+            one.bits = nullptr; one.cnt = nullptr; one.excl = nullptr;
+            one.pick_e = sh.pick1_e;
+            one.pick_w = sh.pick1_w;
+            fz_topk_token(a, 0, one);
+            __syncwarp();
+            asm volatile("bar.arrive 2, %0;" ::"n"(64) : "memory");
+            fz_union_warp(a, sh, one);
+        } else if (warp == 1 && (threadIdx.x & 31) == 0) {
+            sh.xinv[0] = __ldcg(a.xinv8);
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kFzWarps) : "memory");
+        fz_consume<NT, GS>(a, sh, fz_smem, n_units);
+        return;
+    }
     const int n_units = fz_route_union(a, sh, fz_smem);
-    if ((threadIdx.x >> 5) == kFzProducer) fz_produce<GS>(a, sh, fz_smem, n_units);
+    if (warp == kFzProducer) fz_produce<GS>(a, sh, fz_smem, n_units, false);
     else fz_consume<NT, GS>(a, sh, fz_smem, n_units);
 }
 
