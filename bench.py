@@ -436,6 +436,16 @@ def main():
                      if gemm else f"{dominant}_gemv_kernel")
             line["stages_us"] = {n: 1e3 * v for n, v in zip(cm.STAGE_NAMES, stage_mean)}
             line["down_gbs"] = dn_ach
+            if gemm:
+                # tensor work of the dominant launch: gate/up is 2I x H per pair, down H x I
+                pairs = T * (wl.k + wl.n_shared)
+                rows_k = 2 * wl.I * wl.H if dominant == "gateup" else wl.H * wl.I
+                col = 2 if dominant == "gateup" else 3
+                tflops = 2.0 * pairs * rows_k / (st_ms[:, col].mean() / 1e3) / 1e12
+                line["tensor_roofline"] = {"bound": "tensor", "achieved": tflops, "peak": bf16_tf,
+                                           "unit": "TFLOP/s", "frac": tflops / bf16_tf,
+                                           "kernel": kname, "dtype": "f16 x f16 -> f32",
+                                           "peak_source": peak_src}
         traffic = None
         if fused and wl.name == "glm_decode" and T == 1:
             traffic = profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
