@@ -694,8 +694,6 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         ex.err = at<int32_t>(ws, p.err);
         ex.sel = at<float>(ws, p.sel);
         ex.bias = d.router_b;
-        ex.l2_prefetch = static_cast<const uint8_t*>(d.experts) + (int64_t)d.E * layer->L.bytes;
-        ex.l2_prefetch_bytes = (int64_t)d.n_shared * layer->L.bytes;
         if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), nullptr, nullptr, st, &KS, &ex)))
             return rc;
         // the fused kernel is the union, gate/up and down stages at once

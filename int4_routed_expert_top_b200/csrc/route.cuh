@@ -196,11 +196,6 @@ struct RouterExtras {
     // sel receives s + bias instead of the logits
     float* sel = nullptr;
     const float* bias = nullptr;
-    // bytes the dependent kernel reads whatever the routing (the shared
-    // experts' blobs): pulled into L2 by the router CTAs, each its slice, once
-    // their own weight loads are in flight, while HBM is otherwise idle
-    const uint8_t* l2_prefetch = nullptr;
-    int64_t l2_prefetch_bytes = 0;
 };
 
 
@@ -244,17 +239,6 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
 #pragma unroll
         for (int i = 0; i < kRouterMaxSlice / 128; ++i)
             if (i * 128 < SL) wv[i] = __ldg(reinterpret_cast<const float4*>(wrow + i * 128 + lane * 4));
-        if (threadIdx.x == 0 && ex.l2_prefetch) {
-            const int64_t total = ex.l2_prefetch_bytes;
-            const int64_t chunk = ((total + router_blocks - 1) / router_blocks + 255) & ~int64_t(255);
-            const int64_t beg = (int64_t)blockIdx.x * chunk;
-            const int64_t end = beg + chunk < total ? beg + chunk : total;
-            for (int64_t off = beg; off < end; off += 65536) {
-                const uint32_t n = (uint32_t)(end - off < 65536 ? end - off : 65536) & ~15u;
-                if (n) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                                    ::"l"(ex.l2_prefetch + off), "r"(n) : "memory");
-            }
-        }
         // vector loads when the rows are aligned for them (H is a multiple of 128)
         const bool vec = (reinterpret_cast<uintptr_t>(x) & (4 * sizeof(XT) - 1)) == 0;
         for (int t = 0; t < T; ++t) {
@@ -335,17 +319,6 @@ router_row_kernel(const XT* __restrict__ x, int T, int H, const float* __restric
         fence_mbar_init();
         mbar_expect_tx(&bar, (uint32_t)H * 4u);
         bulk_g2s(wrow, wr + (int64_t)e * H, (uint32_t)H * 4u, &bar);
-        if (ex.l2_prefetch) {
-            const int64_t total = ex.l2_prefetch_bytes;
-            const int64_t chunk = ((total + E - 1) / E + 255) & ~int64_t(255);
-            const int64_t beg = (int64_t)e * chunk;
-            const int64_t end = beg + chunk < total ? beg + chunk : total;
-            for (int64_t off = beg; off < end; off += 65536) {
-                const uint32_t n = (uint32_t)(end - off < 65536 ? end - off : 65536) & ~15u;
-                if (n) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                                    ::"l"(ex.l2_prefetch + off), "r"(n) : "memory");
-            }
-        }
     }
     const float bias = (ex.sel && (int)threadIdx.x < T) ? __ldg(ex.bias + e) : 0.0f;
     const bool vec = (reinterpret_cast<uintptr_t>(x) & (4 * sizeof(XT) - 1)) == 0;
