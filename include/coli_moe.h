@@ -226,6 +226,37 @@ int coli_moe_stack_forward(const coli_moe_layer* const* layers, int32_t L,
                            float* x, int32_t T, float eps, coli_path path,
                            void* ws, size_t ws_bytes, coli_stream_t stream);
 
+/* coli_moe_forward_ex (no residual, no routing outputs) for x and y in host
+ * memory: x_host [T, H] (f32 or bf16) is copied into staging at the end of the
+ * workspace, the layer runs on the device, and y [T, H] f32 is copied back into
+ * y_host, all asynchronously on `stream`; y_host holds the result once the
+ * stream has reached the end of the call (synchronise it or wait on an event
+ * recorded after it).  Page-locked host memory that is mapped into the
+ * device's address space (cudaHostAlloc memory on a unified-address system,
+ * or cudaHostRegister with cudaHostRegisterMapped) is read and written by a
+ * small kernel through that mapping, which for the few kilobytes of a decode
+ * step avoids the copy engine's start-up latency; other memory is copied with
+ * cudaMemcpyAsync (pageable memory only outside stream capture).  Page-locked
+ * buffers make the call capturable into a CUDA graph.  ws must cover
+ * coli_moe_host_workspace_size(layer, T) bytes (the forward's workspace plus
+ * the staging of x and y). */
+int coli_moe_host_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes);
+int coli_moe_forward_host(const coli_moe_layer* layer, const void* x_host, coli_dtype xt,
+                          int32_t T, float* y_host, coli_path path, void* ws,
+                          size_t ws_bytes, coli_stream_t stream);
+
+/* coli_moe_stack_forward for a residual stream in host memory: x_host f32
+ * [T, H] is copied into staging in the workspace, the L layers run on it in
+ * place, and the result is copied to y_host (which may equal x_host), with the
+ * same rules as coli_moe_forward_host.  ws must cover
+ * coli_moe_stack_host_workspace_size(layers, L, T) bytes. */
+int coli_moe_stack_host_workspace_size(const coli_moe_layer* const* layers, int32_t L,
+                                       int32_t T, size_t* bytes);
+int coli_moe_stack_forward_host(const coli_moe_layer* const* layers, int32_t L,
+                                const float* x_host, float* y_host, int32_t T, float eps,
+                                coli_path path, void* ws, size_t ws_bytes,
+                                coli_stream_t stream);
+
 /* Device-side status of the most recent coli_moe_forward* call that used this
  * workspace (ws planned for T tokens): copies the error flags to *flags (host)
  * after synchronising `stream`.  Returns COLI_E_TIMEOUT if a bounded wait inside

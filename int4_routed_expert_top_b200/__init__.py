@@ -37,7 +37,8 @@ EXPORTS = (
     "coli_moe_layer_destroy", "coli_moe_workspace_size", "coli_moe_route",
     "coli_moe_union", "coli_moe_forward", "coli_moe_forward_ex", "coli_moe_rmsnorm",
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
-    "coli_moe_forward_noalloc", "coli_moe_status",
+    "coli_moe_forward_noalloc", "coli_moe_status", "coli_moe_host_workspace_size",
+    "coli_moe_forward_host", "coli_moe_stack_host_workspace_size", "coli_moe_stack_forward_host",
 )
 
 
@@ -87,6 +88,12 @@ _SIGS = {
     "coli_moe_dequant_debug": ([_P, _I32, _I32, _P, _P], ctypes.c_int),
     "coli_moe_forward_noalloc": ([_P, _P, ctypes.c_int, _I32, _P, _P], ctypes.c_int),
     "coli_moe_status": ([_P, _I32, _P, ctypes.POINTER(_I32), _P], ctypes.c_int),
+    "coli_moe_host_workspace_size": ([_P, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "coli_moe_forward_host": ([_P, _P, ctypes.c_int, _I32, _P, ctypes.c_int, _P, _SZ, _P],
+                              ctypes.c_int),
+    "coli_moe_stack_host_workspace_size": ([_P, _I32, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "coli_moe_stack_forward_host": ([_P, _I32, _P, _P, _I32, ctypes.c_float, ctypes.c_int, _P,
+                                     _SZ, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -233,6 +240,32 @@ def coli_moe_stack_workspace_size(layers, T: int) -> int:
 def coli_moe_stack_forward(layers, x, T, eps, ws, path=COLI_PATH_AUTO, stream=None):
     _ok(lib.coli_moe_stack_forward(_layer_array(layers), len(layers), _ptr(x), T, eps, path,
                                    _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def coli_moe_host_workspace_size(layer, T: int) -> int:
+    out = _SZ()
+    _ok(lib.coli_moe_host_workspace_size(layer, T, ctypes.byref(out)))
+    return out.value
+
+
+def coli_moe_forward_host(layer, x_host, T, y_host, ws, path=COLI_PATH_AUTO, stream=None):
+    """x_host / y_host: host tensors (page-locked for graph capture); ws on the device."""
+    _ok(lib.coli_moe_forward_host(layer, _ptr(x_host), _xtype(x_host), T, _ptr(y_host), path,
+                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def coli_moe_stack_host_workspace_size(layers, T: int) -> int:
+    out = _SZ()
+    _ok(lib.coli_moe_stack_host_workspace_size(_layer_array(layers), len(layers), T,
+                                               ctypes.byref(out)))
+    return out.value
+
+
+def coli_moe_stack_forward_host(layers, x_host, y_host, T, eps, ws, path=COLI_PATH_AUTO,
+                                stream=None):
+    _ok(lib.coli_moe_stack_forward_host(_layer_array(layers), len(layers), _ptr(x_host),
+                                        _ptr(y_host), T, eps, path, _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def coli_moe_status(layer, T: int, ws, stream=None) -> int:

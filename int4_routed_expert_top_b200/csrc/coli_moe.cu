@@ -148,6 +148,27 @@ int set_smem(const void* fn, int bytes) {
     return COLI_OK;
 }
 
+// Launch as a programmatic dependent of the previous kernel in the stream: the
+// kernel may start while that one finishes and waits (griddepcontrol.wait)
+// before it reads what that one wrote.
+template <typename... Args>
+int launch_pdl(void (*kern)(Args...), dim3 grid, int threads, int smem, cudaStream_t st,
+               const char* what, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) return fail(COLI_E_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return check_launch(what);
+}
+
 // Router logits into zpart ([*ks_out][T][E] K slices; the small-batch router
 // sums its slices itself and reports one).  When xq is non-null the
 // fp16 activation operand is produced as well (by extra CTAs of the small-batch
@@ -165,12 +186,12 @@ int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, f
         const int qblocks = (ex.xq || ex.xq8) ? T : 0;
         const int zblocks = ex.zero_n > 0 ? 1 : 0;
         const dim3 grid(d.E + qblocks + zblocks);
-        if (xt == COLI_F32)
-            router_row_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, zpart, ex);
-        else
-            router_row_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, zpart, ex);
         *ks_out = 1;
-        return check_launch("router");
+        if (xt == COLI_F32)
+            return launch_pdl(router_row_kernel<float>, grid, 256, 0, st, "router", (const float*)x,
+                              T, d.H, d.router_w, d.E, zpart, ex);
+        return launch_pdl(router_row_kernel<__nv_bfloat16>, grid, 256, 0, st, "router",
+                          (const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, zpart, ex);
     }
     int KS = 0;
     if (T <= kRouterMaxT)
@@ -185,12 +206,12 @@ int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, f
         const int qblocks = (ex.xq || ex.xq8) ? T : 0;
         const int zblocks = ex.zero_n > 0 ? 1 : 0;
         const dim3 grid(rblocks + qblocks + zblocks);
-        if (xt == COLI_F32)
-            router_gemv_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
-        else
-            router_gemv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
         *ks_out = 1;
-        return check_launch("router");
+        if (xt == COLI_F32)
+            return launch_pdl(router_gemv_kernel<float>, grid, 256, 0, st, "router",
+                              (const float*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
+        return launch_pdl(router_gemv_kernel<__nv_bfloat16>, grid, 256, 0, st, "router",
+                          (const __nv_bfloat16*)x, T, d.H, d.router_w, d.E, KS, zpart, rblocks, ex);
     } else {
         const int tiles = ((T + 63) / 64) * ((d.E + 63) / 64);
         KS = 1;
@@ -419,23 +440,6 @@ int sm_count() { return gemm_grid(); }
 // Launch with programmatic stream serialisation: the kernel may start while
 // the previous one (router, then fused) finishes; it waits
 // (griddepcontrol.wait) before reading what that kernel wrote.
-template <typename... Args>
-int launch_pdl(void (*kern)(Args...), dim3 grid, int threads, int smem, cudaStream_t st,
-               const char* what, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-    if (e != cudaSuccess) return fail(COLI_E_CUDA, "%s: %s", what, cudaGetErrorString(e));
-    return check_launch(what);
-}
 
 template <int NT, bool GS>
 int launch_fused_t(const FusedArgs& a, cudaStream_t st) {
@@ -803,6 +807,100 @@ int coli_moe_stack_forward(const coli_moe_layer* const* layers, int32_t L, float
             return rc;
     }
     return COLI_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Host-buffer entry points: x is copied into staging at the end of the
+// workspace, the device forward runs, y is copied back; all on one stream.
+// Page-locked memory that is mapped into the device's address space (what
+// cudaHostAlloc gives on a unified-address system) is copied by a small
+// kernel; anything else by cudaMemcpyAsync.
+// ---------------------------------------------------------------------------
+namespace {
+int stage_copy(const void* src, void* dst, size_t bytes, bool h2d, cudaStream_t st) {
+    void* mapped = nullptr;
+    const void* host = h2d ? src : dst;
+    if (bytes % 4 == 0 &&
+        cudaHostGetDevicePointer(&mapped, const_cast<void*>(host), 0) == cudaSuccess && mapped) {
+        const int64_t words = (int64_t)(bytes / 16) + 1;
+        const int grid = (int)std::min<int64_t>(4 * sm_count(), (words + 255) / 256);
+        stage_copy_kernel<<<grid, 256, 0, st>>>(h2d ? mapped : src, h2d ? dst : mapped,
+                                                (int64_t)bytes);
+        return check_launch(h2d ? "stage in" : "stage out");
+    }
+    (void)cudaGetLastError();  // not mapped: clear the query's error, copy by DMA
+    if (cudaMemcpyAsync(dst, src, bytes, h2d ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost,
+                        st) != cudaSuccess)
+        return fail(COLI_E_CUDA, "host copy failed");
+    return COLI_OK;
+}
+}  // namespace
+
+int coli_moe_host_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes) {
+    size_t b;
+    int rc = coli_moe_workspace_size(layer, T, &b);
+    if (rc) return rc;
+    const int64_t row = (int64_t)T * layer->d.H * 4;
+    *bytes = (size_t)(align256((int64_t)b) + 2 * align256(row));
+    return COLI_OK;
+}
+
+int coli_moe_forward_host(const coli_moe_layer* layer, const void* x_host, coli_dtype xt,
+                          int32_t T, float* y_host, coli_path path, void* ws, size_t ws_bytes,
+                          coli_stream_t stream) {
+    if (!layer || !x_host || !y_host) return fail(COLI_E_INVAL, "forward_host: NULL pointer");
+    if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_E_INVAL, "forward_host: bad dtype");
+    size_t need, inner;
+    int rc = coli_moe_host_workspace_size(layer, T, &need);
+    if (rc) return rc;
+    if ((rc = coli_moe_workspace_size(layer, T, &inner))) return rc;
+    if (!ws || ws_bytes < need)
+        return fail(COLI_E_WORKSPACE, "forward_host: workspace %zu < %zu bytes", ws_bytes, need);
+    const int64_t row = (int64_t)T * layer->d.H * 4;
+    char* base = static_cast<char*>(ws);
+    void* xd = base + align256((int64_t)inner);
+    float* yd = reinterpret_cast<float*>(base + align256((int64_t)inner) + align256(row));
+    const size_t xbytes = (size_t)T * layer->d.H * (xt == COLI_F32 ? 4 : 2);
+    if ((rc = stage_copy(x_host, xd, xbytes, true, S(stream)))) return rc;
+    // y mapped into the device's address space: the layer's last kernel writes
+    // it there directly (no path reads y back when there is no residual; the
+    // tensor-core path's combine stores 16-byte vectors, hence the alignment)
+    void* ymap = nullptr;
+    if ((reinterpret_cast<uintptr_t>(y_host) & 15) != 0 ||
+        cudaHostGetDevicePointer(&ymap, y_host, 0) != cudaSuccess || !ymap) {
+        (void)cudaGetLastError();
+        ymap = nullptr;
+    }
+    if ((rc = coli_moe_forward_ex(layer, xd, xt, T, ymap ? static_cast<float*>(ymap) : yd, nullptr,
+                                  path, nullptr, nullptr, nullptr, ws, inner, stream)))
+        return rc;
+    return ymap ? COLI_OK : stage_copy(yd, y_host, (size_t)row, false, S(stream));
+}
+
+int coli_moe_stack_host_workspace_size(const coli_moe_layer* const* layers, int32_t L, int32_t T,
+                                       size_t* bytes) {
+    size_t b;
+    int rc = coli_moe_stack_workspace_size(layers, L, T, &b);
+    if (rc) return rc;
+    *bytes = (size_t)(align256((int64_t)b) + align256((int64_t)T * layers[0]->d.H * 4));
+    return COLI_OK;
+}
+
+int coli_moe_stack_forward_host(const coli_moe_layer* const* layers, int32_t L,
+                                const float* x_host, float* y_host, int32_t T, float eps,
+                                coli_path path, void* ws, size_t ws_bytes, coli_stream_t stream) {
+    if (!x_host || !y_host) return fail(COLI_E_INVAL, "stack_forward_host: NULL pointer");
+    size_t need, inner;
+    int rc = coli_moe_stack_host_workspace_size(layers, L, T, &need);
+    if (rc) return rc;
+    if ((rc = coli_moe_stack_workspace_size(layers, L, T, &inner))) return rc;
+    if (!ws || ws_bytes < need)
+        return fail(COLI_E_WORKSPACE, "stack_forward_host: workspace %zu < %zu bytes", ws_bytes, need);
+    const size_t row = (size_t)T * layers[0]->d.H * 4;
+    float* xd = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((int64_t)inner));
+    if ((rc = stage_copy(x_host, xd, row, true, S(stream)))) return rc;
+    if ((rc = coli_moe_stack_forward(layers, L, xd, T, eps, path, ws, inner, stream))) return rc;
+    return stage_copy(xd, y_host, row, false, S(stream));
 }
 
 int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t which,

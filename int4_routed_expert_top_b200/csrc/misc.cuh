@@ -1,4 +1,5 @@
-// misc.cuh - device quantiser/packer, dequantiser (test helper) and RMSNorm.
+// misc.cuh - device quantiser/packer, dequantiser (test helper), RMSNorm and the
+// staging copies of the host-buffer entry points.
 //
 // Quantiser ("jlnsrk/GLM-5.2-colibri-int4 - Hugging Face": container paragraph
 // and conversion note): per row or per 64 columns s = max|w| / 7, q =
@@ -107,6 +108,29 @@ rmsnorm_kernel(const float* x, int H, float eps, float* out) {
         float4 v = *reinterpret_cast<const float4*>(xr + c);
         v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
         *reinterpret_cast<float4*>(orow + c) = v;
+    }
+}
+
+// Byte copy between page-locked host memory (through its device mapping) and
+// device memory, by SM loads and stores: for the few kilobytes of a decode
+// step this avoids the copy engine's start-up and hand-off latency.  16-byte
+// words when both pointers and the size allow, else 4-byte words (the sizes
+// here are multiples of 4).
+__global__ void __launch_bounds__(256)
+stage_copy_kernel(const void* __restrict__ src, void* __restrict__ dst, int64_t bytes) {
+    // the router (a programmatic dependent) may be scheduled now; it waits for
+    // this grid before reading the staged tokens
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) | (uintptr_t)bytes) & 15) == 0) {
+        const uint4* s = static_cast<const uint4*>(src);
+        uint4* d = static_cast<uint4*>(dst);
+        for (int64_t i = i0; i < bytes / 16; i += stride) d[i] = s[i];
+    } else {
+        const uint32_t* s = static_cast<const uint32_t*>(src);
+        uint32_t* d = static_cast<uint32_t*>(dst);
+        for (int64_t i = i0; i < bytes / 4; i += stride) d[i] = s[i];
     }
 }
 

@@ -208,6 +208,8 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
     // the dependent fused kernel may start its prologue (it waits for this
     // grid's completion before reading anything written here)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // launched as a programmatic dependent: x may come from the previous grid
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if ((int)blockIdx.x >= router_blocks) {
         const int b = blockIdx.x - router_blocks;
         if (b < T) {  // one CTA per token: activation operand
@@ -301,6 +303,8 @@ router_row_kernel(const XT* __restrict__ x, int T, int H, const float* __restric
     __shared__ float part[8][kRouterRowMaxT];
     __shared__ __align__(8) uint64_t bar;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // launched as a programmatic dependent: x may come from the previous grid
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int e = blockIdx.x;
     if (e >= E) {
         const int b = e - E;
