@@ -80,6 +80,25 @@ def test_gemm_path_residual_and_zero_input():
     assert rel_err(out.cpu().numpy() - res.cpu().numpy(), y_ref) <= TOL_TC
 
 
+def test_gemm_path_at_the_largest_batch():
+    """T = 8192, the largest batch a call accepts (16-expert layer): ~2,000
+    pairs per expert, so every unit spans many N tiles.  All outputs against
+    the f32 GEMV path, 64 sampled tokens against the oracle, selected experts
+    exactly."""
+    wl = dataclasses.replace(synth.TINY, T=8192, group=64)
+    wr, b = synth.router(wl)
+    x, idx_ref, w_ref, _ = gap_resampled_tokens(wl, wl.T, wr, b)
+    L = build_layer(wl, router=(wr, b))
+    xd = device_x(x, wl)
+    y, idx, _ = forward(L, xd, wl.T, cm.COLI_PATH_GEMM)
+    same_selection(idx, idx_ref)
+    y_gemv, _, _ = forward(L, xd, wl.T, cm.COLI_PATH_GEMV)
+    assert rel_err(y, y_gemv) <= TOL_TC
+    rows = np.linspace(0, wl.T - 1, 64).astype(int)
+    y_ref = oracle_tokens(wl, OracleExperts(wl), x.numpy()[rows], idx_ref[rows], w_ref[rows])
+    assert rel_err(y[rows], y_ref) <= TOL_TC
+
+
 @pytest.fixture(scope="module")
 def glm_prefill_layer():
     L = build_layer(synth.GLM_PREFILL)
