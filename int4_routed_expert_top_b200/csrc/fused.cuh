@@ -112,18 +112,6 @@ __device__ __forceinline__ void decode_word_s8(uint32_t w, uint32_t& r0, uint32_
     r1 = (w << 4) & 0xF0F0F0F0u;
 }
 
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// order this thread's generic-proxy view before its later async-proxy (bulk
-// copy) reads of global memory
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 }  // namespace coli
 
 namespace coli {

@@ -144,14 +144,6 @@ __device__ __forceinline__ void bulk_g2s_hint_elect(void* dst, const void* src, 
         : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2_elect(const void* src, uint32_t bytes) {
-    asm volatile(
-        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
-        " @e cp.async.bulk.prefetch.L2.global [%0], %1;\n}"
-        ::"l"(src), "r"(bytes)
-        : "memory");
-}
-
 // barrier among the first `threads` threads of the CTA (named barrier 1)
 __device__ __forceinline__ void named_sync(int threads) {
     asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
