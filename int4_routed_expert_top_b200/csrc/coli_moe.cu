@@ -769,8 +769,7 @@ int coli_moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps, float* out
                      coli_stream_t stream) {
     if (!x || !out) return fail(COLI_E_INVAL, "rmsnorm: NULL pointer");
     if (T < 1 || H < 4 || H % 4) return fail(COLI_E_INVAL, "rmsnorm: bad shape");
-    rmsnorm_kernel<<<T, 256, 0, S(stream)>>>(x, H, eps, out);
-    return check_launch("rmsnorm");
+    return launch_pdl(rmsnorm_kernel, dim3(T), 256, 0, S(stream), "rmsnorm", x, (int)H, eps, out);
 }
 
 int coli_moe_stack_workspace_size(const coli_moe_layer* const* layers, int32_t L, int32_t T,

@@ -909,6 +909,9 @@ struct CombineArgs {
 __global__ void __launch_bounds__(1024)
 moe_combine_kernel(CombineArgs c) {
     __shared__ float oj[kFzMaxK + 4][32];
+    // the next kernel may be scheduled now (this library's kernels wait for
+    // this grid before reading y); then wait for the fused kernel's partials
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nw = blockDim.x >> 5;

@@ -87,6 +87,10 @@ dequant_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ scal
 __global__ void __launch_bounds__(256)
 rmsnorm_kernel(const float* x, int H, float eps, float* out) {
     __shared__ float part[8];
+    // a programmatic dependent: the next kernel (the router) may be scheduled
+    // now, and x may come from the previous grid
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t t = blockIdx.x;
     const float* xr = x + t * H;
     float ss = 0.0f;
