@@ -307,6 +307,22 @@ int encode_b_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
     return COLI_OK;
 }
 
+// xq8 of T tokens as [T] rows of 2H bytes read as 32-bit words; boxes of the
+// gate/up stage's 64-column steps (ns x 128 B) of every token, no swizzle
+int encode_act_map(CUtensorMap* m, const void* xq8, int T, int H, int ns) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(COLI_E_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[2] = {(cuuint64_t)(2 * H / 4), (cuuint64_t)T};
+    const cuuint64_t strides[1] = {(cuuint64_t)2 * H};
+    const cuuint32_t box[2] = {(cuuint32_t)(ns * 128 / 4), (cuuint32_t)T};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(xq8), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(COLI_E_CUDA, "activation tensor map encode failed (%d)", (int)r);
+    return COLI_OK;
+}
+
 int gemm_grid() {
     static int sms = 0;
     if (!sms) {
@@ -442,11 +458,12 @@ int sm_count() { return gemm_grid(); }
 // (griddepcontrol.wait) before reading what that kernel wrote.
 
 template <int NT, bool GS>
-int launch_fused_t(const FusedArgs& a, cudaStream_t st) {
+int launch_fused_t(const CUtensorMap& xmap, const FusedArgs& a, cudaStream_t st) {
     const int smem = a.slots * a.slot_bytes;
     int rc = set_smem((const void*)moe_fused_kernel<NT, GS>, smem);
     if (rc) return rc;
-    return launch_pdl(moe_fused_kernel<NT, GS>, dim3(sm_count()), kFzThreads, smem, st, "fused moe", a);
+    return launch_pdl(moe_fused_kernel<NT, GS>, dim3(sm_count()), kFzThreads, smem, st, "fused moe",
+                      xmap, a);
 }
 
 template <typename Mark>
@@ -479,10 +496,18 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     if (a.slots < 2) return fail(COLI_E_UNSUPPORTED, "fused: ring does not fit");
     const bool gs = d.group != 0;
     int rc;
+    // 2 to 4 tokens: one TMA box brings every token's activation slice of a stage
+    CUtensorMap xmap;
+    std::memset(&xmap, 0, sizeof(xmap));
+    a.act_tma = 0;
+    if (T >= 2 && NT == 1) {
+        if ((rc = encode_act_map(&xmap, a.xq8, T, d.H, fz_ns_gateup(d.H)))) return rc;
+        a.act_tma = 1;
+    }
     switch (NT) {
-        case 1: rc = gs ? launch_fused_t<1, true>(a, st) : launch_fused_t<1, false>(a, st); break;
-        case 2: rc = gs ? launch_fused_t<2, true>(a, st) : launch_fused_t<2, false>(a, st); break;
-        default: rc = gs ? launch_fused_t<4, true>(a, st) : launch_fused_t<4, false>(a, st); break;
+        case 1: rc = gs ? launch_fused_t<1, true>(xmap, a, st) : launch_fused_t<1, false>(xmap, a, st); break;
+        case 2: rc = gs ? launch_fused_t<2, true>(xmap, a, st) : launch_fused_t<2, false>(xmap, a, st); break;
+        default: rc = gs ? launch_fused_t<4, true>(xmap, a, st) : launch_fused_t<4, false>(xmap, a, st); break;
     }
     if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;

@@ -85,6 +85,12 @@ struct FusedArgs {
     int T, E, k, n_shared, H, I, group;
     int slots;              // ring stages
     int slot_bytes;
+    // 1: a gate/up stage takes every token's activation slice with one 2-D TMA
+    // box of the kernel's tensor map over xq8 (T rows of 2H bytes read as 32-bit
+    // words, boxes of T x 128 words), stored [token][step][hi 64 B | lo 64 B];
+    // used for 2 <= T <= 4 (one column group).  0: one bulk copy per pair,
+    // stored per pair record.
+    int act_tma;
 };
 
 // row tiles (of 128 H rows) per down stage: the largest of 4, 3, 2, 1 dividing H/128
@@ -466,8 +472,8 @@ __device__ __forceinline__ FzShape fz_shape(const FusedArgs& a) {
 //     [codes, 8 KB per tile | scales (per row: 512 B per tile; gs64: 1 KB)].
 // ---------------------------------------------------------------------------
 template <bool GS>
-__device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, uint8_t* ring,
-                                           int n_units, bool one) {
+__device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap* xmap,
+                                           FusedShared& sh, uint8_t* ring, int n_units, bool one) {
     const int lane = threadIdx.x & 31;
     const FzShape z = fz_shape(a);
     // one token: unit u = item / TG is pick u (slot order), then the shared
@@ -511,7 +517,8 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
                 const int kb0 = st * z.ns_gu;
                 const bool rowsc = !GS && st == z.nst_gu - 1;
                 const uint32_t cb = (uint32_t)z.ns_gu * 4096, sb = GS ? (uint32_t)z.ns_gu * 512 : 0u;
-                mbar_expect_tx_elect(&sh.full[s], 2 * (cb + sb) + (uint32_t)(np * z.ns_gu * 128) +
+                const int nrec = a.act_tma ? a.T : np;  // activation slices of the stage
+                mbar_expect_tx_elect(&sh.full[s], 2 * (cb + sb) + (uint32_t)(nrec * z.ns_gu * 128) +
                                                       (rowsc ? 1024u : 0u));
                 const int64_t coff = frag_unit_offset(tc, kb0, 0, 0, a.H);
                 bulk_g2s_hint_elect(sl, cG + coff, cb, &sh.full[s], pol);
@@ -525,11 +532,15 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, FusedShared& sh, 
                     bulk_g2s_elect(sl + kFzScaleOff, sG + (int64_t)tc * kTileRows, 512u, &sh.full[s]);
                     bulk_g2s_elect(sl + kFzScaleOff + 512, sU + (int64_t)tc * kTileRows, 512u, &sh.full[s]);
                 }
-                for (int pp = 0; pp < np; ++pp) {
-                    const int tok = one ? 0 : sh.pair_tok[p0 + pp];
-                    bulk_g2s_elect(sl + kFzActOff + pp * rec_gu,
-                                   a.xq8 + ((int64_t)tok * (a.H / 64) + kb0) * 128,
-                                   (uint32_t)z.ns_gu * 128, &sh.full[s]);
+                if (a.act_tma) {  // every token's slice, [token][step][128 B] (x in 4-byte units)
+                    tma_load_2d_elect(sl + kFzActOff, xmap, kb0 * 32, 0, &sh.full[s]);
+                } else {
+                    for (int pp = 0; pp < np; ++pp) {
+                        const int tok = one ? 0 : sh.pair_tok[p0 + pp];
+                        bulk_g2s_elect(sl + kFzActOff + pp * rec_gu,
+                                       a.xq8 + ((int64_t)tok * (a.H / 64) + kb0) * 128,
+                                       (uint32_t)z.ns_gu * 128, &sh.full[s]);
+                    }
                 }
             } else {
                 const int rt0 = (st - z.nst_gu) * z.rs;
@@ -577,13 +588,14 @@ namespace coli {
 // ---------------------------------------------------------------------------
 template <int NT, bool GS>
 __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb, int lane,
-                                                int rec_gu, int ntc, int acc_i[2][NT][4],
+                                                int rec_gu, int aoff, int ntc, int acc_i[2][NT][4],
                                                 float acc_f[NT][4]) {
     constexpr int ns = 4;
     const int g = lane >> 2, t = lane & 3;
     const float lanefac = t < 2 ? 256.0f : 1.0f;
     const uint8_t* cp = sl + m * ns * 4096 + rb * 512 + lane * 16;
-    const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + (g & 3) * rec_gu;
+    // aoff: this lane's pair record (column group 0); groups c > 0 follow at 4 c rec_gu
+    const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + aoff;
     const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff + m * ns * 512) + 16 * rb + g;
 #pragma unroll
     for (int j = 0; j < ns; ++j) {
@@ -728,6 +740,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
     uint32_t cphase = 0, lap = 0;
     int s = 0;
     int u = 0, tc = 0, p0 = 0, np = 0;
+    int aoff = 0;  // this lane's activation record in a gate/up stage
     float sw0 = 1.0f, sw1 = 1.0f;  // per-row weight scales of rows g, g + 8
     float hf[NT][2];               // down part: digit and h scale factors
     int dst[NT][2];                //            partial-product offsets
@@ -744,6 +757,12 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
             tc = wk.tc;
             p0 = wk.p0;
             np = wk.np;
+            if (a.act_tma) {  // records by token: the token of this lane's pair
+                const int pp = g & 3;
+                aoff = (pp < np ? sh.pair_tok[p0 + pp] : 0) * (z.ns_gu * 128);
+            } else {
+                aoff = (g & 3) * rec_gu;
+            }
 #pragma unroll
             for (int c = 0; c < NT; ++c)
 #pragma unroll
@@ -751,7 +770,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
         }
         const bool gu = st < z.nst_gu;
         if (gu) {
-            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, (np + 3) >> 2, acc_i, acc_f);
+            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, aoff, (np + 3) >> 2, acc_i, acc_f);
             if (!GS && st == z.nst_gu - 1) {
                 const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
                 sw0 = rsc[0];
@@ -845,7 +864,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
 
 template <int NT, bool GS>
 __global__ void __launch_bounds__(kFzThreads, 1)
-moe_fused_kernel(FusedArgs a) {
+moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
     extern __shared__ __align__(128) uint8_t fz_smem[];
     __shared__ FusedShared sh;
     if (threadIdx.x == 0) {
@@ -866,7 +885,7 @@ moe_fused_kernel(FusedArgs a) {
         const int n_units = a.k + a.n_shared;  // the k picks are distinct experts
         if (warp == kFzProducer) {
             asm volatile("bar.sync 2, %0;" ::"n"(64) : "memory");
-            fz_produce<GS>(a, sh, fz_smem, n_units, true);
+            fz_produce<GS>(a, &xmap, sh, fz_smem, n_units, true);
             return;
         }
         if (warp == 0) {
@@ -886,7 +905,7 @@ moe_fused_kernel(FusedArgs a) {
         return;
     }
     const int n_units = fz_route_union(a, sh, fz_smem);
-    if (warp == kFzProducer) fz_produce<GS>(a, sh, fz_smem, n_units, false);
+    if (warp == kFzProducer) fz_produce<GS>(a, &xmap, sh, fz_smem, n_units, false);
     else fz_consume<NT, GS>(a, sh, fz_smem, n_units);
 }
 

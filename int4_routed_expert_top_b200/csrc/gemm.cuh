@@ -115,14 +115,6 @@ __device__ __forceinline__ void tc_mma_ts_elect(uint32_t d, uint32_t a, uint64_t
         " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}"
         ::"r"(d), "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
-__device__ __forceinline__ void tma_load_2d_elect(void* dst, const CUtensorMap* map, int x, int y,
-                                                  uint64_t* bar) {
-    asm volatile(
-        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
-        " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n}"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-        : "memory");
-}
 __device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t r[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"

@@ -1,7 +1,9 @@
 // pipeline.cuh - shared-memory producer/consumer pipelines on sm_100a:
-// mbarriers, 1-D bulk copies (the TMA engine without a tensor map) and waits
+// mbarriers, 1-D bulk copies and 2-D tiled loads (the TMA engine) and waits
 // that give up after a bounded number of tries instead of hanging.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
@@ -141,6 +143,18 @@ __device__ __forceinline__ void bulk_g2s_hint_elect(void* dst, const void* src, 
         " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1], %2, [%3], %4;\n}"
         ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+
+// 2-D tiled TMA load of the box at (x, y) of `map` into shared memory,
+// completion counted in bytes on `bar` (warp-uniform operands; one elected
+// lane issues).  x times the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d_elect(void* dst, const CUtensorMap* map, int x, int y,
+                                                  uint64_t* bar) {
+    asm volatile(
+        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+        " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n}"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
 
