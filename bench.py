@@ -229,6 +229,26 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# job-wide numbers over ranks (one replica per GPU)
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Length of a timed region as the job sees it: the largest over the ranks
+    (every rank calls this at the same point, so the collectives stay in step)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, job_ms: float) -> float:
+    """Whole-job throughput: the tokens of every rank over the job's time."""
+    return tokens_per_rank * world / (job_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # own arm
 # ---------------------------------------------------------------------------
 def main():
@@ -350,12 +370,8 @@ def main():
     barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)
-    tot = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    job_ms = float(tot.item())
-    tokens_all = T * K * world
-    value = tokens_all / (job_ms / 1e3)
+    job_ms = max_over_ranks(total_ms, world, dev)
+    value = job_tokens_per_s(T * K, world, job_ms)
 
     # per-stage device times: graphs with event nodes at the stage boundaries
     st_ms = []
@@ -406,10 +422,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
-    t2 = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_value = tokens_all / (float(t2.item()) / 1e3)
+    e2e_value = job_tokens_per_s(T * K, world, max_over_ranks(e2e_ms, world, dev))
 
     # bytes: int4 codes + f32 scales of the unique routed experts + shared, per step
     blob = L0.blob_bytes
