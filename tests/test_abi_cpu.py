@@ -134,6 +134,11 @@ def test_workspace_size_and_limits_without_gpu():
         with pytest.raises(cm.ColiError) as e:
             cm.coli_moe_workspace_size(h, 8192)         # union bitmap limit
         assert e.value.code == -4
+        # the host-buffer calls add staging for x and y behind the forward's workspace
+        hb = cm.coli_moe_host_workspace_size(h, 4)
+        assert hb >= cm.coli_moe_workspace_size(h, 4) + 2 * 4 * 6144 * 4
+        sb = cm.coli_moe_stack_host_workspace_size([h, h], 4)
+        assert sb >= cm.coli_moe_stack_workspace_size([h, h], 4) + 4 * 6144 * 4
         # a workspace that is too small is refused before anything is launched
         ws = np.zeros(16, np.uint8)
         with pytest.raises(cm.ColiError) as e:
