@@ -1,6 +1,6 @@
 // fused.cuh - the routed MoE layer after the router for small batches
-// (decode, MTP verify: T <= 16 tokens) in one persistent kernel, plus the
-// kernel that forms y from its partial sums.
+// (decode, MTP verify and batches up to T = 64 tokens) in one persistent
+// kernel, plus the kernel that forms y from its partial sums.
 //
 // Steps (sources are web pages, cited by title and section):
 //   top-k   sigmoid scores, bias-corrected selection of k experts (ties to the
@@ -15,10 +15,16 @@
 // Every CTA (one per SM) first repeats the top-k and the union for the whole
 // batch in its own shared memory; the result is deterministic, so all CTAs
 // agree without exchanging it.  A unit is a distinct routed expert of the batch
-// or a shared expert.  A work item is (unit u, 128-row tile tc of I): the
-// CTA's producer warp streams the item's gate and up rows tc (all of H) and then
-// the matching 128 columns of the down matrix (all H rows) through a ring of
-// 32 KB stages with 1-D bulk copies (the TMA engine).  Sixteen consumer warps
+// or a shared expert.  A work item is (unit u, up to 16 of its pairs, 128-row
+// tile tc of I): the CTA's producer warp streams the item's gate and up rows tc
+// (all of H) and then the matching 128 columns of the down matrix (all H rows)
+// through a ring of ~37 KB stages (32 KB of int4 codes, their scales and the
+// activation digits) with 1-D bulk copies (the TMA engine; for 2 to 4 tokens a
+// 2-D TMA box brings every token's activation slice).  With one token the
+// units are the picks in slot order, so the producer starts streaming as soon
+// as warp 0 has the picks, while warp 0 builds the tables the consumers need;
+// with at most 32 picks the union is one warp's match/ballot/scan, in the
+// order the picks first name their experts (a work order only).  Sixteen consumer warps
 // decode the int4 codes in registers and multiply on the tensor cores
 // (mma.sync s8 x s8 -> s32, exact int32 sums over each 64-column step).  h of
 // the tile never leaves shared memory: the down part of the item multiplies it

@@ -1,5 +1,6 @@
-// route.cuh - router logits, sigmoid + bias-corrected top-k, the batch union,
-// and the fp16 activation operand of the expert kernels.
+// route.cuh - router logits (one kernel per batch-size range), sigmoid +
+// bias-corrected top-k, the batch union, and the activation operands of the
+// expert kernels (fp16 hi/lo digits; s8 digits for the fused kernel).
 //
 // Router ("解密GLM-5.2-colibri-int4-with-int8-mtp" 模型架构深度解析; "github一周涨11k
 // ⭐️！25GB 内存跑 744B GLM-5.2 模型！" 三.1 and 四.3): z = W_r x in f32 (plain FMA on
