@@ -51,9 +51,10 @@ def lib():
                                         ctypes.c_int32, ctypes.c_double, ctypes.c_int,
                                         P, P, P, P, P, P, P, P]
         L.orc_rmsnorm.argtypes = [P, i64, i64, ctypes.c_double, P]
+        L.orc_fp8_block_dequant.argtypes = [P, P, i64, i64, P]
         for f in ("orc_quantize", "orc_dequantize", "orc_route", "orc_union",
                   "orc_expert", "orc_token_forward", "orc_layer_forward",
-                  "orc_rmsnorm"):
+                  "orc_rmsnorm", "orc_fp8_block_dequant"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -78,6 +79,19 @@ def quantize(w, group: int):
     _check(lib().orc_quantize(pw, rows, cols, group, packed.ctypes.data_as(ctypes.c_void_p),
                               scales.ctypes.data_as(ctypes.c_void_p)), "quantize")
     return packed, scales
+
+
+def fp8_block_dequant(codes, block_scales):
+    """FP8 E4M3 codes [R, K] (uint8) with one f32 scale per 128 x 128 block
+    ([ceil(R/128), ceil(K/128)]) -> f32 [R, K]."""
+    codes, pq = _c(codes, np.uint8)
+    bs, pb = _c(block_scales, np.float32)
+    rows, cols = codes.shape
+    assert bs.shape == ((rows + 127) // 128, (cols + 127) // 128)
+    out = np.zeros((rows, cols), np.float32)
+    _check(lib().orc_fp8_block_dequant(pq, pb, rows, cols, out.ctypes.data_as(ctypes.c_void_p)),
+           "fp8_block_dequant")
+    return out
 
 
 def dequantize(packed, scales, cols: int, group: int):

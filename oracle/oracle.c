@@ -66,6 +66,38 @@ int orc_quantize(const float* w, int64_t rows, int64_t cols, int32_t group,
     return 0;
 }
 
+/* FP8 E4M3 code as a float, from the format's definition: sign bit, four
+ * exponent bits with bias 7, three mantissa bits; exponent 0 holds the
+ * subnormals m/8 * 2^-6; S.1111.111 is NaN and there are no infinities.
+ * Every value is exact in f32. */
+static float e4m3_value(uint8_t b) {
+    const int sign = b >> 7, e = (b >> 3) & 0xF, m = b & 7;
+    float v;
+    if (e == 0) v = ldexpf((float)m / 8.0f, -6);
+    else if (e == 15 && m == 7) v = NAN;
+    else v = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return sign ? -v : v;
+}
+
+/* Block-scaled FP8 matrix -> f32: out[r, c] = e4m3(q[r, c]) * bs[r/128, c/128],
+ * one f32 multiply (the checkpoint's 128 x 128 weight blocks, one scale each;
+ * bs is [ceil(rows/128), ceil(cols/128)] row-major).  ["解密GLM-5.2-colibri-int4-
+ * with-int8-mtp", quantisation-config paragraph: fmt e4m3, weight_block_size
+ * [128, 128]; the int4 container is converted from that checkpoint: "GLM-5.2-
+ * colibri-int4专家流技术详解", project-source section.] */
+int orc_fp8_block_dequant(const uint8_t* q, const float* bs, int64_t rows, int64_t cols,
+                          float* out) {
+    if (!q || !bs || !out || rows < 1 || cols < 1) return -1;
+    const int64_t kb = (cols + 127) / 128;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            const float v = e4m3_value(q[r * cols + c]);
+            const float s = bs[(r / 128) * kb + c / 128];
+            out[r * cols + c] = v * s;             /* f32 multiply, round to nearest */
+        }
+    return 0;
+}
+
 static int decode_nibble(uint8_t byte, int high) {
     int n = high ? (byte >> 4) & 0xF : byte & 0xF;
     return n >= 8 ? n - 16 : n;                     /* sign-extend 4 bits */

@@ -94,6 +94,12 @@ int orc_layer_forward(const float* x, int64_t T, int64_t H, int64_t I,
 /* RMSNorm with unit gain: out = v / sqrt(mean(v^2) + eps), per row of [T, H]. */
 int orc_rmsnorm(const float* x, int64_t T, int64_t H, double eps, float* out);
 
+/* FP8 (E4M3) matrix with one f32 scale per 128 x 128 block -> f32:
+ * out[r, c] = e4m3(q[r, c]) * bs[r / 128, c / 128] (bs row-major
+ * [ceil(rows/128), ceil(cols/128)]).  Returns 0, or -1 on bad arguments. */
+int orc_fp8_block_dequant(const uint8_t* q, const float* bs, int64_t rows, int64_t cols,
+                          float* out);
+
 #ifdef __cplusplus
 }
 #endif

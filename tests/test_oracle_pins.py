@@ -302,3 +302,46 @@ def test_rmsnorm_closed_form():
     z = rng.standard_normal((4, 1000)).astype(np.float32)
     o = oracle.rmsnorm(z, 0.0)
     np.testing.assert_allclose((o.astype(np.float64) ** 2).mean(1), 1.0, rtol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3, 128 x 128 block scales) -> f32, the step before the int4 container
+# ---------------------------------------------------------------------------
+
+def test_e4m3_hand_values():
+    codes = np.array([[0x00, 0x80, 0x38, 0x40, 0x3C, 0xB8, 0x7E, 0xFE, 0x08, 0x01, 0x07, 0x30]],
+                     np.uint8)
+    want = [0.0, -0.0, 1.0, 2.0, 1.5, -1.0, 448.0, -448.0, 2.0 ** -6, 2.0 ** -9,
+            7 * 2.0 ** -9, 0.5]
+    got = oracle.fp8_block_dequant(codes, np.ones((1, 1), np.float32))[0]
+    np.testing.assert_array_equal(got, np.array(want, np.float32))
+    assert math.copysign(1.0, got[1]) == -1.0                  # the sign of zero is kept
+    nan = oracle.fp8_block_dequant(np.array([[0x7F, 0xFF]], np.uint8), np.ones((1, 1), np.float32))
+    assert np.isnan(nan).all()                                  # S.1111.111 is NaN
+
+
+def test_e4m3_every_code_matches_torch():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    ours = oracle.fp8_block_dequant(codes, np.ones((1, 2), np.float32))[0]
+    ref = torch.from_numpy(codes[0].copy()).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    finite = ~np.isnan(ref)
+    assert finite.sum() == 254
+    np.testing.assert_array_equal(ours[finite].view(np.uint32), ref[finite].view(np.uint32))
+    assert np.isnan(ours[~finite]).all()
+
+
+def test_fp8_block_scales_cover_ragged_blocks():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(5)
+    R, K = 300, 260                                  # 3 x 3 blocks, the last ones ragged
+    codes = rng.integers(0, 256, (R, K), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C             # finite codes only
+    bs = rng.uniform(1e-4, 1e-2, (3, 3)).astype(np.float32)
+    got = oracle.fp8_block_dequant(codes, bs)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    scale = np.repeat(np.repeat(bs, 128, 0), 128, 1)[:R, :K]
+    np.testing.assert_array_equal(got.view(np.uint32), (vals * scale).view(np.uint32))
+    # the block edges: row 127 uses block row 0, row 128 block row 1
+    assert got[127, 0] == np.float32(vals[127, 0] * bs[0, 0])
+    assert got[128, 259] == np.float32(vals[128, 259] * bs[1, 2])
