@@ -138,6 +138,22 @@ int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group,
                                     const float* down, void* blob,
                                     coli_stream_t stream);
 
+/* coli_moe_quantize_expert_device for an expert given as FP8 E4M3 codes with
+ * one f32 scale per 128 x 128 block (the format of the checkpoint the int4
+ * container is converted from): every weight becomes
+ * w = e4m3(code) * bs[r / 128][c / 128] in f32 (the E4M3 value is exact; one
+ * f32 multiply), then the container's rule applies (s = max|w| / 7 per row or
+ * per 64 columns, q = rint(w / s)).  Device memory: gate, up [I, H] and down
+ * [H, I] as row-major bytes; gate_bs, up_bs [ceil(I/128), ceil(H/128)] and
+ * down_bs [ceil(H/128), ceil(I/128)] row-major f32.  Bit-identical to decoding
+ * on the host and using coli_moe_quantize + coli_moe_pack_expert.  The NaN
+ * codes (S.1111.111) give undefined blobs.  Asynchronous. */
+int coli_moe_quantize_expert_fp8_device(int32_t H, int32_t I, int32_t group,
+                                        const uint8_t* gate, const uint8_t* up,
+                                        const uint8_t* down, const float* gate_bs,
+                                        const float* up_bs, const float* down_bs,
+                                        void* blob, coli_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Layer                                                                     */
 /* ------------------------------------------------------------------------ */

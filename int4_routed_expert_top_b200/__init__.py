@@ -39,6 +39,7 @@ EXPORTS = (
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
     "coli_moe_forward_noalloc", "coli_moe_status", "coli_moe_host_workspace_size",
     "coli_moe_forward_host", "coli_moe_stack_host_workspace_size", "coli_moe_stack_forward_host",
+    "coli_moe_quantize_expert_fp8_device",
 )
 
 
@@ -73,6 +74,8 @@ _SIGS = {
     "coli_moe_expert_bytes": ([_I32, _I32, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
     "coli_moe_pack_expert": ([_I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "coli_moe_quantize_expert_device": ([_I32, _I32, _I32, _P, _P, _P, _P, _P], ctypes.c_int),
+    "coli_moe_quantize_expert_fp8_device": ([_I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P],
+                                            ctypes.c_int),
     "coli_moe_layer_create": ([ctypes.POINTER(Desc), ctypes.POINTER(_P)], ctypes.c_int),
     "coli_moe_layer_destroy": ([_P], ctypes.c_int),
     "coli_moe_workspace_size": ([_P, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
@@ -169,6 +172,14 @@ def coli_moe_pack_expert(H, I, group, gate_codes, gate_scales, up_codes, up_scal
 def coli_moe_quantize_expert_device(H, I, group, gate, up, down, blob, stream=None):
     _ok(lib.coli_moe_quantize_expert_device(H, I, group, _ptr(gate), _ptr(up), _ptr(down),
                                             _ptr(blob), _stream(stream)))
+
+
+def coli_moe_quantize_expert_fp8_device(H, I, group, gate, up, down, gate_bs, up_bs, down_bs,
+                                        blob, stream=None):
+    """FP8 E4M3 codes (uint8 device tensors) with 128 x 128 block scales -> int4 blob."""
+    _ok(lib.coli_moe_quantize_expert_fp8_device(H, I, group, _ptr(gate), _ptr(up), _ptr(down),
+                                                _ptr(gate_bs), _ptr(up_bs), _ptr(down_bs),
+                                                _ptr(blob), _stream(stream)))
 
 
 def coli_moe_layer_create(desc: Desc) -> ctypes.c_void_p:

@@ -609,11 +609,35 @@ int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group, const f
     for (int m = 0; m < 3; ++m) {
         const int R = L.rows[m], K = L.cols[m];
         const int smem = 16 * (K / 2);
-        int rc = set_smem((const void*)quantize_rows_kernel, smem);
+        int rc = set_smem((const void*)quantize_rows_kernel<QzF32>, smem);
         if (rc) return rc;
         quantize_rows_kernel<<<R / 16, 256, smem, S(stream)>>>(
-            src[m], R, K, group, b + L.codes[m], reinterpret_cast<float*>(b + L.scales[m]));
+            QzF32{src[m]}, R, K, group, b + L.codes[m], reinterpret_cast<float*>(b + L.scales[m]));
         if ((rc = check_launch("quantize_rows"))) return rc;
+    }
+    return COLI_OK;
+}
+
+int coli_moe_quantize_expert_fp8_device(int32_t H, int32_t I, int32_t group, const uint8_t* gate,
+                                        const uint8_t* up, const uint8_t* down, const float* gate_bs,
+                                        const float* up_bs, const float* down_bs, void* blob,
+                                        coli_stream_t stream) {
+    if (!gate || !up || !down || !gate_bs || !up_bs || !down_bs || !blob)
+        return fail(COLI_E_INVAL, "quantize_expert_fp8_device: NULL pointer");
+    if (!shape_ok(H, I, group)) return fail(COLI_E_INVAL, "quantize_expert_fp8_device: bad shape");
+    const BlobLayout L = make_blob_layout(H, I, group);
+    uint8_t* b = static_cast<uint8_t*>(blob);
+    const uint8_t* src[3] = {gate, up, down};
+    const float* bsrc[3] = {gate_bs, up_bs, down_bs};
+    for (int m = 0; m < 3; ++m) {
+        const int R = L.rows[m], K = L.cols[m];
+        const int smem = 16 * (K / 2);
+        int rc = set_smem((const void*)quantize_rows_kernel<QzFp8Block>, smem);
+        if (rc) return rc;
+        quantize_rows_kernel<<<R / 16, 256, smem, S(stream)>>>(
+            QzFp8Block{src[m], bsrc[m], (K + 127) / 128}, R, K, group, b + L.codes[m],
+            reinterpret_cast<float*>(b + L.scales[m]));
+        if ((rc = check_launch("quantize_rows_fp8"))) return rc;
     }
     return COLI_OK;
 }

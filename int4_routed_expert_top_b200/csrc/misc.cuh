@@ -7,6 +7,8 @@
 // straight into the tiled device layout.
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 
 namespace coli {
@@ -18,11 +20,31 @@ __device__ __forceinline__ int quant_one(float v, float s) {
     return (int)q;
 }
 
+// Row sources of the device quantiser: f32 masters, or FP8 E4M3 codes with one
+// f32 scale per 128 x 128 block (the checkpoint the container is converted
+// from: "解密GLM-5.2-colibri-int4-with-int8-mtp", quantisation-config
+// paragraph, fmt e4m3 with weight_block_size [128, 128]).  The E4M3 value is
+// exact in half and f32; the block scale is applied by one f32 multiply.
+struct QzF32 {
+    const float* w;
+    __device__ __forceinline__ float at(int64_t r, int c, int K) const { return w[r * K + c]; }
+};
+struct QzFp8Block {
+    const uint8_t* q;   // [R, K] E4M3 codes
+    const float* bs;    // [ceil(R/128), ceil(K/128)] block scales
+    int kb;             // ceil(K / 128)
+    __device__ __forceinline__ float at(int64_t r, int c, int K) const {
+        const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)q[r * K + c], __NV_E4M3);
+        return __fmul_rn(__half2float(__half(h)), bs[(r / 128) * kb + c / 128]);
+    }
+};
+
 // One CTA per 16-row block of a 128-row tile.  Each warp quantises two rows
 // into shared memory in container byte order, then every thread assembles
 // 16-byte fragment-tile units (see common.cuh) and stores them.
+template <typename Src>
 __global__ void __launch_bounds__(256)
-quantize_rows_kernel(const float* __restrict__ w, int R, int K, int group,
+quantize_rows_kernel(Src src, int R, int K, int group,
                      uint8_t* __restrict__ codes, float* __restrict__ scales) {
     extern __shared__ uint4 qz_smem[];
     uint8_t* rows = reinterpret_cast<uint8_t*>(qz_smem);  // [16][K/2]
@@ -33,17 +55,16 @@ quantize_rows_kernel(const float* __restrict__ w, int R, int K, int group,
     const int ng = K / gs;
     for (int lr = warp; lr < 16; lr += 8) {
         const int r = blk * 16 + lr;
-        const float* row = w + (int64_t)r * K;
         uint8_t* buf = rows + (int64_t)lr * (K / 2);
         for (int g = 0; g < ng; ++g) {
             float m = 0.0f;
-            for (int c = g * gs + lane; c < (g + 1) * gs; c += 32) m = fmaxf(m, fabsf(row[c]));
+            for (int c = g * gs + lane; c < (g + 1) * gs; c += 32) m = fmaxf(m, fabsf(src.at(r, c, K)));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             const float s = __fdiv_rn(m, 7.0f);
             if (lane == 0) scales[scale_offset(r, g, ng)] = s;
             for (int cp = g * gs / 2 + lane; cp < (g + 1) * gs / 2; cp += 32) {
-                const int q0 = quant_one(row[2 * cp], s), q1 = quant_one(row[2 * cp + 1], s);
+                const int q0 = quant_one(src.at(r, 2 * cp, K), s), q1 = quant_one(src.at(r, 2 * cp + 1, K), s);
                 buf[cp] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
             }
         }

@@ -62,6 +62,34 @@ def test_device_quantizer_matches_host_packer(group, shape):
 
 
 @pytest.mark.parametrize("group", [0, 64])
+@pytest.mark.parametrize("shape", [(256, 128), (6144, 2048)])
+def test_fp8_block_requantisation_matches_host(group, shape):
+    """FP8 E4M3 experts with 128 x 128 block scales -> int4 container on the
+    device, byte for byte what the oracle's FP8 decode followed by the host
+    quantiser and packer give."""
+    H, I = shape
+    rng = np.random.default_rng(11 + group)
+
+    def fp8(R, K):
+        codes = rng.integers(0, 256, (R, K), dtype=np.uint8)
+        codes[(codes & 0x7F) == 0x7F] = 0x3C              # finite codes only
+        bs = rng.uniform(1e-4, 4e-4, ((R + 127) // 128, (K + 127) // 128)).astype(np.float32)
+        return codes, bs
+
+    mats = [fp8(I, H), fp8(I, H), fp8(H, I)]
+    cont = []
+    for codes, bs in mats:
+        cont += list(oracle.quantize(oracle.fp8_block_dequant(codes, bs), group))
+    host = cm.coli_moe_pack_expert(H, I, group, *cont)
+    dev = [(torch.from_numpy(c).cuda(), torch.from_numpy(b).cuda()) for c, b in mats]
+    blob = torch.empty(cm.coli_moe_expert_bytes(H, I, group), dtype=torch.uint8, device="cuda")
+    cm.coli_moe_quantize_expert_fp8_device(H, I, group, dev[0][0], dev[1][0], dev[2][0],
+                                           dev[0][1], dev[1][1], dev[2][1], blob)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(blob.cpu().numpy(), host)
+
+
+@pytest.mark.parametrize("group", [0, 64])
 def test_dequant_bit_exact(group):
     wl = dataclasses.replace(synth.TINY, group=group)
     L = build_layer(wl)
