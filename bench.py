@@ -187,6 +187,22 @@ class OracleSampler:
         return time.perf_counter() - t0
 
 
+def host_cpu():
+    """The host the CPU baseline ran on: logical CPUs, the ones this process may
+    use, and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    aff = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else None
+    return {"nproc": os.cpu_count(), "affinity": aff, "cpu_model": model}
+
+
 def oracle_sample(wl, budget_s=12.0):
     smp = OracleSampler(wl)
     spent, n = 0.0, 0
@@ -221,7 +237,7 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "tokens_per_step": 1},
             "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "host": host_cpu()},
             "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -504,7 +520,8 @@ def main():
             "value": tok_s, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} tokens of {wl.name} through the oracle ({secs:.1f} s): router over "
                       f"all {wl.E} experts, dequantisation of the {wl.k}+{wl.n_shared} experts "
-                      f"each token uses, SwiGLU, combine; single-threaded (one token)"}
+                      f"each token uses, SwiGLU, combine; single-threaded (one token)",
+            "host": host_cpu()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     for l in layers:
