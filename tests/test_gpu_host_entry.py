@@ -97,3 +97,36 @@ def test_forward_host_rejects_a_short_workspace():
     with pytest.raises(cm.ColiError) as ei:
         cm.coli_moe_forward_host(L.handle, xh, T, yh, short)
     assert ei.value.code == -5      # COLI_E_WORKSPACE
+
+
+@pytest.mark.parametrize("path", ["fused", "gemm"])
+def test_forward_host_pageable_buffers_use_plain_copies(path):
+    """Unpinned host memory is not mapped into the device: the call copies
+    through cudaMemcpyAsync instead, with the same result."""
+    wl = dataclasses.replace(synth.TINY, group=64)
+    L = build_layer(wl)
+    T = 1 if path == "fused" else 24
+    x = torch.randn((T, wl.H))
+    y = torch.empty((T, wl.H), dtype=torch.float32)
+    assert not x.is_pinned() and not y.is_pinned()
+    cm.coli_moe_forward_host(L.handle, x, T, y, host_ws(L, T), path=PATHS[path])
+    torch.cuda.synchronize()
+    ref = device_forward(L, x.cuda(), T, PATHS[path])
+    np.testing.assert_array_equal(y.numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def test_forward_host_misaligned_output_is_staged():
+    """y_host 4 bytes past a 16-byte boundary: the tensor-core path's 16-byte
+    stores cannot target it, so y is staged on the device and copied back."""
+    wl = dataclasses.replace(synth.TINY, group=64)
+    L = build_layer(wl)
+    T = 24
+    x = torch.randn((T, wl.H)).pin_memory()
+    big = torch.zeros((T * wl.H + 4,), dtype=torch.float32).pin_memory()
+    y = big[1:1 + T * wl.H].view(T, wl.H)
+    assert y.data_ptr() % 16 == 4
+    cm.coli_moe_forward_host(L.handle, x, T, y, host_ws(L, T), path=cm.COLI_PATH_GEMM)
+    torch.cuda.synchronize()
+    ref = device_forward(L, x.cuda(), T, cm.COLI_PATH_GEMM)
+    np.testing.assert_array_equal(y.numpy().view(np.uint32), ref.view(np.uint32))
+    assert big[0].item() == 0.0 and big[-3:].abs().sum().item() == 0.0   # nothing outside y
