@@ -67,3 +67,18 @@ def test_reference_arm_runs_on_rank_zero_only():
                        cwd=ROOT, env=env, capture_output=True, timeout=300)
     assert r.returncode == 0, r.stderr.decode()[-500:]
     assert r.stdout.strip() == b""
+
+
+def test_profiled_traffic_only_while_the_kernel_source_matches():
+    """The roofline's traffic comes from the committed ncu summary only while
+    the kernel source still has the hash that summary names."""
+    sys.path.insert(0, ROOT)
+    import bench
+    t = bench.profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
+                               "moe_fused_kernel_glm_decode.md")
+    assert t is not None and t > 170e6                 # at least the algorithmic bytes
+    # another source file has another hash: no traffic
+    assert bench.profiled_traffic("int4_routed_expert_top_b200/csrc/gemm.cuh",
+                                  "moe_fused_kernel_glm_decode.md") is None
+    assert bench.profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
+                                  "no_such_profile.md") is None
