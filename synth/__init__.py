@@ -95,7 +95,7 @@ def normal(seed, layer, tensor, expert, rows, cols, device="cpu", first=0):
 
 
 # ---------------------------------------------------------------------------
-# Workloads (the layer shapes and input recipes; see the design doc for sources)
+# Workloads (the layer shapes and input recipes of the GLM-5.2-shaped layer)
 # ---------------------------------------------------------------------------
 
 @dataclass(frozen=True)
