@@ -52,6 +52,8 @@ def lib():
                                         P, P, P, P, P, P, P, P]
         L.orc_rmsnorm.argtypes = [P, i64, i64, ctypes.c_double, P]
         L.orc_fp8_block_dequant.argtypes = [P, P, i64, i64, P]
+        L.orc_topp_keep.argtypes = [P, P, i64, ctypes.c_double, P]
+        L.orc_topp_keep.restype = i64
         for f in ("orc_quantize", "orc_dequantize", "orc_route", "orc_union",
                   "orc_expert", "orc_token_forward", "orc_layer_forward",
                   "orc_rmsnorm", "orc_fp8_block_dequant"):
@@ -92,6 +94,23 @@ def fp8_block_dequant(codes, block_scales):
     _check(lib().orc_fp8_block_dequant(pq, pb, rows, cols, out.ctypes.data_as(ctypes.c_void_p)),
            "fp8_block_dequant")
     return out
+
+
+def topp_keep(w, idx, p: float):
+    """Adaptive expert top-p: w, idx [T, k] (routing weights, experts, pick
+    order) -> keep [T, k] int32 (1 kept) and the number kept per token."""
+    w, pw = _c(np.atleast_2d(w), np.float32)
+    idx, pi = _c(np.atleast_2d(idx), np.int32)
+    T, k = w.shape
+    keep = np.zeros((T, k), np.int32)
+    n = np.zeros(T, np.int64)
+    for t in range(T):
+        r = lib().orc_topp_keep(w[t].ctypes.data_as(ctypes.c_void_p),
+                                idx[t].ctypes.data_as(ctypes.c_void_p), k, float(p),
+                                keep[t].ctypes.data_as(ctypes.c_void_p))
+        _check(0 if r >= 1 else -1, "topp_keep")
+        n[t] = r
+    return keep, n
 
 
 def dequantize(packed, scales, cols: int, group: int):

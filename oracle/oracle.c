@@ -66,6 +66,35 @@ int orc_quantize(const float* w, int64_t rows, int64_t cols, int32_t group,
     return 0;
 }
 
+/* Adaptive expert top-p of one token ("colibrì 實戰指南" 三 and 五: --topp p reads
+ * 30-40% fewer expert bytes per token; the rule itself is not given): order the
+ * token's k picks by renormalised weight w_j / sum(w), largest first, equal
+ * weights to the lower expert index, and keep the shortest prefix of that order
+ * whose weights add up to at least p (in double).  Kept picks keep their
+ * weights; the others contribute nothing.  keep[j] = 1 for a kept pick j (pick
+ * order), else 0; returns the number kept (k when p >= the total). */
+int64_t orc_topp_keep(const float* w, const int32_t* idx, int64_t k, double p, int32_t* keep) {
+    if (!w || !idx || !keep || k < 1) return -1;
+    double tot = 0.0;
+    for (int64_t j = 0; j < k; ++j) {
+        tot += (double)w[j];
+        keep[j] = 0;
+    }
+    int64_t kept = 0;
+    double mass = 0.0;
+    while (kept < k && (kept == 0 || mass < p)) {
+        int64_t best = -1;   /* largest weight not yet kept, then lower expert index */
+        for (int64_t j = 0; j < k; ++j) {
+            if (keep[j]) continue;
+            if (best < 0 || w[j] > w[best] || (w[j] == w[best] && idx[j] < idx[best])) best = j;
+        }
+        keep[best] = 1;
+        mass += tot > 0.0 ? (double)w[best] / tot : 0.0;
+        ++kept;
+    }
+    return kept;
+}
+
 /* FP8 E4M3 code as a float, from the format's definition: sign bit, four
  * exponent bits with bias 7, three mantissa bits; exponent 0 holds the
  * subnormals m/8 * 2^-6; S.1111.111 is NaN and there are no infinities.

@@ -94,6 +94,12 @@ int orc_layer_forward(const float* x, int64_t T, int64_t H, int64_t I,
 /* RMSNorm with unit gain: out = v / sqrt(mean(v^2) + eps), per row of [T, H]. */
 int orc_rmsnorm(const float* x, int64_t T, int64_t H, double eps, float* out);
 
+/* Adaptive expert top-p of one token: of its k picks (weights w, experts idx,
+ * pick order), keep the shortest run of the largest renormalised weights
+ * (w_j / sum w; equal weights to the lower expert index) whose total reaches p.
+ * keep[j] = 1 for kept picks.  Returns the number kept, or -1 on bad arguments. */
+int64_t orc_topp_keep(const float* w, const int32_t* idx, int64_t k, double p, int32_t* keep);
+
 /* FP8 (E4M3) matrix with one f32 scale per 128 x 128 block -> f32:
  * out[r, c] = e4m3(q[r, c]) * bs[r / 128, c / 128] (bs row-major
  * [ceil(rows/128), ceil(cols/128)]).  Returns 0, or -1 on bad arguments. */

@@ -345,3 +345,51 @@ def test_fp8_block_scales_cover_ragged_blocks():
     # the block edges: row 127 uses block row 0, row 128 block row 1
     assert got[127, 0] == np.float32(vals[127, 0] * bs[0, 0])
     assert got[128, 259] == np.float32(vals[128, 259] * bs[1, 2])
+
+
+# ---------------------------------------------------------------------------
+# adaptive expert top-p (a NEXT row: oracle first)
+# ---------------------------------------------------------------------------
+
+def test_topp_hand_examples():
+    # dyadic weights: every sum below is exact, so p on a boundary is kept exactly
+    w = np.array([[0.5, 0.375, 0.125]], np.float32)
+    idx = np.array([[4, 2, 9]], np.int32)
+    for p, want in [(0.7, [1, 1, 0]), (0.5, [1, 0, 0]), (0.9, [1, 1, 1]), (1.0, [1, 1, 1]),
+                    (0.875, [1, 1, 0]), (0.0, [1, 0, 0])]:   # at least one pick is kept
+        keep, n = oracle.topp_keep(w, idx, p)
+        assert keep[0].tolist() == want, (p, keep)
+        assert n[0] == sum(want)
+    # the order is by weight, not by pick position (the bias changes the selection)
+    keep, _ = oracle.topp_keep(np.array([[0.125, 0.5, 0.375]], np.float32),
+                               np.array([[1, 2, 3]], np.int32), 0.7)
+    assert keep[0].tolist() == [0, 1, 1]
+    # equal weights go to the lower expert index
+    keep, _ = oracle.topp_keep(np.full((1, 4), 0.25, np.float32),
+                               np.array([[7, 3, 9, 1]], np.int32), 0.5)
+    assert keep[0].tolist() == [0, 1, 0, 1]
+    # unnormalised weights: the mass is of the renormalised ones (0.5, 0.25, 0.25)
+    keep, _ = oracle.topp_keep(np.array([[1.0, 0.5, 0.5]], np.float32),
+                               np.array([[0, 2, 1]], np.int32), 0.75)
+    assert keep[0].tolist() == [1, 0, 1]
+
+
+def test_topp_is_the_smallest_set_reaching_p_by_brute_force():
+    import itertools
+    rng = np.random.default_rng(9)
+    k = 6
+    for trial in range(300):
+        w = rng.dirichlet(np.ones(k)).astype(np.float32)
+        idx = rng.permutation(64)[:k].astype(np.int32)
+        p = float(rng.uniform(0.05, 1.0))
+        keep, n = oracle.topp_keep(w[None], idx[None], p)
+        wn = w.astype(np.float64) / w.astype(np.float64).sum()
+        kept = keep[0].astype(bool)
+        # no smaller subset reaches p, and the kept one does (or is everything)
+        best = min((r for r in range(1, k + 1)
+                    if any(wn[list(c)].sum() >= p for c in itertools.combinations(range(k), r))),
+                   default=k)
+        assert n[0] == best, (w, p, keep)
+        assert wn[kept].sum() >= p or n[0] == k
+        # the kept picks are the largest weights
+        assert wn[kept].min() >= wn[~kept].max(initial=-1.0)
