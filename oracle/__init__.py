@@ -53,10 +53,12 @@ def lib():
         L.orc_rmsnorm.argtypes = [P, i64, i64, ctypes.c_double, P]
         L.orc_fp8_block_dequant.argtypes = [P, P, i64, i64, P]
         L.orc_topp_keep.argtypes = [P, P, i64, ctypes.c_double, P]
+        L.orc_quantize8.argtypes = [P, i64, i64, ctypes.c_int32, P, P]
+        L.orc_dequantize8.argtypes = [P, P, i64, i64, ctypes.c_int32, P]
         L.orc_topp_keep.restype = i64
         for f in ("orc_quantize", "orc_dequantize", "orc_route", "orc_union",
                   "orc_expert", "orc_token_forward", "orc_layer_forward",
-                  "orc_rmsnorm", "orc_fp8_block_dequant"):
+                  "orc_rmsnorm", "orc_fp8_block_dequant", "orc_quantize8", "orc_dequantize8"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -93,6 +95,28 @@ def fp8_block_dequant(codes, block_scales):
     out = np.zeros((rows, cols), np.float32)
     _check(lib().orc_fp8_block_dequant(pq, pb, rows, cols, out.ctypes.data_as(ctypes.c_void_p)),
            "fp8_block_dequant")
+    return out
+
+
+def quantize8(w, group: int):
+    """8-bit container: signed byte codes [R, K] and f32 scales [R, K/G]."""
+    w, pw = _c(w, np.float32)
+    rows, cols = w.shape
+    ng = 1 if group == 0 else cols // group
+    codes = np.zeros((rows, cols), np.int8)
+    scales = np.zeros((rows, ng), np.float32)
+    _check(lib().orc_quantize8(pw, rows, cols, group, codes.ctypes.data_as(ctypes.c_void_p),
+                               scales.ctypes.data_as(ctypes.c_void_p)), "quantize8")
+    return codes, scales
+
+
+def dequantize8(codes, scales, group: int):
+    codes, pc = _c(codes, np.int8)
+    scales, ps = _c(scales, np.float32)
+    rows, cols = codes.shape
+    out = np.zeros((rows, cols), np.float32)
+    _check(lib().orc_dequantize8(pc, ps, rows, cols, group, out.ctypes.data_as(ctypes.c_void_p)),
+           "dequantize8")
     return out
 
 

@@ -66,6 +66,56 @@ int orc_quantize(const float* w, int64_t rows, int64_t cols, int32_t group,
     return 0;
 }
 
+/* 8-bit variant of the container (the int8 MTP head: "解密GLM-5.2-colibri-int4-
+ * with-int8-mtp", whose MTP head keeps 8-bit precision; the converter's
+ * --io-bits 8, "GLM-5.2-colibri-int4专家流技术详解" project-source section).
+ * The pages give no further rule; this follows the int4 container's: per row
+ * or per 64 columns s = max|w| / 127 (f32 division), q = rint(w / s) (f32
+ * division, half to even) in [-127, 127], one signed byte per weight. */
+int orc_quantize8(const float* w, int64_t rows, int64_t cols, int32_t group, int8_t* codes,
+                  float* scales) {
+    if (!w || !codes || !scales || rows < 0 || cols <= 0 || (group != 0 && group != 64) ||
+        (group && cols % group))
+        return -1;
+    const int64_t gsz = group == 0 ? cols : group;
+    const int64_t ng = cols / gsz;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* row = w + r * cols;
+        for (int64_t g = 0; g < ng; ++g) {
+            float m = 0.0f;
+            for (int64_t c = g * gsz; c < (g + 1) * gsz; ++c) {
+                const float a = fabsf(row[c]);
+                if (a > m) m = a;
+            }
+            const float s = m / 127.0f;
+            scales[r * ng + g] = s;
+            for (int64_t c = g * gsz; c < (g + 1) * gsz; ++c) {
+                int q = 0;
+                if (s != 0.0f) {
+                    float qf = rintf(row[c] / s);
+                    if (qf > 127.0f) qf = 127.0f;       /* guard only */
+                    if (qf < -127.0f) qf = -127.0f;
+                    q = (int)qf;
+                }
+                codes[r * cols + c] = (int8_t)q;
+            }
+        }
+    }
+    return 0;
+}
+
+int orc_dequantize8(const int8_t* codes, const float* scales, int64_t rows, int64_t cols,
+                    int32_t group, float* out) {
+    if (!codes || !scales || !out || rows < 0 || cols <= 0 || (group != 0 && group != 64) ||
+        (group && cols % group))
+        return -1;
+    const int64_t gsz = group == 0 ? cols : group, ng = cols / gsz;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = (float)codes[r * cols + c] * scales[r * ng + c / gsz];
+    return 0;
+}
+
 /* Adaptive expert top-p of one token ("colibrì 實戰指南" 三 and 五: --topp p reads
  * 30-40% fewer expert bytes per token; the rule itself is not given): order the
  * token's k picks by renormalised weight w_j / sum(w), largest first, equal

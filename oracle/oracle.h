@@ -94,6 +94,14 @@ int orc_layer_forward(const float* x, int64_t T, int64_t H, int64_t I,
 /* RMSNorm with unit gain: out = v / sqrt(mean(v^2) + eps), per row of [T, H]. */
 int orc_rmsnorm(const float* x, int64_t T, int64_t H, double eps, float* out);
 
+/* 8-bit variant of the container: codes[r, c] one signed byte in [-127, 127],
+ * scales[r, g] = max|w| / 127 per row (group 0) or per 64 columns; q = rint(w/s).
+ * dequantize8 writes (float)q * s.  Return 0, or -1 on bad arguments. */
+int orc_quantize8(const float* w, int64_t rows, int64_t cols, int32_t group, int8_t* codes,
+                  float* scales);
+int orc_dequantize8(const int8_t* codes, const float* scales, int64_t rows, int64_t cols,
+                    int32_t group, float* out);
+
 /* Adaptive expert top-p of one token: of its k picks (weights w, experts idx,
  * pick order), keep the shortest run of the largest renormalised weights
  * (w_j / sum w; equal weights to the lower expert index) whose total reaches p.

@@ -393,3 +393,54 @@ def test_topp_is_the_smallest_set_reaching_p_by_brute_force():
         assert wn[kept].sum() >= p or n[0] == k
         # the kept picks are the largest weights
         assert wn[kept].min() >= wn[~kept].max(initial=-1.0)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit variant of the container (a NEXT row: oracle first)
+# ---------------------------------------------------------------------------
+
+def test_quant8_hand_row_half_to_even():
+    # max 127/128 gives s = 1/128 exactly; w/s lands on halves: 2.5 -> 2, 3.5 -> 4
+    row = np.array([[127 / 128, 2.5 / 128, 3.5 / 128, -0.5 / 128, -1.5 / 128, 0.0]], np.float32)
+    codes, scales = oracle.quantize8(row, 0)
+    assert codes[0].tolist() == [127, 2, 4, 0, -2, 0]
+    assert scales[0, 0] == np.float32(1 / 128)
+    z, zs = oracle.quantize8(np.zeros((1, 64), np.float32), 64)      # zero group: s = 0, q = 0
+    assert not z.any() and zs[0, 0] == 0.0
+
+
+@pytest.mark.parametrize("group", [0, 64])
+def test_quant8_roundtrip_and_error_bound(group):
+    rng = np.random.default_rng(21 + group)
+    R, K = 16, 256
+    gs = K if group == 0 else group
+    # codes with +-127 in every group and a power-of-two scale: w = q s is a fixed point
+    q = rng.integers(-127, 128, (R, K))
+    q[:, ::gs] = 127 * rng.choice([-1, 1], (R, K // gs))
+    s = (2.0 ** -rng.integers(4, 12, (R, K // gs))).astype(np.float32)
+    w = (q * np.repeat(s, gs, 1)).astype(np.float32)
+    codes, scales = oracle.quantize8(w, group)
+    np.testing.assert_array_equal(codes, q)
+    np.testing.assert_array_equal(scales, s)
+    np.testing.assert_array_equal(oracle.dequantize8(codes, scales, group), w)
+    # random weights: error within half a step, every code in range
+    w2 = (rng.standard_normal((R, K)) * 0.02).astype(np.float32)
+    c2, s2 = oracle.quantize8(w2, group)
+    err = np.abs(oracle.dequantize8(c2, s2, group) - w2)
+    assert (err <= np.repeat(s2, gs, 1) / 2 * (1 + 1e-6)).all()
+    assert np.abs(c2).max() == 127 and c2.min() >= -127
+
+
+def test_quant8_groups_reduce_to_per_row_and_reject_bad_shapes():
+    rng = np.random.default_rng(3)
+    w = (rng.standard_normal((4, 128)) * 0.02).astype(np.float32)
+    w[:, 0] = 0.1                       # both 64-column groups share the row maximum
+    w[:, 64] = -0.1
+    c0, s0 = oracle.quantize8(w, 0)
+    c64, s64 = oracle.quantize8(w, 64)
+    np.testing.assert_array_equal(c0, c64)
+    np.testing.assert_array_equal(np.repeat(s0, 2, 1), s64)
+    with pytest.raises(RuntimeError):
+        oracle.quantize8(np.zeros((2, 96), np.float32), 64)          # 96 not a multiple of 64
+    with pytest.raises(RuntimeError):
+        oracle.quantize8(np.zeros((2, 64), np.float32), 32)          # group 32 not supported
