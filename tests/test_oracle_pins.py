@@ -444,3 +444,22 @@ def test_quant8_groups_reduce_to_per_row_and_reject_bad_shapes():
         oracle.quantize8(np.zeros((2, 96), np.float32), 64)          # 96 not a multiple of 64
     with pytest.raises(RuntimeError):
         oracle.quantize8(np.zeros((2, 64), np.float32), 32)          # group 32 not supported
+
+
+# ---------------------------------------------------------------------------
+# input recipe: the Zipf-skewed prefill router
+# ---------------------------------------------------------------------------
+
+def test_prefill_zipf_bias_gives_the_stated_load():
+    """The stored bias amplitude routes the prefill workload's own seeded tokens
+    so that the busiest expert takes about 100 of the 512 x 8 picks (+-5); the
+    least popular ones take a handful (5 with this seed)."""
+    import synth
+    wl = synth.GLM_PREFILL
+    wr, b = synth.router(wl, 0)
+    x = synth.tokens(wl, wl.T).numpy()
+    idx, _, _ = oracle.route(x, wr.numpy(), b.numpy(), wl.k)
+    load = np.bincount(idx.reshape(-1), minlength=wl.E)
+    assert 95 <= load.max() <= 105, load.max()
+    assert load.min() <= 8
+    assert load.sum() == wl.T * wl.k
