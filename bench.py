@@ -227,13 +227,17 @@ def run_reference(args):
         secs = smp.step()
         if i >= args.warmup:
             per_step.append(secs)
-    tok_s = len(per_step) / sum(per_step)
+    tok_s = len(per_step) / sum(per_step) / wl.layers
     sample = (f"{len(per_step)} timed steps of 1 token each (router over all {wl.E} experts, "
               f"dequantisation of the {wl.k}+{wl.n_shared} expert matrices it uses, SwiGLU, "
               f"combine) of workload {wl.name}")
+    if wl.layers > 1:
+        sample += (f"; one layer per step, the rate divided by the {wl.layers} layers of the "
+                   f"stack (every layer has the same shapes)")
     line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT,
             "n_gpus": args.gpus, "steps": len(per_step), "warmup": args.warmup,
-            "ms_per_step": 1e3 * sum(per_step) / len(per_step), "higher_is_better": True,
+            "ms_per_step": 1e3 * sum(per_step) / len(per_step) * wl.layers,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "tokens_per_step": 1},
             "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -516,11 +520,13 @@ def main():
                    "d2h_bytes_per_step": int(T * wl.H * 4)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tok_s, n, secs = oracle_sample(wl)
+        stack = (f"; one layer per token, the rate divided by the {wl.layers} layers of the "
+                 f"stack (every layer has the same shapes)" if wl.layers > 1 else "")
         line["cpu_baseline"] = {
-            "value": tok_s, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "value": tok_s / wl.layers, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} tokens of {wl.name} through the oracle ({secs:.1f} s): router over "
                       f"all {wl.E} experts, dequantisation of the {wl.k}+{wl.n_shared} experts "
-                      f"each token uses, SwiGLU, combine; single-threaded (one token)",
+                      f"each token uses, SwiGLU, combine; single-threaded (one token){stack}",
             "host": host_cpu()}
     if rank == 0:
         print(json.dumps(line), flush=True)
