@@ -511,8 +511,8 @@ def main():
         line["int4_weight_frac_of_hbm"] = weight_gbs / hbm_gbs
         line["unique_experts_per_step"] = float(uniq.mean())
         line["gpu_launches"] = (3 if fused else (4 if T < 48 else 9)) * K
-    else:
-        line["gpu_launches"] = 7 * wl.layers * K
+    else:   # per layer: the RMSNorm, then the path's own launches
+        line["gpu_launches"] = (1 + (3 if fused else (4 if T < 48 else 9))) * wl.layers * K
     line["config"] = cfg
     line["clocks"] = clocks.summary()
     line["e2e"] = {"value": e2e_value, "unit": UNIT,
