@@ -138,6 +138,35 @@ int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group,
                                     const float* down, void* blob,
                                     coli_stream_t stream);
 
+/* 8-bit weights (the engine keeps its MTP head at 8 bits): the container's
+ * rule with 127 in place of 7 - per row (group 0) or per 64 columns
+ * s = max|w| / 127 (f32 division), q = rint(w / s) in [-127, 127] (f32
+ * division, half to even), s == 0 gives q = 0.  Host pointers: w and codes
+ * [rows*cols] (one signed byte per weight, row-major), scales [rows*cols/G].
+ * Errors: COLI_E_INVAL as for coli_moe_quantize. */
+int coli_moe_quantize8(const float* w, int64_t rows, int64_t cols, int32_t group,
+                       int8_t* codes, float* scales);
+
+/* Blob of one expert with 8-bit codes: codes_gate, codes_up, codes_down (each
+ * R*K bytes), then the three scale sections as in the 4-bit blob, every
+ * section on a 256-byte boundary.  Codes in 8-bit fragment tiles: blocks of 16
+ * rows x 64 columns ordered [R/128][K/64][8][32 lanes]; lane l of block b in
+ * row tile T and 64-column step s (g = l / 4, u = l % 4) holds 32 bytes: for
+ * each 32-column half h, four words i = 0..3 - i = 0: row r0 = 128T + 16b + g,
+ * columns 64s + 32h + 4u .. +3; i = 1: row r0 + 8, same columns; i = 2: row
+ * r0, columns 64s + 32h + 16 + 4u .. +3; i = 3: row r0 + 8, those columns -
+ * byte j of a word being its first column + j (the lane's mma.sync m16n8k32
+ * s8 A registers).  coli_moe_pack_expert8
+ * re-tiles host codes and scales (as written by coli_moe_quantize8) into a
+ * host blob of coli_moe_expert_bytes8 bytes.  The expert kernels do not read
+ * 8-bit blobs yet. */
+int coli_moe_expert_bytes8(int32_t H, int32_t I, int32_t group, size_t* bytes);
+int coli_moe_pack_expert8(int32_t H, int32_t I, int32_t group,
+                          const int8_t* gate_codes, const float* gate_scales,
+                          const int8_t* up_codes, const float* up_scales,
+                          const int8_t* down_codes, const float* down_scales,
+                          void* blob);
+
 /* coli_moe_quantize_expert_device for an expert given as FP8 E4M3 codes with
  * one f32 scale per 128 x 128 block (the format of the checkpoint the int4
  * container is converted from): every weight becomes

@@ -39,7 +39,8 @@ EXPORTS = (
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
     "coli_moe_forward_noalloc", "coli_moe_status", "coli_moe_host_workspace_size",
     "coli_moe_forward_host", "coli_moe_stack_host_workspace_size", "coli_moe_stack_forward_host",
-    "coli_moe_quantize_expert_fp8_device",
+    "coli_moe_quantize_expert_fp8_device", "coli_moe_quantize8", "coli_moe_expert_bytes8",
+    "coli_moe_pack_expert8",
 )
 
 
@@ -76,6 +77,9 @@ _SIGS = {
     "coli_moe_quantize_expert_device": ([_I32, _I32, _I32, _P, _P, _P, _P, _P], ctypes.c_int),
     "coli_moe_quantize_expert_fp8_device": ([_I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P],
                                             ctypes.c_int),
+    "coli_moe_quantize8": ([_P, _I64, _I64, _I32, _P, _P], ctypes.c_int),
+    "coli_moe_expert_bytes8": ([_I32, _I32, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "coli_moe_pack_expert8": ([_I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "coli_moe_layer_create": ([ctypes.POINTER(Desc), ctypes.POINTER(_P)], ctypes.c_int),
     "coli_moe_layer_destroy": ([_P], ctypes.c_int),
     "coli_moe_workspace_size": ([_P, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
@@ -166,6 +170,32 @@ def coli_moe_pack_expert(H, I, group, gate_codes, gate_scales, up_codes, up_scal
     arrs = [np.ascontiguousarray(a) for a in
             (gate_codes, gate_scales, up_codes, up_scales, down_codes, down_scales)]
     _ok(lib.coli_moe_pack_expert(H, I, group, *[_ptr(a) for a in arrs], _ptr(blob)))
+    return blob
+
+
+def coli_moe_quantize8(w: np.ndarray, group: int):
+    """Host 8-bit quantiser -> (codes int8 [R, K], scales f32 [R, K/G])."""
+    w = np.ascontiguousarray(w, np.float32)
+    R, K = w.shape
+    ng = 1 if group == 0 else max(K // group, 1)
+    codes = np.zeros((R, K), np.int8)
+    scales = np.zeros((R, ng), np.float32)
+    _ok(lib.coli_moe_quantize8(_ptr(w), R, K, group, _ptr(codes), _ptr(scales)))
+    return codes, scales
+
+
+def coli_moe_expert_bytes8(H: int, I: int, group: int) -> int:
+    out = _SZ()
+    _ok(lib.coli_moe_expert_bytes8(H, I, group, ctypes.byref(out)))
+    return out.value
+
+
+def coli_moe_pack_expert8(H, I, group, gate_codes, gate_scales, up_codes, up_scales,
+                          down_codes, down_scales) -> np.ndarray:
+    blob = np.zeros((coli_moe_expert_bytes8(H, I, group),), np.uint8)
+    arrs = [np.ascontiguousarray(a) for a in
+            (gate_codes, gate_scales, up_codes, up_scales, down_codes, down_scales)]
+    _ok(lib.coli_moe_pack_expert8(H, I, group, *[_ptr(a) for a in arrs], _ptr(blob)))
     return blob
 
 

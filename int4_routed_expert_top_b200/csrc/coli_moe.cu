@@ -598,6 +598,63 @@ int coli_moe_pack_expert(int32_t H, int32_t I, int32_t group, const uint8_t* gat
     return COLI_OK;
 }
 
+int coli_moe_quantize8(const float* w, int64_t rows, int64_t cols, int32_t group, int8_t* codes,
+                       float* scales) {
+    if (!w || !codes || !scales) return fail(COLI_E_INVAL, "quantize8: NULL pointer");
+    if (rows < 0 || cols <= 0 || (group != 0 && group != 64) || (group && cols % group))
+        return fail(COLI_E_INVAL, "quantize8: bad shape rows=%lld cols=%lld group=%d",
+                    (long long)rows, (long long)cols, group);
+    const int64_t gs = group ? group : cols, ng = cols / gs;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* row = w + r * cols;
+        for (int64_t g = 0; g < ng; ++g) {
+            float m = 0.0f;
+            for (int64_t c = g * gs; c < (g + 1) * gs; ++c) m = std::fmax(m, std::fabs(row[c]));
+            const float s = m / 127.0f;
+            scales[r * ng + g] = s;
+            for (int64_t c = g * gs; c < (g + 1) * gs; ++c) {
+                int q = 0;
+                if (s != 0.0f) q = (int)std::fmin(std::fmax(std::rint(row[c] / s), -127.0f), 127.0f);
+                codes[r * cols + c] = (int8_t)q;
+            }
+        }
+    }
+    return COLI_OK;
+}
+
+int coli_moe_expert_bytes8(int32_t H, int32_t I, int32_t group, size_t* bytes) {
+    if (!bytes) return fail(COLI_E_INVAL, "expert_bytes8: NULL pointer");
+    if (!shape_ok(H, I, group)) return fail(COLI_E_INVAL, "expert_bytes8: bad shape");
+    *bytes = (size_t)make_blob_layout8(H, I, group).bytes;
+    return COLI_OK;
+}
+
+int coli_moe_pack_expert8(int32_t H, int32_t I, int32_t group, const int8_t* gate_codes,
+                          const float* gate_scales, const int8_t* up_codes, const float* up_scales,
+                          const int8_t* down_codes, const float* down_scales, void* blob) {
+    if (!gate_codes || !gate_scales || !up_codes || !up_scales || !down_codes || !down_scales ||
+        !blob)
+        return fail(COLI_E_INVAL, "pack_expert8: NULL pointer");
+    if (!shape_ok(H, I, group)) return fail(COLI_E_INVAL, "pack_expert8: bad shape");
+    const BlobLayout L = make_blob_layout8(H, I, group);
+    uint8_t* out = static_cast<uint8_t*>(blob);
+    std::memset(out, 0, (size_t)L.bytes);
+    const int8_t* codes[3] = {gate_codes, up_codes, down_codes};
+    const float* scales[3] = {gate_scales, up_scales, down_scales};
+    for (int m = 0; m < 3; ++m) {
+        const int R = L.rows[m], K = L.cols[m], ng = L.ngroups[m];
+        for (int r = 0; r < R; ++r) {
+            for (int c = 0; c < K; ++c)
+                out[L.codes[m] + frag8_byte_offset(r, c, K)] =
+                    (uint8_t)codes[m][(int64_t)r * K + c];
+            for (int g = 0; g < ng; ++g)
+                reinterpret_cast<float*>(out + L.scales[m])[scale_offset(r, g, ng)] =
+                    scales[m][(int64_t)r * ng + g];
+        }
+    }
+    return COLI_OK;
+}
+
 int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group, const float* gate,
                                     const float* up, const float* down, void* blob,
                                     coli_stream_t stream) {

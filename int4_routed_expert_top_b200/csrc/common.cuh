@@ -45,6 +45,41 @@ __host__ __device__ inline BlobLayout make_blob_layout(int H, int I, int group) 
     return L;
 }
 
+// Blob of an expert with 8-bit codes (one signed byte per weight): the same
+// three matrices and scale sections as make_blob_layout, codes R * K bytes.
+__host__ __device__ inline BlobLayout make_blob_layout8(int H, int I, int group) {
+    BlobLayout L;
+    L.rows[0] = I; L.cols[0] = H;
+    L.rows[1] = I; L.cols[1] = H;
+    L.rows[2] = H; L.cols[2] = I;
+    int64_t off = 0;
+    for (int m = 0; m < 3; ++m) {
+        L.codes[m] = off;
+        off = align256(off + (int64_t)L.rows[m] * L.cols[m]);
+    }
+    for (int m = 0; m < 3; ++m) {
+        L.ngroups[m] = group == 0 ? 1 : L.cols[m] / group;
+        L.scales[m] = off;
+        off = align256(off + (int64_t)L.rows[m] * L.ngroups[m] * 4);
+    }
+    L.bytes = off;
+    return L;
+}
+
+// 8-bit fragment tiles: 16-row x 64-column blocks ordered [R/128][K/64][8][32
+// lanes] as for 4-bit codes, 32 bytes per lane: for each 32-column half h of
+// the step, four words i = 0..3 that are the lane's mma.sync m16n8k32 s8 A
+// registers: i = 0 row r0 = 16 b + g, columns 32 h + 4 t .. + 3; i = 1 row
+// r0 + 8, same columns; i = 2 row r0, columns 32 h + 16 + 4 t .. + 3; i = 3 row
+// r0 + 8, those columns; byte j of a word is its first column + j.
+__host__ __device__ inline int64_t frag8_byte_offset(int r, int c, int K) {
+    const int rt = r / 128, b8 = (r % 128) / 16, g = r % 8, upper = (r % 16) / 8;
+    const int kb = c / 64, h = (c % 64) / 32, c32 = c % 32;
+    const int hi16 = c32 / 16, t = (c32 % 16) / 4, j = c32 % 4;
+    const int lane = 4 * g + t, word = 4 * h + 2 * hi16 + upper;
+    return ((((int64_t)rt * (K / 64) + kb) * 8 + b8) * 32 + lane) * 32 + 4 * word + j;
+}
+
 // Fragment tiles.  A matrix [R, K] is cut into 16-row x 64-column blocks; the
 // block is 32 units of 16 bytes, one per lane l = 4*g + t of a warp, so one warp
 // load of 512 bytes fetches a whole block.  Unit l holds rows r0 = 16*b + g and

@@ -147,3 +147,73 @@ def test_workspace_size_and_limits_without_gpu():
         assert e.value.code == -5
     finally:
         cm.coli_moe_layer_destroy(h)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit codes: host quantiser and packer (the expert kernels do not read them yet)
+# ---------------------------------------------------------------------------
+
+def _unpack_blob8(blob, H, I, group):
+    """Read an 8-bit blob back through the layout the header documents."""
+    def sec_align(v):
+        return (v + 255) // 256 * 256
+    mats = [(I, H), (I, H), (H, I)]
+    off, code_off, scale_off = 0, [], []
+    for R, K in mats:
+        code_off.append(off)
+        off = sec_align(off + R * K)
+    for R, K in mats:
+        ng = 1 if group == 0 else K // group
+        scale_off.append(off)
+        off = sec_align(off + R * ng * 4)
+    assert off == blob.size
+    out = []
+    for m, (R, K) in enumerate(mats):
+        ng = 1 if group == 0 else K // group
+        # [T][s][b][lane][h][i][j]: word i of half h, byte j
+        raw = blob[code_off[m]:code_off[m] + R * K].view(np.int8)
+        raw = raw.reshape(R // 128, K // 64, 8, 32, 2, 4, 4)
+        T, s_, b, l, h, i, j = np.meshgrid(*[np.arange(n) for n in raw.shape], indexing="ij")
+        r = 128 * T + 16 * b + l // 4 + 8 * (i % 2)          # i = 1, 3: row r0 + 8
+        c = 64 * s_ + 32 * h + 4 * (l % 4) + 16 * (i // 2) + j  # i = 2, 3: columns + 16
+        q = np.zeros((R, K), np.int8)
+        q[r, c] = raw
+        sc = blob[scale_off[m]:scale_off[m] + R * ng * 4].view(np.float32)
+        sc = sc.reshape(R // 128, ng, 128).transpose(0, 2, 1).reshape(R, ng)
+        out += [q, sc]
+    return out
+
+
+@pytest.mark.parametrize("group", [0, 64])
+def test_quantize8_bit_identical_to_oracle(group):
+    rng = np.random.default_rng(4 + group)
+    w = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    w[3, 10] = 0.0
+    w[5, :] = 0.0                                   # a zero row
+    c, s = cm.coli_moe_quantize8(w, group)
+    co, so = oracle.quantize8(w, group)
+    np.testing.assert_array_equal(c, co)
+    np.testing.assert_array_equal(s.view(np.uint32), so.view(np.uint32))
+    row = np.array([[127 / 128, 2.5 / 128, 3.5 / 128, -0.5 / 128, -1.5 / 128, 0.0]], np.float32)
+    assert cm.coli_moe_quantize8(row, 0)[0][0].tolist() == [127, 2, 4, 0, -2, 0]
+
+
+@pytest.mark.parametrize("group", [0, 64])
+def test_pack_expert8_follows_documented_layout(group):
+    rng = np.random.default_rng(2)
+    H, I = 256, 128
+    mats = [(rng.standard_normal(s) * 0.02).astype(np.float32) for s in ((I, H), (I, H), (H, I))]
+    cont = []
+    for m in mats:
+        cont += list(cm.coli_moe_quantize8(m, group))
+    blob = cm.coli_moe_pack_expert8(H, I, group, *cont)
+    assert blob.size == cm.coli_moe_expert_bytes8(H, I, group)
+    back = _unpack_blob8(blob, H, I, group)
+    for a, b in zip(cont, back):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_expert_bytes8_glm():
+    codes = 3 * 6144 * 2048                       # one byte per weight
+    assert cm.coli_moe_expert_bytes8(6144, 2048, 0) == codes + 40960
+    assert cm.coli_moe_expert_bytes8(6144, 2048, 64) == codes + 2359296
