@@ -34,11 +34,12 @@
 //
 // Activations enter the tensor cores as two signed 8-bit digits of a 15-bit
 // fixed-point value: x16 = rint(x * 2^sh) = 256 * hi + lo with hi in [-64, 64]
-// and lo in [-128, 127], sh a power of two per token (gate/up input) or per
-// (pair, tile) (down input) that puts the largest magnitude in [2^13, 2^14).
-// A weight nibble q enters as the s8 value 16 q (the nibble placed in the high
-// half of a byte), so the int32 sums are exact; the factor 1/16, the weight
-// scales and the activation scales are applied in f32.
+// and lo in [-128, 127], sh a power of two per (token, 256 columns) for the
+// gate/up input and per (pair, tile) for the down input, putting the largest
+// magnitude of its block in [2^13, 2^14).  A weight nibble q enters as the s8
+// value 16 q (the nibble placed in the high half of a byte), so the int32 sums
+// over a stage are exact; the factor 1/16, the weight scales and the
+// activation scales are applied in f32 (once per stage).
 #pragma once
 
 #include "common.cuh"
@@ -80,8 +81,8 @@ struct FusedArgs {
     const float* sel;       // [T][E] selection scores s + bias (router kernel)
     float routed_scale;
     int norm_topk;
-    const int8_t* xq8;      // [T][H/64][128]  hi (64 B) + lo (64 B) per step, permuted
-    const float* xinv8;     // [T] inverse activation scale
+    const int8_t* xq8;      // [T][H/256][kActRec]: per 256 columns 4 steps of hi (64 B) +
+                            //   lo (64 B), permuted, then the f32 inverse scale
     float* part;            // [T][k + n_shared][I/128][H] partial down products
     int32_t* queue;         // work-item counter, zeroed by the router kernel
     int32_t* idx;           // [T*k] picks (written by CTA 0)
@@ -91,9 +92,9 @@ struct FusedArgs {
     int T, E, k, n_shared, H, I, group;
     int slots;              // ring stages
     int slot_bytes;
-    // 1: a gate/up stage takes every token's activation slice with one 2-D TMA
-    // box of the kernel's tensor map over xq8 (T rows of 2H bytes read as 32-bit
-    // words, boxes of T x 128 words), stored [token][step][hi 64 B | lo 64 B];
+    // 1: a gate/up stage takes every token's activation record with one 2-D TMA
+    // box of the kernel's tensor map over xq8 (T rows of H/256 records read as
+    // 32-bit words, boxes of T x kActRec/4 words), stored [token][record];
     // used for 2 <= T <= 4 (one column group).  0: one bulk copy per pair,
     // stored per pair record.
     int act_tma;
@@ -140,7 +141,6 @@ struct FusedShared {
     int u_item0[kFzMaxUnits + 1];                 // first work item of each unit
     int pair_tok[kFzMaxPairs];
     int pair_pick[kFzMaxPairs];                   // t * (k + n_shared) + j of each pair
-    float xinv[kFzMaxT];
     float xch[8][16][kFzChunk];                   // up values for the gate warps
     float wmax[8][kFzChunk];                      // per-warp max |h| of each pair
     __align__(16) int8_t hbuf[kFzChunk * kFzRecH]; // h of the current item, s8 digits
@@ -301,10 +301,6 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
     if (!small)
         for (int e = threadIdx.x; e < a.E; e += kFzThreads) { sc8.cnt[e] = 0; sc8.bits[e] = 0ull; }
     for (int t = warp; t < a.T; t += kAllWarps) fz_topk_token(a, t, sc8);
-    {   // from the last threads, which have no token's top-k before them when T is small
-        const int t = kFzThreads - 1 - (int)threadIdx.x;
-        if (t < a.T) sh.xinv[t] = __ldcg(a.xinv8 + t);
-    }
     __syncthreads();
     if (small) {
         if (warp == 0) fz_union_warp(a, sh, sc8);
@@ -523,8 +519,8 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
                 const int kb0 = st * z.ns_gu;
                 const bool rowsc = !GS && st == z.nst_gu - 1;
                 const uint32_t cb = (uint32_t)z.ns_gu * 4096, sb = GS ? (uint32_t)z.ns_gu * 512 : 0u;
-                const int nrec = a.act_tma ? a.T : np;  // activation slices of the stage
-                mbar_expect_tx_elect(&sh.full[s], 2 * (cb + sb) + (uint32_t)(nrec * z.ns_gu * 128) +
+                const int nrec = a.act_tma ? a.T : np;  // activation records of the stage
+                mbar_expect_tx_elect(&sh.full[s], 2 * (cb + sb) + (uint32_t)(nrec * kActRec) +
                                                       (rowsc ? 1024u : 0u));
                 const int64_t coff = frag_unit_offset(tc, kb0, 0, 0, a.H);
                 bulk_g2s_hint_elect(sl, cG + coff, cb, &sh.full[s], pol);
@@ -538,14 +534,14 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
                     bulk_g2s_elect(sl + kFzScaleOff, sG + (int64_t)tc * kTileRows, 512u, &sh.full[s]);
                     bulk_g2s_elect(sl + kFzScaleOff + 512, sU + (int64_t)tc * kTileRows, 512u, &sh.full[s]);
                 }
-                if (a.act_tma) {  // every token's slice, [token][step][128 B] (x in 4-byte units)
-                    tma_load_2d_elect(sl + kFzActOff, xmap, kb0 * 32, 0, &sh.full[s]);
+                if (a.act_tma) {  // every token's record, [token][kActRec] (x in 4-byte units)
+                    tma_load_2d_elect(sl + kFzActOff, xmap, st * (kActRec / 4), 0, &sh.full[s]);
                 } else {
                     for (int pp = 0; pp < np; ++pp) {
                         const int tok = one ? 0 : sh.pair_tok[p0 + pp];
                         bulk_g2s_elect(sl + kFzActOff + pp * rec_gu,
-                                       a.xq8 + ((int64_t)tok * (a.H / 64) + kb0) * 128,
-                                       (uint32_t)z.ns_gu * 128, &sh.full[s]);
+                                       a.xq8 + ((int64_t)tok * (a.H / 256) + st) * kActRec,
+                                       (uint32_t)kActRec, &sh.full[s]);
                     }
                 }
             } else {
@@ -590,47 +586,72 @@ namespace coli {
 // rb = w % 8 of the tile, every step of the stage.  After an MMA, lane (g, t)
 // holds rows g, g + 8 and columns 2t, 2t + 1 of an 8-column group c: column n
 // carries pair 4c + (n & 3), high digit for n < 4, low digit for n >= 4, so
-// lanes t and t ^ 2 hold the two digits of the same pairs.
+// lanes t and t ^ 2 hold the two digits of the same pairs.  The stage's sum
+// (exact int32 for per-row weight scales; with the weight scale of each step
+// for 64-column groups) is added to acc_f times the activation scale of its
+// pair's 256-column record, the lane's digit factor (256 for high digits) and
+// 1/16 (the nibble sits in the high half of an s8 byte).
+// xsoff[c][q]: offset of the activation record of pair 4c + 2(t & 1) + q.
 // ---------------------------------------------------------------------------
+static_assert(fz_rec_bytes(4) == kActRec, "pair records of a stage are the global records");
+
 template <int NT, bool GS>
 __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb, int lane,
-                                                int rec_gu, int aoff, int ntc, int acc_i[2][NT][4],
-                                                float acc_f[NT][4]) {
+                                                int rec_gu, int aoff, const int (*xsoff)[2],
+                                                int ntc, float acc_f[NT][4]) {
     constexpr int ns = 4;
     const int g = lane >> 2, t = lane & 3;
-    const float lanefac = t < 2 ? 256.0f : 1.0f;
     const uint8_t* cp = sl + m * ns * 4096 + rb * 512 + lane * 16;
     // aoff: this lane's pair record (column group 0); groups c > 0 follow at 4 c rec_gu
     const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + aoff;
     const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff + m * ns * 512) + 16 * rb + g;
+    // per-row scales: exact int32 sums, two chains (even and odd steps) for one
+    // column group, one chain when several groups give independent MMAs
+    constexpr int CH = NT == 1 ? 2 : 1;
+    int acc_i[CH][NT][4];
+    float acc_s[NT][4];    // 64-column scales: the stage's sum with them
 #pragma unroll
     for (int j = 0; j < ns; ++j) {
-        {
-            uint32_t A0[4], A1[4];
-            fz_decode_step(cp + j * 4096, A0, A1);
-            if (GS) {
-                const float s0 = scl[j * 128] * lanefac, s1 = scl[j * 128 + 8] * lanefac;
+        uint32_t A0[4], A1[4];
+        fz_decode_step(cp + j * 4096, A0, A1);
+        float s0 = 0.0f, s1 = 0.0f;
+        if (GS) { s0 = scl[j * 128]; s1 = scl[j * 128 + 8]; }
 #pragma unroll
-                for (int c = 0; c < NT; ++c) {
-                    if (NT > 1 && c >= ntc) break;  // column groups with no pair of this item
-                    const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
-                    int d[4];
-                    mma_s8_16832_zc(d, A0, b.x, b.y);
-                    mma_s8_16832(d, A1, b.z, b.w);
-                    acc_f[c][0] = fmaf((float)d[0], s0, acc_f[c][0]);
-                    acc_f[c][1] = fmaf((float)d[1], s0, acc_f[c][1]);
-                    acc_f[c][2] = fmaf((float)d[2], s1, acc_f[c][2]);
-                    acc_f[c][3] = fmaf((float)d[3], s1, acc_f[c][3]);
+        for (int c = 0; c < NT; ++c) {
+            if (NT > 1 && c >= ntc) break;  // column groups with no pair of this item
+            const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
+            if (GS) {
+                int d[4];
+                mma_s8_16832_zc(d, A0, b.x, b.y);
+                mma_s8_16832(d, A1, b.z, b.w);
+                if (j == 0) {
+                    acc_s[c][0] = (float)d[0] * s0; acc_s[c][1] = (float)d[1] * s0;
+                    acc_s[c][2] = (float)d[2] * s1; acc_s[c][3] = (float)d[3] * s1;
+                } else {
+                    acc_s[c][0] = fmaf((float)d[0], s0, acc_s[c][0]);
+                    acc_s[c][1] = fmaf((float)d[1], s0, acc_s[c][1]);
+                    acc_s[c][2] = fmaf((float)d[2], s1, acc_s[c][2]);
+                    acc_s[c][3] = fmaf((float)d[3], s1, acc_s[c][3]);
                 }
             } else {
-#pragma unroll
-                for (int c = 0; c < NT; ++c) {  // two accumulator chains: even and odd steps
-                    if (NT > 1 && c >= ntc) break;
-                    const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
-                    mma_s8_16832(acc_i[j & 1][c], A0, b.x, b.y);
-                    mma_s8_16832(acc_i[j & 1][c], A1, b.z, b.w);
-                }
+                if (j < CH) mma_s8_16832_zc(acc_i[j % CH][c], A0, b.x, b.y);
+                else mma_s8_16832(acc_i[j % CH][c], A0, b.x, b.y);
+                mma_s8_16832(acc_i[j % CH][c], A1, b.z, b.w);
             }
+        }
+    }
+    const float f = (t < 2 ? 256.0f : 1.0f) * 0.0625f;
+    const uint8_t* xr = sl + kFzActOff + kActRecScale;
+#pragma unroll
+    for (int c = 0; c < NT; ++c) {
+        if (NT > 1 && c >= ntc) break;
+        const float x0 = *reinterpret_cast<const float*>(xr + xsoff[c][0]) * f;
+        const float x1 = *reinterpret_cast<const float*>(xr + xsoff[c][1]) * f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float v = GS ? acc_s[c][i]
+                               : (float)(CH == 2 ? acc_i[0][c][i] + acc_i[CH - 1][c][i] : acc_i[0][c][i]);
+            acc_f[c][i] = fmaf(v, (i & 1) ? x1 : x0, acc_f[c][i]);
         }
     }
 }
@@ -741,16 +762,15 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
     const int rb = warp & 7, m = warp >> 3;
     const FzShape z = fz_shape(a);
     const int rec_gu = fz_rec_bytes(z.ns_gu);
-    const float lanefac = t < 2 ? 256.0f : 1.0f;
     const bool wr = t < 2;  // after the digit combine: lanes holding results
     uint32_t cphase = 0, lap = 0;
     int s = 0;
     int u = 0, tc = 0, p0 = 0, np = 0;
     int aoff = 0;  // this lane's activation record in a gate/up stage
+    int xsoff[NT][2];              // records of the lane's accumulator pairs
     float sw0 = 1.0f, sw1 = 1.0f;  // per-row weight scales of rows g, g + 8
     float hf[NT][2];               // down part: digit and h scale factors
     int dst[NT][2];                //            partial-product offsets
-    int acc_i[2][NT][4];
     float acc_f[NT][4];
     for (;;) {
         if (!fz_wait(&sh.full[s], lap, a.err)) return;
@@ -763,20 +783,24 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
             tc = wk.tc;
             p0 = wk.p0;
             np = wk.np;
-            if (a.act_tma) {  // records by token: the token of this lane's pair
-                const int pp = g & 3;
-                aoff = (pp < np ? sh.pair_tok[p0 + pp] : 0) * (z.ns_gu * 128);
-            } else {
-                aoff = (g & 3) * rec_gu;
+            // records by token (TMA box) or by pair of the item; pairs past np
+            // read pair 0's record (their results are never used)
+            auto rec_of = [&](int pp) {
+                if (pp >= np) pp = 0;
+                return a.act_tma ? sh.pair_tok[p0 + pp] * kActRec : pp * rec_gu;
+            };
+            aoff = rec_of(g & 3);
+#pragma unroll
+            for (int c = 0; c < NT; ++c) {
+                xsoff[c][0] = rec_of(4 * c + 2 * (t & 1));
+                xsoff[c][1] = rec_of(4 * c + 2 * (t & 1) + 1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc_f[c][i] = 0.0f;
             }
-#pragma unroll
-            for (int c = 0; c < NT; ++c)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) { acc_i[0][c][i] = 0; acc_i[1][c][i] = 0; acc_f[c][i] = 0.0f; }
         }
         const bool gu = st < z.nst_gu;
         if (gu) {
-            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, aoff, (np + 3) >> 2, acc_i, acc_f);
+            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, aoff, xsoff, (np + 3) >> 2, acc_f);
             if (!GS && st == z.nst_gu - 1) {
                 const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
                 sw0 = rsc[0];
@@ -797,7 +821,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
         for (int c = 0; c < NT; ++c)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float x = GS ? acc_f[c][i] : (float)(acc_i[0][c][i] + acc_i[1][c][i]) * lanefac;
+                float x = acc_f[c][i];
                 x += __shfl_xor_sync(0xffffffffu, x, 2);  // high digit * 256 + low digit
                 if (!GS) x *= (i >> 1) ? sw1 : sw0;
                 v[c][i] = x;
@@ -808,10 +832,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int pp = 4 * c + 2 * t + (i & 1), rr = g + 8 * (i >> 1);
-                if (wr && pp < np) {
-                    v[c][i] *= sh.xinv[sh.pair_tok[p0 + pp]] * 0.0625f;
-                    if (m == 1) sh.xch[rb][rr][pp] = v[c][i];
-                }
+                if (wr && pp < np && m == 1) sh.xch[rb][rr][pp] = v[c][i];
             }
         if (!fz_cbar(&sh.cbar, cphase, a.err)) return;
         if (m == 0) {
@@ -903,8 +924,6 @@ moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
             __syncwarp();
             asm volatile("bar.arrive 2, %0;" ::"n"(64) : "memory");
             fz_union_warp(a, sh, one);
-        } else if (warp == 1 && (threadIdx.x & 31) == 0) {
-            sh.xinv[0] = __ldcg(a.xinv8);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kFzWarps) : "memory");
         fz_consume<NT, GS>(a, sh, fz_smem, n_units);

@@ -79,7 +79,8 @@ constexpr int kRouterMaxT = 64;        // tokens per call of the small-batch rou
 // ---------------------------------------------------------------------------
 // s8 activation operand of the fused small-batch kernel (fused.cuh): each value
 // becomes two signed 8-bit digits of a 15-bit fixed-point number under one
-// power-of-two scale per token.
+// power-of-two scale per 256 columns (one gate/up stage of that kernel), so a
+// few outlier channels coarsen only the 256-column group they sit in.
 // ---------------------------------------------------------------------------
 // Byte position of column c (0..63) of a 64-column step in the activation
 // operand: lane t's 16 bytes hold columns 4t..4t+3, 16+4t.., 32+4t.., 48+4t..,
@@ -87,6 +88,13 @@ constexpr int kRouterMaxT = 64;        // tokens per call of the small-batch rou
 __host__ __device__ inline int fz_act_pos(int c) {
     return 16 * ((c % 16) / 4) + 4 * (c / 16) + (c % 4);
 }
+
+// Record of one token's 256-column group: 4 steps x (64 hi + 64 lo bytes), the
+// f32 inverse scale at byte 512, zero padding to 576 bytes (a multiple of 16
+// for bulk copies; 64 mod 128 so that records of consecutive tokens in shared
+// memory start in other banks).
+constexpr int kActRec = 576;
+constexpr int kActRecScale = 512;
 
 // Power-of-two scale for a block whose largest magnitude is m: returns sh with
 // m * 2^sh in [2^13, 2^14) and *inv = 2^-sh (1 for an all-zero block).
@@ -106,80 +114,70 @@ __device__ __forceinline__ void fz_split(float v, float sc, int& hi, int& lo) {
     lo = x - 256 * hi;
 }
 
-// s8 activation operand of one token, one CTA of 256 threads: xq8[t][step]
-// (64 hi bytes then 64 lo bytes, columns in fz_act_pos order), xinv8[t].
-// Thread tid owns columns 4 tid + 1024 j; for H <= 8192 the row is read once,
-// with every load in flight together, and kept in registers for both passes.
+// s8 activation operand of one token, one CTA of 256 threads: records
+// xq8[t][H/256][kActRec] as above (H a multiple of 256).  Thread tid owns
+// columns 4 tid + 1024 j; the 64 threads of two consecutive warps cover one
+// 256-column group.  Up to 8 column blocks of 1024 are loaded together (every
+// load in flight at once) and kept in registers for both passes.
 template <typename XT>
 __device__ __forceinline__ void act_quant8_token(const XT* __restrict__ x, int H, int t,
-                                                 int8_t* __restrict__ xq8,
-                                                 float* __restrict__ xinv8) {
+                                                 int8_t* __restrict__ xq8) {
     constexpr int kJ = 8;
-    __shared__ float part8[8];
+    __shared__ float part8[kJ][8];
     const XT* row = x + (int64_t)t * H;
-    const bool in_regs = H <= 1024 * kJ;
     const bool vec = (reinterpret_cast<uintptr_t>(row) & (4 * sizeof(XT) - 1)) == 0;
-    float4 v[kJ];
-    float m = 0.0f;
-    if (in_regs) {
+    const int warp = threadIdx.x >> 5;
+    const int G = H / 256;
+    int8_t* trec = xq8 + (int64_t)t * G * kActRec;
+    for (int j0 = 0; j0 * 1024 < H; j0 += kJ) {
+        float4 v[kJ];
 #pragma unroll
-        for (int j = 0; j < kJ; ++j) {
-            const int c = 4 * threadIdx.x + 1024 * j;
-            v[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int jj = 0; jj < kJ; ++jj) {
+            const int c = 4 * threadIdx.x + 1024 * (j0 + jj);
+            v[jj] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             if (c < H)
-                v[j] = vec ? load4_f32(row + c)
-                           : make_float4(to_f32(row[c]), to_f32(row[c + 1]), to_f32(row[c + 2]),
-                                         to_f32(row[c + 3]));
+                v[jj] = vec ? load4_f32(row + c)
+                            : make_float4(to_f32(row[c]), to_f32(row[c + 1]), to_f32(row[c + 2]),
+                                          to_f32(row[c + 3]));
         }
 #pragma unroll
-        for (int j = 0; j < kJ; ++j)
-            m = fmaxf(m, fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
-    } else {
-        for (int c = threadIdx.x; c < H; c += 256) m = fmaxf(m, fabsf(to_f32(row[c])));
-    }
+        for (int jj = 0; jj < kJ; ++jj) {
+            float m = fmaxf(fmaxf(fabsf(v[jj].x), fabsf(v[jj].y)),
+                            fmaxf(fabsf(v[jj].z), fabsf(v[jj].w)));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) part8[threadIdx.x >> 5] = m;
-    __syncthreads();
-    m = part8[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) m = fmaxf(m, part8[i]);
-    float inv;
-    const float sc = fz_scale(m, &inv);
-    // four consecutive columns per thread -> one 32-bit word of hi, one of lo
-#pragma unroll
-    for (int j = 0; j < kJ; ++j) {
-        const int c = 4 * threadIdx.x + 1024 * j;
-        if (!in_regs || c >= H) break;
-        const float f[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-        uint32_t wh = 0, wl = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            int hi, lo;
-            fz_split(f[i], sc, hi, lo);
-            wh |= (uint32_t)(hi & 0xFF) << (8 * i);
-            wl |= (uint32_t)(lo & 0xFF) << (8 * i);
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if ((threadIdx.x & 31) == 0) part8[jj][warp] = m;
         }
-        int8_t* step = xq8 + ((int64_t)t * (H / 64) + c / 64) * 128;
-        const int pos = fz_act_pos(c % 64);
-        *reinterpret_cast<uint32_t*>(step + pos) = wh;
-        *reinterpret_cast<uint32_t*>(step + 64 + pos) = wl;
-    }
-    for (int c = 4 * threadIdx.x; !in_regs && c < H; c += 1024) {
-        uint32_t wh = 0, wl = 0;
+        __syncthreads();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            int hi, lo;
-            fz_split(to_f32(row[c + i]), sc, hi, lo);
-            wh |= (uint32_t)(hi & 0xFF) << (8 * i);
-            wl |= (uint32_t)(lo & 0xFF) << (8 * i);
+        for (int jj = 0; jj < kJ; ++jj) {
+            const int c = 4 * threadIdx.x + 1024 * (j0 + jj);
+            if (c >= H) break;
+            const float m = fmaxf(part8[jj][warp & ~1], part8[jj][warp | 1]);
+            float inv;
+            const float sc = fz_scale(m, &inv);
+            const float f[4] = {v[jj].x, v[jj].y, v[jj].z, v[jj].w};
+            uint32_t wh = 0, wl = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int hi, lo;
+                fz_split(f[i], sc, hi, lo);
+                wh |= (uint32_t)(hi & 0xFF) << (8 * i);
+                wl |= (uint32_t)(lo & 0xFF) << (8 * i);
+            }
+            int8_t* rec = trec + (int64_t)(c / 256) * kActRec;
+            int8_t* step = rec + ((c % 256) / 64) * 128;
+            const int pos = fz_act_pos(c % 64);
+            *reinterpret_cast<uint32_t*>(step + pos) = wh;
+            *reinterpret_cast<uint32_t*>(step + 64 + pos) = wl;
+            const int lt = threadIdx.x & 63;  // thread within the group
+            if (lt < (kActRec - kActRecScale) / 16) {  // the scale, then zero padding
+                const uint4 z = make_uint4(lt == 0 ? __float_as_uint(inv) : 0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(rec + kActRecScale + 16 * lt) = z;
+            }
         }
-        int8_t* step = xq8 + ((int64_t)t * (H / 64) + c / 64) * 128;
-        const int pos = fz_act_pos(c % 64);
-        *reinterpret_cast<uint32_t*>(step + pos) = wh;
-        *reinterpret_cast<uint32_t*>(step + 64 + pos) = wl;
+        __syncthreads();  // part8 is rewritten by the next block of columns
     }
-    if (threadIdx.x == 0) xinv8[t] = inv;
 }
 
 // Extra blocks after the router's: one per token for the activation operand
@@ -189,7 +187,6 @@ struct RouterExtras {
     __half* xq = nullptr;
     float* xinv = nullptr;
     int8_t* xq8 = nullptr;
-    float* xinv8 = nullptr;
     int32_t* zero = nullptr;
     int zero_n = 0;
     int32_t* err = nullptr;  // device error flags, cleared by the same block
@@ -215,7 +212,7 @@ router_gemv_kernel(const XT* __restrict__ x, int T, int H, const float* __restri
         const int b = blockIdx.x - router_blocks;
         if (b < T) {  // one CTA per token: activation operand
             if (ex.xq) act_quant_token(x, H, b, ex.xq, ex.xinv);
-            if (ex.xq8) act_quant8_token(x, H, b, ex.xq8, ex.xinv8);
+            if (ex.xq8) act_quant8_token(x, H, b, ex.xq8);
         } else {
             for (int i = threadIdx.x; i < ex.zero_n; i += 256) ex.zero[i] = 0;
             if (threadIdx.x == 0 && ex.err) *ex.err = 0;
@@ -311,7 +308,7 @@ router_row_kernel(const XT* __restrict__ x, int T, int H, const float* __restric
         const int b = e - E;
         if (b < T) {
             if (ex.xq) act_quant_token(x, H, b, ex.xq, ex.xinv);
-            if (ex.xq8) act_quant8_token(x, H, b, ex.xq8, ex.xinv8);
+            if (ex.xq8) act_quant8_token(x, H, b, ex.xq8);
         } else {
             for (int i = threadIdx.x; i < ex.zero_n; i += 256) ex.zero[i] = 0;
             if (threadIdx.x == 0 && ex.err) *ex.err = 0;

@@ -111,7 +111,9 @@ def glm_prefill_layer():
 def test_glm_prefill_tensor_core_path(glm_prefill_layer):
     """Prefill, T = 512 bf16 tokens, gs64, Zipf-skewed routing, 257 resident
     experts.  Every output against the f32 GEMV path (itself held to 2e-3 of the
-    oracle); three sampled tokens, all 6144 outputs, against the oracle."""
+    oracle); against the oracle, all 6144 outputs of tokens 0, 255 and 511 and
+    of eight tokens routed to the busiest expert (~100 tokens: its units span
+    two N tiles), the first and last of them included."""
     wl = synth.GLM_PREFILL
     L = glm_prefill_layer
     wr, b = L.router_w.cpu(), L.router_b.cpu()
@@ -121,10 +123,17 @@ def test_glm_prefill_tensor_core_path(glm_prefill_layer):
     same_selection(idx, idx_ref)
     y_gemv, _, _ = forward(L, xd, wl.T, cm.COLI_PATH_GEMV)
     assert rel_err(y, y_gemv) <= TOL_TC
+    import concurrent.futures as cf
     experts = OracleExperts(wl)
     xb = x.numpy()            # already bf16-representable: the device reads the same values
-    for t in (0, 255, 511):
+    hot = int(np.argmax(np.bincount(idx_ref.ravel(), minlength=wl.E)))
+    hot_toks = np.nonzero((idx_ref == hot).any(1))[0]
+    assert hot_toks.size >= 90
+    toks = sorted({0, 255, 511} | set(hot_toks[np.linspace(0, hot_toks.size - 1, 8).astype(int)]))
+    need = sorted({int(e) for t in toks for e in idx_ref[t]} | {wl.E})
+    with cf.ThreadPoolExecutor(16) as ex:
+        list(ex.map(experts, need))
+    for t in toks:
         y_ref = oracle_tokens(wl, experts, xb[t:t + 1], idx_ref[t:t + 1], w_ref[t:t + 1])
         err = rel_err(y[t:t + 1], y_ref)
         assert err <= TOL_TC, (t, err)
-        experts.cache.clear()

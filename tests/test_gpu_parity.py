@@ -332,3 +332,81 @@ def test_glm_mtp_verify_steps(glm_mtp_layer, path):
             err = rel_err(y, y_ref)
             assert err <= TOL_F32, err
             experts.cache.clear()
+
+
+# ---------------------------------------------------------------------------
+# activations with outlier channels and a wide dynamic range
+# ---------------------------------------------------------------------------
+
+def outlier_tokens(wl, wr, b, step, max_rounds=64):
+    """Four tokens on N(0, 1) draws: (0) one channel at 100x, (1) four channels
+    at 1000x, (2) magnitudes 2^u, u uniform in [-10, 10], random signs,
+    (3) sixteen channels at 100x; each then scaled to unit RMS, as a normalised
+    layer input is (the ratios between channels are what the activation
+    encodings must carry; the router keeps its usual operating range).
+    Positions and signs come from a seeded generator; a token whose oracle gap
+    is under 1e-3 is drawn again."""
+    wr_np, b_np = wr.cpu().numpy(), b.cpu().numpy()
+    out = []
+    for case in range(4):
+        for r in range(max_rounds):
+            rng = np.random.default_rng([wl.seed, step, case, r])
+            x = synth.tokens(wl, 1, 0, 1000 + 97 * step + case, [r]).numpy()[0].copy()
+            if case == 2:
+                x = np.where(rng.random(wl.H) < 0.5, -1.0, 1.0) * np.exp2(rng.uniform(-10, 10, wl.H))
+            else:
+                n, amp = {0: (1, 100.0), 1: (4, 1000.0), 3: (16, 100.0)}[case]
+                pos = rng.choice(wl.H, n, replace=False)
+                x[pos] = amp * np.where(rng.random(n) < 0.5, -1.0, 1.0)
+            x = (x / np.sqrt(np.mean(np.square(x, dtype=np.float64)))).astype(np.float32)[None]
+            idx, w, gap = oracle.route(x, wr_np, b_np, wl.k, wl.routed_scale, wl.norm_topk)
+            if gap[0] >= 1e-3:
+                out.append((x[0], idx[0], w[0]))
+                break
+        else:
+            raise RuntimeError("gap rule did not converge")
+    return (np.stack([o[0] for o in out]), np.stack([o[1] for o in out]),
+            np.stack([o[2] for o in out]))
+
+
+def per_element_error(y, ref):
+    """max |y - ref| / max(|ref|, 1e-6 max |ref|), element by element (reported)."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    floor = 1e-6 * np.abs(ref).max()
+    return float((np.abs(y - ref) / np.maximum(np.abs(ref), floor)).max())
+
+
+OUTLIER_PATHS = {"fused": (cm.COLI_PATH_FUSED, TOL_F32), "gemv": (cm.COLI_PATH_GEMV, TOL_F32),
+                 "gemm": (cm.COLI_PATH_GEMM, 1e-2)}
+
+
+def check_outliers(wl, L, step):
+    import concurrent.futures as cf
+    wr, b = L.router_w.cpu(), L.router_b.cpu()
+    x, idx_ref, w_ref = outlier_tokens(wl, wr, b, step)
+    experts = OracleExperts(wl)
+    need = sorted({int(e) for e in idx_ref.ravel()} | {wl.E + s for s in range(wl.n_shared)})
+    with cf.ThreadPoolExecutor(8) as ex:
+        list(ex.map(experts, need))
+    y_ref = oracle_tokens(wl, experts, x, idx_ref, w_ref)
+    xd = torch.from_numpy(x).cuda()
+    for name, (path, tol) in OUTLIER_PATHS.items():
+        y, idx, _ = forward(L, xd, 4, path=path)
+        same_selection(idx, idx_ref)
+        for t in range(4):
+            err = rel_err(y[t], y_ref[t])
+            print(f"{wl.name} {name} token {t}: norm-wise {err:.2e}, "
+                  f"per-element {per_element_error(y[t], y_ref[t]):.2e}")
+            assert err <= tol, (name, t, err)
+    for t in range(4):   # the one-token fused path
+        y, _, _ = forward(L, xd[t:t + 1].contiguous(), 1, path=cm.COLI_PATH_FUSED)
+        assert rel_err(y[0], y_ref[t]) <= TOL_F32, t
+
+
+def test_outlier_activations_per_row(glm_decode_layer):
+    check_outliers(synth.GLM_DECODE, glm_decode_layer, step=0)
+
+
+def test_outlier_activations_gs64(glm_mtp_layer):
+    check_outliers(synth.GLM_MTP, glm_mtp_layer, step=1)
