@@ -305,7 +305,9 @@ int coli_moe_stack_forward_host(const coli_moe_layer* const* layers, int32_t L,
 /* Device-side status of the most recent coli_moe_forward* call that used this
  * workspace (ws planned for T tokens): copies the error flags to *flags (host)
  * after synchronising `stream`.  Returns COLI_E_TIMEOUT if a bounded wait inside
- * a kernel gave up (its outputs are then invalid), else COLI_OK. */
+ * a kernel gave up (its outputs are then invalid), else COLI_OK.  ws == NULL
+ * reads the flags of the built-in scratch array of coli_moe_forward_noalloc on
+ * the current device (T as in that call). */
 int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws,
                     int32_t* flags, coli_stream_t stream);
 
@@ -331,7 +333,11 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert,
  *    fused path for T <= 2).
  *  - The first call on each device looks up that device's copy of the array
  *    (cudaGetSymbolAddress with the device current); make that first call before
- *    any stream capture.  Later calls only launch kernels.
+ *    any stream capture.  Later calls only launch kernels, until the device's
+ *    context is created anew (after cudaDeviceReset), when the next call looks
+ *    the array up again.
+ *  - A bounded device-side wait that gave up is reported by
+ *    coli_moe_status(layer, T, NULL, ...), which reads the array's flags.
  *  - All calls share the one array, and it keeps whatever the previous call left
  *    in it (every value a call needs cleared is cleared by its own kernels).
  *    Calls whose kernels overlap on the GPU (different streams, or different

@@ -310,7 +310,8 @@ def coli_moe_stack_forward_host(layers, x_host, y_host, T, eps, ws, path=COLI_PA
 
 
 def coli_moe_status(layer, T: int, ws, stream=None) -> int:
-    """Error flags of the last forward on this workspace (raises on a timeout)."""
+    """Error flags of the last forward on this workspace (raises on a timeout);
+    ws None: the built-in scratch array of coli_moe_forward_noalloc."""
     flags = _I32(0)
     _ok(lib.coli_moe_status(layer, T, _ptr(ws), ctypes.byref(flags), _stream(stream)))
     return flags.value

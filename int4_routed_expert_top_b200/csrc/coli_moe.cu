@@ -59,7 +59,7 @@ struct WsPlan {
     int64_t zpart, idx, w, offsets, pair_tok, pair_slot, uniq, n_uniq, inv;
     int64_t unit_expert, unit_begin, unit_end, n_units, counters, err;
     int64_t xq, xinv, hq, hinv, o, xg, hg, hmax, hsc;
-    int64_t xq8, xinv8, part, queue, sel;  // fused small-batch kernel (T <= kFzMaxT only)
+    int64_t xq8, part, queue, sel;  // fused small-batch kernel (T <= kFzMaxT only)
     int64_t total;
 };
 
@@ -102,13 +102,12 @@ WsPlan plan_ws(const coli_moe_desc& d, int T, bool with_fused = true) {
     p.hmax = take(P * 4);                       //   per-pair max |h|
     p.hsc = take(P * 4);                        //   per-pair inverse scale of h
     if (with_fused && fused_fits(d, T)) {
-        p.xq8 = take((int64_t)T * d.H * 2);
-        p.xinv8 = take((int64_t)T * 4);
+        p.xq8 = take((int64_t)T * (d.H / 256) * kActRec);
         p.part = take(P * (d.I / 128) * d.H * 4);
         p.queue = take(4);
         p.sel = take((int64_t)T * d.E * 4);
     } else {
-        p.xq8 = p.xinv8 = p.part = p.queue = p.sel = 0;
+        p.xq8 = p.part = p.queue = p.sel = 0;
     }
     p.total = off;
     return p;
@@ -307,14 +306,14 @@ int encode_b_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
     return COLI_OK;
 }
 
-// xq8 of T tokens as [T] rows of 2H bytes read as 32-bit words; boxes of the
-// gate/up stage's 64-column steps (ns x 128 B) of every token, no swizzle
-int encode_act_map(CUtensorMap* m, const void* xq8, int T, int H, int ns) {
+// xq8 of T tokens as [T] rows of H/256 activation records read as 32-bit
+// words; boxes of one record (one gate/up stage) of every token, no swizzle
+int encode_act_map(CUtensorMap* m, const void* xq8, int T, int H) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(COLI_E_CUDA, "cuTensorMapEncodeTiled is not available");
-    const cuuint64_t dims[2] = {(cuuint64_t)(2 * H / 4), (cuuint64_t)T};
-    const cuuint64_t strides[1] = {(cuuint64_t)2 * H};
-    const cuuint32_t box[2] = {(cuuint32_t)(ns * 128 / 4), (cuuint32_t)T};
+    const cuuint64_t dims[2] = {(cuuint64_t)(H / 256 * kActRec / 4), (cuuint64_t)T};
+    const cuuint64_t strides[1] = {(cuuint64_t)(H / 256 * kActRec)};
+    const cuuint32_t box[2] = {(cuuint32_t)(kActRec / 4), (cuuint32_t)T};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(xq8), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -480,7 +479,6 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     a.routed_scale = d.routed_scale;
     a.norm_topk = d.norm_topk;
     a.xq8 = at<int8_t>(ws, p.xq8);
-    a.xinv8 = at<float>(ws, p.xinv8);
     a.part = at<float>(ws, p.part);
     a.queue = at<int32_t>(ws, p.queue);
     a.idx = at<int32_t>(ws, p.idx);
@@ -501,7 +499,7 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     std::memset(&xmap, 0, sizeof(xmap));
     a.act_tma = 0;
     if (T >= 2 && NT == 1) {
-        if ((rc = encode_act_map(&xmap, a.xq8, T, d.H, fz_ns_gateup(d.H)))) return rc;
+        if ((rc = encode_act_map(&xmap, a.xq8, T, d.H))) return rc;
         a.act_tma = 1;
     }
     switch (NT) {
@@ -522,6 +520,65 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     return launch_pdl(moe_combine_kernel, dim3(T * (d.H / 32)), 32 * warps, 0, st, "fused combine", c);
 }
 
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward: the workspace is a scratch array compiled into the
+// library (one copy per device), not memory from the caller.
+// ---------------------------------------------------------------------------
+namespace {
+__device__ __align__(256) unsigned char g_noalloc_scratch[COLI_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+struct NoallocEntry { void* ctx; void* ptr; };
+NoallocEntry g_noalloc[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    });
+    return fn;
+}
+
+// Device address of this device's copy of the scratch array.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// the device current, once per device and context: a context created anew
+// (after cudaDeviceReset, or after the primary context was released) loads the
+// module again, possibly at another address, so the lookup is repeated then.
+int noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return fail(COLI_E_CUDA, "forward_noalloc: no usable current device");
+    CtxGetCurrentFn get = ctx_get_current_fn();
+    if (!get) return fail(COLI_E_CUDA, "forward_noalloc: cuCtxGetCurrent is not available");
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoallocEntry& en = g_noalloc[dev];
+    if (!ctx || en.ctx != (void*)ctx || !en.ptr) {
+        // the lookup also makes the device's primary context current if the
+        // runtime had not created it yet
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(COLI_E_CUDA, "forward_noalloc: scratch lookup failed: %s",
+                        cudaGetErrorString(e));
+        if (get(&ctx) != CUDA_SUCCESS || !ctx)
+            return fail(COLI_E_CUDA, "forward_noalloc: no current context on device %d", dev);
+        en.ctx = (void*)ctx;
+        en.ptr = p;
+    }
+    *out = en.ptr;
+    return COLI_OK;
+}
 }  // namespace
 
 // ===========================================================================
@@ -798,7 +855,6 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         if ((rc = mark(COLI_STAGE_ROUTER))) return rc;
         RouterExtras ex;
         ex.xq8 = at<int8_t>(ws, p.xq8);
-        ex.xinv8 = at<float>(ws, p.xinv8);
         ex.zero = at<int32_t>(ws, p.queue);
         ex.zero_n = 1;
         ex.err = at<int32_t>(ws, p.err);
@@ -1026,9 +1082,14 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t 
 
 int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws, int32_t* flags,
                     coli_stream_t stream) {
-    if (!layer || !ws || !flags) return fail(COLI_E_INVAL, "status: NULL pointer");
+    if (!layer || !flags) return fail(COLI_E_INVAL, "status: NULL pointer");
     int rc = tokens_ok(layer->d, T);
     if (rc) return rc;
+    if (!ws) {  // the built-in scratch array of coli_moe_forward_noalloc
+        void* scratch = nullptr;
+        if ((rc = noalloc_scratch(&scratch))) return rc;
+        ws = scratch;
+    }
     const WsPlan p = plan_ws(layer->d, T);
     cudaStream_t st = S(stream);
     if (cudaMemcpyAsync(flags, static_cast<const char*>(ws) + p.err, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
@@ -1038,37 +1099,6 @@ int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws, int3
     return COLI_OK;
 }
 
-// ---------------------------------------------------------------------------
-// Allocation-free forward: the workspace is a scratch array compiled into the
-// library (one copy per device), not memory from the caller.
-// ---------------------------------------------------------------------------
-namespace {
-__device__ __align__(256) unsigned char g_noalloc_scratch[COLI_NOALLOC_SCRATCH_BYTES];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of this device's copy of the scratch array.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device, with that device current, and cached.
-int noalloc_scratch(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return fail(COLI_E_CUDA, "forward_noalloc: no usable current device");
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || !p)
-            return fail(COLI_E_CUDA, "forward_noalloc: scratch lookup failed: %s",
-                        cudaGetErrorString(e));
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
-    return COLI_OK;
-}
-}  // namespace
 
 int coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x, coli_dtype xt,
                              int32_t T, float* y, coli_stream_t stream) {

@@ -15,29 +15,32 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("group", [0, 64])
 def test_noalloc_forward_matches_workspace_forward(group):
+    """Same path as the ordinary forward (the fused kernel here), so the same
+    bytes, on two calls in a row that share the built-in scratch array; the
+    array's error flags read back clear afterwards."""
     import dataclasses
     wl = dataclasses.replace(synth.TINY, group=group, T=5)
     L = build_layer(wl)
     y_ref = torch.empty((wl.T, wl.H), dtype=torch.float32, device="cuda")
     y = torch.empty_like(y_ref)
-    for call in range(2):           # two calls in a row share the built-in scratch
+    for call in range(2):
         x = synth.tokens(wl, wl.T, step=call).cuda()
         cm.coli_moe_forward(L.handle, x, wl.T, y_ref, L.workspace(wl.T))
         y.fill_(float("nan"))
         cm.coli_moe_forward_noalloc(L.handle, x, wl.T, y)
         torch.cuda.synchronize()
-        err = rel_err(y.cpu().numpy(), y_ref.cpu().numpy())
-        assert err <= 2e-3, (call, err)
-        assert np.isfinite(y.cpu().numpy()).all()
+        np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32),
+                                      y_ref.cpu().numpy().view(np.uint32))
+        assert cm.coli_moe_status(L.handle, wl.T, None) == 0
     L.close()
 
 
 def test_noalloc_rejects_too_many_tokens():
+    """8192 tokens of the tiny layer: even the GEMV path's workspace prefix (its
+    fp16 activation digits alone are T * H * 4 = 8 MiB) exceeds the array."""
     wl = synth.TINY
     L = build_layer(wl)
-    T = 1
-    while cm.coli_moe_workspace_size(L.handle, T) <= cm.NOALLOC_SCRATCH_BYTES:
-        T *= 2
+    T = 8192
     x = torch.zeros((T, wl.H), dtype=torch.float32, device="cuda")
     y = torch.empty_like(x)
     with pytest.raises(cm.ColiError) as e:
