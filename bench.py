@@ -87,12 +87,12 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def profiled_traffic(kernel_src: str, profile: str):
+def profiled_traffic(kernel_src: str, profile: str, profiles_dir: str | None = None):
     """DRAM bytes per launch (read + write) from the ncu summary in profiles/,
     valid only while the kernel source still has the hash the capture names."""
     import hashlib
     try:
-        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        text = open(os.path.join(profiles_dir or os.path.join(ROOT, "profiles"), profile)).read()
         digest = hashlib.sha256(open(os.path.join(ROOT, kernel_src), "rb").read()).hexdigest()
     except OSError:
         return None

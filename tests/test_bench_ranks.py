@@ -69,16 +69,20 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert r.stdout.strip() == b""
 
 
-def test_profiled_traffic_only_while_the_kernel_source_matches():
-    """The roofline's traffic comes from the committed ncu summary only while
-    the kernel source still has the hash that summary names."""
+def test_profiled_traffic_only_while_the_kernel_source_matches(tmp_path):
+    """The roofline's traffic comes from an ncu summary only while the kernel
+    source still has the hash that summary names."""
+    import hashlib
     sys.path.insert(0, ROOT)
     import bench
-    t = bench.profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
-                               "moe_fused_kernel_glm_decode.md")
-    assert t is not None and t > 170e6                 # at least the algorithmic bytes
+    src = "int4_routed_expert_top_b200/csrc/fused.cuh"
+    digest = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+    (tmp_path / "p.md").write_text(
+        f"source sha256 prefix {digest[:16]}\n\n| metric | value |\n|---|---|\n"
+        "| traffic_bytes_per_launch | 173990000 |\n")
+    t = bench.profiled_traffic(src, "p.md", str(tmp_path))
+    assert t == 173990000.0
     # another source file has another hash: no traffic
-    assert bench.profiled_traffic("int4_routed_expert_top_b200/csrc/gemm.cuh",
-                                  "moe_fused_kernel_glm_decode.md") is None
-    assert bench.profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
-                                  "no_such_profile.md") is None
+    assert bench.profiled_traffic("int4_routed_expert_top_b200/csrc/gemm.cuh", "p.md",
+                                  str(tmp_path)) is None
+    assert bench.profiled_traffic(src, "no_such_profile.md", str(tmp_path)) is None

@@ -25,10 +25,14 @@ def masters(wl, layer, e, device="cuda"):
     return tuple(synth.expert_master(wl, layer, t, e, device=device) for t in MATS)
 
 
-def build_layer(wl, layer=0, device="cuda", router=None):
+def build_layer(wl, layer=0, device="cuda", router=None, masters_device=None):
+    """Layer on ``device``; its f32 masters are drawn on ``masters_device``
+    (default: the same device) and quantised by the library on the device."""
     wr, b = router if router is not None else synth.router(wl, layer)
+    md = masters_device or device
     return DeviceLayer(wl.H, wl.I, wl.E, wl.k, wl.n_shared, wl.group, wr, b,
-                       expert_masters=lambda e: masters(wl, layer, e, device),
+                       expert_masters=lambda e: tuple(
+                           m.to(device) for m in masters(wl, layer, e, md)),
                        routed_scale=wl.routed_scale, norm_topk=wl.norm_topk, device=device)
 
 
