@@ -208,6 +208,32 @@ typedef struct coli_moe_layer coli_moe_layer;
 int coli_moe_layer_create(const coli_moe_desc* desc, coli_moe_layer** out);
 int coli_moe_layer_destroy(coli_moe_layer* layer);
 
+/* Adaptive expert top-p for every later forward of this layer ("colibrì 實戰指南"
+ * 三 and 五: `--topp 0.7`, 30-40% fewer expert bytes per token, lossy; the pages
+ * name the option but give no rule).  Rule: of a token's k picks, keep the
+ * shortest run of the largest renormalised weights w_j / sum(w) (equal weights:
+ * the lower expert index first) whose total reaches p, at least one pick; the
+ * kept picks keep their weights w_j, the others add nothing to y.  The totals
+ * are formed in double, in that order, from the f32 weights, and compared with
+ * (double)p.  0 < p <= 1 enables it; p = 0 (the default) disables it; other
+ * values give COLI_E_INVAL.  Forward calls then report w_out = 0 for dropped
+ * picks.  Host-only: changes the handle, not device memory. */
+int coli_moe_layer_set_topp(coli_moe_layer* layer, float p);
+
+/* Expert parallelism: restrict this handle to the routed experts
+ * e_begin <= e < e_end (and to the shared experts when with_shared != 0).
+ * experts (device) then holds only those blobs: e_end - e_begin routed blobs in
+ * expert order, followed by the n_shared shared blobs when with_shared != 0.
+ * Routing still covers all E experts (the router is replicated); a forward
+ * computes y = sum of w_j o_j over the picks whose expert is in the range (and
+ * the shared experts when with_shared, and the residual when given), so the
+ * sum of the y of handles whose ranges partition [0, E), exactly one of them
+ * with the shared experts and the residual, is the layer's output.  Forward
+ * calls report w_out = 0 for picks outside the range.  Workspace sizes follow
+ * the restriction (no shared pairs when with_shared == 0).  Host-only. */
+int coli_moe_layer_set_partition(coli_moe_layer* layer, int32_t e_begin, int32_t e_end,
+                                 int32_t with_shared, const void* experts);
+
 /* Workspace bytes that coli_moe_route / coli_moe_forward need for T tokens
  * (enough for every path; the GEMV and GEMM paths use only a prefix). */
 int coli_moe_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes);
@@ -228,7 +254,9 @@ int coli_moe_union(const int32_t* idx, int32_t T, int32_t k, int32_t E,
                    int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot,
                    int32_t* uniq, int32_t* n_uniq, coli_stream_t stream);
 
-/* Steps 1-5: writes y device f32 [T, H] (overwrites; no accumulation). */
+/* Steps 1-5: writes y device f32 [T, H] (overwrites; no accumulation).  A pick
+ * whose weight is 0 (dropped by top-p, outside the handle's expert range, or a
+ * zero routed weight) is not computed: it would add exactly nothing. */
 int coli_moe_forward(const coli_moe_layer* layer, const void* x, coli_dtype xt,
                      int32_t T, float* y, void* ws, size_t ws_bytes,
                      coli_stream_t stream);
@@ -245,7 +273,9 @@ typedef enum coli_stage {
 
 /* coli_moe_forward with options: path selects the expert kernels; residual
  * (device f32 [T, H] or NULL) is added to the output (it may alias y);
- * idx_out / w_out (device, may be NULL) receive the routing decision.
+ * idx_out / w_out (device, may be NULL) receive the routing decision: the k
+ * experts of every token and the weights as applied (0 for a pick not
+ * computed by this call).
  * events (may be NULL) is an array of COLI_STAGES + 1 cudaEvent_t created by
  * the caller; events[s] is recorded on `stream` just before stage s and
  * events[COLI_STAGES] after the last one, so cudaEventElapsedTime(events[s],

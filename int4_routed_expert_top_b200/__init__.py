@@ -22,6 +22,7 @@ __all__ = [
     "coli_moe_union", "coli_moe_forward", "coli_moe_forward_ex", "coli_moe_rmsnorm",
     "coli_moe_stack_workspace_size", "coli_moe_stack_forward", "coli_moe_dequant_debug",
     "coli_moe_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "coli_moe_status", "Desc",
+    "coli_moe_layer_set_topp", "coli_moe_layer_set_partition",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +41,7 @@ EXPORTS = (
     "coli_moe_forward_noalloc", "coli_moe_status", "coli_moe_host_workspace_size",
     "coli_moe_forward_host", "coli_moe_stack_host_workspace_size", "coli_moe_stack_forward_host",
     "coli_moe_quantize_expert_fp8_device", "coli_moe_quantize8", "coli_moe_expert_bytes8",
-    "coli_moe_pack_expert8",
+    "coli_moe_pack_expert8", "coli_moe_layer_set_topp", "coli_moe_layer_set_partition",
 )
 
 
@@ -82,6 +83,8 @@ _SIGS = {
     "coli_moe_pack_expert8": ([_I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "coli_moe_layer_create": ([ctypes.POINTER(Desc), ctypes.POINTER(_P)], ctypes.c_int),
     "coli_moe_layer_destroy": ([_P], ctypes.c_int),
+    "coli_moe_layer_set_topp": ([_P, ctypes.c_float], ctypes.c_int),
+    "coli_moe_layer_set_partition": ([_P, _I32, _I32, _I32, _P], ctypes.c_int),
     "coli_moe_workspace_size": ([_P, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
     "coli_moe_route": ([_P, _P, ctypes.c_int, _I32, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "coli_moe_union": ([_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P], ctypes.c_int),
@@ -220,6 +223,16 @@ def coli_moe_layer_create(desc: Desc) -> ctypes.c_void_p:
 
 def coli_moe_layer_destroy(layer) -> None:
     _ok(lib.coli_moe_layer_destroy(layer))
+
+
+def coli_moe_layer_set_topp(layer, p: float) -> None:
+    _ok(lib.coli_moe_layer_set_topp(layer, p))
+
+
+def coli_moe_layer_set_partition(layer, e_begin: int, e_end: int, with_shared: bool,
+                                 experts) -> None:
+    _ok(lib.coli_moe_layer_set_partition(layer, e_begin, e_end, int(bool(with_shared)),
+                                         _ptr(experts)))
 
 
 def coli_moe_workspace_size(layer, T: int) -> int:

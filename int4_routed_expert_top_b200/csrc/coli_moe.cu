@@ -22,8 +22,14 @@
 using namespace coli;
 
 struct coli_moe_layer {
-    coli_moe_desc d;
+    coli_moe_desc d;       // as created
     BlobLayout L;
+    // what a forward computes: d with n_shared = 0 on a handle restricted to a
+    // range of routed experts without the shared ones; where the blobs sit;
+    // which picks are computed (top-p, expert range)
+    coli_moe_desc run;
+    ExpertStore store;
+    PickFilter filter;
 };
 
 namespace {
@@ -234,11 +240,11 @@ int launch_router(const coli_moe_desc& d, const void* x, coli_dtype xt, int T, f
     return check_launch("router");
 }
 
-int launch_topk(const coli_moe_desc& d, const float* zpart, int KS, int T, int32_t* idx,
-                float* w, cudaStream_t st) {
+int launch_topk(const coli_moe_desc& d, const PickFilter& f, const float* zpart, int KS, int T,
+                int32_t* idx, float* w, cudaStream_t st) {
     const int smem = kTopkWarps * 2 * d.E * 4;
     topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, 32 * kTopkWarps, smem, st>>>(
-        zpart, KS, T, d.E, d.router_b, d.k, d.routed_scale, d.norm_topk, idx, w);
+        zpart, KS, T, d.E, d.router_b, d.k, d.routed_scale, d.norm_topk, f, idx, w);
     return check_launch("topk");
 }
 
@@ -255,17 +261,17 @@ int launch_union(const int32_t* idx, int T, int k, int E, const UnionOut& o, cud
 }
 
 // top-k + union; one fused single-CTA launch for small batches
-int launch_select(const coli_moe_desc& d, const float* zpart, int KS, int T, int32_t* idx,
-                  float* w, const UnionOut& o, cudaStream_t st) {
+int launch_select(const coli_moe_desc& d, const PickFilter& f, const float* zpart, int KS, int T,
+                  int32_t* idx, float* w, const UnionOut& o, cudaStream_t st) {
     if (T * d.E <= kSmallSelect && T <= kSmallSelect / 32) {
         const int smem = std::max(2 * T * d.E * 4, union_smem_bytes(T, d.E));
         int rc = set_smem((const void*)topk_union_kernel, smem);
         if (rc) return rc;
         topk_union_kernel<<<1, kUnionThreads, smem, st>>>(zpart, KS, T, d.E, d.router_b, d.k,
-                                                          d.routed_scale, d.norm_topk, idx, w, o);
+                                                          d.routed_scale, d.norm_topk, f, idx, w, o);
         return check_launch("topk+union");
     }
-    int rc = launch_topk(d, zpart, KS, T, idx, w, st);
+    int rc = launch_topk(d, f, zpart, KS, T, idx, w, st);
     if (rc) return rc;
     return launch_union(idx, T, d.k, d.E, o, st);
 }
@@ -336,7 +342,7 @@ int gemm_grid() {
 template <typename Mark>
 int launch_gemm(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, cudaStream_t st,
                 Mark&& mark) {
-    const coli_moe_desc& d = l->d;
+    const coli_moe_desc& d = l->run;
     const int P = T * (d.k + d.n_shared);
     int rc;
     {
@@ -348,8 +354,7 @@ int launch_gemm(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, cudaS
     }
     if ((rc = set_smem((const void*)moe_gemm_kernel, kGemmSmem))) return rc;
     GemmArgs g;
-    g.experts = static_cast<const uint8_t*>(d.experts);
-    g.blob_bytes = l->L.bytes;
+    g.store = l->store;
     g.L = l->L;
     g.n_units = at<int32_t>(ws, p.n_units);
     g.unit_expert = at<int32_t>(ws, p.unit_expert);
@@ -408,10 +413,9 @@ int launch_down_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cuda
 template <typename Mark>
 int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const float* residual,
                 float* y, cudaStream_t st, Mark&& mark) {
-    const coli_moe_desc& d = l->d;
+    const coli_moe_desc& d = l->run;
     GemvArgs a;
-    a.experts = static_cast<const uint8_t*>(d.experts);
-    a.blob_bytes = l->L.bytes;
+    a.store = l->store;
     a.L = l->L;
     a.n_units = at<int32_t>(ws, p.n_units);
     a.unit_expert = at<int32_t>(ws, p.unit_expert);
@@ -468,11 +472,11 @@ int launch_fused_t(const CUtensorMap& xmap, const FusedArgs& a, cudaStream_t st)
 template <typename Mark>
 int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int KS,
                  const float* residual, float* y, cudaStream_t st, Mark&& mark) {
-    const coli_moe_desc& d = l->d;
+    const coli_moe_desc& d = l->run;
     FusedArgs a;
-    a.experts = static_cast<const uint8_t*>(d.experts);
-    a.blob_bytes = l->L.bytes;
+    a.store = l->store;
     a.L = l->L;
+    a.filter = l->filter;
     (void)KS;  // the small-batch router leaves one slice: the scores themselves
     a.score = at<float>(ws, p.zpart);
     a.sel = at<float>(ws, p.sel);
@@ -513,6 +517,7 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     CombineArgs c;
     c.part = a.part;
     c.w = a.w;
+    c.inv = a.inv;
     c.residual = residual;
     c.y = y;
     c.T = T; c.k = d.k; c.n_shared = d.n_shared; c.H = d.H; c.TG = d.I / 128;
@@ -768,7 +773,36 @@ int coli_moe_layer_create(const coli_moe_desc* desc, coli_moe_layer** out) {
     if (!l) return fail(COLI_E_NOMEM, "layer_create: out of host memory");
     l->d = d;
     l->L = make_blob_layout(d.H, d.I, d.group);
+    l->run = d;
+    const uint8_t* base = static_cast<const uint8_t*>(d.experts);
+    l->store = ExpertStore{base, base + (int64_t)d.E * l->L.bytes, l->L.bytes, 0, d.E};
+    l->filter = PickFilter{};
+    l->filter.e_hi = d.E;
     *out = l;
+    return COLI_OK;
+}
+
+int coli_moe_layer_set_topp(coli_moe_layer* layer, float p) {
+    if (!layer) return fail(COLI_E_INVAL, "set_topp: NULL layer");
+    if (!(p >= 0.0f && p <= 1.0f)) return fail(COLI_E_INVAL, "set_topp: p=%g outside [0, 1]", (double)p);
+    layer->filter.topp = p;
+    return COLI_OK;
+}
+
+int coli_moe_layer_set_partition(coli_moe_layer* layer, int32_t e_begin, int32_t e_end,
+                                 int32_t with_shared, const void* experts) {
+    if (!layer || !experts) return fail(COLI_E_INVAL, "set_partition: NULL pointer");
+    const coli_moe_desc& d = layer->d;
+    if (e_begin < 0 || e_end < e_begin || e_end > d.E)
+        return fail(COLI_E_INVAL, "set_partition: range [%d, %d) outside [0, %d)", e_begin, e_end, d.E);
+    const uint8_t* base = static_cast<const uint8_t*>(experts);
+    layer->run = d;
+    layer->run.experts = experts;
+    layer->run.n_shared = with_shared ? d.n_shared : 0;
+    layer->store = ExpertStore{base, base + (int64_t)(e_end - e_begin) * layer->L.bytes,
+                               layer->L.bytes, e_begin, d.E};
+    layer->filter.e_lo = e_begin;
+    layer->filter.e_hi = e_end;
     return COLI_OK;
 }
 
@@ -779,9 +813,9 @@ int coli_moe_layer_destroy(coli_moe_layer* layer) {
 
 int coli_moe_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes) {
     if (!layer || !bytes) return fail(COLI_E_INVAL, "workspace_size: NULL pointer");
-    int rc = tokens_ok(layer->d, T);
+    int rc = tokens_ok(layer->run, T);
     if (rc) return rc;
-    *bytes = (size_t)plan_ws(layer->d, T).total;
+    *bytes = (size_t)plan_ws(layer->run, T).total;
     return COLI_OK;
 }
 
@@ -789,16 +823,16 @@ int coli_moe_route(const coli_moe_layer* layer, const void* x, coli_dtype xt, in
                    int32_t* idx, float* w, void* ws, size_t ws_bytes, coli_stream_t stream) {
     if (!layer || !x || !idx || !w) return fail(COLI_E_INVAL, "route: NULL pointer");
     if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_E_INVAL, "route: bad dtype");
-    int rc = tokens_ok(layer->d, T);
+    int rc = tokens_ok(layer->run, T);
     if (rc) return rc;
-    const WsPlan p = plan_ws(layer->d, T);
+    const WsPlan p = plan_ws(layer->run, T);
     if (!ws || ws_bytes < (size_t)p.total)
         return fail(COLI_E_WORKSPACE, "route: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
     int KS;
     if ((rc = launch_router(layer->d, x, xt, T, at<float>(ws, p.zpart), nullptr, nullptr,
                             S(stream), &KS)))
         return rc;
-    return launch_topk(layer->d, at<float>(ws, p.zpart), KS, T, idx, w, S(stream));
+    return launch_topk(layer->d, PickFilter{}, at<float>(ws, p.zpart), KS, T, idx, w, S(stream));
 }
 
 int coli_moe_union(const int32_t* idx, int32_t T, int32_t k, int32_t E, int32_t* offsets,
@@ -824,7 +858,7 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     if (path != COLI_PATH_AUTO && path != COLI_PATH_GEMV && path != COLI_PATH_GEMM &&
         path != COLI_PATH_FUSED)
         return fail(COLI_E_INVAL, "forward: bad path");
-    const coli_moe_desc& d = layer->d;
+    const coli_moe_desc& d = layer->run;
     int rc = tokens_ok(d, T);
     if (rc) return rc;
     if (path == COLI_PATH_FUSED && !fused_fits(d, T))
@@ -894,8 +928,10 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     o.n_counters = d.H / 64;
     o.err = at<int32_t>(ws, p.err);
     o.n_shared = d.n_shared;
+    o.w = w;  // picks of weight 0 (not computed by this call) are left out
     if ((rc = mark(COLI_STAGE_UNION))) return rc;
-    if ((rc = launch_select(d, at<float>(ws, p.zpart), KS, T, idx, w, o, st))) return rc;
+    if ((rc = launch_select(d, layer->filter, at<float>(ws, p.zpart), KS, T, idx, w, o, st)))
+        return rc;
     if ((rc = mark(COLI_STAGE_GATEUP))) return rc;
     if (gemm) {
         if ((rc = launch_gemm(layer, T, ws, p, st, mark))) return rc;
@@ -1067,11 +1103,13 @@ int coli_moe_stack_forward_host(const coli_moe_layer* const* layers, int32_t L,
 int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t which,
                            float* out, coli_stream_t stream) {
     if (!layer || !out) return fail(COLI_E_INVAL, "dequant_debug: NULL pointer");
-    const coli_moe_desc& d = layer->d;
-    if (expert < 0 || expert >= d.E + d.n_shared || which < 0 || which > 2)
+    const coli_moe_desc& d = layer->run;
+    const bool routed_here = expert >= layer->filter.e_lo && expert < layer->filter.e_hi;
+    const bool shared_here = expert >= d.E && expert < d.E + d.n_shared;
+    if (!(routed_here || shared_here) || which < 0 || which > 2)
         return fail(COLI_E_INVAL, "dequant_debug: expert %d / matrix %d out of range", expert, which);
     const BlobLayout& L = layer->L;
-    const uint8_t* blob = static_cast<const uint8_t*>(d.experts) + (int64_t)expert * L.bytes;
+    const uint8_t* blob = layer->store.blob(expert);
     const int R = L.rows[which], K = L.cols[which];
     const int64_t n = (int64_t)R * K;
     dequant_kernel<<<(unsigned)((n + 255) / 256), 256, 0, S(stream)>>>(
@@ -1083,14 +1121,14 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t 
 int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws, int32_t* flags,
                     coli_stream_t stream) {
     if (!layer || !flags) return fail(COLI_E_INVAL, "status: NULL pointer");
-    int rc = tokens_ok(layer->d, T);
+    int rc = tokens_ok(layer->run, T);
     if (rc) return rc;
     if (!ws) {  // the built-in scratch array of coli_moe_forward_noalloc
         void* scratch = nullptr;
         if ((rc = noalloc_scratch(&scratch))) return rc;
         ws = scratch;
     }
-    const WsPlan p = plan_ws(layer->d, T);
+    const WsPlan p = plan_ws(layer->run, T);
     cudaStream_t st = S(stream);
     if (cudaMemcpyAsync(flags, static_cast<const char*>(ws) + p.err, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
@@ -1103,15 +1141,15 @@ int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws, int3
 int coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x, coli_dtype xt,
                              int32_t T, float* y, coli_stream_t stream) {
     if (!layer || !x || !y) return fail(COLI_E_INVAL, "forward_noalloc: NULL pointer");
-    int rc = tokens_ok(layer->d, T);
+    int rc = tokens_ok(layer->run, T);
     if (rc) return rc;
     // the path AUTO would take if its workspace fits the array, else the
     // GEMV/GEMM path, whose workspace is a prefix of the full one
     coli_path path = COLI_PATH_AUTO;
-    int64_t need = plan_ws(layer->d, T, true).total;
+    int64_t need = plan_ws(layer->run, T, true).total;
     if (need > (int64_t)COLI_NOALLOC_SCRATCH_BYTES) {
-        path = gemm_path_preferred(layer->d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV;
-        need = plan_ws(layer->d, T, false).total;
+        path = gemm_path_preferred(layer->run, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV;
+        need = plan_ws(layer->run, T, false).total;
     }
     if (need > (int64_t)COLI_NOALLOC_SCRATCH_BYTES)
         return fail(COLI_E_UNSUPPORTED,

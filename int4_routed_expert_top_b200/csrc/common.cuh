@@ -66,6 +66,65 @@ __host__ __device__ inline BlobLayout make_blob_layout8(int H, int I, int group)
     return L;
 }
 
+// Where the blobs of a layer's experts sit in device memory: routed expert e
+// (e_lo <= e < E) at routed + (e - e_lo) * bytes, shared expert s at shared +
+// s * bytes.  A whole layer has e_lo = 0 and shared = routed + E * bytes; a
+// handle restricted to an expert range (expert parallelism) holds only that
+// range's blobs, then its shared experts, if any.
+struct ExpertStore {
+    const uint8_t* routed;
+    const uint8_t* shared;
+    int64_t bytes;
+    int e_lo, E;
+    __host__ __device__ __forceinline__ const uint8_t* blob(int e) const {
+        return e < E ? routed + (int64_t)(e - e_lo) * bytes : shared + (int64_t)(e - E) * bytes;
+    }
+};
+
+// Which routed picks a call computes.  Adaptive top-p ("colibrì 實戰指南" 三 and
+// 五, `--topp`; the pages give no rule, so: keep the shortest run of the
+// largest renormalised weights w_j / sum(w), equal weights to the lower expert
+// index, whose total reaches p, at least one pick) when 0 < topp <= 1; then
+// only experts e_lo <= e < e_hi (expert parallelism).  A pick not computed gets
+// weight 0 and adds nothing to y.
+struct PickFilter {
+    float topp = 0.0f;  // outside (0, 1]: every pick
+    int e_lo = 0, e_hi = 1 << 30;
+};
+
+// Lane j < k holds pick j (weight w, expert e) of one token; every lane of the
+// warp takes part.  Returns whether lane j's pick is computed (false for lanes
+// >= k).  The top-p rule runs in double, with the weights in the order of the
+// rule and the same divisions as its plain statement, so that the decision
+// equals a double-precision evaluation of the rule on the same f32 weights.
+__device__ __forceinline__ bool pick_kept(const PickFilter& f, int k, float w, int e) {
+    const int lane = threadIdx.x & 31;
+    const bool mine = lane < k;
+    bool keep = mine;
+    if (f.topp > 0.0f && f.topp <= 1.0f) {
+        double tot = 0.0;  // in pick order
+        for (int j = 0; j < k; ++j) tot += (double)__shfl_sync(0xffffffffu, w, j);
+        int rank = 0;      // position in (w descending, expert ascending)
+        for (int j = 0; j < k; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            const int ej = __shfl_sync(0xffffffffu, e, j);
+            rank += (wj > w || (wj == w && ej < e)) ? 1 : 0;
+        }
+        const double p = (double)f.topp;
+        double mass = 0.0;
+        bool kept = false;
+        for (int r = 0; r < k; ++r) {
+            const unsigned who = __ballot_sync(0xffffffffu, mine && rank == r);
+            const float wr = __shfl_sync(0xffffffffu, w, __ffs(who) - 1);
+            const bool take = r == 0 || mass < p;  // decided before adding pick r
+            if (mine && rank == r) kept = take;
+            mass += tot > 0.0 ? (double)wr / tot : 0.0;
+        }
+        keep = mine && kept;
+    }
+    return keep && e >= f.e_lo && e < f.e_hi;
+}
+
 // 8-bit fragment tiles: 16-row x 64-column blocks ordered [R/128][K/64][8][32
 // lanes] as for 4-bit codes, 32 bytes per lane: for each 32-column half h of
 // the step, four words i = 0..3 that are the lane's mma.sync m16n8k32 s8 A

@@ -74,9 +74,9 @@ __host__ __device__ constexpr int fz_rec_bytes(int ns) { return ns * 128 + 64; }
 __host__ __device__ inline int fz_ns_gateup(int) { return 4; }
 
 struct FusedArgs {
-    const uint8_t* experts;
-    int64_t blob_bytes;
+    ExpertStore store;
     BlobLayout L;
+    PickFilter filter;      // picks this call computes (top-p, expert range)
     const float* score;     // [T][E] sigmoid scores s (router kernel)
     const float* sel;       // [T][E] selection scores s + bias (router kernel)
     float routed_scale;
@@ -86,8 +86,8 @@ struct FusedArgs {
     float* part;            // [T][k + n_shared][I/128][H] partial down products
     int32_t* queue;         // work-item counter, zeroed by the router kernel
     int32_t* idx;           // [T*k] picks (written by CTA 0)
-    float* w;               // [T*k] weights
-    int32_t* inv;           // [T*k] pair of (t, j)
+    float* w;               // [T*k] weights as applied (0: pick not computed)
+    int32_t* inv;           // [T*k] pair of (t, j), -1 for a pick not computed
     int32_t* err;
     int T, E, k, n_shared, H, I, group;
     int slots;              // ring stages
@@ -145,7 +145,9 @@ struct FusedShared {
     float wmax[8][kFzChunk];                      // per-warp max |h| of each pair
     __align__(16) int8_t hbuf[kFzChunk * kFzRecH]; // h of the current item, s8 digits
     int pick1_e[kFzMaxK];                         // one token: its picks (outside the ring,
-    float pick1_w[kFzMaxK];                       // which fills while they are read)
+    float pick1_w[kFzMaxK];                       // which fills while they are read),
+    int unit1_e[kFzMaxK];                         // the computed ones in slot order
+    int n_kept1;                                  // and their number
     int n_uniq, n_items;
 };
 
@@ -156,7 +158,9 @@ struct FzScratch {
     unsigned long long* bits;
     int* excl;
     int* pick_e;
-    float* pick_w;
+    float* pick_w;           // weight as applied: 0 for a pick this call does not compute
+    int* unit_e = nullptr;   // one token: computed picks' experts, compacted (or nullptr)
+    int* n_kept = nullptr;
 };
 __device__ __forceinline__ FzScratch fz_scratch(uint8_t* ring, int E) {
     FzScratch r;
@@ -215,9 +219,17 @@ __device__ __forceinline__ void fz_topk_token(const FusedArgs& a, int t, const F
     }
     float denom = 0.0f;  // over the picks in pick order
     for (int j = 0; j < a.k; ++j) denom += __shfl_sync(0xffffffffu, mine, j);
+    const float wgt = (a.norm_topk ? mine / denom : mine) * a.routed_scale;
+    // computed: kept by the pick filter and with a weight that can add something
+    const bool kept = pick_kept(a.filter, a.k, wgt, mine_e) && wgt != 0.0f;
     if (lane < a.k) {
         sc8.pick_e[t * a.k + lane] = mine_e;
-        sc8.pick_w[t * a.k + lane] = (a.norm_topk ? mine / denom : mine) * a.routed_scale;
+        sc8.pick_w[t * a.k + lane] = kept ? wgt : 0.0f;
+    }
+    if (sc8.unit_e) {
+        const unsigned km = __ballot_sync(0xffffffffu, kept);
+        if (kept) sc8.unit_e[__popc(km & ((1u << lane) - 1u))] = mine_e;
+        if (lane == 0) *sc8.n_kept = __popc(km);
     }
 }
 
@@ -232,9 +244,10 @@ __device__ __forceinline__ void fz_union_warp(const FusedArgs& a, FusedShared& s
                                               const FzScratch& sc8) {
     const int lane = threadIdx.x & 31;
     const int Tk = a.T * a.k, TG = a.I / 128;
-    const bool valid = lane < Tk;
-    const int e = valid ? sc8.pick_e[lane] : 0;
-    const int t = valid ? lane / a.k : 0;
+    const bool pick = lane < Tk;
+    const bool valid = pick && sc8.pick_w[lane] != 0.0f;  // a pick this call computes
+    const int e = pick ? sc8.pick_e[lane] : 0;
+    const int t = pick ? lane / a.k : 0;
     const unsigned lt = (1u << lane) - 1u;
     const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1);  // idle lanes: one group
     const bool first = valid && (same & lt) == 0u;
@@ -264,11 +277,11 @@ __device__ __forceinline__ void fz_union_warp(const FusedArgs& a, FusedShared& s
     if (valid) {
         sh.pair_tok[p] = t;
         sh.pair_pick[p] = t * (a.k + a.n_shared) + (lane - t * a.k);
-        if (blockIdx.x == 0) {
-            a.idx[lane] = e;
-            a.w[lane] = sc8.pick_w[lane];
-            a.inv[lane] = p;
-        }
+    }
+    if (pick && blockIdx.x == 0) {
+        a.idx[lane] = e;
+        a.w[lane] = sc8.pick_w[lane];
+        a.inv[lane] = valid ? p : -1;
     }
     const int per_shared = (a.T + kFzChunk - 1) / kFzChunk * TG;
     if (lane < a.n_shared) {
@@ -308,6 +321,7 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
         return sh.n_uniq + a.n_shared;
     }
     for (int i = threadIdx.x; i < Tk; i += kFzThreads) {
+        if (sc8.pick_w[i] == 0.0f) continue;  // not computed by this call
         const int e = sc8.pick_e[i];
         atomicAdd(&sc8.cnt[e], 1);
         atomicOr(&sc8.bits[e], 1ull << (i / a.k));
@@ -359,13 +373,16 @@ __device__ __forceinline__ int fz_route_union(const FusedArgs& a, FusedShared& s
     const int nu = sh.n_uniq;
     for (int i = threadIdx.x; i < Tk; i += kFzThreads) {
         const int t = i / a.k, e = sc8.pick_e[i];
+        const bool valid = sc8.pick_w[i] != 0.0f;
         const int p = sc8.excl[e] + __popcll(sc8.bits[e] & ((1ull << t) - 1ull));
-        sh.pair_tok[p] = t;
-        sh.pair_pick[p] = t * (a.k + a.n_shared) + (i - t * a.k);
+        if (valid) {
+            sh.pair_tok[p] = t;
+            sh.pair_pick[p] = t * (a.k + a.n_shared) + (i - t * a.k);
+        }
         if (blockIdx.x == 0) {
             a.idx[i] = e;
             a.w[i] = sc8.pick_w[i];
-            a.inv[i] = p;
+            a.inv[i] = valid ? p : -1;
         }
     }
     for (int s = threadIdx.x; s < a.n_shared; s += kFzThreads) {
@@ -478,9 +495,10 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
                                            FusedShared& sh, uint8_t* ring, int n_units, bool one) {
     const int lane = threadIdx.x & 31;
     const FzShape z = fz_shape(a);
-    // one token: unit u = item / TG is pick u (slot order), then the shared
-    // experts, one pair each (pair u, token 0); no tables needed
+    // one token: unit u = item / TG is the u-th computed pick (slot order),
+    // then the shared experts, one pair each (token 0); no tables needed
     const int n_items = one ? n_units * z.TG : sh.n_items;
+    const int n_kept = n_units - a.n_shared;
     const int rec_gu = fz_rec_bytes(z.ns_gu);
     const int ngH = GS ? a.H / 64 : 1, ngI = GS ? a.I / 64 : 1;
     const uint64_t pol = l2_evict_first_policy();
@@ -496,13 +514,13 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
             wk.tc = item - wk.u * z.TG;
             wk.p0 = wk.u;
             wk.np = 1;
-            e = wk.u < a.k ? sh.pick1_e[wk.u] : a.E + (wk.u - a.k);
+            e = wk.u < n_kept ? sh.unit1_e[wk.u] : a.E + (wk.u - n_kept);
         } else {
             wk = fz_work(sh, n_units, z.TG, item);
             e = sh.u_exp[wk.u];
         }
         const int tc = wk.tc, p0 = wk.p0, np = wk.np;
-        const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
+        const uint8_t* blob = a.store.blob(e);
         const uint8_t* cG = blob + a.L.codes[0];
         const uint8_t* cU = blob + a.L.codes[1];
         const uint8_t* cD = blob + a.L.codes[2];
@@ -909,10 +927,10 @@ moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
         // 0 and the producer), so it starts streaming while warp 0 writes the
         // unit and pair tables for the consumer warps (named barrier 1).
         __syncthreads();  // barrier initialisation, before any wait on them
-        const int n_units = a.k + a.n_shared;  // the k picks are distinct experts
         if (warp == kFzProducer) {
             asm volatile("bar.sync 2, %0;" ::"n"(64) : "memory");
-            fz_produce<GS>(a, &xmap, sh, fz_smem, n_units, true);
+            // the computed picks are distinct experts: one unit each
+            fz_produce<GS>(a, &xmap, sh, fz_smem, sh.n_kept1 + a.n_shared, true);
             return;
         }
         if (warp == 0) {
@@ -920,13 +938,15 @@ moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
             one.bits = nullptr; one.cnt = nullptr; one.excl = nullptr;
             one.pick_e = sh.pick1_e;
             one.pick_w = sh.pick1_w;
+            one.unit_e = sh.unit1_e;
+            one.n_kept = &sh.n_kept1;
             fz_topk_token(a, 0, one);
             __syncwarp();
             asm volatile("bar.arrive 2, %0;" ::"n"(64) : "memory");
             fz_union_warp(a, sh, one);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kFzWarps) : "memory");
-        fz_consume<NT, GS>(a, sh, fz_smem, n_units);
+        fz_consume<NT, GS>(a, sh, fz_smem, sh.n_uniq + a.n_shared);
         return;
     }
     const int n_units = fz_route_union(a, sh, fz_smem);
@@ -945,6 +965,7 @@ constexpr int kCombineMaxTiles = 32;  // I <= 4096
 struct CombineArgs {
     const float* part;     // [T][k + n_shared][TG][H]
     const float* w;        // [T*k]
+    const int32_t* inv;    // [T*k], < 0 for a pick the fused kernel did not compute
     const float* residual; // [T][H] or nullptr
     float* y;              // [T][H]
     int T, k, n_shared, H, TG;
@@ -963,6 +984,7 @@ moe_combine_kernel(CombineArgs c) {
     const int t = blockIdx.x / nrg, r = (blockIdx.x - t * nrg) * 32 + lane;
     const int J = c.k + c.n_shared;
     for (int j = warp; j < J; j += nw) {
+        if (j < c.k && __ldcg(c.inv + t * c.k + j) < 0) continue;  // not computed: adds nothing
         const float* src = c.part + ((int64_t)t * J + j) * c.TG * c.H + r;
         float pv[kCombineMaxTiles];
 #pragma unroll
@@ -977,7 +999,8 @@ moe_combine_kernel(CombineArgs c) {
     __syncthreads();
     if (warp == 0) {
         float acc = 0.0f;
-        for (int j = 0; j < c.k; ++j) acc += oj[j][lane];
+        for (int j = 0; j < c.k; ++j)
+            if (__ldcg(c.inv + t * c.k + j) >= 0) acc += oj[j][lane];
         for (int s = 0; s < c.n_shared; ++s) acc += oj[c.k + s][lane];
         if (c.residual) acc = c.residual[(int64_t)t * c.H + r] + acc;
         c.y[(int64_t)t * c.H + r] = acc;

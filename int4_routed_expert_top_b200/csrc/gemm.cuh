@@ -58,8 +58,7 @@ static_assert(kStageBytes % 1024 == 0, "stages must stay 1 KB aligned for the sw
 constexpr uint32_t kTmemCols = 512;
 
 struct GemmArgs {
-    const uint8_t* experts;
-    int64_t blob_bytes;
+    ExpertStore store;
     BlobLayout L;
     DecodeK dk;
     const int32_t* n_units;
@@ -242,7 +241,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
         int u = 0;
         int p0, n, rt;
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x) {
-            const uint8_t* blob = a.experts + (int64_t)a.unit_expert[cur.u] * a.blob_bytes;
+            const uint8_t* blob = a.store.blob(a.unit_expert[cur.u]);
             const uint8_t* c0 = blob + a.L.codes[mA];
             const uint8_t* c1 = blob + a.L.codes[1];
             const float* s0 = reinterpret_cast<const float*>(blob + a.L.scales[mA]);
@@ -322,7 +321,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x, ++tcount) {
             const int buf = tcount & 1;
             const int row = rt * kTileRows + 32 * q + lane;
-            const uint8_t* blob = a.experts + (int64_t)a.unit_expert[cur.u] * a.blob_bytes;
+            const uint8_t* blob = a.store.blob(a.unit_expert[cur.u]);
             const float srow0 = a.group ? 1.0f
                 : __ldg(reinterpret_cast<const float*>(blob + a.L.scales[mA]) + scale_offset(row, 0, 1));
             const float srow1 = (a.group || !a.two) ? 1.0f
@@ -480,6 +479,7 @@ combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ inv,
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
         const int p = inv[(int64_t)t * k + j];
+        if (p < 0) continue;  // a pick this call does not compute
         const float wj = w[(int64_t)t * k + j];
         const float4 v = *reinterpret_cast<const float4*>(o + (int64_t)p * H + c);
         acc.x = fmaf(wj, v.x, acc.x); acc.y = fmaf(wj, v.y, acc.y);

@@ -40,8 +40,7 @@ constexpr int kGemvMaxNT = 2;   // up to 2 column groups of 8: 8 tokens per pass
 constexpr int kDownSplit = 2;   // the down reduction is split in halves
 
 struct GemvArgs {
-    const uint8_t* experts;
-    int64_t blob_bytes;
+    ExpertStore store;
     BlobLayout L;
     DecodeK dk;
     const int32_t* n_units;
@@ -288,7 +287,7 @@ gateup_gemv_kernel(GemvArgs a) {
     const int u = blockIdx.x / nrb, rb64 = blockIdx.x % nrb;
     if (u >= *a.n_units) return;
     const int e = a.unit_expert[u], p0 = a.unit_begin[u], p1 = a.unit_end[u];
-    const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
+    const uint8_t* blob = a.store.blob(e);
     const uint8_t* codesA = blob + a.L.codes[0];
     const uint8_t* codesB = blob + a.L.codes[1];
     const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[0]);
@@ -409,9 +408,19 @@ down_gemv_kernel(GemvArgs a) {
     const int rem = blockIdx.x % (nrb * kDownSplit);
     const int rb64 = rem / kDownSplit, half = rem % kDownSplit;
     const int n_units = *a.n_units;
-    if (u >= n_units) return;
+    if (u >= n_units) {
+        if (n_units == 0 && u == 0 && half == 0) {
+            // nothing to compute for this call (every pick elsewhere, no shared
+            // expert): y of this 64-row block is the residual, or zero
+            for (int q = threadIdx.x; q < a.T * 64; q += blockDim.x) {
+                const int64_t o = (int64_t)(q / 64) * a.H + rb64 * 64 + q % 64;
+                a.y[o] = a.residual ? a.residual[o] : 0.0f;
+            }
+        }
+        return;
+    }
     const int e = a.unit_expert[u], p0 = a.unit_begin[u], p1 = a.unit_end[u];
-    const uint8_t* blob = a.experts + (int64_t)e * a.blob_bytes;
+    const uint8_t* blob = a.store.blob(e);
     const uint8_t* codesA = blob + a.L.codes[2];
     const float* sA = reinterpret_cast<const float*>(blob + a.L.scales[2]);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -477,6 +486,7 @@ down_gemv_kernel(GemvArgs a) {
         float acc = 0.0f;
         for (int j = 0; j < a.k; ++j) {
             const int p = __ldcg(a.inv + (int64_t)tt * a.k + j);
+            if (p < 0) continue;  // a pick this call does not compute
             acc = fmaf(__ldcg(a.w + (int64_t)tt * a.k + j), __ldcg(a.o + (int64_t)p * a.H + r), acc);
         }
         for (int s = 0; s < a.n_shared; ++s)

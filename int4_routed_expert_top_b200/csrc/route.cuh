@@ -426,7 +426,8 @@ router_tiled_kernel(const XT* __restrict__ x, int T, int H, const float* __restr
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void topk_token(const float* __restrict__ zpart, int KS, int T, int E,
                                            const float* __restrict__ bias, int k,
-                                           float routed_scale, int norm_topk, int t, float* sel,
+                                           float routed_scale, int norm_topk,
+                                           const PickFilter& filter, int t, float* sel,
                                            float* sc, int32_t* __restrict__ idx,
                                            float* __restrict__ w) {
     const int lane = threadIdx.x & 31;
@@ -466,9 +467,11 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ zpart, int 
     }
     float denom = 0.0f;  // renormalise over the k picks in pick order
     for (int j = 0; j < k; ++j) denom += __shfl_sync(0xffffffffu, mine, j);
+    const float wgt = (norm_topk ? mine / denom : mine) * routed_scale;
+    const bool kept = pick_kept(filter, k, wgt, mine_e);  // weight 0: not computed
     if (lane < k) {
         idx[(int64_t)t * k + lane] = mine_e;
-        w[(int64_t)t * k + lane] = (norm_topk ? mine / denom : mine) * routed_scale;
+        w[(int64_t)t * k + lane] = kept ? wgt : 0.0f;
     }
 }
 
@@ -477,13 +480,13 @@ constexpr int kTopkWarps = 4;
 __global__ void __launch_bounds__(32 * kTopkWarps)
 topk_kernel(const float* __restrict__ zpart, int KS, int T, int E,
             const float* __restrict__ bias, int k, float routed_scale, int norm_topk,
-            int32_t* __restrict__ idx, float* __restrict__ w) {
+            PickFilter filter, int32_t* __restrict__ idx, float* __restrict__ w) {
     extern __shared__ float tk_smem[];
     const int warp = threadIdx.x >> 5;
     const int t = blockIdx.x * kTopkWarps + warp;
     if (t >= T) return;
     float* sel = tk_smem + (int64_t)warp * 2 * E;
-    topk_token(zpart, KS, T, E, bias, k, routed_scale, norm_topk, t, sel, sel + E, idx, w);
+    topk_token(zpart, KS, T, E, bias, k, routed_scale, norm_topk, filter, t, sel, sel + E, idx, w);
 }
 
 // ---------------------------------------------------------------------------
@@ -509,6 +512,8 @@ struct UnionOut {
     int32_t n_counters;
     int32_t* err;          // device error flags to clear, or nullptr
     int32_t n_shared;
+    const float* w = nullptr;  // [T*k] pick weights: a pick of weight 0 is left out
+                               //   (inv = -1), or nullptr: every pick
 };
 
 constexpr int kUnionThreads = 1024;
@@ -531,7 +536,7 @@ __device__ __forceinline__ void union_body(const int32_t* idx, int T, int k, int
     const int P = T * k;
     for (int i = tid; i < P; i += kUnionThreads) {
         const int e = idx[i];
-        if (e < 0 || e >= E) continue;
+        if (e < 0 || e >= E || (o.w && o.w[i] == 0.0f)) continue;
         const int t = i / k;
         atomicAdd(&cnt[e], 1);
         atomicOr(&bits[(int64_t)e * W + t / 32], 1u << (t % 32));
@@ -579,7 +584,10 @@ __device__ __forceinline__ void union_body(const int32_t* idx, int T, int k, int
     __syncthreads();
     for (int i = tid; i < P; i += kUnionThreads) {
         const int e = idx[i];
-        if (e < 0 || e >= E) continue;
+        if (e < 0 || e >= E || (o.w && o.w[i] == 0.0f)) {
+            if (o.inv) o.inv[i] = -1;
+            continue;
+        }
         const int t = i / k, j = i % k;
         const uint32_t* row = bits + (int64_t)e * W;
         int rank = __popc(row[t / 32] & ((1u << (t % 32)) - 1u));
@@ -588,6 +596,14 @@ __device__ __forceinline__ void union_body(const int32_t* idx, int T, int k, int
         o.pair_tok[p] = t;
         o.pair_slot[p] = j;
         if (o.inv) o.inv[i] = p;
+    }
+    if (o.w) {  // pairs left free by picks not computed: token 0, so that
+                // kernels sweeping every pair index read valid rows
+        const int used = excl[E - 1] + cnt[E - 1];
+        for (int p = used + tid; p < P; p += kUnionThreads) {
+            o.pair_tok[p] = 0;
+            o.pair_slot[p] = 0;
+        }
     }
     if (o.unit_expert) {
         for (int e = tid; e < E; e += kUnionThreads) {
@@ -625,7 +641,7 @@ constexpr int kSmallSelect = 4096;
 __global__ void __launch_bounds__(kUnionThreads)
 topk_union_kernel(const float* __restrict__ zpart, int KS, int T, int E,
                   const float* __restrict__ bias, int k, float routed_scale, int norm_topk,
-                  int32_t* idx, float* w, UnionOut o) {
+                  PickFilter filter, int32_t* idx, float* w, UnionOut o) {
     extern __shared__ uint32_t un_smem[];
     float* sc = reinterpret_cast<float*>(un_smem);  // [T][E] sigmoid scores
     float* sel = sc + T * E;                         // [T][E] selection scores
@@ -653,12 +669,19 @@ topk_union_kernel(const float* __restrict__ zpart, int KS, int T, int E,
         if (r < k) { pick_e[t][r] = e; pick_s[t][r] = sc[i]; }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < T * k; i += kUnionThreads) {
-        const int t = i / k, j = i - t * k;
-        float denom = 0.0f;  // in pick order
+    // one warp per token: weights (denominator in pick order), then the pick filter
+    for (int t = threadIdx.x >> 5; t < T; t += kUnionThreads / 32) {
+        const int j = threadIdx.x & 31;
+        float denom = 0.0f;
         for (int q = 0; q < k; ++q) denom += pick_s[t][q];
-        idx[i] = pick_e[t][j];
-        w[i] = (norm_topk ? pick_s[t][j] / denom : pick_s[t][j]) * routed_scale;
+        const float sj = j < k ? pick_s[t][j] : 0.0f;
+        const int ej = j < k ? pick_e[t][j] : 0;
+        const float wgt = (norm_topk ? sj / denom : sj) * routed_scale;
+        const bool kept = pick_kept(filter, k, wgt, ej);
+        if (j < k) {
+            idx[t * k + j] = ej;
+            w[t * k + j] = kept ? wgt : 0.0f;
+        }
     }
     __threadfence_block();
     __syncthreads();

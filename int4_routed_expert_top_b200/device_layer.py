@@ -8,8 +8,8 @@ import ctypes
 import numpy as np
 
 from . import (Desc, coli_moe_expert_bytes, coli_moe_layer_create, coli_moe_layer_destroy,
-               coli_moe_pack_expert, coli_moe_quantize, coli_moe_quantize_expert_device,
-               coli_moe_workspace_size)
+               coli_moe_layer_set_partition, coli_moe_pack_expert, coli_moe_quantize,
+               coli_moe_quantize_expert_device, coli_moe_workspace_size)
 
 
 class DeviceLayer:
@@ -24,28 +24,38 @@ class DeviceLayer:
 
     def __init__(self, H, I, E, k, n_shared, group, router_w, router_b, *,
                  expert_masters=None, container=None, routed_scale=1.0, norm_topk=True,
-                 device="cuda"):
+                 device="cuda", expert_range=None, with_shared=True):
+        """expert_range=(lo, hi): hold and compute only routed experts lo <= e < hi
+        (and the shared experts when with_shared), as one rank of an
+        expert-parallel layer (coli_moe_layer_set_partition)."""
         import torch
         self.H, self.I, self.E, self.k = H, I, E, k
         self.n_shared, self.group = n_shared, group
         self.routed_scale, self.norm_topk = routed_scale, norm_topk
         self.blob_bytes = coli_moe_expert_bytes(H, I, group)
-        n = E + n_shared
+        lo, hi = expert_range if expert_range is not None else (0, E)
+        self.expert_range = (lo, hi)
+        self.with_shared = with_shared or expert_range is None
+        ids = list(range(lo, hi)) + (list(range(E, E + n_shared)) if self.with_shared else [])
+        self.expert_ids = ids
         self.router_w = router_w.to(device=device, dtype=torch.float32).contiguous()
         self.router_b = router_b.to(device=device, dtype=torch.float32).contiguous()
-        self.experts = torch.empty((n, self.blob_bytes), dtype=torch.uint8, device=device)
-        for e in range(n):
+        self.experts = torch.empty((max(len(ids), 1), self.blob_bytes), dtype=torch.uint8,
+                                   device=device)
+        for slot, e in enumerate(ids):
             if expert_masters is not None:
                 g, u, d = expert_masters(e)
                 coli_moe_quantize_expert_device(H, I, group, g.contiguous(), u.contiguous(),
-                                                d.contiguous(), self.experts[e])
+                                                d.contiguous(), self.experts[slot])
             else:
                 blob = coli_moe_pack_expert(H, I, group, *container(e))
-                self.experts[e].copy_(torch.from_numpy(blob))
+                self.experts[slot].copy_(torch.from_numpy(blob))
         self.desc = Desc(H, I, E, k, n_shared, group, routed_scale, int(norm_topk),
                          self.router_w.data_ptr(), self.router_b.data_ptr(),
                          self.experts.data_ptr())
         self.handle = coli_moe_layer_create(self.desc)
+        if expert_range is not None:
+            coli_moe_layer_set_partition(self.handle, lo, hi, self.with_shared, self.experts)
 
     def workspace_bytes(self, T: int) -> int:
         return coli_moe_workspace_size(self.handle, T)
