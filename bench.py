@@ -124,7 +124,7 @@ def token_pool(wl, T, n_batches, rank, device):
     return x.contiguous()
 
 
-def build_layers(wl, device):
+def build_layers(wl, device, bits=4):
     import synth
     from int4_routed_expert_top_b200.device_layer import DeviceLayer
     layers = []
@@ -135,7 +135,7 @@ def build_layers(wl, device):
             wl.H, wl.I, wl.E, wl.k, wl.n_shared, wl.group, wr, b,
             expert_masters=lambda e, l=l: tuple(synth.expert_master(wl, l, t, e, device=device)
                                                 for t in mats),
-            routed_scale=wl.routed_scale, norm_topk=wl.norm_topk, device=device))
+            routed_scale=wl.routed_scale, norm_topk=wl.norm_topk, device=device, bits=bits))
     return layers
 
 
@@ -434,6 +434,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="override routed experts (small-footprint profiling layers)")
+    ap.add_argument("--bits", type=int, default=4, choices=(4, 8),
+                    help="bits per expert weight code (8: the 8-bit container, fused path)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: each rank holds E/N routed experts (rank 0 the "
                          "shared ones), one all-reduce of y per step")
@@ -473,7 +475,7 @@ def main():
     fused = args.path == "fused" or (
         args.path == "auto" and T <= 64 and T * (wl.k + wl.n_shared) <= 640 and wl.E <= 256
         and wl.k <= 32 and wl.n_shared <= 4 and wl.H % 256 == 0 and wl.I <= 4096)
-    layers = build_layers(wl, dev)
+    layers = build_layers(wl, dev, args.bits)
     L0 = layers[0]
     n_pool = 64 if T <= 16 else 2
     xpool = token_pool(wl, T, n_pool, rank, dev)
@@ -613,7 +615,7 @@ def main():
     cfg = {"workload": wl.name, "tokens_per_step": T, "hidden": wl.H, "experts": wl.E,
            "top_k": wl.k, "intermediate": wl.I, "shared": wl.n_shared,
            "scale_group": wl.group or "per-row", "layers": wl.layers,
-           "x_dtype": wl.x_dtype, "path": args.path,
+           "x_dtype": wl.x_dtype, "path": args.path, "weight_bits": args.bits,
            "l2": "256 MiB buffer written between timed steps (flush), not timed",
            "launch": "one CUDA graph per token slot, replayed",
            "e2e_launch": ("coli_moe_forward_host / coli_moe_stack_forward_host (pinned host x "
@@ -625,8 +627,8 @@ def main():
         weight_gbs = nbytes.sum() / (total_ms / 1e3) / 1e9
         ng_h = 1 if wl.group == 0 else wl.H // wl.group
         ng_i = 1 if wl.group == 0 else wl.I // wl.group
-        gu_bytes_unit = 2 * (wl.I * wl.H // 2 + wl.I * ng_h * 4)
-        dn_bytes_unit = wl.H * wl.I // 2 + wl.H * ng_i * 4
+        gu_bytes_unit = 2 * (wl.I * wl.H * args.bits // 8 + wl.I * ng_h * 4)
+        dn_bytes_unit = wl.H * wl.I * args.bits // 8 + wl.H * ng_i * 4
         units = uniq_slot[st_ms[:, -1].astype(int)] + wl.n_shared
         stage_mean = st_ms[:, :-1].mean(0)
         if fused:

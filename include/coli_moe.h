@@ -93,9 +93,9 @@ typedef enum coli_path {
     COLI_PATH_GEMM = 2,  /* tcgen05 grouped GEMM, fp16 operands, f32 accumulate */
     COLI_PATH_FUSED = 3  /* one persistent kernel for top-k, union and experts,
                             then a combine kernel (mma.sync s8, exact int32
-                            step sums); T <= 64, T * (k + n_shared) <= 640,
+                            sums per stage); T <= 64, T * (k + n_shared) <= 640,
                             E <= 256, k <= 32, n_shared <= 4, H a multiple
-                            of 256, I <= 4096                                 */
+                            of 256, I <= 4096; the only path of 8-bit layers */
 } coli_path;
 
 /* Thread-local description of the last error returned on this thread. */
@@ -158,14 +158,23 @@ int coli_moe_quantize8(const float* w, int64_t rows, int64_t cols, int32_t group
  * byte j of a word being its first column + j (the lane's mma.sync m16n8k32
  * s8 A registers).  coli_moe_pack_expert8
  * re-tiles host codes and scales (as written by coli_moe_quantize8) into a
- * host blob of coli_moe_expert_bytes8 bytes.  The expert kernels do not read
- * 8-bit blobs yet. */
+ * host blob of coli_moe_expert_bytes8 bytes.  A layer created with bits = 8
+ * reads such blobs on the fused path (the codes are the tensor-core operands
+ * as they are: no decode). */
 int coli_moe_expert_bytes8(int32_t H, int32_t I, int32_t group, size_t* bytes);
 int coli_moe_pack_expert8(int32_t H, int32_t I, int32_t group,
                           const int8_t* gate_codes, const float* gate_scales,
                           const int8_t* up_codes, const float* up_scales,
                           const int8_t* down_codes, const float* down_scales,
                           void* blob);
+
+/* Device-side 8-bit quantise + pack of one expert from f32 masters (as for
+ * coli_moe_quantize_expert_device): bit-identical to coli_moe_quantize8
+ * followed by coli_moe_pack_expert8.  Asynchronous. */
+int coli_moe_quantize_expert8_device(int32_t H, int32_t I, int32_t group,
+                                     const float* gate, const float* up,
+                                     const float* down, void* blob,
+                                     coli_stream_t stream);
 
 /* coli_moe_quantize_expert_device for an expert given as FP8 E4M3 codes with
  * one f32 scale per 128 x 128 block (the format of the checkpoint the int4
@@ -199,6 +208,9 @@ typedef struct coli_moe_desc {
     const float* router_w; /* device f32 [E, H]                              */
     const float* router_b; /* device f32 [E], selection bias                 */
     const void* experts;   /* device, (E + n_shared) blobs back to back      */
+    int32_t bits;          /* bits per weight code: 0 or 4 (int4 blobs of
+                              coli_moe_pack_expert), 8 (8-bit blobs of
+                              coli_moe_pack_expert8; fused path only)         */
 } coli_moe_desc;
 
 typedef struct coli_moe_layer coli_moe_layer;
@@ -233,6 +245,17 @@ int coli_moe_layer_set_topp(coli_moe_layer* layer, float p);
  * the restriction (no shared pairs when with_shared == 0).  Host-only. */
 int coli_moe_layer_set_partition(coli_moe_layer* layer, int32_t e_begin, int32_t e_end,
                                  int32_t with_shared, const void* experts);
+
+/* Test of the device-side bounded waits (no counterpart on the source pages):
+ * on later fused-path forwards of this layer, CTA 0's producer skips ring
+ * stage withhold_stage (0 = its first; < 0 = none), so nothing ever completes
+ * that stage and the consumer warps' wait on it gives up; every wait of the
+ * fused kernel gives up after wait_tries tries (0 = the default, about a
+ * second).  The call then returns normally, its outputs are invalid and
+ * coli_moe_status reports COLI_E_TIMEOUT; the next call without the option is
+ * unaffected.  Never needed in normal use.  Host-only. */
+int coli_moe_layer_set_wait_test(coli_moe_layer* layer, int32_t withhold_stage,
+                                 uint32_t wait_tries);
 
 /* Workspace bytes that coli_moe_route / coli_moe_forward need for T tokens
  * (enough for every path; the GEMV and GEMM paths use only a prefix). */

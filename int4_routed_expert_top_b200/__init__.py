@@ -42,6 +42,7 @@ EXPORTS = (
     "coli_moe_forward_host", "coli_moe_stack_host_workspace_size", "coli_moe_stack_forward_host",
     "coli_moe_quantize_expert_fp8_device", "coli_moe_quantize8", "coli_moe_expert_bytes8",
     "coli_moe_pack_expert8", "coli_moe_layer_set_topp", "coli_moe_layer_set_partition",
+    "coli_moe_quantize_expert8_device", "coli_moe_layer_set_wait_test",
 )
 
 
@@ -56,7 +57,8 @@ class Desc(ctypes.Structure):
                 ("k", ctypes.c_int32), ("n_shared", ctypes.c_int32),
                 ("group", ctypes.c_int32), ("routed_scale", ctypes.c_float),
                 ("norm_topk", ctypes.c_int32), ("router_w", ctypes.c_void_p),
-                ("router_b", ctypes.c_void_p), ("experts", ctypes.c_void_p)]
+                ("router_b", ctypes.c_void_p), ("experts", ctypes.c_void_p),
+                ("bits", ctypes.c_int32)]
 
 
 from . import build as _build  # noqa: E402
@@ -76,6 +78,7 @@ _SIGS = {
     "coli_moe_expert_bytes": ([_I32, _I32, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
     "coli_moe_pack_expert": ([_I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "coli_moe_quantize_expert_device": ([_I32, _I32, _I32, _P, _P, _P, _P, _P], ctypes.c_int),
+    "coli_moe_quantize_expert8_device": ([_I32, _I32, _I32, _P, _P, _P, _P, _P], ctypes.c_int),
     "coli_moe_quantize_expert_fp8_device": ([_I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P],
                                             ctypes.c_int),
     "coli_moe_quantize8": ([_P, _I64, _I64, _I32, _P, _P], ctypes.c_int),
@@ -84,6 +87,7 @@ _SIGS = {
     "coli_moe_layer_create": ([ctypes.POINTER(Desc), ctypes.POINTER(_P)], ctypes.c_int),
     "coli_moe_layer_destroy": ([_P], ctypes.c_int),
     "coli_moe_layer_set_topp": ([_P, ctypes.c_float], ctypes.c_int),
+    "coli_moe_layer_set_wait_test": ([_P, _I32, ctypes.c_uint32], ctypes.c_int),
     "coli_moe_layer_set_partition": ([_P, _I32, _I32, _I32, _P], ctypes.c_int),
     "coli_moe_workspace_size": ([_P, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
     "coli_moe_route": ([_P, _P, ctypes.c_int, _I32, _P, _P, _P, _SZ, _P], ctypes.c_int),
@@ -207,6 +211,11 @@ def coli_moe_quantize_expert_device(H, I, group, gate, up, down, blob, stream=No
                                             _ptr(blob), _stream(stream)))
 
 
+def coli_moe_quantize_expert8_device(H, I, group, gate, up, down, blob, stream=None):
+    _ok(lib.coli_moe_quantize_expert8_device(H, I, group, _ptr(gate), _ptr(up), _ptr(down),
+                                             _ptr(blob), _stream(stream)))
+
+
 def coli_moe_quantize_expert_fp8_device(H, I, group, gate, up, down, gate_bs, up_bs, down_bs,
                                         blob, stream=None):
     """FP8 E4M3 codes (uint8 device tensors) with 128 x 128 block scales -> int4 blob."""
@@ -223,6 +232,11 @@ def coli_moe_layer_create(desc: Desc) -> ctypes.c_void_p:
 
 def coli_moe_layer_destroy(layer) -> None:
     _ok(lib.coli_moe_layer_destroy(layer))
+
+
+def coli_moe_layer_set_wait_test(layer, withhold_stage: int, wait_tries: int) -> None:
+    """Test only: make the fused kernel's bounded waits run out (see the header)."""
+    _ok(lib.coli_moe_layer_set_wait_test(layer, withhold_stage, wait_tries))
 
 
 def coli_moe_layer_set_topp(layer, p: float) -> None:

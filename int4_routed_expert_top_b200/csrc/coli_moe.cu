@@ -23,6 +23,7 @@ using namespace coli;
 
 struct coli_moe_layer {
     coli_moe_desc d;       // as created
+    int bits;              // 4 or 8 (bits per weight code)
     BlobLayout L;
     // what a forward computes: d with n_shared = 0 on a handle restricted to a
     // range of routed experts without the shared ones; where the blobs sit;
@@ -30,6 +31,9 @@ struct coli_moe_layer {
     coli_moe_desc run;
     ExpertStore store;
     PickFilter filter;
+    // test of the bounded waits (coli_moe_layer_set_wait_test)
+    uint32_t wait_tries = kWaitTries;
+    int withhold = -1;
 };
 
 namespace {
@@ -460,13 +464,22 @@ int sm_count() { return gemm_grid(); }
 // the previous one (router, then fused) finishes; it waits
 // (griddepcontrol.wait) before reading what that kernel wrote.
 
-template <int NT, bool GS>
+template <int NT, bool GS, bool W8>
 int launch_fused_t(const CUtensorMap& xmap, const FusedArgs& a, cudaStream_t st) {
     const int smem = a.slots * a.slot_bytes;
-    int rc = set_smem((const void*)moe_fused_kernel<NT, GS>, smem);
+    int rc = set_smem((const void*)moe_fused_kernel<NT, GS, W8>, smem);
     if (rc) return rc;
-    return launch_pdl(moe_fused_kernel<NT, GS>, dim3(sm_count()), kFzThreads, smem, st, "fused moe",
-                      xmap, a);
+    return launch_pdl(moe_fused_kernel<NT, GS, W8>, dim3(sm_count()), kFzThreads, smem, st,
+                      "fused moe", xmap, a);
+}
+
+template <bool W8>
+int launch_fused_w(int NT, bool gs, const CUtensorMap& xmap, const FusedArgs& a, cudaStream_t st) {
+    switch (NT) {
+        case 1: return gs ? launch_fused_t<1, true, W8>(xmap, a, st) : launch_fused_t<1, false, W8>(xmap, a, st);
+        case 2: return gs ? launch_fused_t<2, true, W8>(xmap, a, st) : launch_fused_t<2, false, W8>(xmap, a, st);
+        default: return gs ? launch_fused_t<4, true, W8>(xmap, a, st) : launch_fused_t<4, false, W8>(xmap, a, st);
+    }
 }
 
 template <typename Mark>
@@ -477,6 +490,8 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     a.store = l->store;
     a.L = l->L;
     a.filter = l->filter;
+    a.wait_tries = l->wait_tries;
+    a.withhold = l->withhold;
     (void)KS;  // the small-batch router leaves one slice: the scores themselves
     a.score = at<float>(ws, p.zpart);
     a.sel = at<float>(ws, p.sel);
@@ -492,7 +507,7 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     a.T = T; a.E = d.E; a.k = d.k; a.n_shared = d.n_shared;
     a.H = d.H; a.I = d.I; a.group = d.group;
     const int NT = T <= 4 ? 1 : (T <= 8 ? 2 : 4);
-    a.slot_bytes = (int)align256(kFzActOff + 4 * NT * fz_rec_bytes(fz_ns_gateup(d.H)));
+    a.slot_bytes = (int)align256(kFzActOff + 4 * NT * kActRec);
     const int budget = 227 * 1024 - (int)sizeof(FusedShared) - 1024;
     a.slots = std::min(kFzSlots, budget / a.slot_bytes);
     if (a.slots < 2) return fail(COLI_E_UNSUPPORTED, "fused: ring does not fit");
@@ -506,11 +521,8 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
         if ((rc = encode_act_map(&xmap, a.xq8, T, d.H))) return rc;
         a.act_tma = 1;
     }
-    switch (NT) {
-        case 1: rc = gs ? launch_fused_t<1, true>(xmap, a, st) : launch_fused_t<1, false>(xmap, a, st); break;
-        case 2: rc = gs ? launch_fused_t<2, true>(xmap, a, st) : launch_fused_t<2, false>(xmap, a, st); break;
-        default: rc = gs ? launch_fused_t<4, true>(xmap, a, st) : launch_fused_t<4, false>(xmap, a, st); break;
-    }
+    rc = l->bits == 8 ? launch_fused_w<true>(NT, gs, xmap, a, st)
+                      : launch_fused_w<false>(NT, gs, xmap, a, st);
     if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;
     if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
@@ -737,6 +749,26 @@ int coli_moe_quantize_expert_device(int32_t H, int32_t I, int32_t group, const f
     return COLI_OK;
 }
 
+int coli_moe_quantize_expert8_device(int32_t H, int32_t I, int32_t group, const float* gate,
+                                     const float* up, const float* down, void* blob,
+                                     coli_stream_t stream) {
+    if (!gate || !up || !down || !blob) return fail(COLI_E_INVAL, "quantize_expert8_device: NULL pointer");
+    if (!shape_ok(H, I, group)) return fail(COLI_E_INVAL, "quantize_expert8_device: bad shape");
+    const BlobLayout L = make_blob_layout8(H, I, group);
+    uint8_t* b = static_cast<uint8_t*>(blob);
+    const float* src[3] = {gate, up, down};
+    for (int m = 0; m < 3; ++m) {
+        const int R = L.rows[m], K = L.cols[m];
+        const int smem = 16 * K;
+        int rc = set_smem((const void*)quantize_rows8_kernel<QzF32>, smem);
+        if (rc) return rc;
+        quantize_rows8_kernel<<<R / 16, 256, smem, S(stream)>>>(
+            QzF32{src[m]}, R, K, group, b + L.codes[m], reinterpret_cast<float*>(b + L.scales[m]));
+        if ((rc = check_launch("quantize_rows8"))) return rc;
+    }
+    return COLI_OK;
+}
+
 int coli_moe_quantize_expert_fp8_device(int32_t H, int32_t I, int32_t group, const uint8_t* gate,
                                         const uint8_t* up, const uint8_t* down, const float* gate_bs,
                                         const float* up_bs, const float* down_bs, void* blob,
@@ -769,16 +801,27 @@ int coli_moe_layer_create(const coli_moe_desc* desc, coli_moe_layer** out) {
         return fail(COLI_E_INVAL, "layer_create: need 1<=k<=min(E,32), E<=1024, 0<=n_shared<=4");
     if (!d.router_w || !d.router_b || !d.experts) return fail(COLI_E_INVAL, "layer_create: NULL device pointer");
     if (!(std::isfinite(d.routed_scale))) return fail(COLI_E_INVAL, "layer_create: routed_scale not finite");
+    if (d.bits != 0 && d.bits != 4 && d.bits != 8)
+        return fail(COLI_E_INVAL, "layer_create: bits must be 0 (4), 4 or 8, got %d", d.bits);
     coli_moe_layer* l = new (std::nothrow) coli_moe_layer;
     if (!l) return fail(COLI_E_NOMEM, "layer_create: out of host memory");
     l->d = d;
-    l->L = make_blob_layout(d.H, d.I, d.group);
+    l->bits = d.bits == 8 ? 8 : 4;
+    l->L = l->bits == 8 ? make_blob_layout8(d.H, d.I, d.group) : make_blob_layout(d.H, d.I, d.group);
     l->run = d;
     const uint8_t* base = static_cast<const uint8_t*>(d.experts);
     l->store = ExpertStore{base, base + (int64_t)d.E * l->L.bytes, l->L.bytes, 0, d.E};
     l->filter = PickFilter{};
     l->filter.e_hi = d.E;
     *out = l;
+    return COLI_OK;
+}
+
+int coli_moe_layer_set_wait_test(coli_moe_layer* layer, int32_t withhold_stage,
+                                 uint32_t wait_tries) {
+    if (!layer) return fail(COLI_E_INVAL, "set_wait_test: NULL layer");
+    layer->withhold = withhold_stage < 0 ? -1 : withhold_stage;
+    layer->wait_tries = wait_tries == 0 ? kWaitTries : wait_tries;
     return COLI_OK;
 }
 
@@ -865,6 +908,10 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         return fail(COLI_E_UNSUPPORTED,
                     "forward: fused path needs T<=%d, T*(k+n_shared)<=%d, E<=%d, k<=%d, n_shared<=4, "
                     "H%%256==0, I<=4096", kFzMaxT, kFzMaxPairs, kFzMaxE, kFzMaxK);
+    if (layer->bits == 8 && (path == COLI_PATH_GEMV || path == COLI_PATH_GEMM ||
+                             (path == COLI_PATH_AUTO && !fused_fits(d, T))))
+        return fail(COLI_E_UNSUPPORTED, "forward: 8-bit experts run on the fused path only (T<=%d, "
+                    "T*(k+n_shared)<=%d, E<=%d, H%%256==0, I<=4096)", kFzMaxT, kFzMaxPairs, kFzMaxE);
     if (path == COLI_PATH_AUTO)
         path = fused_fits(d, T) ? COLI_PATH_FUSED
                                 : (gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV);
@@ -1112,7 +1159,8 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t 
     const uint8_t* blob = layer->store.blob(expert);
     const int R = L.rows[which], K = L.cols[which];
     const int64_t n = (int64_t)R * K;
-    dequant_kernel<<<(unsigned)((n + 255) / 256), 256, 0, S(stream)>>>(
+    auto kern = layer->bits == 8 ? dequant8_kernel : dequant_kernel;
+    kern<<<(unsigned)((n + 255) / 256), 256, 0, S(stream)>>>(
         blob + L.codes[which], reinterpret_cast<const float*>(blob + L.scales[which]), R, K,
         d.group, out);
     return check_launch("dequant");

@@ -69,9 +69,12 @@ constexpr int kFzRecH = 320;                     // h record of a pair: 2 steps 
 // records are 64 bytes apart modulo 128 (conflict-free 16-byte shared loads).
 __host__ __device__ constexpr int fz_rec_bytes(int ns) { return ns * 128 + 64; }
 
-// Steps (64 columns) per gate/up stage (both matrices); the fused path needs
-// H to be a multiple of 256.
-__host__ __device__ inline int fz_ns_gateup(int) { return 4; }
+// Steps (64 columns) per gate/up stage (both matrices): 32 KB of codes, 4 steps
+// of 4-bit codes or 2 of 8-bit ones; the fused path needs H to be a multiple of
+// 256 (one activation record per 256 columns).
+template <bool W8> __host__ __device__ constexpr int fz_ns_gateup() { return W8 ? 2 : 4; }
+// code bytes of one 64-column step of a 128-row tile
+template <bool W8> __host__ __device__ constexpr int fz_step_bytes() { return W8 ? 8192 : 4096; }
 
 struct FusedArgs {
     ExpertStore store;
@@ -98,11 +101,18 @@ struct FusedArgs {
     // used for 2 <= T <= 4 (one column group).  0: one bulk copy per pair,
     // stored per pair record.
     int act_tma;
+    // bounded waits: tries before a wait gives up (kWaitTries normally); a
+    // test may also have CTA 0's producer withhold ring stage withhold (its
+    // copies are never issued, so the consumers' wait on it runs out), -1: none
+    uint32_t wait_tries;
+    int withhold;
 };
 
-// row tiles (of 128 H rows) per down stage: the largest of 4, 3, 2, 1 dividing H/128
-__host__ __device__ inline int fz_down_tiles(int H) {
+// row tiles (of 128 H rows) per down stage: the largest of 4, 3, 2, 1 dividing
+// H/128 (4-bit codes, 8 KB per tile) or of 2, 1 (8-bit codes, 16 KB per tile)
+__host__ __device__ inline int fz_down_tiles(int H, bool w8) {
     const int n = H / 128;
+    if (w8) return n % 2 == 0 ? 2 : 1;
     return n % 4 == 0 ? 4 : (n % 3 == 0 ? 3 : (n % 2 == 0 ? 2 : 1));
 }
 
@@ -433,9 +443,10 @@ __device__ __forceinline__ void mma_s8_16832_zc(int d[4], const uint32_t a[4], u
 
 // Warp-wide bounded wait on an mbarrier phase; every lane returns the result
 // and is ordered after lane 0's acquire.
-__device__ __forceinline__ bool fz_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
+__device__ __forceinline__ bool fz_wait(uint64_t* bar, uint32_t parity, int32_t* err,
+                                        uint32_t tries) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, tries) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
@@ -443,10 +454,11 @@ __device__ __forceinline__ bool fz_wait(uint64_t* bar, uint32_t parity, int32_t*
 
 // Barrier of the consumer warps on an mbarrier (count kFzWarps) with a bounded
 // wait, so that a failed warp cannot leave the others blocked for good.
-__device__ __forceinline__ bool fz_cbar(uint64_t* bar, uint32_t& phase, int32_t* err) {
+__device__ __forceinline__ bool fz_cbar(uint64_t* bar, uint32_t& phase, int32_t* err,
+                                        uint32_t tries) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-    const bool ok = fz_wait(bar, phase, err);
+    const bool ok = fz_wait(bar, phase, err, tries);
     phase ^= 1u;
     return ok;
 }
@@ -471,11 +483,12 @@ struct FzShape {
     int rs, nst_dn;      // 128-row tiles per down stage; down stages
     int TG;              // 128-row tiles of I (items per unit)
 };
+template <bool W8>
 __device__ __forceinline__ FzShape fz_shape(const FusedArgs& a) {
     FzShape z;
-    z.ns_gu = fz_ns_gateup(a.H);
+    z.ns_gu = fz_ns_gateup<W8>();
     z.nst_gu = a.H / 64 / z.ns_gu;
-    z.rs = fz_down_tiles(a.H);
+    z.rs = fz_down_tiles(a.H, W8);
     z.nst_dn = a.H / 128 / z.rs;
     z.TG = a.I / 128;
     return z;
@@ -484,22 +497,24 @@ __device__ __forceinline__ FzShape fz_shape(const FusedArgs& a) {
 // ---------------------------------------------------------------------------
 // Producer warp: claim items (u, tc), stream their stages, then the end marker.
 // Ring position: slot s, lap parity lap (flips whenever s wraps to 0).
-//   gate/up stage st: rows tc of gate and of up, steps 4 st .. 4 st + 3
-//     [codes gate | codes up | gs64 scales gate, up | x slices of the pairs]
-//     and, on the last one, the tile's per-row scales of gate and up;
+//   gate/up stage st: rows tc of gate and of up, steps ns st .. ns st + ns - 1
+//     [codes gate | codes up | gs64 scales gate, up | activation records of
+//     the pairs (the 256-column record holding these steps)] and, on the last
+//     one, the tile's per-row scales of gate and up;
 //   down stage: rs tiles of 128 H rows, columns 128 tc .. 128 tc + 127
-//     [codes, 8 KB per tile | scales (per row: 512 B per tile; gs64: 1 KB)].
+//     [codes, 8 or 16 KB per tile | scales (per row: 512 B per tile; gs64: 1 KB)].
 // ---------------------------------------------------------------------------
-template <bool GS>
+template <bool GS, bool W8>
 __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap* xmap,
                                            FusedShared& sh, uint8_t* ring, int n_units, bool one) {
     const int lane = threadIdx.x & 31;
-    const FzShape z = fz_shape(a);
+    const FzShape z = fz_shape<W8>(a);
+    constexpr uint32_t kStep = fz_step_bytes<W8>();
     // one token: unit u = item / TG is the u-th computed pick (slot order),
     // then the shared experts, one pair each (token 0); no tables needed
     const int n_items = one ? n_units * z.TG : sh.n_items;
     const int n_kept = n_units - a.n_shared;
-    const int rec_gu = fz_rec_bytes(z.ns_gu);
+    const int rec_gu = kActRec;
     const int ngH = GS ? a.H / 64 : 1, ngI = GS ? a.I / 64 : 1;
     const uint64_t pol = l2_evict_first_policy();
     int s = 0, issued = 0;
@@ -529,18 +544,24 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
         const float* sD = reinterpret_cast<const float*>(blob + a.L.scales[2]);
         const int nst = z.nst_gu + z.nst_dn;
         for (int st = 0; st < nst; ++st) {
-            if (issued >= a.slots && !fz_wait(&sh.empty[s], lap ^ 1u, a.err)) { ok = false; break; }
+            if (issued >= a.slots && !fz_wait(&sh.empty[s], lap ^ 1u, a.err, a.wait_tries)) {
+                ok = false;
+                break;
+            }
             if (lane == 0) { sh.meta_item[s] = item; sh.meta_st[s] = st; }
             __syncwarp();
             uint8_t* sl = ring + (int64_t)s * a.slot_bytes;
-            if (st < z.nst_gu) {
+            if (issued == a.withhold && blockIdx.x == 0) {
+                // nothing is copied and the stage's barrier never completes
+            } else if (st < z.nst_gu) {
                 const int kb0 = st * z.ns_gu;
+                const int rec = kb0 / 4;  // the activation record of these steps
                 const bool rowsc = !GS && st == z.nst_gu - 1;
-                const uint32_t cb = (uint32_t)z.ns_gu * 4096, sb = GS ? (uint32_t)z.ns_gu * 512 : 0u;
+                const uint32_t cb = (uint32_t)z.ns_gu * kStep, sb = GS ? (uint32_t)z.ns_gu * 512 : 0u;
                 const int nrec = a.act_tma ? a.T : np;  // activation records of the stage
                 mbar_expect_tx_elect(&sh.full[s], 2 * (cb + sb) + (uint32_t)(nrec * kActRec) +
                                                       (rowsc ? 1024u : 0u));
-                const int64_t coff = frag_unit_offset(tc, kb0, 0, 0, a.H);
+                const int64_t coff = (int64_t)tc * (a.H / 64) * kStep + (int64_t)kb0 * kStep;
                 bulk_g2s_hint_elect(sl, cG + coff, cb, &sh.full[s], pol);
                 bulk_g2s_hint_elect(sl + cb, cU + coff, cb, &sh.full[s], pol);
                 if (GS) {
@@ -553,23 +574,24 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
                     bulk_g2s_elect(sl + kFzScaleOff + 512, sU + (int64_t)tc * kTileRows, 512u, &sh.full[s]);
                 }
                 if (a.act_tma) {  // every token's record, [token][kActRec] (x in 4-byte units)
-                    tma_load_2d_elect(sl + kFzActOff, xmap, st * (kActRec / 4), 0, &sh.full[s]);
+                    tma_load_2d_elect(sl + kFzActOff, xmap, rec * (kActRec / 4), 0, &sh.full[s]);
                 } else {
                     for (int pp = 0; pp < np; ++pp) {
                         const int tok = one ? 0 : sh.pair_tok[p0 + pp];
                         bulk_g2s_elect(sl + kFzActOff + pp * rec_gu,
-                                       a.xq8 + ((int64_t)tok * (a.H / 256) + st) * kActRec,
+                                       a.xq8 + ((int64_t)tok * (a.H / 256) + rec) * kActRec,
                                        (uint32_t)kActRec, &sh.full[s]);
                     }
                 }
             } else {
                 const int rt0 = (st - z.nst_gu) * z.rs;
                 const uint32_t sb = GS ? 1024u : 512u;
-                mbar_expect_tx_elect(&sh.full[s], (uint32_t)z.rs * (8192u + sb));
+                mbar_expect_tx_elect(&sh.full[s], (uint32_t)z.rs * (2 * kStep + sb));
                 for (int q = 0; q < z.rs; ++q) {
                     const int rt = rt0 + q;
-                    bulk_g2s_hint_elect(sl + q * 8192, cD + frag_unit_offset(rt, 2 * tc, 0, 0, a.I),
-                                        8192u, &sh.full[s], pol);
+                    bulk_g2s_hint_elect(sl + q * 2 * kStep,
+                                        cD + (int64_t)rt * (a.I / 64) * kStep + (int64_t)2 * tc * kStep,
+                                        2 * kStep, &sh.full[s], pol);
                     if (GS)
                         bulk_g2s_elect(sl + kFzScaleOff + q * 1024,
                                        sD + ((int64_t)rt * ngI + 2 * tc) * kTileRows, 1024u, &sh.full[s]);
@@ -584,7 +606,7 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
         if (lane == 0) item = (int)gridDim.x + atomicAdd(a.queue, 1);
         item = __shfl_sync(0xffffffffu, item, 0);
     }
-    if (ok && (issued < a.slots || fz_wait(&sh.empty[s], lap ^ 1u, a.err))) {  // end marker
+    if (ok && (issued < a.slots || fz_wait(&sh.empty[s], lap ^ 1u, a.err, a.wait_tries))) {  // end marker
         if (lane == 0) sh.meta_item[s] = -1;
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.full[s]);
@@ -592,7 +614,7 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
     }
     // leave only once every copy issued into the ring has landed
     for (int j = issued > a.slots ? issued - a.slots : 0; j < issued; ++j)
-        fz_wait(&sh.full[j % a.slots], (j / a.slots) & 1, nullptr);
+        fz_wait(&sh.full[j % a.slots], (j / a.slots) & 1, nullptr, a.wait_tries);
 }
 
 }  // namespace coli
@@ -607,21 +629,37 @@ namespace coli {
 // lanes t and t ^ 2 hold the two digits of the same pairs.  The stage's sum
 // (exact int32 for per-row weight scales; with the weight scale of each step
 // for 64-column groups) is added to acc_f times the activation scale of its
-// pair's 256-column record, the lane's digit factor (256 for high digits) and
-// 1/16 (the nibble sits in the high half of an s8 byte).
-// xsoff[c][q]: offset of the activation record of pair 4c + 2(t & 1) + q.
+// pair's 256-column record, the lane's digit factor (256 for high digits) and,
+// for 4-bit codes, 1/16 (the nibble sits in the high half of an s8 byte).
+// xsoff[c][q]: offset of the activation record of pair 4c + 2(t & 1) + q; jo:
+// the first of the stage's steps within that record.
 // ---------------------------------------------------------------------------
 static_assert(fz_rec_bytes(4) == kActRec, "pair records of a stage are the global records");
 
-template <int NT, bool GS>
+// A registers of one 64-column step (both k32 halves) of one lane: 4-bit codes
+// are expanded to s8 in registers, 8-bit codes are the registers already
+template <bool W8>
+__device__ __forceinline__ void fz_load_step(const uint8_t* p, uint32_t A0[4], uint32_t A1[4]) {
+    if (W8) {
+        const uint4 u0 = *reinterpret_cast<const uint4*>(p);
+        const uint4 u1 = *reinterpret_cast<const uint4*>(p + 16);
+        A0[0] = u0.x; A0[1] = u0.y; A0[2] = u0.z; A0[3] = u0.w;
+        A1[0] = u1.x; A1[1] = u1.y; A1[2] = u1.z; A1[3] = u1.w;
+    } else {
+        fz_decode_step(p, A0, A1);
+    }
+}
+
+template <int NT, bool GS, bool W8>
 __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb, int lane,
                                                 int rec_gu, int aoff, const int (*xsoff)[2],
-                                                int ntc, float acc_f[NT][4]) {
-    constexpr int ns = 4;
+                                                int jo, int ntc, float acc_f[NT][4]) {
+    constexpr int ns = fz_ns_gateup<W8>();
+    constexpr int kStep = fz_step_bytes<W8>();
     const int g = lane >> 2, t = lane & 3;
-    const uint8_t* cp = sl + m * ns * 4096 + rb * 512 + lane * 16;
+    const uint8_t* cp = sl + m * ns * kStep + rb * (kStep / 8) + lane * (kStep / 256);
     // aoff: this lane's pair record (column group 0); groups c > 0 follow at 4 c rec_gu
-    const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + aoff;
+    const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + aoff + jo * 128;
     const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff + m * ns * 512) + 16 * rb + g;
     // per-row scales: exact int32 sums, two chains (even and odd steps) for one
     // column group, one chain when several groups give independent MMAs
@@ -631,7 +669,7 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
 #pragma unroll
     for (int j = 0; j < ns; ++j) {
         uint32_t A0[4], A1[4];
-        fz_decode_step(cp + j * 4096, A0, A1);
+        fz_load_step<W8>(cp + j * kStep, A0, A1);
         float s0 = 0.0f, s1 = 0.0f;
         if (GS) { s0 = scl[j * 128]; s1 = scl[j * 128 + 8]; }
 #pragma unroll
@@ -658,7 +696,7 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
             }
         }
     }
-    const float f = (t < 2 ? 256.0f : 1.0f) * 0.0625f;
+    const float f = (t < 2 ? 256.0f : 1.0f) * (W8 ? 1.0f : 0.0625f);
     const uint8_t* xr = sl + kFzActOff + kActRecScale;
 #pragma unroll
     for (int c = 0; c < NT; ++c) {
@@ -675,13 +713,14 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
 }
 
 // ---------------------------------------------------------------------------
-// Down stage of a consumer warp: tile q = w / 4 of the stage's rs tiles,
-// 16-row blocks 2 (w % 4) and 2 (w % 4) + 1, both steps (the tile's 128
-// columns of I) against h of the item in shared memory.  Writes the partial
-// products of pairs p0 .. p0 + np - 1 for these 32 rows.
+// Down stage of a consumer warp: 16-row blocks B = BPW w .. BPW w + BPW - 1 of
+// the stage's rs tiles (block B: tile B / 8, block B % 8 of it; BPW = 2 for
+// 4-bit codes, 1 for 8-bit ones), both steps (the tile's 128 columns of I)
+// against h of the item in shared memory.  Writes the partial products of
+// pairs p0 .. p0 + np - 1 for these rows.
 // ---------------------------------------------------------------------------
-template <int NT>
-// hf[c][q]: lanefac * (inverse scale of h) / 16 of pair 4c + 2(t & 1) + q;
+template <int NT, bool W8>
+// hf[c][q]: lanefac * (inverse scale of h) (/ 16 for 4-bit codes) of pair 4c + 2(t & 1) + q;
 // dst[c][q]: element offset in part of that pair's row 0 (-1: not written by
 // this lane).  Both are constant over the down stages of an item.
 __device__ __forceinline__ void fz_stage_down_prep(const FusedArgs& a, const FusedShared& sh,
@@ -693,25 +732,29 @@ __device__ __forceinline__ void fz_stage_down_prep(const FusedArgs& a, const Fus
     for (int c = 0; c < NT; ++c)
         for (int q = 0; q < 2; ++q) {
             const int ph = 4 * c + 2 * (t & 1) + q;  // pair of this lane's digit columns
-            hf[c][q] = lanefac * *reinterpret_cast<const float*>(sh.hbuf + ph * kFzRecH + 256) * 0.0625f;
+            hf[c][q] = lanefac * *reinterpret_cast<const float*>(sh.hbuf + ph * kFzRecH + 256) *
+                       (W8 ? 1.0f : 0.0625f);
             const int pw = 4 * c + 2 * t + q;         // pair this lane writes (t < 2)
             dst[c][q] = (t < 2 && pw < np) ? (sh.pair_pick[p0 + pw] * TG + tc) * a.H : -1;
         }
 }
 
-template <int NT, bool GS>
+template <int NT, bool GS, bool W8>
 __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedShared& sh,
                                               const uint8_t* sl, int rs, int rt0, int ntc,
                                               const float (*hf)[2], const int (*dst)[2],
                                               int warp, int lane) {
-    const int q = warp >> 2;
+    constexpr int BPW = W8 ? 1 : 2;
+    constexpr int WPT = 8 / BPW;  // warps per tile
+    constexpr int kStep = fz_step_bytes<W8>();
+    const int q = warp / WPT;
     if (q >= rs) return;
     const int g = lane >> 2, t = lane & 3;
     const int8_t* hb = sh.hbuf + (g >> 2) * 64 + t * 16 + (g & 3) * kFzRecH;
 #pragma unroll
-    for (int bb = 0; bb < 2; ++bb) {
-        const int b8 = 2 * (warp & 3) + bb;
-        const uint8_t* cp = sl + q * 8192 + b8 * 512 + lane * 16;
+    for (int bb = 0; bb < BPW; ++bb) {
+        const int b8 = BPW * (warp % WPT) + bb;
+        const uint8_t* cp = sl + q * 2 * kStep + b8 * (kStep / 8) + lane * (kStep / 256);
         const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff) +
                            (GS ? q * 256 : q * 128) + 16 * b8 + g;
         float v[NT][4];
@@ -723,7 +766,7 @@ __device__ __forceinline__ void fz_stage_down(const FusedArgs& a, const FusedSha
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             uint32_t A0[4], A1[4];
-            fz_decode_step(cp + j * 4096, A0, A1);
+            fz_load_step<W8>(cp + j * kStep, A0, A1);
 #pragma unroll
             for (int c = 0; c < NT; ++c) {
                 if (NT > 1 && c >= ntc) break;
@@ -772,14 +815,14 @@ namespace coli {
 // tile (SwiGLU of the two accumulators) becomes s8 digits in shared memory
 // with one power-of-two scale per pair.
 // ---------------------------------------------------------------------------
-template <int NT, bool GS>
+template <int NT, bool GS, bool W8>
 __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, uint8_t* ring,
                                            int n_units) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int rb = warp & 7, m = warp >> 3;
-    const FzShape z = fz_shape(a);
-    const int rec_gu = fz_rec_bytes(z.ns_gu);
+    const FzShape z = fz_shape<W8>(a);
+    const int rec_gu = kActRec;
     const bool wr = t < 2;  // after the digit combine: lanes holding results
     uint32_t cphase = 0, lap = 0;
     int s = 0;
@@ -791,7 +834,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
     int dst[NT][2];                //            partial-product offsets
     float acc_f[NT][4];
     for (;;) {
-        if (!fz_wait(&sh.full[s], lap, a.err)) return;
+        if (!fz_wait(&sh.full[s], lap, a.err, a.wait_tries)) return;
         const int item = sh.meta_item[s], st = sh.meta_st[s];
         if (item < 0) return;
         const uint8_t* sl = ring + (int64_t)s * a.slot_bytes;
@@ -818,14 +861,15 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
         }
         const bool gu = st < z.nst_gu;
         if (gu) {
-            fz_stage_gateup<NT, GS>(sl, m, rb, lane, rec_gu, aoff, xsoff, (np + 3) >> 2, acc_f);
+            fz_stage_gateup<NT, GS, W8>(sl, m, rb, lane, rec_gu, aoff, xsoff,
+                                        W8 ? (st & 1) * 2 : 0, (np + 3) >> 2, acc_f);
             if (!GS && st == z.nst_gu - 1) {
                 const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
                 sw0 = rsc[0];
                 sw1 = rsc[8];
             }
         } else {
-            fz_stage_down<NT, GS>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, (np + 3) >> 2, hf, dst, warp,
+            fz_stage_down<NT, GS, W8>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, (np + 3) >> 2, hf, dst, warp,
                                   lane);
         }
         __syncwarp();
@@ -852,7 +896,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 const int pp = 4 * c + 2 * t + (i & 1), rr = g + 8 * (i >> 1);
                 if (wr && pp < np && m == 1) sh.xch[rb][rr][pp] = v[c][i];
             }
-        if (!fz_cbar(&sh.cbar, cphase, a.err)) return;
+        if (!fz_cbar(&sh.cbar, cphase, a.err, a.wait_tries)) return;
         if (m == 0) {
 #pragma unroll
             for (int c = 0; c < NT; ++c) {
@@ -876,7 +920,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 }
             }
         }
-        if (!fz_cbar(&sh.cbar, cphase, a.err)) return;
+        if (!fz_cbar(&sh.cbar, cphase, a.err, a.wait_tries)) return;
         if (m == 0 && wr) {
             const int j = rb / 4;  // 64-column step of the down part holding these rows of h
 #pragma unroll
@@ -902,12 +946,12 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                     if (rb == 0 && g == 0) *reinterpret_cast<float*>(rec + 256) = inv;
                 }
         }
-        if (!fz_cbar(&sh.cbar, cphase, a.err)) return;  // h complete before the down stages
-        fz_stage_down_prep<NT>(a, sh, tc, p0, np, lane, hf, dst);
+        if (!fz_cbar(&sh.cbar, cphase, a.err, a.wait_tries)) return;  // h complete before the down stages
+        fz_stage_down_prep<NT, W8>(a, sh, tc, p0, np, lane, hf, dst);
     }
 }
 
-template <int NT, bool GS>
+template <int NT, bool GS, bool W8>
 __global__ void __launch_bounds__(kFzThreads, 1)
 moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
     extern __shared__ __align__(128) uint8_t fz_smem[];
@@ -930,7 +974,7 @@ moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
         if (warp == kFzProducer) {
             asm volatile("bar.sync 2, %0;" ::"n"(64) : "memory");
             // the computed picks are distinct experts: one unit each
-            fz_produce<GS>(a, &xmap, sh, fz_smem, sh.n_kept1 + a.n_shared, true);
+            fz_produce<GS, W8>(a, &xmap, sh, fz_smem, sh.n_kept1 + a.n_shared, true);
             return;
         }
         if (warp == 0) {
@@ -946,12 +990,12 @@ moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
             fz_union_warp(a, sh, one);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kFzWarps) : "memory");
-        fz_consume<NT, GS>(a, sh, fz_smem, sh.n_uniq + a.n_shared);
+        fz_consume<NT, GS, W8>(a, sh, fz_smem, sh.n_uniq + a.n_shared);
         return;
     }
     const int n_units = fz_route_union(a, sh, fz_smem);
-    if (warp == kFzProducer) fz_produce<GS>(a, &xmap, sh, fz_smem, n_units, false);
-    else fz_consume<NT, GS>(a, sh, fz_smem, n_units);
+    if (warp == kFzProducer) fz_produce<GS, W8>(a, &xmap, sh, fz_smem, n_units, false);
+    else fz_consume<NT, GS, W8>(a, sh, fz_smem, n_units);
 }
 
 // ---------------------------------------------------------------------------

@@ -89,6 +89,70 @@ quantize_rows_kernel(Src src, int R, int K, int group,
     }
 }
 
+// 8-bit codes (the engine keeps its MTP head at 8 bits: "解密GLM-5.2-colibri-
+// int4-with-int8-mtp"): the container's rule with 127 in place of 7, one signed
+// byte per weight, written into 8-bit fragment tiles (common.cuh).
+__device__ __forceinline__ int quant_one8(float v, float s) {
+    if (s == 0.0f) return 0;
+    float q = rintf(__fdiv_rn(v, s));
+    q = fminf(fmaxf(q, -127.0f), 127.0f);
+    return (int)q;
+}
+
+template <typename Src>
+__global__ void __launch_bounds__(256)
+quantize_rows8_kernel(Src src, int R, int K, int group,
+                      uint8_t* __restrict__ codes, float* __restrict__ scales) {
+    extern __shared__ uint4 qz_smem[];
+    int8_t* rows = reinterpret_cast<int8_t*>(qz_smem);  // [16][K]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int blk = blockIdx.x;                           // 16-row block index
+    const int rt = blk / 8, b8 = blk % 8;
+    const int gs = group ? group : K;
+    const int ng = K / gs;
+    for (int lr = warp; lr < 16; lr += 8) {
+        const int r = blk * 16 + lr;
+        int8_t* buf = rows + (int64_t)lr * K;
+        for (int g = 0; g < ng; ++g) {
+            float m = 0.0f;
+            for (int c = g * gs + lane; c < (g + 1) * gs; c += 32) m = fmaxf(m, fabsf(src.at(r, c, K)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const float s = __fdiv_rn(m, 127.0f);
+            if (lane == 0) scales[scale_offset(r, g, ng)] = s;
+            for (int c = g * gs + lane; c < (g + 1) * gs; c += 32)
+                buf[c] = (int8_t)quant_one8(src.at(r, c, K), s);
+        }
+    }
+    __syncthreads();
+    // lane l's 32 bytes of each 64-column step: words i = 4h + 2 hi16 + upper
+    for (int i = threadIdx.x; i < (K / 64) * 32; i += 256) {
+        const int kb = i / 32, l = i % 32, g = l >> 2, t = l & 3;
+        uint32_t wd[8];
+        for (int w = 0; w < 8; ++w) {
+            const int h = w >> 2, hi16 = (w >> 1) & 1, upper = w & 1;
+            const int lr = g + 8 * upper, c0 = kb * 64 + 32 * h + 16 * hi16 + 4 * t;
+            wd[w] = *reinterpret_cast<const uint32_t*>(rows + (int64_t)lr * K + c0);
+        }
+        uint8_t* dst = codes + ((((int64_t)rt * (K / 64) + kb) * 8 + b8) * 32 + l) * 32;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        *reinterpret_cast<uint4*>(dst + 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+    }
+}
+
+// one thread per element of an 8-bit matrix: out[r, c] = (float)q * s
+__global__ void __launch_bounds__(256)
+dequant8_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ scales,
+                int R, int K, int group, float* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    if (i >= (int64_t)R * K) return;
+    const int r = (int)(i / K), c = (int)(i % K);
+    const int ng = group ? K / group : 1;
+    const int q = (int8_t)codes[frag8_byte_offset(r, c, K)];
+    const float s = scales[scale_offset(r, group ? c / group : 0, ng)];
+    out[i] = __fmul_rn((float)q, s);
+}
+
 // one thread per element: out[r, c] = (float)q * s
 __global__ void __launch_bounds__(256)
 dequant_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ scales,

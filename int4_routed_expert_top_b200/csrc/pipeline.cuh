@@ -52,8 +52,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // abandoned, kErrWaitTimeout is or-ed into *err and false is returned.
 constexpr uint32_t kWaitTries = 1u << 22;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
-    for (uint32_t i = 0; i < kWaitTries; ++i)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err,
+                                          uint32_t tries = kWaitTries) {
+    for (uint32_t i = 0; i < tries; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     if (err) atomicOr(err, kErrWaitTimeout);
     return false;

@@ -7,8 +7,9 @@ import ctypes
 
 import numpy as np
 
-from . import (Desc, coli_moe_expert_bytes, coli_moe_layer_create, coli_moe_layer_destroy,
-               coli_moe_layer_set_partition, coli_moe_pack_expert, coli_moe_quantize,
+from . import (Desc, coli_moe_expert_bytes, coli_moe_expert_bytes8, coli_moe_layer_create,
+               coli_moe_layer_destroy, coli_moe_layer_set_partition, coli_moe_pack_expert,
+               coli_moe_pack_expert8, coli_moe_quantize, coli_moe_quantize_expert8_device,
                coli_moe_quantize_expert_device, coli_moe_workspace_size)
 
 
@@ -24,15 +25,18 @@ class DeviceLayer:
 
     def __init__(self, H, I, E, k, n_shared, group, router_w, router_b, *,
                  expert_masters=None, container=None, routed_scale=1.0, norm_topk=True,
-                 device="cuda", expert_range=None, with_shared=True):
+                 device="cuda", expert_range=None, with_shared=True, bits=4):
         """expert_range=(lo, hi): hold and compute only routed experts lo <= e < hi
         (and the shared experts when with_shared), as one rank of an
-        expert-parallel layer (coli_moe_layer_set_partition)."""
+        expert-parallel layer (coli_moe_layer_set_partition).  bits=8: 8-bit
+        expert codes (quantised by coli_moe_quantize_expert8_device or packed by
+        coli_moe_pack_expert8 from the container arrays of coli_moe_quantize8)."""
         import torch
         self.H, self.I, self.E, self.k = H, I, E, k
         self.n_shared, self.group = n_shared, group
         self.routed_scale, self.norm_topk = routed_scale, norm_topk
-        self.blob_bytes = coli_moe_expert_bytes(H, I, group)
+        self.bits = bits
+        self.blob_bytes = (coli_moe_expert_bytes8 if bits == 8 else coli_moe_expert_bytes)(H, I, group)
         lo, hi = expert_range if expert_range is not None else (0, E)
         self.expert_range = (lo, hi)
         self.with_shared = with_shared or expert_range is None
@@ -45,14 +49,16 @@ class DeviceLayer:
         for slot, e in enumerate(ids):
             if expert_masters is not None:
                 g, u, d = expert_masters(e)
-                coli_moe_quantize_expert_device(H, I, group, g.contiguous(), u.contiguous(),
-                                                d.contiguous(), self.experts[slot])
+                quant = coli_moe_quantize_expert8_device if bits == 8 else coli_moe_quantize_expert_device
+                quant(H, I, group, g.contiguous(), u.contiguous(), d.contiguous(),
+                      self.experts[slot])
             else:
-                blob = coli_moe_pack_expert(H, I, group, *container(e))
+                pack = coli_moe_pack_expert8 if bits == 8 else coli_moe_pack_expert
+                blob = pack(H, I, group, *container(e))
                 self.experts[slot].copy_(torch.from_numpy(blob))
         self.desc = Desc(H, I, E, k, n_shared, group, routed_scale, int(norm_topk),
                          self.router_w.data_ptr(), self.router_b.data_ptr(),
-                         self.experts.data_ptr())
+                         self.experts.data_ptr(), bits)
         self.handle = coli_moe_layer_create(self.desc)
         if expert_range is not None:
             coli_moe_layer_set_partition(self.handle, lo, hi, self.with_shared, self.experts)

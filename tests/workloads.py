@@ -25,15 +25,17 @@ def masters(wl, layer, e, device="cuda"):
     return tuple(synth.expert_master(wl, layer, t, e, device=device) for t in MATS)
 
 
-def build_layer(wl, layer=0, device="cuda", router=None, masters_device=None):
+def build_layer(wl, layer=0, device="cuda", router=None, masters_device=None, bits=4):
     """Layer on ``device``; its f32 masters are drawn on ``masters_device``
-    (default: the same device) and quantised by the library on the device."""
+    (default: the same device) and quantised by the library on the device
+    (4-bit codes, or 8-bit ones with bits=8)."""
     wr, b = router if router is not None else synth.router(wl, layer)
     md = masters_device or device
     return DeviceLayer(wl.H, wl.I, wl.E, wl.k, wl.n_shared, wl.group, wr, b,
                        expert_masters=lambda e: tuple(
                            m.to(device) for m in masters(wl, layer, e, md)),
-                       routed_scale=wl.routed_scale, norm_topk=wl.norm_topk, device=device)
+                       routed_scale=wl.routed_scale, norm_topk=wl.norm_topk, device=device,
+                       bits=bits)
 
 
 def gap_resampled_tokens(wl, T, wr, b, layer=0, step=0, max_rounds=64):
@@ -54,10 +56,11 @@ def gap_resampled_tokens(wl, T, wr, b, layer=0, step=0, max_rounds=64):
 
 
 class OracleExperts:
-    """Dequantised expert matrices computed by the oracle, cached per expert."""
+    """Dequantised expert matrices computed by the oracle (the int4 container,
+    or the 8-bit one with bits=8), cached per expert."""
 
-    def __init__(self, wl, layer=0, device="cuda"):
-        self.wl, self.layer, self.device = wl, layer, device
+    def __init__(self, wl, layer=0, device="cuda", bits=4):
+        self.wl, self.layer, self.device, self.bits = wl, layer, device, bits
         self.cache = {}
 
     def __call__(self, e):
@@ -65,8 +68,12 @@ class OracleExperts:
             mats = []
             for m in masters(self.wl, self.layer, e, self.device):
                 m = m.cpu().numpy()
-                p, s = oracle.quantize(m, self.wl.group)
-                mats.append(oracle.dequantize(p, s, m.shape[1], self.wl.group))
+                if self.bits == 8:
+                    q, s = oracle.quantize8(m, self.wl.group)
+                    mats.append(oracle.dequantize8(q, s, self.wl.group))
+                else:
+                    p, s = oracle.quantize(m, self.wl.group)
+                    mats.append(oracle.dequantize(p, s, m.shape[1], self.wl.group))
             self.cache[e] = tuple(mats)
         return self.cache[e]
 
