@@ -248,14 +248,15 @@ int coli_moe_layer_set_partition(coli_moe_layer* layer, int32_t e_begin, int32_t
 
 /* Test of the device-side bounded waits (no counterpart on the source pages):
  * on later fused-path forwards of this layer, CTA 0's producer skips ring
- * stage withhold_stage (0 = its first; < 0 = none), so nothing ever completes
- * that stage and the consumer warps' wait on it gives up; every wait of the
- * fused kernel gives up after wait_tries tries (0 = the default, about a
- * second).  The call then returns normally, its outputs are invalid and
- * coli_moe_status reports COLI_E_TIMEOUT; the next call without the option is
- * unaffected.  Never needed in normal use.  Host-only. */
-int coli_moe_layer_set_wait_test(coli_moe_layer* layer, int32_t withhold_stage,
-                                 uint32_t wait_tries);
+ * stage withhold_stage (0 = its first; < 0 = none, the default), so nothing
+ * ever completes that stage and the consumer warps' wait on it gives up; with
+ * the option set, every wait of the fused kernel gives up after 4096 tries
+ * instead of the default (about a second).  The call then returns normally,
+ * its outputs are invalid and coli_moe_status reports COLI_E_TIMEOUT; the
+ * next call without the option is unaffected.  4-bit layers only (a fused
+ * forward of an 8-bit layer with the option set returns COLI_E_UNSUPPORTED).
+ * Never needed in normal use.  Host-only. */
+int coli_moe_layer_set_wait_test(coli_moe_layer* layer, int32_t withhold_stage);
 
 /* Workspace bytes that coli_moe_route / coli_moe_forward need for T tokens
  * (enough for every path; the GEMV and GEMM paths use only a prefix). */

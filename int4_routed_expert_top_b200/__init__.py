@@ -87,7 +87,7 @@ _SIGS = {
     "coli_moe_layer_create": ([ctypes.POINTER(Desc), ctypes.POINTER(_P)], ctypes.c_int),
     "coli_moe_layer_destroy": ([_P], ctypes.c_int),
     "coli_moe_layer_set_topp": ([_P, ctypes.c_float], ctypes.c_int),
-    "coli_moe_layer_set_wait_test": ([_P, _I32, ctypes.c_uint32], ctypes.c_int),
+    "coli_moe_layer_set_wait_test": ([_P, _I32], ctypes.c_int),
     "coli_moe_layer_set_partition": ([_P, _I32, _I32, _I32, _P], ctypes.c_int),
     "coli_moe_workspace_size": ([_P, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
     "coli_moe_route": ([_P, _P, ctypes.c_int, _I32, _P, _P, _P, _SZ, _P], ctypes.c_int),
@@ -234,9 +234,9 @@ def coli_moe_layer_destroy(layer) -> None:
     _ok(lib.coli_moe_layer_destroy(layer))
 
 
-def coli_moe_layer_set_wait_test(layer, withhold_stage: int, wait_tries: int) -> None:
+def coli_moe_layer_set_wait_test(layer, withhold_stage: int) -> None:
     """Test only: make the fused kernel's bounded waits run out (see the header)."""
-    _ok(lib.coli_moe_layer_set_wait_test(layer, withhold_stage, wait_tries))
+    _ok(lib.coli_moe_layer_set_wait_test(layer, withhold_stage))
 
 
 def coli_moe_layer_set_topp(layer, p: float) -> None:

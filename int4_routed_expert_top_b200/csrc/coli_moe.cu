@@ -32,7 +32,6 @@ struct coli_moe_layer {
     ExpertStore store;
     PickFilter filter;
     // test of the bounded waits (coli_moe_layer_set_wait_test)
-    uint32_t wait_tries = kWaitTries;
     int withhold = -1;
 };
 
@@ -464,21 +463,21 @@ int sm_count() { return gemm_grid(); }
 // the previous one (router, then fused) finishes; it waits
 // (griddepcontrol.wait) before reading what that kernel wrote.
 
-template <int NT, bool GS, bool W8>
+template <int NT, bool GS, bool W8, bool TW>
 int launch_fused_t(const CUtensorMap& xmap, const FusedArgs& a, cudaStream_t st) {
     const int smem = a.slots * a.slot_bytes;
-    int rc = set_smem((const void*)moe_fused_kernel<NT, GS, W8>, smem);
+    int rc = set_smem((const void*)moe_fused_kernel<NT, GS, W8, TW>, smem);
     if (rc) return rc;
-    return launch_pdl(moe_fused_kernel<NT, GS, W8>, dim3(sm_count()), kFzThreads, smem, st,
+    return launch_pdl(moe_fused_kernel<NT, GS, W8, TW>, dim3(sm_count()), kFzThreads, smem, st,
                       "fused moe", xmap, a);
 }
 
-template <bool W8>
+template <bool W8, bool TW>
 int launch_fused_w(int NT, bool gs, const CUtensorMap& xmap, const FusedArgs& a, cudaStream_t st) {
     switch (NT) {
-        case 1: return gs ? launch_fused_t<1, true, W8>(xmap, a, st) : launch_fused_t<1, false, W8>(xmap, a, st);
-        case 2: return gs ? launch_fused_t<2, true, W8>(xmap, a, st) : launch_fused_t<2, false, W8>(xmap, a, st);
-        default: return gs ? launch_fused_t<4, true, W8>(xmap, a, st) : launch_fused_t<4, false, W8>(xmap, a, st);
+        case 1: return gs ? launch_fused_t<1, true, W8, TW>(xmap, a, st) : launch_fused_t<1, false, W8, TW>(xmap, a, st);
+        case 2: return gs ? launch_fused_t<2, true, W8, TW>(xmap, a, st) : launch_fused_t<2, false, W8, TW>(xmap, a, st);
+        default: return gs ? launch_fused_t<4, true, W8, TW>(xmap, a, st) : launch_fused_t<4, false, W8, TW>(xmap, a, st);
     }
 }
 
@@ -490,7 +489,6 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
     a.store = l->store;
     a.L = l->L;
     a.filter = l->filter;
-    a.wait_tries = l->wait_tries;
     a.withhold = l->withhold;
     (void)KS;  // the small-batch router leaves one slice: the scores themselves
     a.score = at<float>(ws, p.zpart);
@@ -521,8 +519,12 @@ int launch_fused(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, int 
         if ((rc = encode_act_map(&xmap, a.xq8, T, d.H))) return rc;
         a.act_tma = 1;
     }
-    rc = l->bits == 8 ? launch_fused_w<true>(NT, gs, xmap, a, st)
-                      : launch_fused_w<false>(NT, gs, xmap, a, st);
+    // the wait test has its own instantiation (4-bit layers only)
+    if (l->withhold >= 0 && l->bits == 8)
+        return fail(COLI_E_UNSUPPORTED, "wait test: 4-bit layers only");
+    rc = l->bits == 8 ? launch_fused_w<true, false>(NT, gs, xmap, a, st)
+                      : (l->withhold >= 0 ? launch_fused_w<false, true>(NT, gs, xmap, a, st)
+                                          : launch_fused_w<false, false>(NT, gs, xmap, a, st));
     if (rc) return rc;
     if ((rc = mark(COLI_STAGE_DOWN))) return rc;
     if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
@@ -817,11 +819,9 @@ int coli_moe_layer_create(const coli_moe_desc* desc, coli_moe_layer** out) {
     return COLI_OK;
 }
 
-int coli_moe_layer_set_wait_test(coli_moe_layer* layer, int32_t withhold_stage,
-                                 uint32_t wait_tries) {
+int coli_moe_layer_set_wait_test(coli_moe_layer* layer, int32_t withhold_stage) {
     if (!layer) return fail(COLI_E_INVAL, "set_wait_test: NULL layer");
     layer->withhold = withhold_stage < 0 ? -1 : withhold_stage;
-    layer->wait_tries = wait_tries == 0 ? kWaitTries : wait_tries;
     return COLI_OK;
 }
 

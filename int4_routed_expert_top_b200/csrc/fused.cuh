@@ -101,10 +101,9 @@ struct FusedArgs {
     // used for 2 <= T <= 4 (one column group).  0: one bulk copy per pair,
     // stored per pair record.
     int act_tma;
-    // bounded waits: tries before a wait gives up (kWaitTries normally); a
-    // test may also have CTA 0's producer withhold ring stage withhold (its
-    // copies are never issued, so the consumers' wait on it runs out), -1: none
-    uint32_t wait_tries;
+    // test of the bounded waits (kernels instantiated with TW only): CTA 0's
+    // producer withholds ring stage withhold (its copies are never issued, so
+    // the consumers' wait on it runs out) and every wait takes a short limit
     int withhold;
 };
 
@@ -443,10 +442,12 @@ __device__ __forceinline__ void mma_s8_16832_zc(int d[4], const uint32_t a[4], u
 
 // Warp-wide bounded wait on an mbarrier phase; every lane returns the result
 // and is ordered after lane 0's acquire.
-__device__ __forceinline__ bool fz_wait(uint64_t* bar, uint32_t parity, int32_t* err,
-                                        uint32_t tries) {
+// test: the wait test (a stage withheld): a short limit instead of the default
+constexpr uint32_t kFzTestWaitTries = 1u << 12;
+__device__ __forceinline__ bool fz_wait(uint64_t* bar, uint32_t parity, int32_t* err, bool test) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, tries) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait(bar, parity, err, test ? kFzTestWaitTries : kWaitTries) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
@@ -454,11 +455,10 @@ __device__ __forceinline__ bool fz_wait(uint64_t* bar, uint32_t parity, int32_t*
 
 // Barrier of the consumer warps on an mbarrier (count kFzWarps) with a bounded
 // wait, so that a failed warp cannot leave the others blocked for good.
-__device__ __forceinline__ bool fz_cbar(uint64_t* bar, uint32_t& phase, int32_t* err,
-                                        uint32_t tries) {
+__device__ __forceinline__ bool fz_cbar(uint64_t* bar, uint32_t& phase, int32_t* err, bool test) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-    const bool ok = fz_wait(bar, phase, err, tries);
+    const bool ok = fz_wait(bar, phase, err, test);
     phase ^= 1u;
     return ok;
 }
@@ -504,7 +504,7 @@ __device__ __forceinline__ FzShape fz_shape(const FusedArgs& a) {
 //   down stage: rs tiles of 128 H rows, columns 128 tc .. 128 tc + 127
 //     [codes, 8 or 16 KB per tile | scales (per row: 512 B per tile; gs64: 1 KB)].
 // ---------------------------------------------------------------------------
-template <bool GS, bool W8>
+template <bool GS, bool W8, bool TW>
 __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap* xmap,
                                            FusedShared& sh, uint8_t* ring, int n_units, bool one) {
     const int lane = threadIdx.x & 31;
@@ -544,14 +544,14 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
         const float* sD = reinterpret_cast<const float*>(blob + a.L.scales[2]);
         const int nst = z.nst_gu + z.nst_dn;
         for (int st = 0; st < nst; ++st) {
-            if (issued >= a.slots && !fz_wait(&sh.empty[s], lap ^ 1u, a.err, a.wait_tries)) {
+            if (issued >= a.slots && !fz_wait(&sh.empty[s], lap ^ 1u, a.err, TW)) {
                 ok = false;
                 break;
             }
             if (lane == 0) { sh.meta_item[s] = item; sh.meta_st[s] = st; }
             __syncwarp();
             uint8_t* sl = ring + (int64_t)s * a.slot_bytes;
-            if (issued == a.withhold && blockIdx.x == 0) {
+            if (TW && issued == a.withhold && blockIdx.x == 0) {
                 // nothing is copied and the stage's barrier never completes
             } else if (st < z.nst_gu) {
                 const int kb0 = st * z.ns_gu;
@@ -606,7 +606,7 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
         if (lane == 0) item = (int)gridDim.x + atomicAdd(a.queue, 1);
         item = __shfl_sync(0xffffffffu, item, 0);
     }
-    if (ok && (issued < a.slots || fz_wait(&sh.empty[s], lap ^ 1u, a.err, a.wait_tries))) {  // end marker
+    if (ok && (issued < a.slots || fz_wait(&sh.empty[s], lap ^ 1u, a.err, TW))) {  // end marker
         if (lane == 0) sh.meta_item[s] = -1;
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.full[s]);
@@ -614,7 +614,7 @@ __device__ __forceinline__ void fz_produce(const FusedArgs& a, const CUtensorMap
     }
     // leave only once every copy issued into the ring has landed
     for (int j = issued > a.slots ? issued - a.slots : 0; j < issued; ++j)
-        fz_wait(&sh.full[j % a.slots], (j / a.slots) & 1, nullptr, a.wait_tries);
+        fz_wait(&sh.full[j % a.slots], (j / a.slots) & 1, nullptr, TW);
 }
 
 }  // namespace coli
@@ -631,7 +631,7 @@ namespace coli {
 // for 64-column groups) is added to acc_f times the activation scale of its
 // pair's 256-column record, the lane's digit factor (256 for high digits) and,
 // for 4-bit codes, 1/16 (the nibble sits in the high half of an s8 byte).
-// xsoff[c][q]: offset of the activation record of pair 4c + 2(t & 1) + q; jo:
+// xsoff0[q]: offset of the activation record of pair 2(t & 1) + q; jo:
 // the first of the stage's steps within that record.
 // ---------------------------------------------------------------------------
 static_assert(fz_rec_bytes(4) == kActRec, "pair records of a stage are the global records");
@@ -652,8 +652,8 @@ __device__ __forceinline__ void fz_load_step(const uint8_t* p, uint32_t A0[4], u
 
 template <int NT, bool GS, bool W8>
 __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb, int lane,
-                                                int rec_gu, int aoff, const int (*xsoff)[2],
-                                                int jo, int ntc, float acc_f[NT][4]) {
+                                                int rec_gu, int aoff, const int* xsoff0, int np,
+                                                int jo, int ntc, bool last, float acc_f[NT][4]) {
     constexpr int ns = fz_ns_gateup<W8>();
     constexpr int kStep = fz_step_bytes<W8>();
     const int g = lane >> 2, t = lane & 3;
@@ -661,11 +661,32 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
     // aoff: this lane's pair record (column group 0); groups c > 0 follow at 4 c rec_gu
     const uint8_t* ap = sl + kFzActOff + (g >> 2) * 64 + t * 16 + aoff + jo * 128;
     const float* scl = reinterpret_cast<const float*>(sl + kFzScaleOff + m * ns * 512) + 16 * rb + g;
+    const uint8_t* xr = sl + kFzActOff;
+    // the records of the lane's two accumulator pairs: column group 0 from the
+    // item's table (records by token or by pair); later groups (several column
+    // groups: records by pair) at fixed offsets from the lane's first pair.  A
+    // pair past np reads a record the stage did not fill (inside the slot): it
+    // only scales that pair's own columns, whose results are never used.
+    const uint8_t* xr_lane = xr + 2 * (t & 1) * kActRec;
+    auto rec_at = [&](int c, int q) -> const uint8_t* {
+        if (c == 0) return xr + xsoff0[q];
+        return xr_lane + (4 * c + q) * kActRec;
+    };
+    // entering a new record (a new 256-column group of activations): the
+    // running sums move to its units, an exact power-of-two rescale
+    if (jo == 0) {
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+            if (NT > 1 && c >= ntc) break;
+            const float r0 = *reinterpret_cast<const float*>(rec_at(c, 0) + kActRecRatio);
+            const float r1 = *reinterpret_cast<const float*>(rec_at(c, 1) + kActRecRatio);
+            acc_f[c][0] *= r0; acc_f[c][1] *= r1; acc_f[c][2] *= r0; acc_f[c][3] *= r1;
+        }
+    }
     // per-row scales: exact int32 sums, two chains (even and odd steps) for one
     // column group, one chain when several groups give independent MMAs
     constexpr int CH = NT == 1 ? 2 : 1;
     int acc_i[CH][NT][4];
-    float acc_s[NT][4];    // 64-column scales: the stage's sum with them
 #pragma unroll
     for (int j = 0; j < ns; ++j) {
         uint32_t A0[4], A1[4];
@@ -676,19 +697,14 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
         for (int c = 0; c < NT; ++c) {
             if (NT > 1 && c >= ntc) break;  // column groups with no pair of this item
             const uint4 b = *reinterpret_cast<const uint4*>(ap + 4 * c * rec_gu + j * 128);
-            if (GS) {
+            if (GS) {  // 64-column weight scales: each step into f32 at once
                 int d[4];
                 mma_s8_16832_zc(d, A0, b.x, b.y);
                 mma_s8_16832(d, A1, b.z, b.w);
-                if (j == 0) {
-                    acc_s[c][0] = (float)d[0] * s0; acc_s[c][1] = (float)d[1] * s0;
-                    acc_s[c][2] = (float)d[2] * s1; acc_s[c][3] = (float)d[3] * s1;
-                } else {
-                    acc_s[c][0] = fmaf((float)d[0], s0, acc_s[c][0]);
-                    acc_s[c][1] = fmaf((float)d[1], s0, acc_s[c][1]);
-                    acc_s[c][2] = fmaf((float)d[2], s1, acc_s[c][2]);
-                    acc_s[c][3] = fmaf((float)d[3], s1, acc_s[c][3]);
-                }
+                acc_f[c][0] = fmaf((float)d[0], s0, acc_f[c][0]);
+                acc_f[c][1] = fmaf((float)d[1], s0, acc_f[c][1]);
+                acc_f[c][2] = fmaf((float)d[2], s1, acc_f[c][2]);
+                acc_f[c][3] = fmaf((float)d[3], s1, acc_f[c][3]);
             } else {
                 if (j < CH) mma_s8_16832_zc(acc_i[j % CH][c], A0, b.x, b.y);
                 else mma_s8_16832(acc_i[j % CH][c], A0, b.x, b.y);
@@ -696,18 +712,24 @@ __device__ __forceinline__ void fz_stage_gateup(const uint8_t* sl, int m, int rb
             }
         }
     }
-    const float f = (t < 2 ? 256.0f : 1.0f) * (W8 ? 1.0f : 0.0625f);
-    const uint8_t* xr = sl + kFzActOff + kActRecScale;
+    if (!GS) {
 #pragma unroll
-    for (int c = 0; c < NT; ++c) {
-        if (NT > 1 && c >= ntc) break;
-        const float x0 = *reinterpret_cast<const float*>(xr + xsoff[c][0]) * f;
-        const float x1 = *reinterpret_cast<const float*>(xr + xsoff[c][1]) * f;
+        for (int c = 0; c < NT; ++c) {
+            if (NT > 1 && c >= ntc) break;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float v = GS ? acc_s[c][i]
-                               : (float)(CH == 2 ? acc_i[0][c][i] + acc_i[CH - 1][c][i] : acc_i[0][c][i]);
-            acc_f[c][i] = fmaf(v, (i & 1) ? x1 : x0, acc_f[c][i]);
+            for (int i = 0; i < 4; ++i)
+                acc_f[c][i] += (float)(CH == 2 ? acc_i[0][c][i] + acc_i[CH - 1][c][i] : acc_i[0][c][i]);
+        }
+    }
+    if (last) {  // out of record units: the last record's scale, the digit factor
+                 // (and 1/16 for nibbles)
+        const float f = (t < 2 ? 256.0f : 1.0f) * (W8 ? 1.0f : 0.0625f);
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+            if (NT > 1 && c >= ntc) break;
+            const float x0 = *reinterpret_cast<const float*>(rec_at(c, 0) + kActRecScale) * f;
+            const float x1 = *reinterpret_cast<const float*>(rec_at(c, 1) + kActRecScale) * f;
+            acc_f[c][0] *= x0; acc_f[c][1] *= x1; acc_f[c][2] *= x0; acc_f[c][3] *= x1;
         }
     }
 }
@@ -815,7 +837,7 @@ namespace coli {
 // tile (SwiGLU of the two accumulators) becomes s8 digits in shared memory
 // with one power-of-two scale per pair.
 // ---------------------------------------------------------------------------
-template <int NT, bool GS, bool W8>
+template <int NT, bool GS, bool W8, bool TW>
 __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, uint8_t* ring,
                                            int n_units) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -828,13 +850,13 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
     int s = 0;
     int u = 0, tc = 0, p0 = 0, np = 0;
     int aoff = 0;  // this lane's activation record in a gate/up stage
-    int xsoff[NT][2];              // records of the lane's accumulator pairs
+    int xsoff0[2];                 // records of the lane's accumulator pairs (group 0)
     float sw0 = 1.0f, sw1 = 1.0f;  // per-row weight scales of rows g, g + 8
     float hf[NT][2];               // down part: digit and h scale factors
     int dst[NT][2];                //            partial-product offsets
-    float acc_f[NT][4];
+    float acc_f[NT][4];            // running gate/up sums, in the current record's units
     for (;;) {
-        if (!fz_wait(&sh.full[s], lap, a.err, a.wait_tries)) return;
+        if (!fz_wait(&sh.full[s], lap, a.err, TW)) return;
         const int item = sh.meta_item[s], st = sh.meta_st[s];
         if (item < 0) return;
         const uint8_t* sl = ring + (int64_t)s * a.slot_bytes;
@@ -851,26 +873,26 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 return a.act_tma ? sh.pair_tok[p0 + pp] * kActRec : pp * rec_gu;
             };
             aoff = rec_of(g & 3);
+            xsoff0[0] = rec_of(2 * (t & 1));
+            xsoff0[1] = rec_of(2 * (t & 1) + 1);
 #pragma unroll
-            for (int c = 0; c < NT; ++c) {
-                xsoff[c][0] = rec_of(4 * c + 2 * (t & 1));
-                xsoff[c][1] = rec_of(4 * c + 2 * (t & 1) + 1);
+            for (int c = 0; c < NT; ++c)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc_f[c][i] = 0.0f;
-            }
         }
         const bool gu = st < z.nst_gu;
         if (gu) {
-            fz_stage_gateup<NT, GS, W8>(sl, m, rb, lane, rec_gu, aoff, xsoff,
-                                        W8 ? (st & 1) * 2 : 0, (np + 3) >> 2, acc_f);
+            fz_stage_gateup<NT, GS, W8>(sl, m, rb, lane, rec_gu, aoff, xsoff0, np,
+                                        W8 ? (st & 1) * 2 : 0, (np + 3) >> 2, st == z.nst_gu - 1,
+                                        acc_f);
             if (!GS && st == z.nst_gu - 1) {
                 const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
                 sw0 = rsc[0];
                 sw1 = rsc[8];
             }
         } else {
-            fz_stage_down<NT, GS, W8>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, (np + 3) >> 2, hf, dst, warp,
-                                  lane);
+            fz_stage_down<NT, GS, W8>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, (np + 3) >> 2, hf, dst,
+                                      warp, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[s]);
@@ -896,7 +918,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 const int pp = 4 * c + 2 * t + (i & 1), rr = g + 8 * (i >> 1);
                 if (wr && pp < np && m == 1) sh.xch[rb][rr][pp] = v[c][i];
             }
-        if (!fz_cbar(&sh.cbar, cphase, a.err, a.wait_tries)) return;
+        if (!fz_cbar(&sh.cbar, cphase, a.err, TW)) return;
         if (m == 0) {
 #pragma unroll
             for (int c = 0; c < NT; ++c) {
@@ -920,7 +942,7 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 }
             }
         }
-        if (!fz_cbar(&sh.cbar, cphase, a.err, a.wait_tries)) return;
+        if (!fz_cbar(&sh.cbar, cphase, a.err, TW)) return;
         if (m == 0 && wr) {
             const int j = rb / 4;  // 64-column step of the down part holding these rows of h
 #pragma unroll
@@ -946,12 +968,16 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                     if (rb == 0 && g == 0) *reinterpret_cast<float*>(rec + 256) = inv;
                 }
         }
-        if (!fz_cbar(&sh.cbar, cphase, a.err, a.wait_tries)) return;  // h complete before the down stages
+        if (!fz_cbar(&sh.cbar, cphase, a.err, TW)) return;  // h complete before the down stages
         fz_stage_down_prep<NT, W8>(a, sh, tc, p0, np, lane, hf, dst);
     }
 }
 
-template <int NT, bool GS, bool W8>
+// TW: the wait test (coli_moe_layer_set_wait_test): CTA 0's producer withholds
+// one ring stage and every wait takes a short limit.  A separate instantiation,
+// so that the default launches keep compile-time limits (a limit chosen at run
+// time made the consumer loop ~12% slower).
+template <int NT, bool GS, bool W8, bool TW>
 __global__ void __launch_bounds__(kFzThreads, 1)
 moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
     extern __shared__ __align__(128) uint8_t fz_smem[];
@@ -974,7 +1000,7 @@ moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
         if (warp == kFzProducer) {
             asm volatile("bar.sync 2, %0;" ::"n"(64) : "memory");
             // the computed picks are distinct experts: one unit each
-            fz_produce<GS, W8>(a, &xmap, sh, fz_smem, sh.n_kept1 + a.n_shared, true);
+            fz_produce<GS, W8, TW>(a, &xmap, sh, fz_smem, sh.n_kept1 + a.n_shared, true);
             return;
         }
         if (warp == 0) {
@@ -990,12 +1016,12 @@ moe_fused_kernel(const __grid_constant__ CUtensorMap xmap, FusedArgs a) {
             fz_union_warp(a, sh, one);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kFzWarps) : "memory");
-        fz_consume<NT, GS, W8>(a, sh, fz_smem, sh.n_uniq + a.n_shared);
+        fz_consume<NT, GS, W8, TW>(a, sh, fz_smem, sh.n_uniq + a.n_shared);
         return;
     }
     const int n_units = fz_route_union(a, sh, fz_smem);
-    if (warp == kFzProducer) fz_produce<GS, W8>(a, &xmap, sh, fz_smem, n_units, false);
-    else fz_consume<NT, GS, W8>(a, sh, fz_smem, n_units);
+    if (warp == kFzProducer) fz_produce<GS, W8, TW>(a, &xmap, sh, fz_smem, n_units, false);
+    else fz_consume<NT, GS, W8, TW>(a, sh, fz_smem, n_units);
 }
 
 // ---------------------------------------------------------------------------

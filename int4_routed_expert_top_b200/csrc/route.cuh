@@ -90,11 +90,17 @@ __host__ __device__ inline int fz_act_pos(int c) {
 }
 
 // Record of one token's 256-column group: 4 steps x (64 hi + 64 lo bytes), the
-// f32 inverse scale at byte 512, zero padding to 576 bytes (a multiple of 16
-// for bulk copies; 64 mod 128 so that records of consecutive tokens in shared
-// memory start in other banks).
+// f32 inverse scale 2^-sh at byte 512, at byte 516 the ratio of the previous
+// group's inverse scale to this one's (a power of two; 1 for the first group),
+// zero padding to 576 bytes (a multiple of 16 for bulk copies; 64 mod 128 so
+// that records of consecutive tokens in shared memory start in other banks).
+// A consumer summing over the groups keeps its running sum in the current
+// group's units and multiplies it by the ratio on entering the next group,
+// which is exact.
 constexpr int kActRec = 576;
 constexpr int kActRecScale = 512;
+constexpr int kActRecRatio = 516;
+constexpr int kActMaxGroups = 64;  // H <= 16384 on the fused path
 
 // Power-of-two scale for a block whose largest magnitude is m: returns sh with
 // m * 2^sh in [2^13, 2^14) and *inv = 2^-sh (1 for an all-zero block).
@@ -115,30 +121,34 @@ __device__ __forceinline__ void fz_split(float v, float sc, int& hi, int& lo) {
 }
 
 // s8 activation operand of one token, one CTA of 256 threads: records
-// xq8[t][H/256][kActRec] as above (H a multiple of 256).  Thread tid owns
-// columns 4 tid + 1024 j; the 64 threads of two consecutive warps cover one
-// 256-column group.  Up to 8 column blocks of 1024 are loaded together (every
-// load in flight at once) and kept in registers for both passes.
+// xq8[t][H/256][kActRec] as above (H a multiple of 256, at most 16384).
+// Thread tid owns columns 4 tid + 1024 j; the 64 threads of two consecutive
+// warps cover one 256-column group.  First every group's largest magnitude
+// (the row read once, up to 8 blocks of 1024 columns in flight together), then
+// the digits, scales and ratios.
 template <typename XT>
 __device__ __forceinline__ void act_quant8_token(const XT* __restrict__ x, int H, int t,
                                                  int8_t* __restrict__ xq8) {
     constexpr int kJ = 8;
     __shared__ float part8[kJ][8];
+    __shared__ float ginv[kActMaxGroups];
     const XT* row = x + (int64_t)t * H;
     const bool vec = (reinterpret_cast<uintptr_t>(row) & (4 * sizeof(XT) - 1)) == 0;
     const int warp = threadIdx.x >> 5;
     const int G = H / 256;
     int8_t* trec = xq8 + (int64_t)t * G * kActRec;
+    auto load = [&](int c) {
+        return vec ? load4_f32(row + c)
+                   : make_float4(to_f32(row[c]), to_f32(row[c + 1]), to_f32(row[c + 2]),
+                                 to_f32(row[c + 3]));
+    };
+    // pass 1: the inverse scale of every group
     for (int j0 = 0; j0 * 1024 < H; j0 += kJ) {
         float4 v[kJ];
 #pragma unroll
         for (int jj = 0; jj < kJ; ++jj) {
             const int c = 4 * threadIdx.x + 1024 * (j0 + jj);
-            v[jj] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (c < H)
-                v[jj] = vec ? load4_f32(row + c)
-                            : make_float4(to_f32(row[c]), to_f32(row[c + 1]), to_f32(row[c + 2]),
-                                          to_f32(row[c + 3]));
+            v[jj] = c < H ? load(c) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
 #pragma unroll
         for (int jj = 0; jj < kJ; ++jj) {
@@ -149,34 +159,44 @@ __device__ __forceinline__ void act_quant8_token(const XT* __restrict__ x, int H
             if ((threadIdx.x & 31) == 0) part8[jj][warp] = m;
         }
         __syncthreads();
-#pragma unroll
-        for (int jj = 0; jj < kJ; ++jj) {
-            const int c = 4 * threadIdx.x + 1024 * (j0 + jj);
-            if (c >= H) break;
-            const float m = fmaxf(part8[jj][warp & ~1], part8[jj][warp | 1]);
-            float inv;
-            const float sc = fz_scale(m, &inv);
-            const float f[4] = {v[jj].x, v[jj].y, v[jj].z, v[jj].w};
-            uint32_t wh = 0, wl = 0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int hi, lo;
-                fz_split(f[i], sc, hi, lo);
-                wh |= (uint32_t)(hi & 0xFF) << (8 * i);
-                wl |= (uint32_t)(lo & 0xFF) << (8 * i);
-            }
-            int8_t* rec = trec + (int64_t)(c / 256) * kActRec;
-            int8_t* step = rec + ((c % 256) / 64) * 128;
-            const int pos = fz_act_pos(c % 64);
-            *reinterpret_cast<uint32_t*>(step + pos) = wh;
-            *reinterpret_cast<uint32_t*>(step + 64 + pos) = wl;
-            const int lt = threadIdx.x & 63;  // thread within the group
-            if (lt < (kActRec - kActRecScale) / 16) {  // the scale, then zero padding
-                const uint4 z = make_uint4(lt == 0 ? __float_as_uint(inv) : 0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(rec + kActRecScale + 16 * lt) = z;
+        if (threadIdx.x < kJ * 4) {  // group 4 (j0 + jj) + w2 of this block of columns
+            const int jj = threadIdx.x >> 2, w2 = threadIdx.x & 3;
+            const int g = 4 * (j0 + jj) + w2;
+            if (g < G) {
+                float inv;
+                fz_scale(fmaxf(part8[jj][2 * w2], part8[jj][2 * w2 + 1]), &inv);
+                ginv[g] = inv;
             }
         }
-        __syncthreads();  // part8 is rewritten by the next block of columns
+        __syncthreads();
+    }
+    // pass 2: digits (the row again, now from L1/L2), scales, ratios
+    for (int c = 4 * threadIdx.x; c < H; c += 1024) {
+        const float4 v = load(c);
+        const int g = c / 256;
+        const float inv = ginv[g];
+        const float sc = 1.0f / inv;  // a power of two: exact
+        const float f[4] = {v.x, v.y, v.z, v.w};
+        uint32_t wh = 0, wl = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int hi, lo;
+            fz_split(f[i], sc, hi, lo);
+            wh |= (uint32_t)(hi & 0xFF) << (8 * i);
+            wl |= (uint32_t)(lo & 0xFF) << (8 * i);
+        }
+        int8_t* rec = trec + (int64_t)g * kActRec;
+        int8_t* step = rec + ((c % 256) / 64) * 128;
+        const int pos = fz_act_pos(c % 64);
+        *reinterpret_cast<uint32_t*>(step + pos) = wh;
+        *reinterpret_cast<uint32_t*>(step + 64 + pos) = wl;
+        const int lt = (c % 256) / 4;  // thread within the group
+        if (lt < (kActRec - kActRecScale) / 16) {  // scale, ratio, then zero padding
+            const float ratio = g == 0 ? 1.0f : ginv[g - 1] / inv;
+            const uint4 z = lt == 0 ? make_uint4(__float_as_uint(inv), __float_as_uint(ratio), 0u, 0u)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(rec + kActRecScale + 16 * lt) = z;
+        }
     }
 }
 

@@ -33,13 +33,13 @@ def test_wait_gives_up_and_the_next_call_is_correct(T, group):
     y_clean = y.cpu().numpy().copy()
     assert cm.coli_moe_status(L.handle, T, ws) == 0
 
-    cm.coli_moe_layer_set_wait_test(L.handle, 0, 1 << 12)
+    cm.coli_moe_layer_set_wait_test(L.handle, 0)
     cm.coli_moe_forward_ex(L.handle, xd, T, y, ws, path=cm.COLI_PATH_FUSED)
     with pytest.raises(cm.ColiError) as e:
         cm.coli_moe_status(L.handle, T, ws)
     assert e.value.code == -6                                  # COLI_E_TIMEOUT
 
-    cm.coli_moe_layer_set_wait_test(L.handle, -1, 0)
+    cm.coli_moe_layer_set_wait_test(L.handle, -1)
     y.fill_(float("nan"))
     cm.coli_moe_forward_ex(L.handle, xd, T, y, ws, path=cm.COLI_PATH_FUSED)
     torch.cuda.synchronize()
