@@ -436,6 +436,8 @@ def main():
                     help="override routed experts (small-footprint profiling layers)")
     ap.add_argument("--bits", type=int, default=4, choices=(4, 8),
                     help="bits per expert weight code (8: the 8-bit container, fused path)")
+    ap.add_argument("--topp", type=float, default=0.0,
+                    help="adaptive expert top-p (0: every pick; coli_moe_layer_set_topp)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: each rank holds E/N routed experts (rank 0 the "
                          "shared ones), one all-reduce of y per step")
@@ -476,6 +478,9 @@ def main():
         args.path == "auto" and T <= 64 and T * (wl.k + wl.n_shared) <= 640 and wl.E <= 256
         and wl.k <= 32 and wl.n_shared <= 4 and wl.H % 256 == 0 and wl.I <= 4096)
     layers = build_layers(wl, dev, args.bits)
+    if args.topp:
+        for l in layers:
+            cm.coli_moe_layer_set_topp(l.handle, args.topp)
     L0 = layers[0]
     n_pool = 64 if T <= 16 else 2
     xpool = token_pool(wl, T, n_pool, rank, dev)
@@ -489,13 +494,15 @@ def main():
                      dtype=torch.uint8, device=dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
     idx_all = torch.empty((max(args.steps, n_pool), T, wl.k), dtype=torch.int32, device=dev)
+    w_all = torch.empty((max(args.steps, n_pool), T, wl.k), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(i, events=None, record_idx=False):
         xi = xpool[i % n_pool]
         if wl.layers == 1:
             cm.coli_moe_forward_ex(L0.handle, xi, T, y, ws, path=path,
-                                   idx_out=idx_all[i] if record_idx else None, events=events)
+                                   idx_out=idx_all[i] if record_idx else None,
+                                   w_out=w_all[i] if record_idx else None, events=events)
         else:
             xs.copy_(xi)
             cm.coli_moe_stack_forward([l.handle for l in layers], xs, T, wl.eps, ws, path=path)
@@ -509,6 +516,8 @@ def main():
         step(j, record_idx=True)
     torch.cuda.synchronize()
     slot_idx = idx_all[:n_pool].cpu().numpy() if wl.layers == 1 else None
+    # picks of weight 0 (dropped by top-p) are not computed: their experts are not read
+    slot_w = w_all[:n_pool].cpu().numpy() if wl.layers == 1 else None
 
     # one CUDA graph per token slot: the forward as a deployment would replay it
     graphs = []
@@ -616,12 +625,13 @@ def main():
            "top_k": wl.k, "intermediate": wl.I, "shared": wl.n_shared,
            "scale_group": wl.group or "per-row", "layers": wl.layers,
            "x_dtype": wl.x_dtype, "path": args.path, "weight_bits": args.bits,
+           "topp": args.topp or None,
            "l2": "256 MiB buffer written between timed steps (flush), not timed",
            "launch": "one CUDA graph per token slot, replayed",
            "e2e_launch": ("coli_moe_forward_host / coli_moe_stack_forward_host (pinned host x "
                           "and y), captured as one CUDA graph per token slot, replayed")}
     if wl.layers == 1:
-        uniq_slot = np.array([len(np.unique(slot_idx[j])) for j in range(n_pool)])
+        uniq_slot = np.array([len(np.unique(slot_idx[j][slot_w[j] != 0])) for j in range(n_pool)])
         uniq = uniq_slot[np.arange(K) % n_pool]
         nbytes = (uniq + wl.n_shared) * blob
         weight_gbs = nbytes.sum() / (total_ms / 1e3) / 1e9
