@@ -671,9 +671,10 @@ def main():
                                            "kernel": kname, "dtype": "f16 x f16 -> f32",
                                            "peak_source": peak_src}
         traffic = None
-        if fused and wl.name == "glm_decode" and T == 1:
+        if fused and wl.name == "glm_decode" and T == 1 and not args.topp:
             traffic = profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
-                                       "moe_fused_kernel_glm_decode.md")
+                                       "moe_fused_kernel_glm_decode_int8.md" if args.bits == 8
+                                       else "moe_fused_kernel_glm_decode.md")
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
                             "frac": ach / hbm_gbs, "traffic": traffic, "kernel": kname,
                             "peak_source": peak_src,

@@ -365,6 +365,18 @@ int coli_moe_stack_forward_host(const coli_moe_layer* const* layers, int32_t L,
 int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws,
                     int32_t* flags, coli_stream_t stream);
 
+/* Test helper: the batch union a forward built, read back from its workspace
+ * (ws planned for T tokens; device i32 outputs, each may be NULL): offsets
+ * [E+1], pair_tok and pair_slot [T*k] (pairs of computed picks grouped by
+ * expert, experts ascending, tokens ascending), uniq [E] (first n_uniq
+ * entries), n_uniq [1] after a GEMV- or GEMM-path forward; inv [T*k] (the
+ * pair of each pick, -1 for a pick not computed) after any path.  The fused
+ * path keeps its union in shared memory, in the order the picks first name
+ * their experts: only inv describes it.  Asynchronous. */
+int coli_moe_union_readback(const coli_moe_layer* layer, int32_t T, const void* ws,
+                            int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot,
+                            int32_t* uniq, int32_t* n_uniq, int32_t* inv, coli_stream_t stream);
+
 /* Test helper: dequantise matrix `which` (0 gate, 1 up, 2 down) of expert
  * `expert` (0 .. E + n_shared - 1) from the device blob into out (device f32,
  * row-major [R, K] in container order). */

@@ -42,7 +42,7 @@ EXPORTS = (
     "coli_moe_forward_host", "coli_moe_stack_host_workspace_size", "coli_moe_stack_forward_host",
     "coli_moe_quantize_expert_fp8_device", "coli_moe_quantize8", "coli_moe_expert_bytes8",
     "coli_moe_pack_expert8", "coli_moe_layer_set_topp", "coli_moe_layer_set_partition",
-    "coli_moe_quantize_expert8_device", "coli_moe_layer_set_wait_test",
+    "coli_moe_quantize_expert8_device", "coli_moe_layer_set_wait_test", "coli_moe_union_readback",
 )
 
 
@@ -100,6 +100,7 @@ _SIGS = {
     "coli_moe_stack_forward": ([_P, _I32, _P, _I32, ctypes.c_float, ctypes.c_int, _P, _SZ,
                                 _P], ctypes.c_int),
     "coli_moe_dequant_debug": ([_P, _I32, _I32, _P, _P], ctypes.c_int),
+    "coli_moe_union_readback": ([_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "coli_moe_forward_noalloc": ([_P, _P, ctypes.c_int, _I32, _P, _P], ctypes.c_int),
     "coli_moe_status": ([_P, _I32, _P, ctypes.POINTER(_I32), _P], ctypes.c_int),
     "coli_moe_host_workspace_size": ([_P, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
@@ -342,6 +343,14 @@ def coli_moe_status(layer, T: int, ws, stream=None) -> int:
     flags = _I32(0)
     _ok(lib.coli_moe_status(layer, T, _ptr(ws), ctypes.byref(flags), _stream(stream)))
     return flags.value
+
+
+def coli_moe_union_readback(layer, T: int, ws, offsets=None, pair_tok=None, pair_slot=None,
+                            uniq=None, n_uniq=None, inv=None, stream=None):
+    """Test helper: the union the last forward on ws built (see the header)."""
+    _ok(lib.coli_moe_union_readback(layer, T, _ptr(ws), _ptr(offsets), _ptr(pair_tok),
+                                    _ptr(pair_slot), _ptr(uniq), _ptr(n_uniq), _ptr(inv),
+                                    _stream(stream)))
 
 
 def coli_moe_dequant_debug(layer, expert: int, which: int, out, stream=None):

@@ -1166,6 +1166,26 @@ int coli_moe_dequant_debug(const coli_moe_layer* layer, int32_t expert, int32_t 
     return check_launch("dequant");
 }
 
+int coli_moe_union_readback(const coli_moe_layer* layer, int32_t T, const void* ws,
+                            int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot,
+                            int32_t* uniq, int32_t* n_uniq, int32_t* inv, coli_stream_t stream) {
+    if (!layer || !ws) return fail(COLI_E_INVAL, "union_readback: NULL pointer");
+    int rc = tokens_ok(layer->run, T);
+    if (rc) return rc;
+    const coli_moe_desc& d = layer->run;
+    const WsPlan p = plan_ws(d, T);
+    const char* w = static_cast<const char*>(ws);
+    const int64_t Tk = (int64_t)T * d.k;
+    struct { void* dst; int64_t off, n; } parts[] = {
+        {offsets, p.offsets, d.E + 1}, {pair_tok, p.pair_tok, Tk}, {pair_slot, p.pair_slot, Tk},
+        {uniq, p.uniq, d.E}, {n_uniq, p.n_uniq, 1}, {inv, p.inv, Tk}};
+    for (auto& q : parts)
+        if (q.dst && cudaMemcpyAsync(q.dst, w + q.off, (size_t)q.n * 4, cudaMemcpyDeviceToDevice,
+                                     S(stream)) != cudaSuccess)
+            return fail(COLI_E_CUDA, "union_readback: copy failed");
+    return COLI_OK;
+}
+
 int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws, int32_t* flags,
                     coli_stream_t stream) {
     if (!layer || !flags) return fail(COLI_E_INVAL, "status: NULL pointer");

@@ -40,6 +40,9 @@ namespace coli {
 constexpr int kGemmThreads = 768;
 constexpr int kGemmStages = 3;                        // shared-memory ring (68 KB stages)
 constexpr int kGemmAStages = 4;                       // TMEM A ring
+constexpr int kGemmAccBufs = 2;                       // TMEM accumulator buffers (128 columns each)
+constexpr int kGemmABase = 128 * kGemmAccBufs;        // first TMEM column of the A ring
+static_assert(kGemmABase + 64 * kGemmAStages <= 512, "TMEM holds 512 columns");
 constexpr int kGemmMaxN = 64;                         // tokens per tile
 constexpr int kGemmDecodeWarp0 = 8;
 constexpr int kGemmDecodeWarps = 16;
@@ -199,7 +202,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gm_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages];
     __shared__ __align__(8) uint64_t afull[kGemmAStages], aempty[kGemmAStages];
-    __shared__ __align__(8) uint64_t accfull[2], accempty[2];
+    __shared__ __align__(8) uint64_t accfull[kGemmAccBufs], accempty[kGemmAccBufs];
     __shared__ uint32_t tmem_slot;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_units = *a.n_units;
@@ -222,7 +225,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
             mbar_init(&afull[s], kGemmDecodeWarps);
             mbar_init(&aempty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kGemmAccBufs; ++b) {
             mbar_init(&accfull[b], 1);
             mbar_init(&accempty[b], 4);
         }
@@ -277,8 +280,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x, ++tcount) {
             const int np = (n + 15) / 16 * 16;  // N: multiple of 16 for M = 128
             const uint32_t idesc = idesc_f16_f32(np);
-            const int buf = tcount & 1;
-            if (tcount >= 2 && ok && !mbar_wait_warp_sleep(&accempty[buf], ((tcount >> 1) - 1) & 1, a.err)) ok = false;
+            const int buf = tcount % kGemmAccBufs;
+            if (tcount >= kGemmAccBufs && ok &&
+                !mbar_wait_warp_sleep(&accempty[buf], ((tcount / kGemmAccBufs) - 1) & 1, a.err))
+                ok = false;
             tc_fence_after();
             const uint32_t dacc = tmem + 128 * buf;
             for (int ka = 0; ka < KA; ++ka, ++u) {
@@ -288,7 +293,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
                 if (ok && !mbar_wait_warp_sleep(&full[s], (su / kGemmStages) & 1, a.err)) ok = false;
                 tc_fence_after();
                 uint8_t* st = smem + s * kStageBytes;
-                const uint32_t a0 = tmem + 256 + 64 * as;
+                const uint32_t a0 = tmem + kGemmABase + 64 * as;
                 if (a.two) {
                     const uint64_t bdesc = smem_desc_sw128(st + w * kAtomBytes);
 #pragma unroll
@@ -319,7 +324,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
         int tcount = 0;
         int p0, n, rt;
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x, ++tcount) {
-            const int buf = tcount & 1;
+            const int buf = tcount % kGemmAccBufs;
             const int row = rt * kTileRows + 32 * q + lane;
             const uint8_t* blob = a.store.blob(a.unit_expert[cur.u]);
             const float srow0 = a.group ? 1.0f
@@ -338,7 +343,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
                                     : __ldg(a.act_inv + p);
                 }
             }
-            if (ok && !mbar_wait_warp_sleep(&accfull[buf], (tcount >> 1) & 1, a.err)) ok = false;
+            if (ok && !mbar_wait_warp_sleep(&accfull[buf], (tcount / kGemmAccBufs) & 1, a.err)) ok = false;
             tc_fence_after();
             const uint32_t dacc = tmem + lane_off + 128 * buf;
             for (int c0 = 0; c0 < n; c0 += 16) {
@@ -380,7 +385,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap bmap, GemmArgs a) {
         const int g = lane >> 2;
         const DecodeK dk = a.dk;
         const uint32_t sbase = smem_u32(smem);
-        const uint32_t tlane = tmem + ((uint32_t)(32 * q + 16 * hb) << 16) + 256 + 32 * slot;
+        const uint32_t tlane = tmem + ((uint32_t)(32 * q + 16 * hb) << 16) + kGemmABase + 32 * slot;
         int u = 0;
         int p0, n, rt;
         for (int tile = blockIdx.x; cur.next(a, n_units, RT, tile, p0, n, rt); tile += gridDim.x) {
