@@ -6,9 +6,11 @@ checks the one the layer itself uses: on the GEMV and tensor-core paths the
 expert offsets, the (token, slot) pairs grouped by expert and the unique-expert
 list equal the oracle's stable grouping of the picks the call computes (all
 picks, or those top-p or an expert range keep), and every pick's pair index
-names its own (token, slot).  The fused path keeps its union in shared memory;
-its pair indices must cover the computed picks once each, one contiguous run
-per expert, tokens ascending inside a run."""
+names its own (token, slot).  The fused path keeps its union in shared memory
+and publishes each pick's pair index: with more than 32 picks its grouping is
+the same (experts ascending), with at most 32 the experts come in the order
+the picks first name them (token, then slot); both are rebuilt here from their
+definitions and compared index for index."""
 import dataclasses
 
 import numpy as np
@@ -84,6 +86,33 @@ def check_inv(idx, w, inv_flat):
         assert (np.diff(t_of[sel][order]) > 0).all(), e             # tokens ascending
 
 
+def inv_from_pairs(shape, ptok, pslot):
+    inv = np.full(shape, -1, np.int32)
+    inv[ptok, pslot] = np.arange(ptok.size, dtype=np.int32)
+    return inv
+
+
+def fused_inv_ref(idx, w, E):
+    """Pair index of every pick in the fused kernel's union."""
+    T, k = idx.shape
+    if T * k > 32:
+        _, ptok, pslot, _, _ = kept_union(idx, w, E)
+        return inv_from_pairs(idx.shape, ptok, pslot)
+    order = []                                   # experts by first naming
+    for t in range(T):
+        for j in range(k):
+            if w[t, j] != 0 and idx[t, j] not in order:
+                order.append(int(idx[t, j]))
+    ptok, pslot = [], []
+    for e in order:
+        for t in range(T):
+            for j in range(k):
+                if w[t, j] != 0 and idx[t, j] == e:
+                    ptok.append(t)
+                    pslot.append(j)
+    return inv_from_pairs(idx.shape, np.array(ptok, np.int64), np.array(pslot, np.int64))
+
+
 CASES = [dict(T=1), dict(T=5), dict(T=40, group=64), dict(T=60, k=8, E=32, group=64),
          dict(T=150, k=8, E=32, group=64)]
 
@@ -106,6 +135,7 @@ def test_forward_union_matches_oracle(case, topp):
     if wl.T * (wl.k + wl.n_shared) <= 640:                     # the fused path's limit
         idx, w, u = forward(L, x.cuda(), wl.T, cm.COLI_PATH_FUSED)
         check_inv(idx, w, u["inv"])
+        np.testing.assert_array_equal(u["inv"].reshape(idx.shape), fused_inv_ref(idx, w, wl.E))
     L.close()
 
 
@@ -124,6 +154,8 @@ def test_forward_union_of_an_expert_range(T):
         np.testing.assert_array_equal(w != 0, inside)
         if path == cm.COLI_PATH_FUSED:
             check_inv(idx, w, u["inv"])
+            np.testing.assert_array_equal(u["inv"].reshape(idx.shape),
+                                          fused_inv_ref(idx, w, wl.E))
         else:
             check_grouped(idx, w, u, wl.E)
             assert ((u["uniq"][: int(u["n_uniq"][0])] >= 16) &
