@@ -109,6 +109,41 @@ def profiled_traffic(kernel_src: str, profile: str, profiles_dir: str | None = N
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
+def path_ids():
+    import int4_routed_expert_top_b200 as cm
+    return {"auto": cm.COLI_PATH_AUTO, "gemv": cm.COLI_PATH_GEMV, "gemm": cm.COLI_PATH_GEMM,
+            "fused": cm.COLI_PATH_FUSED, "twopass": cm.COLI_PATH_TWOPASS}
+
+
+def resolve_path(wl, T, path_name, bits=4):
+    """The path a forward takes (AUTO resolved as include/coli_moe.h states)."""
+    if path_name != "auto":
+        return path_name
+    if (T <= 64 and T * (wl.k + wl.n_shared) <= 640 and wl.E <= 256 and wl.k <= 32
+            and wl.n_shared <= 4 and wl.H % 256 == 0 and wl.I <= 4096):
+        return "fused"
+    if (bits == 4 and 64 < T <= 1024 and wl.E <= 256 and wl.n_shared <= 4
+            and wl.H % 256 == 0 and wl.I % 256 == 0):
+        return "twopass"
+    return "gemv" if T < 48 else "gemm"
+
+
+def launches_per_layer(wl, T, path_name, fused):
+    """This library's kernel launches in one forward of one layer."""
+    path_name = resolve_path(wl, T, path_name)
+    if fused or path_name == "fused":
+        return 3                                  # router, fused kernel, combine
+    select = 1 if T * wl.E <= 4096 and T <= 128 else 2   # top-k and union together or apart
+    if path_name == "twopass":
+        # router, select, x records, gate/up pass, h records, down pass, combine
+        return 1 + select + 5
+    if path_name == "gemv":
+        return 1 + select + 2                     # router, select, gate/up GEMV, down GEMV
+    # router (+ the fp16 activation operand past 64 tokens), select, gather,
+    # GEMM, h, GEMM, combine
+    return (2 if T > 64 else 1) + select + 5
+
+
 def workload(name):
     import synth
     return synth.WORKLOADS[name]
@@ -333,8 +368,7 @@ def run_ep(args):
     if wl.layers != 1:
         raise SystemExit("--ep times one layer")
     T = args.tokens or wl.T
-    path = {"auto": cm.COLI_PATH_AUTO, "gemv": cm.COLI_PATH_GEMV, "gemm": cm.COLI_PATH_GEMM,
-            "fused": cm.COLI_PATH_FUSED}[args.path]
+    path = path_ids()[args.path]
     lo, hi = ep.expert_range(wl.E, rank, world)
     wr, b = synth.router(wl, 0)
     mats = (synth.T_GATE, synth.T_UP, synth.T_DOWN)
@@ -410,7 +444,7 @@ def run_ep(args):
                        "l2": "256 MiB buffer written between timed steps, not timed",
                        "launch": "eager (no graph)"},
             "clocks": clocks.summary(),
-            "gpu_launches": (3 if T <= 64 else 9) * K,
+            "gpu_launches": launches_per_layer(wl, T, args.path, T <= 64) * K,
             "e2e": {"value": T / (e2e_med / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": int(xpool[0].numel() * xpool.element_size()),
                     "d2h_bytes_per_step": int(T * wl.H * 4)}}
@@ -429,7 +463,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="glm_decode")
     ap.add_argument("--tokens", type=int, default=0, help="override tokens per step")
-    ap.add_argument("--path", default="auto", choices=("auto", "gemv", "gemm", "fused"))
+    ap.add_argument("--path", default="auto", choices=("auto", "gemv", "gemm", "fused", "twopass"))
     ap.add_argument("--impl", default="own", choices=("own", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
@@ -471,12 +505,10 @@ def main():
         import dataclasses
         wl = dataclasses.replace(wl, E=args.experts)
     T = args.tokens or wl.T
-    path = {"auto": cm.COLI_PATH_AUTO, "gemv": cm.COLI_PATH_GEMV, "gemm": cm.COLI_PATH_GEMM,
-            "fused": cm.COLI_PATH_FUSED}[args.path]
-    # the path AUTO resolves to (include/coli_moe.h): the fused kernel for small batches
-    fused = args.path == "fused" or (
-        args.path == "auto" and T <= 64 and T * (wl.k + wl.n_shared) <= 640 and wl.E <= 256
-        and wl.k <= 32 and wl.n_shared <= 4 and wl.H % 256 == 0 and wl.I <= 4096)
+    path = path_ids()[args.path]
+    # the path AUTO resolves to (include/coli_moe.h)
+    resolved = resolve_path(wl, T, args.path, args.bits)
+    fused = resolved == "fused"
     layers = build_layers(wl, dev, args.bits)
     if args.topp:
         for l in layers:
@@ -624,7 +656,8 @@ def main():
     cfg = {"workload": wl.name, "tokens_per_step": T, "hidden": wl.H, "experts": wl.E,
            "top_k": wl.k, "intermediate": wl.I, "shared": wl.n_shared,
            "scale_group": wl.group or "per-row", "layers": wl.layers,
-           "x_dtype": wl.x_dtype, "path": args.path, "weight_bits": args.bits,
+           "x_dtype": wl.x_dtype, "path": args.path, "path_taken": resolved,
+           "weight_bits": args.bits,
            "topp": args.topp or None,
            "l2": "256 MiB buffer written between timed steps (flush), not timed",
            "launch": "one CUDA graph per token slot, replayed",
@@ -655,21 +688,33 @@ def main():
             dominant = "gateup" if stage_mean[2] >= stage_mean[3] else "down"
             ach = gu_ach if dominant == "gateup" else dn_ach
             kern_bytes = units * (gu_bytes_unit if dominant == "gateup" else dn_bytes_unit)
-            gemm = args.path == "gemm" or (args.path == "auto" and T >= 48)
-            kname = (f"moe_gemm_kernel ({'gate/up' if dominant == 'gateup' else 'down'})"
-                     if gemm else f"{dominant}_gemv_kernel")
+            gemm = resolved == "gemm"
+            two = resolved == "twopass"
+            part = "gate/up" if dominant == "gateup" else "down"
+            kname = (f"moe_gemm_kernel ({part})" if gemm else
+                     (f"moe_split_kernel ({part} pass)" if two else f"{dominant}_gemv_kernel"))
             line["stages_us"] = {n: 1e3 * v for n, v in zip(cm.STAGE_NAMES, stage_mean)}
             line["down_gbs"] = dn_ach
-            if gemm:
+            if gemm or two:
                 # tensor work of the dominant launch: gate/up is 2I x H per pair, down H x I
                 pairs = T * (wl.k + wl.n_shared)
                 rows_k = 2 * wl.I * wl.H if dominant == "gateup" else wl.H * wl.I
                 col = 2 if dominant == "gateup" else 3
                 tflops = 2.0 * pairs * rows_k / (st_ms[:, col].mean() / 1e3) / 1e12
-                line["tensor_roofline"] = {"bound": "tensor", "achieved": tflops, "peak": bf16_tf,
-                                           "unit": "TFLOP/s", "frac": tflops / bf16_tf,
-                                           "kernel": kname, "dtype": "f16 x f16 -> f32",
-                                           "peak_source": peak_src}
+                if gemm:
+                    line["tensor_roofline"] = {"bound": "tensor", "achieved": tflops,
+                                               "peak": bf16_tf, "unit": "TFLOP/s",
+                                               "frac": tflops / bf16_tf, "kernel": kname,
+                                               "dtype": "f16 x f16 -> f32", "peak_source": peak_src}
+                else:
+                    # mma.sync s8 with two activation digits: two s8 products per
+                    # product of the layer; peak: the measured bf16 peak x 2
+                    # (the nominal dense int8 : bf16 ratio)
+                    line["tensor_roofline"] = {"bound": "tensor", "achieved": tflops,
+                                               "peak": 2 * bf16_tf, "unit": "TOP/s",
+                                               "frac": tflops / (2 * bf16_tf), "kernel": kname,
+                                               "dtype": "s8 x s8 -> s32 (two activation digits)",
+                                               "peak_source": peak_src + " bf16 x 2"}
         traffic = None
         if fused and wl.name == "glm_decode" and T == 1 and not args.topp:
             traffic = profiled_traffic("int4_routed_expert_top_b200/csrc/fused.cuh",
@@ -686,9 +731,9 @@ def main():
         line["int4_weight_frac_of_hbm"] = weight_gbs / hbm_gbs
         line["int4_weight_frac_of_spec"] = weight_gbs / SPEC_HBM_GBS
         line["unique_experts_per_step"] = float(uniq.mean())
-        line["gpu_launches"] = (3 if fused else (4 if T < 48 else 9)) * K
+        line["gpu_launches"] = launches_per_layer(wl, T, args.path, fused) * K
     else:   # per layer: the RMSNorm, then the path's own launches
-        line["gpu_launches"] = (1 + (3 if fused else (4 if T < 48 else 9))) * wl.layers * K
+        line["gpu_launches"] = (1 + launches_per_layer(wl, T, args.path, fused)) * wl.layers * K
     line["config"] = cfg
     line["clocks"] = clocks.summary()
     line["e2e"] = {"value": e2e_value, "unit": UNIT,

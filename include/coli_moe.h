@@ -86,16 +86,23 @@ typedef enum coli_status {
 typedef enum coli_dtype { COLI_F32 = 0, COLI_BF16 = 1 } coli_dtype;
 
 typedef enum coli_path {
-    COLI_PATH_AUTO = 0,  /* FUSED when it applies, else GEMV below 48 tokens,
-                            else GEMM                                          */
+    COLI_PATH_AUTO = 0,  /* FUSED when it applies; else TWOPASS for 65 to 1024
+                            tokens where it applies; else GEMV below 48
+                            tokens, else GEMM                                  */
     COLI_PATH_GEMV = 1,  /* per-unit int4 GEMV kernels (mma.sync, fp16 hi/lo
                             activation digits, f32 accumulation)               */
     COLI_PATH_GEMM = 2,  /* tcgen05 grouped GEMM, fp16 operands, f32 accumulate */
-    COLI_PATH_FUSED = 3  /* one persistent kernel for top-k, union and experts,
+    COLI_PATH_FUSED = 3, /* one persistent kernel for top-k, union and experts,
                             then a combine kernel (mma.sync s8, exact int32
                             sums per stage); T <= 64, T * (k + n_shared) <= 640,
                             E <= 256, k <= 32, n_shared <= 4, H a multiple
                             of 256, I <= 4096; the only path of 8-bit layers */
+    COLI_PATH_TWOPASS = 4 /* large batches: router and union kernels, then a
+                            gate/up pass writing h and a down pass writing
+                            each pair's output (the fused kernel's mma.sync s8
+                            stage on chunks of 16 of a unit's pairs), then the
+                            combine; E <= 256, n_shared <= 4, H and I
+                            multiples of 256; 4-bit layers                     */
 } coli_path;
 
 /* Thread-local description of the last error returned on this thread. */

@@ -15,7 +15,7 @@ import numpy as np
 
 __all__ = [
     "ColiError", "COLI_F32", "COLI_BF16", "COLI_PATH_AUTO", "COLI_PATH_GEMV",
-    "COLI_PATH_GEMM", "COLI_PATH_FUSED", "lib", "EXPORTS",
+    "COLI_PATH_GEMM", "COLI_PATH_FUSED", "COLI_PATH_TWOPASS", "lib", "EXPORTS",
     "coli_moe_last_error", "coli_moe_quantize", "coli_moe_expert_bytes",
     "coli_moe_pack_expert", "coli_moe_quantize_expert_device", "coli_moe_layer_create",
     "coli_moe_layer_destroy", "coli_moe_workspace_size", "coli_moe_route",
@@ -29,7 +29,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcolimoe.so")
 
 COLI_F32, COLI_BF16 = 0, 1
-COLI_PATH_AUTO, COLI_PATH_GEMV, COLI_PATH_GEMM, COLI_PATH_FUSED = 0, 1, 2, 3
+COLI_PATH_AUTO, COLI_PATH_GEMV, COLI_PATH_GEMM, COLI_PATH_FUSED, COLI_PATH_TWOPASS = 0, 1, 2, 3, 4
 
 # every symbol include/coli_moe.h declares
 EXPORTS = (

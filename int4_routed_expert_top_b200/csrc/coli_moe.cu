@@ -18,6 +18,7 @@
 #include "gemv.cuh"
 #include "misc.cuh"
 #include "route.cuh"
+#include "split.cuh"
 
 using namespace coli;
 
@@ -69,17 +70,31 @@ struct WsPlan {
     int64_t unit_expert, unit_begin, unit_end, n_units, counters, err;
     int64_t xq, xinv, hq, hinv, o, xg, hg, hmax, hsc;
     int64_t xq8, part, queue, sel;  // fused small-batch kernel (T <= kFzMaxT only)
+    int64_t hrec, squeue;           // two-pass path (xq8 as well)
     int64_t total;
 };
+
+// workspace layouts: the GEMV/GEMM base, the base with the fused path's
+// buffers where that path applies (else with the two-pass path's), the base
+// with the two-pass path's buffers.  Where the fused path applies its buffers
+// are larger than the two-pass path's, so the full layout covers every path.
+enum PlanKind { kPlanBase = 0, kPlanFull = 1, kPlanSplit = 2 };
 
 bool fused_fits(const coli_moe_desc& d, int T) {
     return T <= kFzMaxT && T * (d.k + d.n_shared) <= kFzMaxPairs && d.E <= kFzMaxE &&
            d.k <= kFzMaxK && d.n_shared <= 4 && d.H % 256 == 0 && d.I / 128 <= kCombineMaxTiles;
 }
 
+// the two-pass path: activation records along H and along I, the unit table
+// of the fused kernel's size
+bool split_fits(const coli_moe_desc& d) {
+    return d.E <= kFzMaxE && d.n_shared <= 4 && d.H % 256 == 0 && d.I % 256 == 0 &&
+           d.H <= 256 * kActMaxGroups && d.I <= 256 * kActMaxGroups;
+}
+
 // with_fused: also the fused path's buffers (placed last, so the plan without
 // them is a prefix of the plan with them)
-WsPlan plan_ws(const coli_moe_desc& d, int T, bool with_fused = true) {
+WsPlan plan_ws(const coli_moe_desc& d, int T, int kind = kPlanFull) {
     WsPlan p;
     int64_t off = 0;
     auto take = [&](int64_t bytes) { const int64_t at = off; off = align256(off + bytes); return at; };
@@ -110,13 +125,16 @@ WsPlan plan_ws(const coli_moe_desc& d, int T, bool with_fused = true) {
     p.hg = take(P * d.I * 2);                   //   fp16 h of every pair
     p.hmax = take(P * 4);                       //   per-pair max |h|
     p.hsc = take(P * 4);                        //   per-pair inverse scale of h
-    if (with_fused && fused_fits(d, T)) {
+    p.xq8 = p.part = p.queue = p.sel = p.hrec = p.squeue = 0;
+    if (kind == kPlanFull && fused_fits(d, T)) {
         p.xq8 = take((int64_t)T * (d.H / 256) * kActRec);
         p.part = take(P * (d.I / 128) * d.H * 4);
         p.queue = take(4);
         p.sel = take((int64_t)T * d.E * 4);
-    } else {
-        p.xq8 = p.part = p.queue = p.sel = 0;
+    } else if (kind != kPlanBase && split_fits(d)) {
+        p.xq8 = take((int64_t)T * (d.H / 256) * kActRec);
+        p.hrec = take(P * (d.I / 256) * kActRec);
+        p.squeue = take(2 * 4);
     }
     p.total = off;
     return p;
@@ -395,6 +413,16 @@ int launch_gemm(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, cudaS
 constexpr int kGemmMinTokens = 48;
 bool gemm_path_preferred(const coli_moe_desc&, int T) { return T >= kGemmMinTokens; }
 
+// AUTO past the fused path's limits: the two-pass path up to kSplitMaxT tokens
+// (GLM-5.2 prefill shapes on B200: 1.33 ms against the GEMM path's 3.93 ms at
+// 128 tokens, 2.67 against 4.17 ms at 512; the GEMM path wins at 2048, 6.7
+// against 9.5 ms, once units hold enough tokens to fill its 64-token tiles)
+constexpr int kSplitMaxT = 1024;
+coli_path large_batch_path(const coli_moe_desc& d, int bits, int T) {
+    if (bits == 4 && split_fits(d) && T <= kSplitMaxT && T > kFzMaxT) return COLI_PATH_TWOPASS;
+    return gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV;
+}
+
 template <int NT, bool GS>
 int launch_gateup_t(const coli_moe_desc& d, int units_max, const GemvArgs& a, cudaStream_t st) {
     const int smem = gemv_ring_bytes<true, GS>() + gemv_act_bytes(a.tok_cap, d.H);
@@ -458,6 +486,63 @@ int launch_gemv(const coli_moe_layer* l, int T, void* ws, const WsPlan& p, const
 // fused small-batch path
 // ---------------------------------------------------------------------------
 int sm_count() { return gemm_grid(); }
+
+// ---------------------------------------------------------------------------
+// two-pass path: x records, gate/up pass (h in f32), h records, down pass (o)
+// ---------------------------------------------------------------------------
+template <bool GS>
+int launch_split_t(const SplitArgs& a, cudaStream_t st, const char* what) {
+    const int smem = a.slots * a.slot_bytes;
+    int rc = set_smem((const void*)moe_split_kernel<GS>, smem);
+    if (rc) return rc;
+    return launch_pdl(moe_split_kernel<GS>, dim3(sm_count()), kFzThreads, smem, st, what, a);
+}
+
+template <typename Mark>
+int launch_split(const coli_moe_layer* l, const void* x, coli_dtype xt, int T, void* ws,
+                 const WsPlan& p, cudaStream_t st, Mark&& mark) {
+    const coli_moe_desc& d = l->run;
+    const int P = T * (d.k + d.n_shared);
+    int8_t* xrec = at<int8_t>(ws, p.xq8);
+    int rc = xt == COLI_F32
+        ? launch_pdl(act_records_kernel<float>, dim3(T), 256, 0, st, "x records",
+                     (const float*)x, d.H, xrec)
+        : launch_pdl(act_records_kernel<__nv_bfloat16>, dim3(T), 256, 0, st, "x records",
+                     (const __nv_bfloat16*)x, d.H, xrec);
+    if (rc) return rc;
+    SplitArgs a;
+    a.store = l->store;
+    a.L = l->L;
+    a.n_units = at<int32_t>(ws, p.n_units);
+    a.unit_expert = at<int32_t>(ws, p.unit_expert);
+    a.unit_begin = at<int32_t>(ws, p.unit_begin);
+    a.unit_end = at<int32_t>(ws, p.unit_end);
+    a.pair_tok = at<int32_t>(ws, p.pair_tok);
+    a.err = at<int32_t>(ws, p.err);
+    a.H = d.H; a.I = d.I;
+    a.slot_bytes = (int)align256(kFzActOff + kFzChunk * kActRec);
+    const int budget = 227 * 1024 - (int)sizeof(SplitShared) - 1024;
+    a.slots = std::min(kSpSlots, budget / a.slot_bytes);
+    if (a.slots < 2) return fail(COLI_E_UNSUPPORTED, "two-pass: ring does not fit");
+    const bool gs = d.group != 0;
+    float* hf = at<float>(ws, p.hq);                 // [P][I] f32
+    int8_t* hrec = at<int8_t>(ws, p.hrec);
+    a.act = xrec;
+    a.out = hf;
+    a.queue = at<int32_t>(ws, p.squeue);
+    a.down = 0;
+    if ((rc = gs ? launch_split_t<true>(a, st, "gate/up pass") : launch_split_t<false>(a, st, "gate/up pass")))
+        return rc;
+    if ((rc = mark(COLI_STAGE_DOWN))) return rc;
+    if ((rc = launch_pdl(act_records_kernel<float>, dim3(P), 256, 0, st, "h records",
+                         (const float*)hf, d.I, hrec)))
+        return rc;
+    a.act = hrec;
+    a.out = at<float>(ws, p.o);                      // [P][H] f32
+    a.queue = at<int32_t>(ws, p.squeue) + 1;
+    a.down = 1;
+    return gs ? launch_split_t<true>(a, st, "down pass") : launch_split_t<false>(a, st, "down pass");
+}
 
 // Launch with programmatic stream serialisation: the kernel may start while
 // the previous one (router, then fused) finishes; it waits
@@ -899,7 +984,7 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     if (!layer || !x || !y) return fail(COLI_E_INVAL, "forward: NULL pointer");
     if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_E_INVAL, "forward: bad dtype");
     if (path != COLI_PATH_AUTO && path != COLI_PATH_GEMV && path != COLI_PATH_GEMM &&
-        path != COLI_PATH_FUSED)
+        path != COLI_PATH_FUSED && path != COLI_PATH_TWOPASS)
         return fail(COLI_E_INVAL, "forward: bad path");
     const coli_moe_desc& d = layer->run;
     int rc = tokens_ok(d, T);
@@ -908,15 +993,19 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         return fail(COLI_E_UNSUPPORTED,
                     "forward: fused path needs T<=%d, T*(k+n_shared)<=%d, E<=%d, k<=%d, n_shared<=4, "
                     "H%%256==0, I<=4096", kFzMaxT, kFzMaxPairs, kFzMaxE, kFzMaxK);
+    if (path == COLI_PATH_TWOPASS && !split_fits(d))
+        return fail(COLI_E_UNSUPPORTED, "forward: two-pass path needs E<=%d, n_shared<=4, "
+                    "H%%256==0, I%%256==0", kFzMaxE);
     if (layer->bits == 8 && (path == COLI_PATH_GEMV || path == COLI_PATH_GEMM ||
+                             path == COLI_PATH_TWOPASS ||
                              (path == COLI_PATH_AUTO && !fused_fits(d, T))))
         return fail(COLI_E_UNSUPPORTED, "forward: 8-bit experts run on the fused path only (T<=%d, "
                     "T*(k+n_shared)<=%d, E<=%d, H%%256==0, I<=4096)", kFzMaxT, kFzMaxPairs, kFzMaxE);
     if (path == COLI_PATH_AUTO)
-        path = fused_fits(d, T) ? COLI_PATH_FUSED
-                                : (gemm_path_preferred(d, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV);
+        path = fused_fits(d, T) ? COLI_PATH_FUSED : large_batch_path(d, layer->bits, T);
     // the GEMV and GEMM paths need only a prefix of the full workspace
-    const WsPlan p = plan_ws(d, T, path == COLI_PATH_FUSED);
+    const WsPlan p = plan_ws(d, T, path == COLI_PATH_FUSED ? kPlanFull
+                                   : (path == COLI_PATH_TWOPASS ? kPlanSplit : kPlanBase));
     if (!ws || ws_bytes < (size_t)p.total)
         return fail(COLI_E_WORKSPACE, "forward: workspace %zu < %lld bytes", ws_bytes, (long long)p.total);
     cudaStream_t st = S(stream);
@@ -957,8 +1046,10 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
         return COLI_OK;
     }
     if ((rc = mark(COLI_STAGE_ROUTER))) return rc;
-    if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), at<__half>(ws, p.xq),
-                            at<float>(ws, p.xinv), st, &KS)))
+    const bool split = path == COLI_PATH_TWOPASS;
+    // the two-pass path makes its own activation records after the union
+    if ((rc = launch_router(d, x, xt, T, at<float>(ws, p.zpart), split ? nullptr : at<__half>(ws, p.xq),
+                            split ? nullptr : at<float>(ws, p.xinv), st, &KS)))
         return rc;
     UnionOut o{};
     o.offsets = at<int32_t>(ws, p.offsets);
@@ -971,8 +1062,8 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     o.unit_begin = at<int32_t>(ws, p.unit_begin);
     o.unit_end = at<int32_t>(ws, p.unit_end);
     o.n_units = at<int32_t>(ws, p.n_units);
-    o.counters = at<int32_t>(ws, p.counters);
-    o.n_counters = d.H / 64;
+    o.counters = at<int32_t>(ws, split ? p.squeue : p.counters);
+    o.n_counters = split ? 2 : d.H / 64;
     o.err = at<int32_t>(ws, p.err);
     o.n_shared = d.n_shared;
     o.w = w;  // picks of weight 0 (not computed by this call) are left out
@@ -980,8 +1071,10 @@ int coli_moe_forward_ex(const coli_moe_layer* layer, const void* x, coli_dtype x
     if ((rc = launch_select(d, layer->filter, at<float>(ws, p.zpart), KS, T, idx, w, o, st)))
         return rc;
     if ((rc = mark(COLI_STAGE_GATEUP))) return rc;
-    if (gemm) {
-        if ((rc = launch_gemm(layer, T, ws, p, st, mark))) return rc;
+    if (gemm || split) {
+        if ((rc = split ? launch_split(layer, x, xt, T, ws, p, st, mark)
+                        : launch_gemm(layer, T, ws, p, st, mark)))
+            return rc;
         if ((rc = mark(COLI_STAGE_COMBINE))) return rc;
         const int64_t n4 = (int64_t)T * (d.H / 4);
         combine_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
@@ -1214,10 +1307,10 @@ int coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x, coli_dt
     // the path AUTO would take if its workspace fits the array, else the
     // GEMV/GEMM path, whose workspace is a prefix of the full one
     coli_path path = COLI_PATH_AUTO;
-    int64_t need = plan_ws(layer->run, T, true).total;
+    int64_t need = plan_ws(layer->run, T, kPlanFull).total;
     if (need > (int64_t)COLI_NOALLOC_SCRATCH_BYTES) {
         path = gemm_path_preferred(layer->run, T) ? COLI_PATH_GEMM : COLI_PATH_GEMV;
-        need = plan_ws(layer->run, T, false).total;
+        need = plan_ws(layer->run, T, kPlanBase).total;
     }
     if (need > (int64_t)COLI_NOALLOC_SCRATCH_BYTES)
         return fail(COLI_E_UNSUPPORTED,

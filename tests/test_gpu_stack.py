@@ -30,7 +30,8 @@ from tests.workloads import OracleExperts, build_layer
 
 pytestmark = pytest.mark.gpu
 
-TOL = {cm.COLI_PATH_FUSED: 2e-3, cm.COLI_PATH_GEMV: 2e-3, cm.COLI_PATH_GEMM: 1e-2}
+TOL = {cm.COLI_PATH_FUSED: 2e-3, cm.COLI_PATH_GEMV: 2e-3, cm.COLI_PATH_GEMM: 1e-2,
+       cm.COLI_PATH_TWOPASS: 2e-3}
 THREADS = max(1, min(16, os.cpu_count() or 1))
 
 
@@ -150,6 +151,34 @@ def test_tiny_stack_teacher_forced(tiny_stack, path, T):
     assert excluded <= T * TINY_STACK.layers // 2
 
 
+# the two-pass path needs I to be a multiple of 256
+TINY_STACK_I256 = dataclasses.replace(TINY_STACK, I=256, seed=5102)
+
+
+@pytest.fixture(scope="module")
+def tiny_stack_i256():
+    layers = [build_layer(TINY_STACK_I256, layer=l) for l in range(TINY_STACK_I256.layers)]
+    yield layers
+    for L in layers:
+        L.close()
+
+
+@pytest.mark.parametrize("T", [3, 90])
+def test_tiny_stack_two_pass(tiny_stack_i256, T):
+    x0 = stack_tokens(TINY_STACK_I256, T, step=200 + T).cuda()
+    worst, excluded = check_stack(TINY_STACK_I256, tiny_stack_i256, x0, cm.COLI_PATH_TWOPASS)
+    print(f"tiny stack two-pass T={T}: worst layer error {worst:.2e}, excluded tokens {excluded}")
+    assert excluded <= T * TINY_STACK_I256.layers // 2
+
+
+def test_tiny_stack_auto_takes_two_pass_past_the_fused_limit(tiny_stack_i256):
+    handles = [L.handle for L in tiny_stack_i256]
+    x0 = stack_tokens(TINY_STACK_I256, 90, step=390).cuda()
+    a, _ = run_stack(handles, x0, 90, TINY_STACK_I256.eps, cm.COLI_PATH_AUTO)
+    b, _ = run_stack(handles, x0, 90, TINY_STACK_I256.eps, cm.COLI_PATH_TWOPASS)
+    np.testing.assert_array_equal(a.cpu().numpy().view(np.uint32), b.cpu().numpy().view(np.uint32))
+
+
 def test_tiny_stack_auto_equals_chosen_path(tiny_stack):
     """AUTO takes the fused kernel at 4 tokens and the tensor-core path at 80:
     the same bytes as asking for those paths."""
@@ -210,6 +239,23 @@ def test_glm_stack16_sixteen_tokens(glm_stack):
                                   sample=lambda l, idx: (l % 16, (l + 7) % 16))
     print(f"GLM stack T=16: worst layer error {worst:.2e}, excluded {excluded}")
     assert excluded <= 16 * wl.layers // 2
+
+
+def test_glm_stack16_prefill_two_pass(glm_stack):
+    """512 tokens on the two-pass path (what AUTO takes there): the same samples
+    as the tensor-core test below, at the s8 path's tolerance."""
+    wl = synth.GLM_STACK
+
+    def sample(l, idx):
+        counts = np.bincount(idx.ravel(), minlength=wl.E)
+        hot = int(np.argmax(counts))
+        last_hot = int(np.nonzero((idx == hot).any(1))[0][-1])
+        return (last_hot, 256 + (37 * l) % 256)
+
+    x0 = stack_tokens(wl, 512, step=2).cuda()
+    worst, excluded = check_stack(wl, glm_stack, x0, cm.COLI_PATH_TWOPASS, sample=sample)
+    print(f"GLM stack T=512 two-pass: worst layer error {worst:.2e}, excluded {excluded}")
+    assert excluded <= 512 * wl.layers // 2
 
 
 def test_glm_stack16_prefill_tensor_cores(glm_stack):
