@@ -881,18 +881,47 @@ __device__ __forceinline__ void fz_consume(const FusedArgs& a, FusedShared& sh, 
                 for (int i = 0; i < 4; ++i) acc_f[c][i] = 0.0f;
         }
         const bool gu = st < z.nst_gu;
+        const int ntc = (np + 3) >> 2;  // column groups holding the item's pairs
         if (gu) {
-            fz_stage_gateup<NT, GS, W8>(sl, m, rb, lane, rec_gu, aoff, xsoff0, np,
-                                        W8 ? (st & 1) * 2 : 0, (np + 3) >> 2, st == z.nst_gu - 1,
-                                        acc_f);
+            // the column-group count as a compile-time constant: no branch inside
+            // the unrolled MMA loops
+            const int jo = W8 ? (st & 1) * 2 : 0;
+            const bool lst = st == z.nst_gu - 1;
+#define FZ_GU(K) fz_stage_gateup<K, GS, W8>(sl, m, rb, lane, rec_gu, aoff, xsoff0, np, jo, K, lst, acc_f)
+            if constexpr (NT == 1) {
+                FZ_GU(1);
+            } else if constexpr (NT == 2) {
+                if (ntc == 1) FZ_GU(1); else FZ_GU(2);
+            } else {
+                switch (ntc) {
+                    case 1: FZ_GU(1); break;
+                    case 2: FZ_GU(2); break;
+                    case 3: FZ_GU(3); break;
+                    default: FZ_GU(4); break;
+                }
+            }
+#undef FZ_GU
             if (!GS && st == z.nst_gu - 1) {
                 const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
                 sw0 = rsc[0];
                 sw1 = rsc[8];
             }
         } else {
-            fz_stage_down<NT, GS, W8>(a, sh, sl, z.rs, (st - z.nst_gu) * z.rs, (np + 3) >> 2, hf, dst,
-                                      warp, lane);
+            const int rt0 = (st - z.nst_gu) * z.rs;
+#define FZ_DN(K) fz_stage_down<K, GS, W8>(a, sh, sl, z.rs, rt0, K, hf, dst, warp, lane)
+            if constexpr (NT == 1) {
+                FZ_DN(1);
+            } else if constexpr (NT == 2) {
+                if (ntc == 1) FZ_DN(1); else FZ_DN(2);
+            } else {
+                switch (ntc) {
+                    case 1: FZ_DN(1); break;
+                    case 2: FZ_DN(2); break;
+                    case 3: FZ_DN(3); break;
+                    default: FZ_DN(4); break;
+                }
+            }
+#undef FZ_DN
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[s]);

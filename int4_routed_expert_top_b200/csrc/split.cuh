@@ -247,8 +247,14 @@ __device__ __forceinline__ void sp_consume(const SplitArgs& a, SplitShared& sh, 
                 for (int i = 0; i < 4; ++i) acc_f[c][i] = 0.0f;
         }
         const bool last = st == nst - 1;
-        fz_stage_gateup<NT, GS, false>(sl, m, rb, lane, kActRec, aoff, xsoff0, np, 0, (np + 3) >> 2,
-                                       last, acc_f);
+        // the chunk's column groups as a compile-time count: no branch inside
+        // the unrolled MMA loops
+        switch ((np + 3) >> 2) {
+            case 1: fz_stage_gateup<1, GS, false>(sl, m, rb, lane, kActRec, aoff, xsoff0, np, 0, 1, last, acc_f); break;
+            case 2: fz_stage_gateup<2, GS, false>(sl, m, rb, lane, kActRec, aoff, xsoff0, np, 0, 2, last, acc_f); break;
+            case 3: fz_stage_gateup<3, GS, false>(sl, m, rb, lane, kActRec, aoff, xsoff0, np, 0, 3, last, acc_f); break;
+            default: fz_stage_gateup<4, GS, false>(sl, m, rb, lane, kActRec, aoff, xsoff0, np, 0, 4, last, acc_f); break;
+        }
         if (!GS && last) {
             const float* rsc = reinterpret_cast<const float*>(sl + kFzScaleOff + m * 512) + 16 * rb + g;
             sw0 = rsc[0];
