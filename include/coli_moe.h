@@ -266,7 +266,8 @@ int coli_moe_layer_set_partition(coli_moe_layer* layer, int32_t e_begin, int32_t
 int coli_moe_layer_set_wait_test(coli_moe_layer* layer, int32_t withhold_stage);
 
 /* Workspace bytes that coli_moe_route / coli_moe_forward need for T tokens
- * (enough for every path; the GEMV and GEMM paths use only a prefix). */
+ * (enough for every path; the GEMV and GEMM paths use only a prefix, the
+ * fused and two-pass paths that prefix and their own buffers after it). */
 int coli_moe_workspace_size(const coli_moe_layer* layer, int32_t T, size_t* bytes);
 
 /* Step 1 alone.  x device [T, H] (f32 or bf16); idx device i32 [T, k] ordered
@@ -376,7 +377,7 @@ int coli_moe_status(const coli_moe_layer* layer, int32_t T, const void* ws,
  * (ws planned for T tokens; device i32 outputs, each may be NULL): offsets
  * [E+1], pair_tok and pair_slot [T*k] (pairs of computed picks grouped by
  * expert, experts ascending, tokens ascending), uniq [E] (first n_uniq
- * entries), n_uniq [1] after a GEMV- or GEMM-path forward; inv [T*k] (the
+ * entries), n_uniq [1] after a GEMV-, GEMM- or two-pass forward; inv [T*k] (the
  * pair of each pick, -1 for a pick not computed) after any path.  The fused
  * path keeps its union in shared memory, in the order the picks first name
  * their experts: only inv describes it.  Asynchronous. */

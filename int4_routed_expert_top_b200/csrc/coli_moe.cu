@@ -415,8 +415,8 @@ bool gemm_path_preferred(const coli_moe_desc&, int T) { return T >= kGemmMinToke
 
 // AUTO past the fused path's limits: the two-pass path up to kSplitMaxT tokens
 // (GLM-5.2 prefill shapes on B200: 1.33 ms against the GEMM path's 3.93 ms at
-// 128 tokens, 2.67 against 4.17 ms at 512; the GEMM path wins at 2048, 6.7
-// against 9.5 ms, once units hold enough tokens to fill its 64-token tiles)
+// 128 tokens, 2.28 against 4.17 ms at 512; the GEMM path wins at 2048, 6.7
+// against 8.1 ms, once units hold enough tokens to fill its 64-token tiles)
 constexpr int kSplitMaxT = 1024;
 coli_path large_batch_path(const coli_moe_desc& d, int bits, int T) {
     if (bits == 4 && split_fits(d) && T <= kSplitMaxT && T > kFzMaxT) return COLI_PATH_TWOPASS;

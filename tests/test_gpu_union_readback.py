@@ -161,3 +161,18 @@ def test_forward_union_of_an_expert_range(T):
             assert ((u["uniq"][: int(u["n_uniq"][0])] >= 16) &
                     (u["uniq"][: int(u["n_uniq"][0])] < 48)).all()
     L.close()
+
+
+@pytest.mark.parametrize("topp", [0.0, 0.7])
+@pytest.mark.parametrize("T,E,k", [(70, 16, 4), (300, 8, 2)])
+def test_two_pass_forward_union_matches_oracle(T, E, k, topp):
+    """The two-pass path (I a multiple of 256) builds the same union as the
+    GEMV/GEMM paths: units of many 16-pair chunks included."""
+    wl = dataclasses.replace(synth.TINY, I=256, T=T, E=E, k=k, group=64)
+    router = synth.router(wl)
+    x, _, _, _ = gap_resampled_tokens(wl, T, *router)
+    L = build_layer(wl, router=router)
+    cm.coli_moe_layer_set_topp(L.handle, topp)
+    idx, w, u = forward(L, x.cuda(), T, cm.COLI_PATH_TWOPASS)
+    check_grouped(idx, w, u, wl.E)
+    L.close()
