@@ -644,6 +644,21 @@ def main():
     barrier()
     e2e_med = statistics.median(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
     e2e_value = job_tokens_per_s(T, world, max_over_ranks(e2e_med, world, dev))
+    # the same steps on the host's clock: each replay is submitted and waited
+    # for (after the flush has finished), so host submission counts too
+    wall = []
+    barrier()
+    for i in range(K):
+        flush.zero_()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e2e_graphs[i % n_pool].replay()
+        torch.cuda.synchronize()
+        wall.append((time.perf_counter() - t0) * 1e3)
+    barrier()
+    wall_ms = max_over_ranks(statistics.median(wall), world, dev)
+    e2e_wall = {"value": job_tokens_per_s(T, world, wall_ms), "unit": UNIT, "ms_per_step": wall_ms,
+                "timing": "host perf_counter around each replay and its synchronize, median"}
 
     # bytes: int4 codes + f32 scales of the unique routed experts + shared, per step
     blob = L0.blob_bytes
@@ -738,7 +753,8 @@ def main():
     line["clocks"] = clocks.summary()
     line["e2e"] = {"value": e2e_value, "unit": UNIT,
                    "h2d_bytes_per_step": int(xpool[0].numel() * xpool.element_size()),
-                   "d2h_bytes_per_step": int(T * wl.H * 4)}
+                   "d2h_bytes_per_step": int(T * wl.H * 4),
+                   "wall_clock": e2e_wall}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tok_s, n, secs, smp = oracle_sample(wl)
         threads = oracle_threads()
